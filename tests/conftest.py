@@ -1,0 +1,16 @@
+"""Shared pytest configuration.
+
+Marker `gpu`: the test needs a CUDA device (B200, sm_100a) and the built
+CUDA library. Everything else runs on the CPU.
+"""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device and the built sm_100a library")
+    config.addinivalue_line("markers", "slow: long-running CPU test")
