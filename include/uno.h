@@ -1,0 +1,209 @@
+/*
+ * uno.h — C ABI of the sm_100a (B200) Psi-Spec linear decode step.
+ *
+ * The method ("Uno", diffusion-augmented LLMs with the Psi-Spec sampler):
+ *   - every AR weight matrix carries a LoRA adapter theta_Delta; drafting uses
+ *     theta_AR + theta_Delta, verification theta_AR alone (hyper.ai page,
+ *     section "方法", the paragraph on theta_Delta);
+ *   - one forward serves both paths through a per-row gate that switches the
+ *     adapter off on clean rows and on for noisy rows (same section, the
+ *     gated-LoRA paragraph; ainews page: "conditional LoRA");
+ *   - the linear sampler drafts one block from the draft path's per-position
+ *     marginals, and rejection sampling against the AR distribution keeps the
+ *     longest accepted prefix (same section, the Psi-Spec paragraph);
+ *   - "lossless" means the output follows the AR distribution (ainews page).
+ *
+ * Conventions for every call
+ *   - Pointers named as device pointers must be device memory of the current
+ *     device, 16-byte aligned. The caller owns every buffer; the library never
+ *     allocates device memory on these calls (scratch comes from `workspace`,
+ *     sized by the matching *_workspace query).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls
+ *     only enqueue work on it and return; results are ready when the stream
+ *     reaches them.
+ *   - Errors found on the host return a status at once and launch nothing;
+ *     uno_last_error() describes the last one on the calling thread.
+ *     Conditions found on the device (a draft id outside the vocabulary, a NaN
+ *     logit, a bounded wait that gave up) OR bits into `dev_status` (where the
+ *     call has one) and into the library's device status word (see
+ *     uno_device_status); no kernel traps.
+ *   - Row-major layouts throughout. bf16 is IEEE bfloat16 bits; f32 is float.
+ */
+#ifndef UNO_H_
+#define UNO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  UNO_OK = 0,
+  UNO_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or value */
+  UNO_ERR_UNSUPPORTED = 2,  /* valid but outside the supported range */
+  UNO_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  UNO_ERR_TIMEOUT = 4,      /* reported through uno_device_status */
+  UNO_ERR_DEVICE_FLAG = 5,  /* reported through uno_device_status */
+  UNO_ERR_WORKSPACE = 6     /* workspace NULL or smaller than the query says */
+} uno_status;
+
+typedef enum { UNO_BF16 = 0, UNO_F32 = 1 } uno_dtype;
+
+/* Device status bits (dev_status words and uno_device_status). */
+#define UNO_DEV_BAD_DRAFT 1 /* a draft id outside [0, V): that sequence's outputs are -1 */
+#define UNO_DEV_NAN 2       /* a NaN logit in a row that was read: outputs are -1 */
+#define UNO_DEV_TIMEOUT 4   /* a bounded on-device wait gave up (kernel returned early) */
+
+/* Message for the last failed call on this thread (static storage, valid
+ * until the next call on this thread). Never NULL. */
+const char* uno_last_error(void);
+
+/* Library version string. */
+const char* uno_version(void);
+
+/* Read the library-wide device status word of the current device into
+ * *bits_out (synchronises `stream`), clearing it when `clear` != 0. */
+uno_status uno_device_status(int32_t* bits_out, int32_t clear, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Gated-LoRA linear (hyper.ai page, section "方法": LoRA adapter on every AR
+ * matrix, gated per row in one forward pass):
+ *
+ *     y = x W^T + scale * g (.) ((x A^T) Bl^T)
+ *
+ *   x [M,K], W [N,K], A [r,K], Bl [N,r] (nn.Linear / PEFT layout), all `dt`;
+ *   gate [M] uint8 in {0,1} (0 = adapter off: the verify path theta_AR;
+ *   1 = adapter on: the draft path theta_AR + theta_Delta); y [M,N] `dt`.
+ *   fp32 accumulation. The rank-r product x A^T is rounded to `dt` before the
+ *   up-projection, which runs in the same tensor-core pass as x W^T, so W is
+ *   read from HBM once.
+ *   Sizes: M >= 0 (M = 0 launches nothing), K >= 1, N >= 1, 0 <= r <= 256.
+ *   bf16: K, N, r multiples of 8; f32: multiples of 4 (16-byte row strides).
+ *   f32 inputs run on the tf32 tensor-core path (10-bit mantissa products).
+ *   workspace: >= uno_gated_lora_linear_workspace(...) bytes of device memory.
+ * ------------------------------------------------------------------------- */
+size_t uno_gated_lora_linear_workspace(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r);
+
+uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r,
+                                 const void* x, const void* W, const void* A, const void* Bl,
+                                 const uint8_t* gate, float scale, void* y, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Psi-Spec verification of one drafted block per sequence (hyper.ai page,
+ * section "方法", the Psi-Spec paragraph: rejection sampling against the base
+ * AR distribution, longest valid prefix; ainews page: lossless).
+ *
+ *   p_logits [B,k_p,V]: AR logits for the k drafted positions (k_p = k) plus,
+ *     when k_p = k+1, the position after the block (bonus draw).
+ *   q_logits [B,k,V]: draft logits; draft [B,k] int32: the drafted ids.
+ *   With p = softmax(p_logits / T), q = softmax(q_logits / T) per position
+ *   and uniforms u from Philox4x32-10 (counter = (b_global*k + j, step lo,
+ *   step hi, stream), key = (seed lo, seed hi), u = (word0 >> 8) * 2^-24,
+ *   b_global = seq_offset + b; stream 1 accept, 2 residual, 3 bonus):
+ *     accept position j iff u1 * q_j(d_j) < p_j(d_j);
+ *     n = first rejected position (k if none)          -> accepted_len[b]
+ *     out_tokens[b] = d_0..d_{n-1}, then
+ *       if n < k: r = smallest v with C(v) > u2 * C(V-1), C the inclusive
+ *                 cumulative sum of max(p_n - q_n, 0) in ascending id (p_n
+ *                 itself if that sum is 0);
+ *       if n = k and k_p = k+1: the bonus, same rule on p_k with u3;
+ *     padded with -1; out_count[b] = number of tokens written.
+ *   out_tokens is [B, k+1]. T > 0. 1 <= k <= 32, 2 <= V <= 196608.
+ *   dev_status: optional int32 device word, OR-ed with UNO_DEV_* bits.
+ * ------------------------------------------------------------------------- */
+size_t uno_psi_verify_workspace(int32_t B, int32_t k, int32_t k_p, int32_t V);
+
+uno_status uno_psi_verify(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32_t V,
+                          const void* p_logits, const void* q_logits, const int32_t* draft,
+                          float temperature, uint64_t seed, uint64_t step, uint64_t seq_offset,
+                          int32_t* accepted_len, int32_t* out_tokens, int32_t* out_count,
+                          int32_t* dev_status, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Linear-sampler draft (hyper.ai page, section "方法": the linear sampler
+ * draws one candidate block from the per-position marginals):
+ *   draft[b,j] = smallest v with C(v) > u0 * C(V-1), C the inclusive
+ *   cumulative sum of softmax(q_logits[b,j] / T) in ascending id; u0 from
+ *   Philox stream 0 at index (seq_offset + b)*k + j.
+ *   q_logits [B,k,V] `dt`; draft [B,k] int32 (device).
+ * ------------------------------------------------------------------------- */
+size_t uno_draft_sample_workspace(int32_t B, int32_t k, int32_t V);
+
+uno_status uno_draft_sample(uno_dtype dt, int32_t B, int32_t k, int32_t V, const void* q_logits,
+                            float temperature, uint64_t seed, uint64_t step, uint64_t seq_offset,
+                            int32_t* draft, int32_t* dev_status, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Philox uniforms, exposed so the generator can be checked bit for bit:
+ *   words[i] = Philox4x32-10 word 0 at counter (index0 + i, step lo, step hi,
+ *   stream), key (seed lo, seed hi); u[i] = (words[i] >> 8) * 2^-24.
+ *   Either output may be NULL. n >= 0, index0 + n <= 2^32.
+ * ------------------------------------------------------------------------- */
+uno_status uno_philox_uniforms(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,
+                               int64_t n, uint32_t* words, float* u, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Synthetic decode step (the linear decode step of Psi-Spec on a stand-in
+ * decoder stack: gated-LoRA projections of every layer, no attention; the
+ * model-side rules come from hyper.ai page, section "方法", the shapes from
+ * section "实验" — rank-128 adapters on Qwen3-8B):
+ *
+ *   per layer:  n = rmsnorm(h); q = L_q(n); k = L_k(n); v = L_v(n) (unused);
+ *               h = h + L_o(q); n = rmsnorm(h);
+ *               h = h + L_down(silu(L_gate(n)) * L_up(n))
+ *   logits = L_head(rmsnorm(h)), rmsnorm(x) = x / sqrt(mean(x^2) + 1e-6)
+ *
+ * with L = the gated-LoRA linear above, bf16 storage between operations.
+ *
+ * Model handle: holds device pointers and cached launch descriptors only;
+ * the caller owns (and keeps alive) the weight memory. `weights` lists, for
+ * each layer in order, the (W, A, Bl) device pointers of q, k, v, o, gate, up,
+ * down (21 per layer), then those of the LM head: 21 * n_layers + 3 pointers.
+ * Shapes: q [q_out, hidden], k and v [kv_out, hidden], o [hidden, q_out],
+ * gate and up [inter, hidden], down [hidden, inter], head [vocab, hidden];
+ * A [r, in], Bl [out, r]. All bf16.
+ * ------------------------------------------------------------------------- */
+typedef struct uno_model uno_model;
+
+uno_status uno_model_create(uno_model** out, int32_t n_layers, int32_t hidden, int32_t q_out,
+                            int32_t kv_out, int32_t inter, int32_t vocab, int32_t r, float scale,
+                            const void* const* weights);
+void uno_model_destroy(uno_model* m);
+
+/* One step for B sequences with block size k (M = B(2k+1) rows):
+ *   h_in [M, hidden] bf16: rows 0..B(k+1)-1 are the verify rows (gate 0,
+ *     sequence-major: anchor + k drafted tokens), then B*k mask rows
+ *     (gate 1) that produce the next block's draft distributions.
+ *   Verifies the previous block (q_prev [B,k,V] bf16, d_prev [B,k] int32)
+ *   against this step's AR rows p [B,k+1,V] (bonus enabled), as
+ *   uno_psi_verify with k_p = k+1 and the same seed/step; then drafts the next
+ *   block from the mask rows as uno_draft_sample (same seed/step) into
+ *   d_next [B,k], and writes their logits to q_next [B,k,V] bf16.
+ *   logits_out: optional [B(k+1), V] bf16 copy target for the AR rows (NULL
+ *   to skip). accepted_len [B], out_tokens [B,k+1], out_count [B] as in
+ *   uno_psi_verify. q_next must not alias q_prev. */
+size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k);
+
+uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, const void* q_prev,
+                        const int32_t* d_prev, float temperature, uint64_t seed, uint64_t step,
+                        void* q_next, int32_t* d_next, void* logits_out, int32_t* accepted_len,
+                        int32_t* out_tokens, int32_t* out_count, int32_t* dev_status,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The step's glue operations, exposed for testing (all bf16, device):
+ *   uno_rmsnorm:  y[m,:] = x[m,:] / sqrt(mean(x[m,:]^2) + eps)      x, y [M,D]
+ *   uno_silu_mul: y = silu(a) * b = a / (1 + exp(-a)) * b           [n]
+ * ------------------------------------------------------------------------- */
+uno_status uno_rmsnorm(int64_t M, int64_t D, const void* x, void* y, float eps, void* stream);
+uno_status uno_silu_mul(int64_t n, const void* a, const void* b, void* y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UNO_H_ */

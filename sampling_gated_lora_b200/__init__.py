@@ -1,0 +1,293 @@
+"""Python binding of libuno.so — the sm_100a Psi-Spec linear decode step.
+
+Argument marshalling only: every operation runs in the library's CUDA kernels
+(include/uno.h). PyTorch supplies device memory and streams. There is no CPU
+fallback: if libuno.so is missing or cannot load, every call raises.
+
+Functions mirror the C ABI:
+    gated_lora_linear  y = x W^T + s g (x A^T) Bl^T
+    psi_verify         accept u q(d) < p(d), longest prefix, residual / bonus draw
+    draft_sample       linear-sampler draft from softmax(q / T)
+    philox_uniforms    the generator's words and uniforms, for bit-exact checks
+    rmsnorm, silu_mul  the step's glue operations
+    Model              synthetic decoder stack + LM head; Model.step = uno_psi_step
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libuno.so")
+
+UNO_BF16, UNO_F32 = 0, 1
+DEV_BAD_DRAFT, DEV_NAN, DEV_TIMEOUT = 1, 2, 4
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT",
+                5: "DEVICE_FLAG", 6: "WORKSPACE"}
+
+EXPORTS = [
+    "uno_last_error", "uno_version", "uno_device_status",
+    "uno_gated_lora_linear_workspace", "uno_gated_lora_linear",
+    "uno_psi_verify_workspace", "uno_psi_verify",
+    "uno_draft_sample_workspace", "uno_draft_sample",
+    "uno_philox_uniforms",
+    "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
+    "uno_rmsnorm", "uno_silu_mul",
+]
+
+
+class UnoError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def load():
+    """Load libuno.so (raises if it is missing or broken)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m sampling_gated_lora_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, u32, u64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                       ctypes.c_uint32, ctypes.c_uint64, ctypes.c_float,
+                                       ctypes.c_size_t)
+    sig = {
+        "uno_last_error": (ctypes.c_char_p, []),
+        "uno_version": (ctypes.c_char_p, []),
+        "uno_device_status": (i32, [vp, i32, vp]),
+        "uno_gated_lora_linear_workspace": (sz, [i32, i64, i64, i64, i32]),
+        "uno_gated_lora_linear": (i32, [i32, i64, i64, i64, i32, vp, vp, vp, vp, vp, f32, vp, vp,
+                                        sz, vp]),
+        "uno_psi_verify_workspace": (sz, [i32, i32, i32, i32]),
+        "uno_psi_verify": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, f32, u64, u64, u64, vp, vp,
+                                 vp, vp, vp, sz, vp]),
+        "uno_draft_sample_workspace": (sz, [i32, i32, i32]),
+        "uno_draft_sample": (i32, [i32, i32, i32, i32, vp, f32, u64, u64, u64, vp, vp, vp, sz, vp]),
+        "uno_philox_uniforms": (i32, [u64, u64, u32, u32, i64, vp, vp, vp]),
+        "uno_model_create": (i32, [vp, i32, i32, i32, i32, i32, i32, i32, f32, vp]),
+        "uno_model_destroy": (None, [vp]),
+        "uno_psi_step_workspace": (sz, [vp, i32, i32]),
+        "uno_psi_step": (i32, [vp, i32, i32, vp, vp, vp, f32, u64, u64, vp, vp, vp, vp, vp, vp, vp,
+                               vp, sz, vp]),
+        "uno_rmsnorm": (i32, [i64, i64, vp, vp, f32, vp]),
+        "uno_silu_mul": (i32, [i64, vp, vp, vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def version() -> str:
+    return load().uno_version().decode()
+
+
+def _check(st: int):
+    if st != 0:
+        raise UnoError(st, load().uno_last_error().decode())
+
+
+# ---------------------------------------------------------------- marshalling helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return UNO_BF16
+    if t.dtype == torch.float32:
+        return UNO_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must be on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def _workspace(nbytes, device, workspace):
+    torch = _torch()
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+# ---------------------------------------------------------------- operations
+
+def gated_lora_linear(x, W, A, Bl, gate, scale=1.0, y=None, workspace=None, stream=None):
+    """y [M,N] = x W^T + scale * gate (x A^T) Bl^T (bf16 or f32 tensors, uint8 gate)."""
+    torch = _torch()
+    L = load()
+    M, K = x.shape
+    N = W.shape[0]
+    r = A.shape[0] if A is not None else 0
+    if y is None:
+        y = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    _dev(x, W, A, Bl, gate, y)
+    dt = _dtype(x)
+    need = L.uno_gated_lora_linear_workspace(dt, M, K, N, r)
+    ws, wsb = _workspace(need, x.device, workspace)
+    _check(L.uno_gated_lora_linear(dt, M, K, N, r, _ptr(x), _ptr(W), _ptr(A), _ptr(Bl),
+                                   _ptr(gate), float(scale), _ptr(y), _ptr(ws), wsb,
+                                   _stream(stream)))
+    return y
+
+
+def psi_verify(p_logits, q_logits, draft, temperature, seed, step, seq_offset=0,
+               accepted_len=None, out_tokens=None, out_count=None, dev_status=None,
+               workspace=None, stream=None):
+    """Verify one block per sequence; returns (accepted_len [B], out_tokens [B,k+1], out_count [B])."""
+    torch = _torch()
+    L = load()
+    B, k_p, V = p_logits.shape
+    k = q_logits.shape[1]
+    dev = p_logits.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    accepted_len = torch.empty(B, **i32) if accepted_len is None else accepted_len
+    out_tokens = torch.empty((B, k + 1), **i32) if out_tokens is None else out_tokens
+    out_count = torch.empty(B, **i32) if out_count is None else out_count
+    _dev(p_logits, q_logits, draft, accepted_len, out_tokens, out_count, dev_status)
+    need = L.uno_psi_verify_workspace(B, k, k_p, V)
+    ws, wsb = _workspace(need, dev, workspace)
+    _check(L.uno_psi_verify(_dtype(p_logits), B, k, k_p, V, _ptr(p_logits), _ptr(q_logits),
+                            _ptr(draft), float(temperature), int(seed), int(step), int(seq_offset),
+                            _ptr(accepted_len), _ptr(out_tokens), _ptr(out_count),
+                            _ptr(dev_status), _ptr(ws), wsb, _stream(stream)))
+    return accepted_len, out_tokens, out_count
+
+
+def draft_sample(q_logits, temperature, seed, step, seq_offset=0, draft=None, dev_status=None,
+                 stream=None):
+    """Linear-sampler draft: draft [B,k] int32 from softmax(q_logits / T)."""
+    torch = _torch()
+    L = load()
+    B, k, V = q_logits.shape
+    draft = torch.empty((B, k), dtype=torch.int32, device=q_logits.device) if draft is None else draft
+    _dev(q_logits, draft, dev_status)
+    _check(L.uno_draft_sample(_dtype(q_logits), B, k, V, _ptr(q_logits), float(temperature),
+                              int(seed), int(step), int(seq_offset), _ptr(draft), _ptr(dev_status),
+                              None, 0, _stream(stream)))
+    return draft
+
+
+def philox_uniforms(seed, step, stream_id, index0, n, device="cuda", stream=None):
+    """(words uint32 as int64 tensor, u float32) of Philox word 0 at indices index0..index0+n-1."""
+    torch = _torch()
+    L = load()
+    words = torch.empty(n, dtype=torch.int32, device=device)
+    u = torch.empty(n, dtype=torch.float32, device=device)
+    _check(L.uno_philox_uniforms(int(seed), int(step), int(stream_id), int(index0), int(n),
+                                 _ptr(words), _ptr(u), _stream(stream)))
+    return words.to(torch.int64) & 0xFFFFFFFF, u
+
+
+def rmsnorm(x, eps=1e-6, y=None, stream=None):
+    torch = _torch()
+    L = load()
+    y = torch.empty_like(x) if y is None else y
+    _dev(x, y)
+    M, D = x.shape
+    _check(L.uno_rmsnorm(M, D, _ptr(x), _ptr(y), float(eps), _stream(stream)))
+    return y
+
+
+def silu_mul(a, b, y=None, stream=None):
+    torch = _torch()
+    L = load()
+    y = torch.empty_like(a) if y is None else y
+    _dev(a, b, y)
+    _check(L.uno_silu_mul(a.numel(), _ptr(a), _ptr(b), _ptr(y), _stream(stream)))
+    return y
+
+
+def device_status(clear=True, stream=None) -> int:
+    """The library-wide device status bits (UNO_DEV_*), optionally cleared."""
+    L = load()
+    v = ctypes.c_int32(0)
+    _check(L.uno_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)))
+    return v.value
+
+
+LINEAR_NAMES = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+class Model:
+    """Handle over caller-owned bf16 weights of the synthetic decoder stack.
+
+    layers: list of dicts name -> (W, A, Bl) for the names in LINEAR_NAMES;
+    head: (W, A, Bl) of the LM head. The tensors must stay alive with the model.
+    """
+
+    def __init__(self, layers, head, hidden, q_out, kv_out, inter, vocab, r, scale=1.0):
+        L = load()
+        self._keep = (layers, head)
+        ptrs = []
+        for lw in layers:
+            for name in LINEAR_NAMES:
+                for t in lw[name]:
+                    _dev(t)
+                    ptrs.append(t.data_ptr())
+        for t in head:
+            _dev(t)
+            ptrs.append(t.data_ptr())
+        arr = (ctypes.c_void_p * len(ptrs))(*ptrs)
+        h = ctypes.c_void_p()
+        _check(L.uno_model_create(ctypes.byref(h), len(layers), hidden, q_out, kv_out, inter,
+                                  vocab, r, float(scale), arr))
+        self._h = h
+        self.n_layers, self.hidden, self.vocab, self.r = len(layers), hidden, vocab, r
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            load().uno_model_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, B, k):
+        return load().uno_psi_step_workspace(self._h, B, k)
+
+    def step(self, B, k, h_in, q_prev, d_prev, temperature, seed, step, q_next, d_next,
+             accepted_len, out_tokens, out_count, workspace, logits_out=None, dev_status=None,
+             stream=None):
+        """uno_psi_step on caller-provided device buffers (see include/uno.h)."""
+        _dev(h_in, q_prev, d_prev, q_next, d_next, accepted_len, out_tokens, out_count, workspace,
+             logits_out, dev_status)
+        wsb = workspace.numel() * workspace.element_size()
+        _check(load().uno_psi_step(self._h, B, k, _ptr(h_in), _ptr(q_prev), _ptr(d_prev),
+                                   float(temperature), int(seed), int(step), _ptr(q_next),
+                                   _ptr(d_next), _ptr(logits_out), _ptr(accepted_len),
+                                   _ptr(out_tokens), _ptr(out_count), _ptr(dev_status),
+                                   _ptr(workspace), wsb, _stream(stream)))

@@ -1,0 +1,589 @@
+// C ABI of the library (include/uno.h): argument validation, error reporting,
+// the model handle and the orchestration of one synthetic decode step.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <memory>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace uno {
+
+namespace {
+thread_local char g_err[512] = "no error";
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t dt_size(uno_dtype dt) { return dt == UNO_F32 ? 4 : 2; }
+
+bool valid_dtype(uno_dtype dt) { return dt == UNO_BF16 || dt == UNO_F32; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+}  // namespace
+
+uno_status set_error(uno_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+uno_status cuda_error(cudaError_t e, const char* what) {
+  return set_error(UNO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- gated linear
+
+namespace {
+
+struct LinearLayout {
+  size_t t_off, total;
+};
+
+LinearLayout linear_layout(uno_dtype dt, int64_t M, int32_t r) {
+  LinearLayout l{};
+  l.t_off = 0;
+  l.total = align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * dt_size(dt));
+  return l;
+}
+
+uno_status check_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (!valid_dtype(dt)) return set_error(UNO_ERR_INVALID_ARG, "unknown dtype %d", dt);
+  if (M < 0 || K < 1 || N < 1 || r < 0)
+    return set_error(UNO_ERR_INVALID_ARG, "bad sizes M=%lld K=%lld N=%lld r=%d",
+                     static_cast<long long>(M), static_cast<long long>(K),
+                     static_cast<long long>(N), r);
+  const int64_t q = dt == UNO_F32 ? 4 : 8;
+  if (K % q || N % q || r % q)
+    return set_error(UNO_ERR_UNSUPPORTED,
+                     "K, N and r must be multiples of %lld (16-byte rows): K=%lld N=%lld r=%d",
+                     static_cast<long long>(q), static_cast<long long>(K),
+                     static_cast<long long>(N), r);
+  if (r > 256) return set_error(UNO_ERR_UNSUPPORTED, "rank r=%d > 256", r);
+  if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30))
+    return set_error(UNO_ERR_UNSUPPORTED, "sizes above 2^30");
+  return UNO_OK;
+}
+
+// Two launches: the gated down-projection t = scale * g * (x A^T), then the
+// base product with t folded in as extra K-blocks.
+uno_status linear_prepare(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r,
+                          const void* x, const void* W, const void* A, const void* Bl,
+                          const uint8_t* gate, int64_t gate_row0, float scale, void* t_buf,
+                          int mode, void* y, void* y1, int64_t M0, GemmLaunch* down,
+                          GemmLaunch* main, bool* has_down) {
+  *has_down = r > 0;
+  if (r > 0) {
+    GemmProblem d{};
+    d.dt = dt;
+    d.M = M;
+    d.N = r;
+    d.K = K;
+    d.r = 0;
+    d.x = x;
+    d.W = A;
+    d.mode = kEpiRowScale;
+    d.y = t_buf;
+    d.y1 = t_buf;
+    d.M0 = M;
+    d.ldy = r;
+    d.gate = gate;
+    d.gate_row0 = gate_row0;
+    d.scale = scale;
+    uno_status s = gemm_prepare(d, down);
+    if (s != UNO_OK) return s;
+  }
+  GemmProblem p{};
+  p.dt = dt;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.x = x;
+  p.W = W;
+  p.t = t_buf;
+  p.Bl = Bl;
+  p.mode = mode;
+  p.y = y;
+  p.y1 = y1 ? y1 : y;
+  p.M0 = y1 ? M0 : M;
+  p.ldy = N;
+  return gemm_prepare(p, main);
+}
+
+}  // namespace
+
+}  // namespace uno
+
+using namespace uno;
+
+extern "C" {
+
+const char* uno_last_error(void) { return g_err; }
+
+const char* uno_version(void) { return "uno-psispec-b200 0.1 (sm_100a)"; }
+
+uno_status uno_device_status(int32_t* bits_out, int32_t clear, void* stream) {
+  if (!bits_out) return set_error(UNO_ERR_INVALID_ARG, "bits_out is NULL");
+  cudaStream_t s = as_stream(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(v), 0,
+                                            cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "reading the device status word");
+  if (clear) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_error(e, "clearing the device status word");
+  }
+  *bits_out = v;
+  return UNO_OK;
+}
+
+size_t uno_gated_lora_linear_workspace(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r) {
+  (void)K;
+  (void)N;
+  if (M < 0 || r < 0) return 0;
+  return linear_layout(dt, M, r).total;
+}
+
+uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r,
+                                 const void* x, const void* W, const void* A, const void* Bl,
+                                 const uint8_t* gate, float scale, void* y, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  uno_status s = check_linear(dt, M, K, N, r);
+  if (s != UNO_OK) return s;
+  if (M == 0) return UNO_OK;
+  if (!x || !W || !y) return set_error(UNO_ERR_INVALID_ARG, "x, W and y must be non-NULL");
+  if (r > 0 && (!A || !Bl || !gate))
+    return set_error(UNO_ERR_INVALID_ARG, "A, Bl and gate must be non-NULL when r > 0");
+  if (!aligned16(x) || !aligned16(W) || !aligned16(y) || (r > 0 && (!aligned16(A) || !aligned16(Bl))))
+    return set_error(UNO_ERR_INVALID_ARG, "x, W, A, Bl and y must be 16-byte aligned");
+  const LinearLayout L = linear_layout(dt, M, r);
+  if (r > 0 && (!workspace || ws_bytes < L.total || !aligned16(workspace)))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", L.total,
+                     ws_bytes);
+  void* t_buf = r > 0 ? static_cast<char*>(workspace) + L.t_off : nullptr;
+  GemmLaunch down, main;
+  bool has_down = false;
+  s = linear_prepare(dt, M, K, N, r, x, W, A, Bl, gate, 0, scale, t_buf, kEpiStore, y, nullptr,
+                     M, &down, &main, &has_down);
+  if (s != UNO_OK) return s;
+  if (has_down && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
+  return gemm_run(main, as_stream(stream));
+}
+
+// ---------------------------------------------------------------- sampler
+
+size_t uno_psi_verify_workspace(int32_t B, int32_t k, int32_t k_p, int32_t V) {
+  if (B < 0 || k < 1 || V < 1 || (k_p != k && k_p != k + 1)) return 0;
+  return align_up(verify_workspace(B, k, k_p, V));
+}
+
+static uno_status check_sampler(uno_dtype dt, int32_t B, int32_t k, int32_t V, float T) {
+  if (!valid_dtype(dt)) return set_error(UNO_ERR_INVALID_ARG, "unknown dtype %d", dt);
+  if (B < 0) return set_error(UNO_ERR_INVALID_ARG, "B=%d < 0", B);
+  if (k < 1 || k > 32) return set_error(UNO_ERR_UNSUPPORTED, "block size k=%d outside [1, 32]", k);
+  if (V < 2 || V > 196608) return set_error(UNO_ERR_UNSUPPORTED, "vocabulary V=%d outside [2, 196608]", V);
+  if (!(T > 0.f) || !(T < 1e30f)) return set_error(UNO_ERR_INVALID_ARG, "temperature must be > 0 (got %g)", T);
+  return UNO_OK;
+}
+
+uno_status uno_psi_verify(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32_t V,
+                          const void* p_logits, const void* q_logits, const int32_t* draft,
+                          float temperature, uint64_t seed, uint64_t step, uint64_t seq_offset,
+                          int32_t* accepted_len, int32_t* out_tokens, int32_t* out_count,
+                          int32_t* dev_status, void* workspace, size_t ws_bytes, void* stream) {
+  uno_status s = check_sampler(dt, B, k, V, temperature);
+  if (s != UNO_OK) return s;
+  if (k_p != k && k_p != k + 1) return set_error(UNO_ERR_INVALID_ARG, "k_p=%d must be k or k+1", k_p);
+  if (B == 0) return UNO_OK;
+  if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k + 1) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * (k + 1) must be <= 2^32");
+  if (!p_logits || !q_logits || !draft || !accepted_len || !out_tokens || !out_count)
+    return set_error(UNO_ERR_INVALID_ARG, "NULL input or output pointer");
+  if (!aligned16(p_logits) || !aligned16(q_logits))
+    return set_error(UNO_ERR_INVALID_ARG, "logits must be 16-byte aligned");
+  const size_t need = uno_psi_verify_workspace(B, k, k_p, V);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
+  VerifyArgs a{};
+  a.dt = dt;
+  a.B = B;
+  a.k = k;
+  a.k_p = k_p;
+  a.V = V;
+  a.p_logits = p_logits;
+  a.q_logits = q_logits;
+  a.draft = draft;
+  a.temperature = temperature;
+  a.seed = seed;
+  a.step = step;
+  a.seq_offset = seq_offset;
+  a.accepted_len = accepted_len;
+  a.out_tokens = out_tokens;
+  a.out_count = out_count;
+  a.dev_status = dev_status;
+  return verify_launch(a, workspace, as_stream(stream));
+}
+
+size_t uno_draft_sample_workspace(int32_t B, int32_t k, int32_t V) {
+  (void)B;
+  (void)k;
+  (void)V;
+  return 0;
+}
+
+uno_status uno_draft_sample(uno_dtype dt, int32_t B, int32_t k, int32_t V, const void* q_logits,
+                            float temperature, uint64_t seed, uint64_t step, uint64_t seq_offset,
+                            int32_t* draft, int32_t* dev_status, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  uno_status s = check_sampler(dt, B, k, V, temperature);
+  if (s != UNO_OK) return s;
+  if (B == 0) return UNO_OK;
+  if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * k must be <= 2^32");
+  if (!q_logits || !draft) return set_error(UNO_ERR_INVALID_ARG, "NULL q_logits or draft");
+  DraftArgs a{};
+  a.dt = dt;
+  a.B = B;
+  a.k = k;
+  a.V = V;
+  a.q_logits = q_logits;
+  a.temperature = temperature;
+  a.seed = seed;
+  a.step = step;
+  a.seq_offset = seq_offset;
+  a.draft = draft;
+  a.dev_status = dev_status;
+  return draft_launch(a, as_stream(stream));
+}
+
+uno_status uno_philox_uniforms(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,
+                               int64_t n, uint32_t* words, float* u, void* stream) {
+  if (n < 0) return set_error(UNO_ERR_INVALID_ARG, "n < 0");
+  if (static_cast<uint64_t>(index0) + static_cast<uint64_t>(n) > (1ull << 32))
+    return set_error(UNO_ERR_INVALID_ARG, "index0 + n > 2^32");
+  return philox_launch(seed, step, stream_id, index0, n, words, u, as_stream(stream));
+}
+
+uno_status uno_rmsnorm(int64_t M, int64_t D, const void* x, void* y, float eps, void* stream) {
+  if (M < 0 || D < 1) return set_error(UNO_ERR_INVALID_ARG, "bad sizes");
+  if (M > 0 && (!x || !y)) return set_error(UNO_ERR_INVALID_ARG, "NULL pointer");
+  if (M > 0 && (!aligned16(x) || !aligned16(y))) return set_error(UNO_ERR_INVALID_ARG, "unaligned pointer");
+  if (M > 0x7fffffffll || D > (1ll << 30)) return set_error(UNO_ERR_UNSUPPORTED, "sizes too large");
+  return rmsnorm_launch(M, D, x, y, eps, as_stream(stream));
+}
+
+uno_status uno_silu_mul(int64_t n, const void* a, const void* b, void* y, void* stream) {
+  if (n < 0) return set_error(UNO_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && (!a || !b || !y)) return set_error(UNO_ERR_INVALID_ARG, "NULL pointer");
+  if (n > 0 && (!aligned16(a) || !aligned16(b) || !aligned16(y)))
+    return set_error(UNO_ERR_INVALID_ARG, "unaligned pointer");
+  return silu_mul_launch(n, a, b, y, as_stream(stream));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- model + step
+
+namespace uno {
+namespace {
+
+constexpr int kLinPerLayer = 7;   // q, k, v, o, gate, up, down
+enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
+
+struct StepLayout {
+  size_t h, n, q, kv, g, u, t, logits, vstat, total;
+};
+
+}  // namespace
+}  // namespace uno
+
+struct uno_model {
+  int32_t n_layers, hidden, q_out, kv_out, inter, vocab, r;
+  float scale;
+  std::vector<const void*> w;   // 21 * n_layers + 3
+
+  // Launch descriptors of one (B, k, buffers) combination, in step order.
+  struct Plan {
+    int32_t B, k;
+    const void* ws;
+    const void* q_next;
+    const void* logits_out;
+    std::vector<GemmLaunch> down, main;
+    std::vector<char> has_down;
+  };
+  std::mutex mu;
+  std::vector<std::unique_ptr<Plan>> plans;   // most recently used last
+
+  int lin_in(int i) const { return i == uno::kO ? q_out : (i == uno::kDown ? inter : hidden); }
+  int lin_out(int i) const {
+    switch (i) {
+      case uno::kQ: return q_out;
+      case uno::kK:
+      case uno::kV: return kv_out;
+      case uno::kGate:
+      case uno::kUp: return inter;
+      default: return hidden;
+    }
+  }
+  const void* wp(int layer, int i, int part) const {
+    return w[static_cast<size_t>(layer * uno::kLinPerLayer + i) * 3 + part];
+  }
+  const void* head(int part) const {
+    return w[static_cast<size_t>(n_layers) * uno::kLinPerLayer * 3 + part];
+  }
+};
+
+namespace uno {
+namespace {
+
+StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
+  const size_t M = static_cast<size_t>(B) * (2 * k + 1);
+  const size_t Mv = static_cast<size_t>(B) * (k + 1);
+  StepLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  };
+  L.h = take(M * m->hidden * 2);
+  L.n = take(M * m->hidden * 2);
+  L.q = take(M * m->q_out * 2);
+  L.kv = take(M * m->kv_out * 2);
+  L.g = take(M * m->inter * 2);
+  L.u = take(M * m->inter * 2);
+  L.t = take(M * m->r * 2);
+  L.logits = take(Mv * static_cast<size_t>(m->vocab) * 2);
+  L.vstat = take(verify_workspace(B, k, k + 1, m->vocab));
+  L.total = off;
+  return L;
+}
+
+// Input and output buffers of linear i of a layer, within the workspace.
+void lin_io(const uno_model* m, const StepLayout& L, char* base, int i, const void** x, void** y,
+            int* mode) {
+  *mode = kEpiStore;
+  switch (i) {
+    case kQ: *x = base + L.n; *y = base + L.q; break;
+    case kK:
+    case kV: *x = base + L.n; *y = base + L.kv; break;
+    case kO: *x = base + L.q; *y = base + L.h; *mode = kEpiAdd; break;
+    case kGate: *x = base + L.n; *y = base + L.g; break;
+    case kUp: *x = base + L.n; *y = base + L.u; break;
+    default: *x = base + L.g; *y = base + L.h; *mode = kEpiAdd; break;
+  }
+  (void)m;
+}
+
+uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
+                      void* logits_out, uno_model::Plan* P) {
+  const StepLayout L = step_layout(m, B, k);
+  char* base = static_cast<char*>(ws);
+  const int64_t M = static_cast<int64_t>(B) * (2 * k + 1);
+  const int64_t Mv = static_cast<int64_t>(B) * (k + 1);
+  const size_t n_lin = static_cast<size_t>(m->n_layers) * kLinPerLayer + 1;
+  P->B = B;
+  P->k = k;
+  P->ws = ws;
+  P->q_next = q_next;
+  P->logits_out = logits_out;
+  P->down.assign(n_lin, GemmLaunch{});
+  P->main.assign(n_lin, GemmLaunch{});
+  P->has_down.assign(n_lin, 0);
+  void* t_buf = base + L.t;
+  for (int l = 0; l < m->n_layers; ++l) {
+    for (int i = 0; i < kLinPerLayer; ++i) {
+      const void* x;
+      void* y;
+      int mode;
+      lin_io(m, L, base, i, &x, &y, &mode);
+      const size_t idx = static_cast<size_t>(l) * kLinPerLayer + i;
+      bool hd = false;
+      const uno_status s = linear_prepare(
+          UNO_BF16, M, m->lin_in(i), m->lin_out(i), m->r, x, m->wp(l, i, 0), m->wp(l, i, 1),
+          m->wp(l, i, 2), nullptr, Mv, m->scale, t_buf, mode, y, nullptr, M, &P->down[idx],
+          &P->main[idx], &hd);
+      if (s != UNO_OK) return s;
+      P->has_down[idx] = hd;
+    }
+  }
+  // LM head: AR rows -> logits (caller's buffer or the workspace), mask rows -> q_next
+  void* p_dst = logits_out ? logits_out : base + L.logits;
+  bool hd = false;
+  const uno_status s = linear_prepare(UNO_BF16, M, m->hidden, m->vocab, m->r, base + L.n,
+                                      m->head(0), m->head(1), m->head(2), nullptr, Mv, m->scale,
+                                      t_buf, kEpiStore, p_dst, q_next, Mv, &P->down[n_lin - 1],
+                                      &P->main[n_lin - 1], &hd);
+  if (s != UNO_OK) return s;
+  P->has_down[n_lin - 1] = hd;
+  return UNO_OK;
+}
+
+uno_model::Plan* find_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
+                           void* logits_out, uno_status* st) {
+  for (size_t i = 0; i < m->plans.size(); ++i) {
+    uno_model::Plan* p = m->plans[i].get();
+    if (p->B == B && p->k == k && p->ws == ws && p->q_next == q_next &&
+        p->logits_out == logits_out) {
+      if (i + 1 != m->plans.size()) {
+        std::unique_ptr<uno_model::Plan> keep = std::move(m->plans[i]);
+        m->plans.erase(m->plans.begin() + static_cast<long>(i));
+        m->plans.push_back(std::move(keep));
+      }
+      *st = UNO_OK;
+      return m->plans.back().get();
+    }
+  }
+  std::unique_ptr<uno_model::Plan> p(new uno_model::Plan());
+  *st = build_plan(m, B, k, ws, q_next, logits_out, p.get());
+  if (*st != UNO_OK) return nullptr;
+  if (m->plans.size() >= 4) m->plans.erase(m->plans.begin());
+  m->plans.push_back(std::move(p));
+  return m->plans.back().get();
+}
+
+}  // namespace
+}  // namespace uno
+
+extern "C" {
+
+uno_status uno_model_create(uno_model** out, int32_t n_layers, int32_t hidden, int32_t q_out,
+                            int32_t kv_out, int32_t inter, int32_t vocab, int32_t r, float scale,
+                            const void* const* weights) {
+  if (!out) return set_error(UNO_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (n_layers < 0 || hidden < 8 || q_out < 8 || kv_out < 8 || inter < 8 || vocab < 2 || r < 0)
+    return set_error(UNO_ERR_INVALID_ARG, "bad model sizes");
+  if (hidden % 8 || q_out % 8 || kv_out % 8 || inter % 8 || vocab % 8 || r % 8)
+    return set_error(UNO_ERR_UNSUPPORTED, "model sizes must be multiples of 8");
+  if (r > 256) return set_error(UNO_ERR_UNSUPPORTED, "rank r=%d > 256", r);
+  if (vocab > 196608) return set_error(UNO_ERR_UNSUPPORTED, "vocab=%d > 196608", vocab);
+  if (!weights) return set_error(UNO_ERR_INVALID_ARG, "weights is NULL");
+  const size_t nw = static_cast<size_t>(n_layers) * kLinPerLayer * 3 + 3;
+  for (size_t i = 0; i < nw; ++i) {
+    const bool lora_part = (i % 3) != 0;
+    if ((!weights[i] && !(lora_part && r == 0)) || (weights[i] && !aligned16(weights[i])))
+      return set_error(UNO_ERR_INVALID_ARG, "weight pointer %zu is NULL or unaligned", i);
+  }
+  uno_model* m = new uno_model();
+  m->n_layers = n_layers;
+  m->hidden = hidden;
+  m->q_out = q_out;
+  m->kv_out = kv_out;
+  m->inter = inter;
+  m->vocab = vocab;
+  m->r = r;
+  m->scale = scale;
+  m->w.assign(weights, weights + nw);
+  *out = m;
+  return UNO_OK;
+}
+
+void uno_model_destroy(uno_model* m) { delete m; }
+
+size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k) {
+  if (!m || B < 1 || k < 1 || k > 32) return 0;
+  return step_layout(m, B, k).total;
+}
+
+uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, const void* q_prev,
+                        const int32_t* d_prev, float temperature, uint64_t seed, uint64_t step,
+                        void* q_next, int32_t* d_next, void* logits_out, int32_t* accepted_len,
+                        int32_t* out_tokens, int32_t* out_count, int32_t* dev_status,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  if (!m) return set_error(UNO_ERR_INVALID_ARG, "model is NULL");
+  uno_status s = check_sampler(UNO_BF16, B, k, m->vocab, temperature);
+  if (s != UNO_OK) return s;
+  if (B < 1) return set_error(UNO_ERR_INVALID_ARG, "B must be >= 1");
+  if (static_cast<uint64_t>(B) * static_cast<uint64_t>(k + 1) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "B * (k + 1) must be <= 2^32");
+  if (static_cast<int64_t>(B) * (2 * k + 1) > (1ll << 30))
+    return set_error(UNO_ERR_UNSUPPORTED, "too many rows");
+  if (!h_in || !q_prev || !d_prev || !q_next || !d_next || !accepted_len || !out_tokens ||
+      !out_count)
+    return set_error(UNO_ERR_INVALID_ARG, "NULL input or output pointer");
+  if (!aligned16(h_in) || !aligned16(q_prev) || !aligned16(q_next) ||
+      (logits_out && !aligned16(logits_out)))
+    return set_error(UNO_ERR_INVALID_ARG, "h_in, q_prev, q_next and logits_out must be 16-byte aligned");
+  if (q_prev == q_next) return set_error(UNO_ERR_INVALID_ARG, "q_next must not alias q_prev");
+  const StepLayout L = step_layout(m, B, k);
+  if (!workspace || ws_bytes < L.total || !aligned16(workspace))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", L.total, ws_bytes);
+
+  std::lock_guard<std::mutex> lock(m->mu);
+  uno_model::Plan* P = find_plan(m, B, k, workspace, q_next, logits_out, &s);
+  if (!P) return s;
+  cudaStream_t st = as_stream(stream);
+  char* base = static_cast<char*>(workspace);
+  const int64_t M = static_cast<int64_t>(B) * (2 * k + 1);
+  cudaError_t e = cudaMemcpyAsync(base + L.h, h_in, static_cast<size_t>(M) * m->hidden * 2,
+                                  cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return cuda_error(e, "copying h_in");
+  auto lin = [&](size_t idx) -> uno_status {
+    uno_status r2;
+    if (P->has_down[idx] && (r2 = gemm_run(P->down[idx], st)) != UNO_OK) return r2;
+    return gemm_run(P->main[idx], st);
+  };
+  for (int l = 0; l < m->n_layers; ++l) {
+    const size_t b0 = static_cast<size_t>(l) * kLinPerLayer;
+    if ((s = rmsnorm_launch(M, m->hidden, base + L.h, base + L.n, 1e-6f, st)) != UNO_OK) return s;
+    for (int i = kQ; i <= kO; ++i)
+      if ((s = lin(b0 + i)) != UNO_OK) return s;
+    if ((s = rmsnorm_launch(M, m->hidden, base + L.h, base + L.n, 1e-6f, st)) != UNO_OK) return s;
+    if ((s = lin(b0 + kGate)) != UNO_OK) return s;
+    if ((s = lin(b0 + kUp)) != UNO_OK) return s;
+    if ((s = silu_mul_launch(M * m->inter, base + L.g, base + L.u, base + L.g, st)) != UNO_OK)
+      return s;
+    if ((s = lin(b0 + kDown)) != UNO_OK) return s;
+  }
+  if ((s = rmsnorm_launch(M, m->hidden, base + L.h, base + L.n, 1e-6f, st)) != UNO_OK) return s;
+  if ((s = lin(static_cast<size_t>(m->n_layers) * kLinPerLayer)) != UNO_OK) return s;
+
+  VerifyArgs va{};
+  va.dt = UNO_BF16;
+  va.B = B;
+  va.k = k;
+  va.k_p = k + 1;
+  va.V = m->vocab;
+  va.p_logits = logits_out ? logits_out : static_cast<const void*>(base + L.logits);
+  va.q_logits = q_prev;
+  va.draft = d_prev;
+  va.temperature = temperature;
+  va.seed = seed;
+  va.step = step;
+  va.seq_offset = 0;
+  va.accepted_len = accepted_len;
+  va.out_tokens = out_tokens;
+  va.out_count = out_count;
+  va.dev_status = dev_status;
+  if ((s = verify_launch(va, base + L.vstat, st)) != UNO_OK) return s;
+
+  DraftArgs da{};
+  da.dt = UNO_BF16;
+  da.B = B;
+  da.k = k;
+  da.V = m->vocab;
+  da.q_logits = q_next;
+  da.temperature = temperature;
+  da.seed = seed;
+  da.step = step;
+  da.seq_offset = 0;
+  da.draft = d_next;
+  da.dev_status = dev_status;
+  return draft_launch(da, st);
+}
+
+}  // extern "C"

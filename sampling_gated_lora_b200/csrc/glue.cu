@@ -1,0 +1,117 @@
+// Glue between the gated projections of the synthetic decode step (bf16,
+// HBM-bound): RMSNorm without weight and silu(gate) * up.
+#include "common.cuh"
+#include "internal.h"
+
+namespace uno {
+
+namespace {
+
+constexpr int kNormThreads = 256;
+
+// One CTA per row: y = x / sqrt(mean(x^2) + eps), fp32 arithmetic.
+__global__ void __launch_bounds__(kNormThreads)
+    rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y, int D,
+                   float eps) {
+  const size_t row = blockIdx.x;
+  const __nv_bfloat16* xr = x + row * D;
+  __nv_bfloat16* yr = y + row * D;
+  const bool vec = (D % 8) == 0;
+  float ss = 0.f;
+  if (vec) {
+    for (int i = threadIdx.x; i < D / 8; i += kNormThreads) {
+      const uint4 w = reinterpret_cast<const uint4*>(xr)[i];
+      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = bf16_lo(a[e]), hi = bf16_hi(a[e]);
+        ss += lo * lo + hi * hi;
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < D; i += kNormThreads) {
+      const float v = __bfloat162float(xr[i]);
+      ss += v * v;
+    }
+  }
+  ss = warp_sum(ss);
+  __shared__ float red[kNormThreads / 32];
+  __shared__ float s_inv;
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kNormThreads / 32; ++w) t += red[w];
+    s_inv = 1.0f / sqrtf(t / static_cast<float>(D) + eps);
+  }
+  __syncthreads();
+  const float inv = s_inv;
+  if (vec) {
+    for (int i = threadIdx.x; i < D / 8; i += kNormThreads) {
+      const uint4 w = reinterpret_cast<const uint4*>(xr)[i];
+      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(bf16_lo(a[e]) * inv, bf16_hi(a[e]) * inv);
+        o[e] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(yr)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  } else {
+    for (int i = threadIdx.x; i < D; i += kNormThreads)
+      yr[i] = __float2bfloat16_rn(__bfloat162float(xr[i]) * inv);
+  }
+}
+
+__device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.0f + expf(-a)) * b; }
+
+__global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
+                                const __nv_bfloat16* __restrict__ b,
+                                __nv_bfloat16* __restrict__ y, int64_t n) {
+  const int64_t nv = n / 8;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+       i += stride) {
+    const uint4 wa = reinterpret_cast<const uint4*>(a)[i];
+    const uint4 wb = reinterpret_cast<const uint4*>(b)[i];
+    const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xb[4] = {wb.x, wb.y, wb.z, wb.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(silu_mul(bf16_lo(xa[e]), bf16_lo(xb[e])),
+                                               silu_mul(bf16_hi(xa[e]), bf16_hi(xb[e])));
+      o[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    reinterpret_cast<uint4*>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  for (int64_t i = nv * 8 + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += stride)
+    y[i] = __float2bfloat16_rn(silu_mul(__bfloat162float(a[i]), __bfloat162float(b[i])));
+}
+
+}  // namespace
+
+uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
+                          cudaStream_t s) {
+  if (M == 0) return UNO_OK;
+  rmsnorm_kernel<<<static_cast<unsigned>(M), kNormThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), static_cast<int>(D),
+      eps);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "rmsnorm launch");
+}
+
+uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s) {
+  if (n == 0) return UNO_OK;
+  const int threads = 256;
+  const int64_t want = (n / 8 + threads - 1) / threads + 1;
+  const int blocks = static_cast<int>(std::min<int64_t>(want, 16 * device_sm_count()));
+  silu_mul_kernel<<<blocks, threads, 0, s>>>(static_cast<const __nv_bfloat16*>(a),
+                                             static_cast<const __nv_bfloat16*>(b),
+                                             static_cast<__nv_bfloat16*>(y), n);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "silu_mul launch");
+}
+
+}  // namespace uno

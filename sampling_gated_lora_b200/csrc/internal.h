@@ -1,0 +1,99 @@
+// Host-side declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/uno.h"
+
+namespace uno {
+
+// ---------------------------------------------------------------- errors
+uno_status set_error(uno_status st, const char* fmt, ...);
+uno_status cuda_error(cudaError_t e, const char* what);
+
+// ---------------------------------------------------------------- gated GEMM
+
+enum EpilogueMode : int {
+  kEpiStore = 0,     // y = acc
+  kEpiAdd = 1,       // y = y + acc (in place)
+  kEpiRowScale = 2,  // y = scale * gate[m] * acc   (the gated LoRA down-projection)
+};
+
+// One launch of the gated-LoRA GEMM:
+//   y[m, n] = epi( sum_k x[m,k] W[n,k] + sum_j t[m,j] Bl[n,j] )
+// Rows m >= M0 are written to y1 (row m - M0) instead of y.
+struct GemmProblem {
+  uno_dtype dt;
+  int64_t M, N, K;
+  int32_t r;              // 0: no LoRA term
+  const void* x;          // [M, K]
+  const void* W;          // [N, K]
+  const void* t;          // [M, r]  (rank-r activations, already gated and scaled)
+  const void* Bl;         // [N, r]
+  int mode;
+  void* y;
+  void* y1;
+  int64_t M0;             // rows >= M0 go to y1
+  int64_t ldy;
+  const uint8_t* gate;    // kEpiRowScale; NULL: gate[m] = (m >= gate_row0)
+  int64_t gate_row0;
+  float scale;            // kEpiRowScale
+};
+
+// Cached launch of a GemmProblem (tensor maps + grid); valid while the
+// pointers of the problem stay the same.
+struct GemmLaunch {
+  CUtensorMap tm[4];
+  alignas(8) unsigned char params[128];
+  int swap;
+  int grid_x, grid_y, splits;
+  int smem_bytes;
+  int dtype;
+};
+
+uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out);
+uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream);
+
+// ---------------------------------------------------------------- sampler
+
+struct VerifyArgs {
+  uno_dtype dt;
+  int32_t B, k, k_p, V;
+  const void* p_logits;
+  const void* q_logits;
+  const int32_t* draft;
+  float temperature;
+  uint64_t seed, step, seq_offset;
+  int32_t* accepted_len;
+  int32_t* out_tokens;
+  int32_t* out_count;
+  int32_t* dev_status;
+};
+size_t verify_workspace(int32_t B, int32_t k, int32_t k_p, int32_t V);
+uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s);
+
+struct DraftArgs {
+  uno_dtype dt;
+  int32_t B, k, V;
+  const void* q_logits;
+  float temperature;
+  uint64_t seed, step, seq_offset;
+  int32_t* draft;
+  int32_t* dev_status;
+};
+uno_status draft_launch(const DraftArgs& a, cudaStream_t s);
+
+uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,
+                         int64_t n, uint32_t* words, float* u, cudaStream_t s);
+
+// ---------------------------------------------------------------- glue
+uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
+                          cudaStream_t s);
+uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s);
+
+int device_sm_count();
+
+}  // namespace uno

@@ -1,0 +1,631 @@
+// Psi-Spec verification and the linear-sampler draft (sm_100a).
+//
+// Method (hyper.ai page, section "方法", the Psi-Spec paragraph; ainews page):
+// the draft path proposes a block from its per-position marginals q_j; the
+// block is checked against the AR distributions p_j by rejection sampling and
+// the longest accepted prefix is kept; the result follows p exactly.
+//
+// Kernels
+//   row_stats_kernel     for every logit row (p rows, then q rows) and vocab
+//                        chunk: the chunk max m and s = sum exp((z - m) / T).
+//                        Streams the logits once with 16-byte loads; this is
+//                        where the HBM time goes.
+//   verify_finalize      one thread-block cluster per sequence: merge the
+//                        chunk stats, test u1 q(d) < p(d) per position (lane
+//                        j of warp 0), ballot -> first rejection n, then the
+//                        residual (or bonus) inverse-CDF draw split over the
+//                        cluster's CTAs (chunk totals exchanged through
+//                        distributed shared memory).
+//   draft_sample_kernel  one cluster per (sequence, position): chunk max ->
+//                        cluster max -> weights exp((z - max) / T) -> the same
+//                        inverse-CDF draw.
+// Uniforms: Philox4x32-10 word 0 at counter (index, step lo, step hi,
+// stream), key (seed lo, seed hi); u = (x >> 8) 2^-24. The counter depends on
+// (sequence, position, stream) only, never on the launch shape.
+#include <algorithm>
+#include <cfloat>
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace uno {
+
+__device__ int32_t g_device_status = 0;
+
+namespace {
+
+constexpr int kStatThreads = 256;
+constexpr int kDrawThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <typename T>
+struct Vec;   // 16-byte vector of logits
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int n = 4;
+  __device__ static void load(const float* p, float (&v)[4]) {
+    const float4 w = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+  }
+};
+
+// Online (max, sum of exp2((z - max) * c)) of one thread.
+struct OnlineStat {
+  float m = -INFINITY;
+  float s = 0.f;
+  __device__ __forceinline__ void add(const float* v, int n, float c) {
+    float mx = v[0];
+    for (int e = 1; e < n; ++e) mx = fmaxf(mx, v[e]);
+    if (mx > m) {
+      s *= fast_exp2((m - mx) * c);
+      m = mx;
+    }
+    for (int e = 0; e < n; ++e) s += fast_exp2((v[e] - m) * c);
+  }
+};
+
+// Merge (m1, s1) with (m2, s2); s is relative to m, exp base 2 with scale c.
+__device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s2, float c) {
+  if (isnan(s2) || isnan(s)) {   // keep a NaN seen anywhere
+    s = NAN;
+    m = fmaxf(m, m2);
+    return;
+  }
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = m2;
+    s = s2;
+    return;
+  }
+  const float mx = fmaxf(m, m2);
+  s = s * fast_exp2((m - mx) * c) + s2 * fast_exp2((m2 - mx) * c);
+  m = mx;
+}
+
+// Grid: (chunks, rows). Row r < rows_p reads p_logits row r, else q_logits
+// row r - rows_p. Writes stats[r * chunks + chunk] = (m, s).
+template <typename T>
+__global__ void __launch_bounds__(kStatThreads)
+    row_stats_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits, int rows_p,
+                     int V, int chunk_len, float c, float2* __restrict__ stats) {
+  const int row = blockIdx.y;
+  const T* z = row < rows_p ? p_logits + static_cast<size_t>(row) * V
+                            : q_logits + static_cast<size_t>(row - rows_p) * V;
+  const int lo = blockIdx.x * chunk_len;
+  const int hi = min(V, lo + chunk_len);
+  constexpr int kN = Vec<T>::n;
+  OnlineStat st;
+  // aligned body [a0, a1) in whole 16-byte vectors; scalar head and tail
+  int a0 = lo;
+  while (a0 < hi && (reinterpret_cast<uintptr_t>(z + a0) & 15u)) ++a0;
+  const int nvec = (hi - a0) / kN;
+  const int a1 = a0 + nvec * kN;
+  for (int v = lo + threadIdx.x; v < a0; v += kStatThreads) {
+    float x = to_f32<T>(z[v]);
+    st.add(&x, 1, c);
+  }
+  constexpr int kUnroll = 4;
+  int i = threadIdx.x;
+  for (; i + (kUnroll - 1) * kStatThreads < nvec; i += kUnroll * kStatThreads) {
+    float v[kUnroll][kN];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) Vec<T>::load(z + a0 + (i + u * kStatThreads) * kN, v[u]);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) st.add(v[u], kN, c);
+  }
+  for (; i < nvec; i += kStatThreads) {
+    float v[kN];
+    Vec<T>::load(z + a0 + i * kN, v);
+    st.add(v, kN, c);
+  }
+  for (int v = a1 + threadIdx.x; v < hi; v += kStatThreads) {
+    float x = to_f32<T>(z[v]);
+    st.add(&x, 1, c);
+  }
+  // block reduction
+  float m = st.m, s = st.s;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    merge_stat(m, s, m2, s2, c);
+  }
+  __shared__ float sm[kStatThreads / 32], ss[kStatThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sm[warp] = m;
+    ss[warp] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float M = sm[0], S = ss[0];
+    for (int w = 1; w < kStatThreads / 32; ++w) merge_stat(M, S, sm[w], ss[w], c);
+    // a NaN anywhere in the chunk makes S NaN (fmaxf skips it in the max)
+    stats[static_cast<size_t>(row) * gridDim.x + blockIdx.x] = make_float2(M, S);
+  }
+}
+
+// Merge the chunk stats of one row.
+__device__ __forceinline__ float2 row_stat(const float2* stats, int row, int chunks, float c) {
+  float m = -INFINITY, s = 0.f;
+  bool nan = false;
+  for (int i = 0; i < chunks; ++i) {
+    const float2 v = stats[static_cast<size_t>(row) * chunks + i];
+    nan |= isnan(v.y);
+    merge_stat(m, s, v.x, v.y, c);
+  }
+  return make_float2(m, nan ? NAN : s);
+}
+
+// ------------------------------------------------------------------ cluster inverse-CDF draw
+
+// Shared state of one draw (per CTA).
+struct DrawSmem {
+  double segsum[kDrawThreads];
+  double seg_prefix[kDrawThreads + 1];
+  double chunk_total;
+  int token;
+};
+
+// Inverse-CDF draw over the cluster: this CTA holds `len` weights w(i) of
+// vocab ids [lo, lo + len) (computed on demand by wfn, deterministic). Returns
+// in every CTA: the drawn vocab id if this CTA owns it, -1 otherwise; sets
+// *zero_total when the cluster-wide total is 0. All threads of all CTAs of the
+// cluster must call it (it contains cluster barriers). No CTA reads another
+// CTA's shared memory after the last barrier inside, so callers may exit.
+template <typename WFn>
+__device__ int cluster_draw(DrawSmem& sh, const WFn& wfn, int lo, int len, double u,
+                            bool* zero_total) {
+  const int t = threadIdx.x;
+  const int seg = (len + kDrawThreads - 1) / kDrawThreads;
+  const int s0 = min(len, t * seg), s1 = min(len, s0 + seg);
+  double my = 0.0;
+  for (int i = s0; i < s1; ++i) my += static_cast<double>(wfn(i));
+  // exclusive prefix of the segment sums, sequential (one thread), so that the
+  // search below sees exactly the same partial sums
+  sh.segsum[t] = my;
+  __syncthreads();
+  if (t == 0) {
+    double run = 0.0;
+    for (int i = 0; i < kDrawThreads; ++i) {
+      sh.seg_prefix[i] = run;
+      run += sh.segsum[i];
+    }
+    sh.seg_prefix[kDrawThreads] = run;
+    sh.chunk_total = run;
+    sh.token = -1;
+  }
+  cluster_sync();
+  // every CTA reads the chunk totals in rank order -> identical prefixes
+  const uint32_t nrank = cluster_nctarank();
+  const uint32_t myrank = cluster_ctarank();
+  const uint32_t tot_addr = smem_u32(&sh.chunk_total);
+  double Z = 0.0, my_prefix = 0.0;
+  bool later_mass = false;
+  for (uint32_t r = 0; r < nrank; ++r) {
+    const double v = ld_cluster_f64(map_shared_rank(tot_addr, r));
+    if (r == myrank) my_prefix = Z;
+    if (r > myrank && v > 0.0) later_mass = true;
+    Z += v;
+  }
+  cluster_sync();   // totals read everywhere before anyone reuses the slot or exits
+  if (!(Z > 0.0)) {
+    *zero_total = true;
+    return -1;
+  }
+  *zero_total = false;
+  const double thr = u * Z;
+  const double mine = sh.chunk_total;
+  // owning CTA: my_prefix <= thr < my_prefix + mine (the last CTA with
+  // positive mass also owns thresholds that rounding pushed past the end)
+  bool own = (mine > 0.0) && (thr >= my_prefix) && (thr < my_prefix + mine);
+  if (!own && mine > 0.0 && thr >= my_prefix + mine && !later_mass) own = true;
+  if (own) {
+    const double tl = thr - my_prefix;
+    const double lo_s = sh.seg_prefix[t], hi_s = sh.seg_prefix[t + 1];
+    bool mine_seg = hi_s > lo_s && tl >= lo_s && tl < hi_s;
+    if (!mine_seg && hi_s > lo_s && tl >= hi_s) {
+      // rounding past the chunk total: the last segment with mass owns it
+      bool last = true;
+      for (int i = t + 1; i < kDrawThreads && last; ++i)
+        last = !(sh.seg_prefix[i + 1] > sh.seg_prefix[i]);
+      mine_seg = last;
+    }
+    if (mine_seg) {
+      const double tt = tl - lo_s;
+      double run = 0.0;
+      int pick = -1, last_nz = -1;
+      for (int i = s0; i < s1; ++i) {
+        const float w = wfn(i);
+        if (w > 0.f) last_nz = i;
+        run += static_cast<double>(w);
+        if (run > tt) {
+          pick = i;
+          break;
+        }
+      }
+      if (pick < 0) pick = last_nz;
+      sh.token = lo + pick;
+    }
+  }
+  __syncthreads();
+  return own ? sh.token : -1;
+}
+
+// Vocab range of CTA `rank` among `n`: chunks are multiples of 8 ids.
+__device__ __forceinline__ void chunk_range(int V, int n, int rank, int* lo, int* len) {
+  int per = (V + n - 1) / n;
+  per = (per + 7) & ~7;
+  const int a = min(V, rank * per);
+  *lo = a;
+  *len = min(V, a + per) - a;
+}
+
+template <typename T>
+__device__ __forceinline__ void load_chunk(T* dst, const T* src, int len) {
+  for (int i = threadIdx.x; i < len; i += blockDim.x) dst[i] = src[i];
+}
+
+struct FinalizeParams {
+  int B, k, k_p, V, chunks;
+  float c;   // log2(e) / T
+  uint64_t seed, step, seq_offset;
+  const int32_t* draft;
+  const float2* stats;
+  int32_t* accepted_len;
+  int32_t* out_tokens;
+  int32_t* out_count;
+  int32_t* status;
+  int chunk_elems;   // per-CTA smem capacity in elements (per row)
+};
+
+// One cluster per sequence; blockDim = kDrawThreads.
+template <typename T>
+__global__ void __launch_bounds__(kDrawThreads)
+    verify_finalize_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits,
+                           const FinalizeParams a) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ DrawSmem sh;
+  __shared__ int s_n, s_bad, s_nan;
+  __shared__ float s_stat[4];   // Mp, Sp, Mq, Sq of the drawing row(s)
+
+  const uint32_t nrank = cluster_nctarank();
+  const uint32_t rank = cluster_ctarank();
+  const int b = blockIdx.x / nrank;
+  const int k = a.k, V = a.V;
+  const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
+  const int rows_p = a.B * a.k_p;
+
+  if (threadIdx.x < 32) {
+    const int j = threadIdx.x;
+    bool acc = true, bad = false, nan = false;
+    if (j < k) {
+      const int d = a.draft[b * k + j];
+      bad = d < 0 || d >= V;
+      const int prow = b * a.k_p + j, qrow = rows_p + b * k + j;
+      const float2 sp = row_stat(a.stats, prow, a.chunks, a.c);
+      const float2 sq = row_stat(a.stats, qrow, a.chunks, a.c);
+      nan = isnan(sp.y) || isnan(sq.y);
+      if (!bad && !nan) {
+        const float zp = to_f32<T>(p_logits[static_cast<size_t>(prow) * V + d]);
+        const float zq = to_f32<T>(q_logits[static_cast<size_t>(b * k + j) * V + d]);
+        const float pd = fast_exp2((zp - sp.x) * a.c) / sp.y;
+        const float qd = fast_exp2((zq - sq.x) * a.c) / sq.y;
+        const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + j);
+        const float u1 = uniform24(philox_word0(a.seed, a.step, kStreamAccept, idx));
+        acc = (qd == 0.f) || (u1 * qd < pd);
+      }
+    }
+    const uint32_t in_k = k >= 32 ? 0xffffffffu : ((1u << k) - 1u);
+    const uint32_t rej = __ballot_sync(0xffffffffu, !acc) & in_k;
+    const uint32_t badm = __ballot_sync(0xffffffffu, bad) & in_k;
+    const uint32_t nanm = __ballot_sync(0xffffffffu, nan) & in_k;
+    if (j == 0) {
+      s_n = rej ? __ffs(rej) - 1 : k;
+      s_bad = badm != 0;
+      s_nan = nanm != 0;
+    }
+  }
+  __syncthreads();
+  const int n = s_n;
+  int32_t* tok = a.out_tokens + static_cast<size_t>(b) * (k + 1);
+  if (s_bad || s_nan) {
+    if (rank == 0) {
+      if (threadIdx.x == 0) {
+        a.accepted_len[b] = -1;
+        a.out_count[b] = -1;
+        raise_status(a.status, (s_bad ? kDevBadDraft : 0) | (s_nan ? kDevNaN : 0));
+      }
+      for (int i = threadIdx.x; i <= k; i += blockDim.x) tok[i] = -1;
+    }
+    return;   // uniform over the cluster: every CTA saw the same flags
+  }
+  const bool residual = n < k;
+  const bool bonus = !residual && a.k_p == k + 1;
+  const bool draw = residual || bonus;
+  if (rank == 0) {
+    if (threadIdx.x == 0) {
+      a.accepted_len[b] = n;
+      a.out_count[b] = n + (draw ? 1 : 0);
+    }
+    for (int i = threadIdx.x; i <= k; i += blockDim.x) {
+      if (i < n) tok[i] = a.draft[b * k + i];
+      else if (i > n || !draw) tok[i] = -1;
+    }
+  }
+  if (!draw) return;
+
+  // Rows of the draw: residual at position n (p row and q row), or the bonus p row k.
+  const int prow = b * a.k_p + (residual ? n : k);
+  const int qrow_local = b * k + n;   // q row index within q_logits
+  if (threadIdx.x == 0) {
+    const float2 sp = row_stat(a.stats, prow, a.chunks, a.c);
+    s_stat[0] = sp.x;
+    s_stat[1] = sp.y;
+    if (residual) {
+      const float2 sq = row_stat(a.stats, rows_p + qrow_local, a.chunks, a.c);
+      s_stat[2] = sq.x;
+      s_stat[3] = sq.y;
+    }
+  }
+  int lo, len;
+  chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
+  T* zp = reinterpret_cast<T*>(dyn);
+  T* zq = zp + a.chunk_elems;
+  load_chunk(zp, p_logits + static_cast<size_t>(prow) * V + lo, len);
+  if (residual) load_chunk(zq, q_logits + static_cast<size_t>(qrow_local) * V + lo, len);
+  __syncthreads();
+  const float Mp = s_stat[0], inv_sp = 1.f / s_stat[1];
+  const float Mq = s_stat[2], inv_sq = residual ? 1.f / s_stat[3] : 0.f;
+  const float c = a.c;
+  const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + (residual ? n : k));
+  const double u = static_cast<double>(uniform24(
+      philox_word0(a.seed, a.step, residual ? kStreamResidual : kStreamBonus, idx)));
+
+  bool zero = false;
+  int token;
+  if (residual) {
+    auto w_res = [&](int i) {
+      const float p = fast_exp2((to_f32<T>(zp[i]) - Mp) * c) * inv_sp;
+      const float q = fast_exp2((to_f32<T>(zq[i]) - Mq) * c) * inv_sq;
+      return fmaxf(p - q, 0.f);
+    };
+    token = cluster_draw(sh, w_res, lo, len, u, &zero);
+  } else {
+    auto w_p = [&](int i) { return fast_exp2((to_f32<T>(zp[i]) - Mp) * c); };
+    token = cluster_draw(sh, w_p, lo, len, u, &zero);
+  }
+  if (zero) {   // residual mass 0 (only through rounding): draw from p_n
+    auto w_p = [&](int i) { return fast_exp2((to_f32<T>(zp[i]) - Mp) * c); };
+    token = cluster_draw(sh, w_p, lo, len, u, &zero);
+  }
+  if (token >= 0 && threadIdx.x == 0) tok[n] = token;
+}
+
+struct DraftParams {
+  int k, V;
+  float c;
+  uint64_t seed, step, seq_offset;
+  int32_t* draft;
+  int32_t* status;
+};
+
+// One cluster per (sequence, position) row of q; blockDim = kDrawThreads.
+template <typename T>
+__global__ void __launch_bounds__(kDrawThreads)
+    draft_sample_kernel(const T* __restrict__ q_logits, const DraftParams a) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ DrawSmem sh;
+  __shared__ float s_max;
+  __shared__ float s_cmax[kDrawThreads / 32];
+  const uint32_t nrank = cluster_nctarank();
+  const uint32_t rank = cluster_ctarank();
+  const int row = blockIdx.x / nrank;
+  const int V = a.V;
+  int lo, len;
+  chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
+  T* z = reinterpret_cast<T*>(dyn);
+  const T* src = q_logits + static_cast<size_t>(row) * V + lo;
+  float mx = -INFINITY;
+  bool nan = false;
+  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+    const T v = src[i];
+    z[i] = v;
+    const float f = to_f32<T>(v);
+    nan |= isnan(f);
+    mx = fmaxf(mx, f);
+  }
+  mx = warp_max(mx);
+  nan = __any_sync(0xffffffffu, nan);
+  if ((threadIdx.x & 31) == 0) s_cmax[threadIdx.x >> 5] = nan ? NAN : mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = -INFINITY;
+    bool any_nan = false;
+    for (int w = 0; w < kDrawThreads / 32; ++w) {
+      any_nan |= isnan(s_cmax[w]);
+      m = fmaxf(m, s_cmax[w]);
+    }
+    s_max = any_nan ? NAN : m;
+  }
+  cluster_sync();
+  // cluster-wide max (NaN if any chunk saw a NaN)
+  float M = -INFINITY;
+  bool any_nan = false;
+  const uint32_t addr = smem_u32(&s_max);
+  for (uint32_t r = 0; r < nrank; ++r) {
+    const float v = ld_cluster_f32(map_shared_rank(addr, r));
+    any_nan |= isnan(v);
+    M = fmaxf(M, v);
+  }
+  cluster_sync();
+  if (any_nan || M == -INFINITY) {
+    if (rank == 0 && threadIdx.x == 0) {
+      a.draft[row] = -1;
+      raise_status(a.status, kDevNaN);
+    }
+    return;
+  }
+  const int b = row / a.k, j = row % a.k;
+  const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
+  const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(a.k) + j);
+  const double u = static_cast<double>(uniform24(philox_word0(a.seed, a.step, kStreamDraft, idx)));
+  const float c = a.c;
+  auto w = [&](int i) { return fast_exp2((to_f32<T>(z[i]) - M) * c); };
+  bool zero = false;
+  const int token = cluster_draw(sh, w, lo, len, u, &zero);
+  if (token >= 0 && threadIdx.x == 0) a.draft[row] = token;
+}
+
+__global__ void philox_kernel(uint64_t seed, uint64_t step, uint32_t stream, uint32_t index0,
+                              int64_t n, uint32_t* words, float* u) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t w = philox_word0(seed, step, stream, index0 + static_cast<uint32_t>(i));
+    if (words) words[i] = w;
+    if (u) u[i] = uniform24(w);
+  }
+}
+
+// Cluster width for a vocabulary: enough CTAs that one chunk (two rows of
+// logits) fits comfortably in shared memory, at most 8 (portable).
+int draw_cluster(int V, int esz, int* chunk_elems) {
+  int n = 1;
+  while (n < 8 && (static_cast<int64_t>((V + n - 1) / n) * esz * 2 > 48 * 1024)) n <<= 1;
+  int per = (V + n - 1) / n;
+  per = (per + 7) & ~7;
+  *chunk_elems = per;
+  return n;
+}
+
+template <typename Kern, typename... Args>
+uno_status launch_cluster(Kern kern, int grid, int cluster, size_t smem, cudaStream_t s,
+                          Args... args) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute(draw smem)");
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kDrawThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) return cuda_error(e, "sampler launch");
+  return UNO_OK;
+}
+
+int stat_chunks(int rows, int V) {
+  const int target = 4 * device_sm_count();
+  int c = (target + rows - 1) / rows;
+  c = std::min(c, std::max(1, V / 2048));
+  return std::max(1, c);
+}
+
+}  // namespace
+
+size_t verify_workspace(int32_t B, int32_t k, int32_t k_p, int32_t V) {
+  const int rows = B * k_p + B * k;
+  const int chunks = stat_chunks(rows, V);
+  return static_cast<size_t>(rows) * chunks * sizeof(float2);
+}
+
+uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s) {
+  const int rows = a.B * a.k_p + a.B * a.k;
+  const int chunks = stat_chunks(rows, a.V);
+  const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
+  const float c = kLog2e / a.temperature;
+  float2* stats = static_cast<float2*>(ws);
+  const int esz = a.dt == UNO_F32 ? 4 : 2;
+  int chunk_elems = 0;
+  const int cl = draw_cluster(a.V, esz, &chunk_elems);
+  FinalizeParams fp{};
+  fp.B = a.B;
+  fp.k = a.k;
+  fp.k_p = a.k_p;
+  fp.V = a.V;
+  fp.chunks = chunks;
+  fp.c = c;
+  fp.seed = a.seed;
+  fp.step = a.step;
+  fp.seq_offset = a.seq_offset;
+  fp.draft = a.draft;
+  fp.stats = stats;
+  fp.accepted_len = a.accepted_len;
+  fp.out_tokens = a.out_tokens;
+  fp.out_count = a.out_count;
+  fp.status = a.dev_status;
+  fp.chunk_elems = chunk_elems;
+  const size_t smem = static_cast<size_t>(chunk_elems) * esz * 2;
+  const dim3 grid(chunks, rows);
+  if (a.dt == UNO_F32) {
+    row_stats_kernel<float><<<grid, kStatThreads, 0, s>>>(
+        static_cast<const float*>(a.p_logits), static_cast<const float*>(a.q_logits),
+        a.B * a.k_p, a.V, chunk_len, c, stats);
+  } else {
+    row_stats_kernel<__nv_bfloat16><<<grid, kStatThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(a.p_logits),
+        static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.k_p, a.V, chunk_len, c, stats);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_error(e, "row_stats launch");
+  if (a.dt == UNO_F32)
+    return launch_cluster(verify_finalize_kernel<float>, a.B * cl, cl, smem, s,
+                          static_cast<const float*>(a.p_logits),
+                          static_cast<const float*>(a.q_logits), fp);
+  return launch_cluster(verify_finalize_kernel<__nv_bfloat16>, a.B * cl, cl, smem, s,
+                        static_cast<const __nv_bfloat16*>(a.p_logits),
+                        static_cast<const __nv_bfloat16*>(a.q_logits), fp);
+}
+
+uno_status draft_launch(const DraftArgs& a, cudaStream_t s) {
+  const int esz = a.dt == UNO_F32 ? 4 : 2;
+  int chunk_elems = 0;
+  const int cl = draw_cluster(a.V, esz, &chunk_elems);
+  DraftParams dp{};
+  dp.k = a.k;
+  dp.V = a.V;
+  dp.c = kLog2e / a.temperature;
+  dp.seed = a.seed;
+  dp.step = a.step;
+  dp.seq_offset = a.seq_offset;
+  dp.draft = a.draft;
+  dp.status = a.dev_status;
+  const size_t smem = static_cast<size_t>(chunk_elems) * esz;
+  const int rows = a.B * a.k;
+  if (a.dt == UNO_F32)
+    return launch_cluster(draft_sample_kernel<float>, rows * cl, cl, smem, s,
+                          static_cast<const float*>(a.q_logits), dp);
+  return launch_cluster(draft_sample_kernel<__nv_bfloat16>, rows * cl, cl, smem, s,
+                        static_cast<const __nv_bfloat16*>(a.q_logits), dp);
+}
+
+uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,
+                         int64_t n, uint32_t* words, float* u, cudaStream_t s) {
+  if (n == 0) return UNO_OK;
+  const int threads = 256;
+  const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 8 * device_sm_count());
+  philox_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(seed, step, stream_id, index0, n,
+                                                             words, u);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_error(e, "philox launch");
+  return UNO_OK;
+}
+
+}  // namespace uno

@@ -1,0 +1,132 @@
+"""The C-ABI library loads, exports every symbol of include/uno.h, and rejects
+bad arguments on the host (no GPU needed: these calls return before any CUDA work)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sampling_gated_lora_b200 as U
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "uno.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(uno_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_what_binding_uses():
+    assert set(_declared()) == set(U.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = U.load()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert "sm_100a" in U.version()
+
+
+def _status(st):
+    return st, U.load().uno_last_error().decode()
+
+
+def test_linear_rejects_bad_arguments():
+    L = U.load()
+    null = None
+    # K not a multiple of 8 (bf16 rows must be 16-byte multiples)
+    st, msg = _status(L.uno_gated_lora_linear(U.UNO_BF16, 4, 12, 16, 8, null, null, null, null, null,
+                                              1.0, null, null, 0, null))
+    assert st == 2 and "multiples" in msg
+    st, _ = _status(L.uno_gated_lora_linear(U.UNO_BF16, -1, 16, 16, 8, null, null, null, null, null,
+                                            1.0, null, null, 0, null))
+    assert st == 1
+    st, msg = _status(L.uno_gated_lora_linear(U.UNO_BF16, 4, 16, 16, 264, null, null, null, null, null,
+                                              1.0, null, null, 0, null))
+    assert st == 2 and "rank" in msg
+    st, _ = _status(L.uno_gated_lora_linear(7, 4, 16, 16, 8, null, null, null, null, null,
+                                            1.0, null, null, 0, null))
+    assert st == 1
+    # M = 0 is a valid empty call that launches nothing
+    assert L.uno_gated_lora_linear(U.UNO_BF16, 0, 16, 16, 8, null, null, null, null, null,
+                                   1.0, null, null, 0, null) == 0
+    # NULL inputs with M > 0
+    st, _ = _status(L.uno_gated_lora_linear(U.UNO_BF16, 4, 16, 16, 8, null, null, null, null, null,
+                                            1.0, null, null, 0, null))
+    assert st == 1
+    # misaligned pointers
+    fake = ctypes.c_void_p(0x1008)
+    st, msg = _status(L.uno_gated_lora_linear(U.UNO_BF16, 4, 16, 16, 8, fake, fake, fake, fake, fake,
+                                              1.0, fake, fake, 1 << 20, null))
+    assert st == 1 and "aligned" in msg
+    # workspace too small
+    ok = ctypes.c_void_p(0x10000)
+    st, _ = _status(L.uno_gated_lora_linear(U.UNO_BF16, 4, 16, 16, 8, ok, ok, ok, ok, ok,
+                                            1.0, ok, ok, 1, null))
+    assert st == 6
+    assert L.uno_gated_lora_linear_workspace(U.UNO_BF16, 9, 4096, 4096, 128) >= 9 * 128 * 2
+
+
+def test_verify_rejects_bad_arguments():
+    L = U.load()
+    null = None
+    ok = ctypes.c_void_p(0x10000)
+    args = lambda dt, B, k, kp, V, T: L.uno_psi_verify(dt, B, k, kp, V, ok, ok, ok, T, 0, 0, 0, ok,
+                                                     ok, ok, null, ok, 1 << 30, null)
+    assert _status(args(U.UNO_BF16, 2, 4, 4, 1024, 0.0))[0] == 1        # T <= 0
+    assert _status(args(U.UNO_BF16, 2, 4, 4, 1024, -1.0))[0] == 1
+    assert _status(args(U.UNO_BF16, 2, 33, 33, 1024, 1.0))[0] == 2      # k > 32
+    assert _status(args(U.UNO_BF16, 2, 0, 0, 1024, 1.0))[0] == 2        # k < 1
+    assert _status(args(U.UNO_BF16, 2, 4, 6, 1024, 1.0))[0] == 1        # k_p not k or k+1
+    assert _status(args(U.UNO_BF16, 2, 4, 4, 1, 1.0))[0] == 2           # V < 2
+    assert _status(args(U.UNO_BF16, 2, 4, 4, 300000, 1.0))[0] == 2      # V too large
+    assert _status(args(U.UNO_BF16, -1, 4, 4, 1024, 1.0))[0] == 1
+    assert args(U.UNO_BF16, 0, 4, 4, 1024, 1.0) == 0                    # empty batch
+    st = L.uno_psi_verify(U.UNO_BF16, 2, 4, 4, 1024, null, ok, ok, 1.0, 0, 0, 0, ok, ok, ok, null,
+                          ok, 1 << 30, null)
+    assert st == 1
+    st = L.uno_psi_verify(U.UNO_BF16, 2, 4, 4, 1024, ok, ok, ok, 1.0, 0, 0, 0, ok, ok, ok, null,
+                          ok, 0, null)
+    assert st == 6
+    assert L.uno_psi_verify_workspace(256, 16, 16, 151936) > 0
+    assert L.uno_psi_verify_workspace(2, 4, 7, 1024) == 0
+
+
+def test_draft_and_misc_reject_bad_arguments():
+    L = U.load()
+    null = None
+    ok = ctypes.c_void_p(0x10000)
+    assert L.uno_draft_sample(U.UNO_BF16, 2, 4, 1024, ok, 0.0, 0, 0, 0, ok, null, null, 0, null) == 1
+    assert L.uno_draft_sample(U.UNO_BF16, 2, 4, 1024, null, 1.0, 0, 0, 0, ok, null, null, 0, null) == 1
+    assert L.uno_philox_uniforms(0, 0, 0, 0xFFFFFFFF, 2, ok, ok, null) == 1
+    assert L.uno_philox_uniforms(0, 0, 0, 0, -1, ok, ok, null) == 1
+    assert L.uno_rmsnorm(-1, 8, ok, ok, 1e-6, null) == 1
+    assert L.uno_silu_mul(-1, ok, ok, ok, null) == 1
+    assert L.uno_device_status(null, 0, null) == 1
+
+
+def test_model_create_validates():
+    L = U.load()
+    h = ctypes.c_void_p()
+    assert L.uno_model_create(ctypes.byref(h), 1, 12, 16, 16, 16, 16, 8, 1.0, None) == 2
+    assert L.uno_model_create(ctypes.byref(h), 1, 16, 16, 16, 16, 16, 8, 1.0, None) == 1
+    ptrs = (ctypes.c_void_p * 24)(*([0x10000] * 24))
+    ptrs[5] = 0x10008    # misaligned
+    assert L.uno_model_create(ctypes.byref(h), 1, 16, 16, 16, 16, 16, 8, 1.0, ptrs) == 1
+    ptrs[5] = 0x10000
+    assert L.uno_model_create(ctypes.byref(h), 1, 16, 16, 16, 16, 16, 8, 1.0, ptrs) == 0
+    assert h.value
+    assert L.uno_psi_step_workspace(h, 2, 4) > 0
+    st = L.uno_psi_step(h, 2, 4, None, None, None, 1.0, 0, 0, None, None, None, None, None, None,
+                        None, None, 0, None)
+    assert st == 1
+    L.uno_model_destroy(h)
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(U, "_lib", None)
+    monkeypatch.setattr(U, "LIB_PATH", "/nonexistent/libuno.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        U.load()

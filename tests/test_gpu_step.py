@@ -1,0 +1,98 @@
+"""One synthetic decode step (uno_psi_step) on a small model.
+
+Logits of every row are compared with the fp64 oracle stack (bf16 storage at
+the same points). The step's tokens are checked by composition: they must
+equal uno_psi_verify / uno_draft_sample run on the step's own logits (those
+two kernels have their own oracle parity tests)."""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import sampling as S
+from oracle import stack as O
+from gpu_util import check_close, dev_tensor, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _model(shape, seed):
+    import sampling_gated_lora_b200 as U
+    layers_np, head_np = W.model_weights_np(shape, seed=seed)
+    tl = lambda wab: tuple(dev_tensor(a, "bf16") for a in wab)
+    layers = [{k: tl(v) for k, v in lw.items()} for lw in layers_np]
+    head = tl(head_np)
+    m = U.Model(layers, head, shape.hidden, shape.q_out, shape.kv_out, shape.inter, shape.vocab,
+                shape.r, shape.scale)
+    return m, layers_np, head_np
+
+
+def _buffers(B, k, V, dev="cuda"):
+    import torch
+    i32 = dict(dtype=torch.int32, device=dev)
+    return dict(q_next=torch.empty((B, k, V), dtype=torch.bfloat16, device=dev),
+                d_next=torch.empty((B, k), **i32), acc=torch.empty(B, **i32),
+                tok=torch.empty((B, k + 1), **i32), cnt=torch.empty(B, **i32),
+                logits=torch.empty((B * (k + 1), V), dtype=torch.bfloat16, device=dev),
+                status=torch.zeros(1, **i32))
+
+
+@pytest.mark.parametrize("B,k,T", [(2, 4, 1.0), (3, 8, 0.7), (1, 1, 1.0)])
+def test_tiny_step(B, k, T):
+    import torch
+    import sampling_gated_lora_b200 as U
+    shape = W.TINY_SHAPE
+    m, layers_np, head_np = _model(shape, seed=1)
+    V = shape.vocab
+    h = W.step_hidden(B, k, shape.hidden, seed=2)
+    qp = W.logits_case(B, k, V, ar_std=2.0, sigma=1.0, peak_frac=0.0, seed=3)
+    q_prev = qp.q_logits
+    d_prev = S.draft_sample(q_prev, T, 7, 4)             # drafted at the previous step
+    buf = _buffers(B, k, V)
+    ws = torch.empty(m.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
+    Q_prev = dev_tensor(q_prev, "bf16")
+    D_prev = dev_tensor(d_prev, "i32")
+    m.step(B, k, dev_tensor(h, "bf16"), Q_prev, D_prev, T, 7, 5, buf["q_next"], buf["d_next"],
+           buf["acc"], buf["tok"], buf["cnt"], ws, logits_out=buf["logits"],
+           dev_status=buf["status"])
+    torch.cuda.synchronize()
+    assert int(buf["status"].item()) == 0
+    # logits of every row vs the oracle stack
+    ref = O.stack_logits(h, layers_np, head_np, O.step_gate(B, k), shape.scale)
+    got = np.concatenate([host_f64(buf["logits"]), host_f64(buf["q_next"]).reshape(B * k, V)])
+    check_close(got, ref, what="step logits")
+    # tokens: same as the verify / draft kernels on the step's own logits
+    acc, tok, cnt = U.psi_verify(buf["logits"].reshape(B, k + 1, V), Q_prev, D_prev, T, 7, 5)
+    np.testing.assert_array_equal(buf["acc"].cpu().numpy(), acc.cpu().numpy())
+    np.testing.assert_array_equal(buf["tok"].cpu().numpy(), tok.cpu().numpy())
+    np.testing.assert_array_equal(buf["cnt"].cpu().numpy(), cnt.cpu().numpy())
+    d = U.draft_sample(buf["q_next"], T, 7, 5)
+    np.testing.assert_array_equal(buf["d_next"].cpu().numpy(), d.cpu().numpy())
+    m.close()
+
+
+def test_zero_adapter_step_accepts_its_own_drafts():
+    """Bl = 0 everywhere: q_next equals the drafted-token verify rows, so verifying the
+    step's own drafts against its AR rows accepts every block."""
+    import torch
+    import sampling_gated_lora_b200 as U
+    shape = W.TINY_SHAPE
+    layers_np, head_np = W.model_weights_np(shape, seed=4)
+    zero = lambda wab: (wab[0], wab[1], np.zeros_like(wab[2]))
+    layers_np = [{k: zero(v) for k, v in lw.items()} for lw in layers_np]
+    head_np = zero(head_np)
+    tl = lambda wab: tuple(dev_tensor(a, "bf16") for a in wab)
+    m = U.Model([{k: tl(v) for k, v in lw.items()} for lw in layers_np], tl(head_np), shape.hidden,
+                shape.q_out, shape.kv_out, shape.inter, shape.vocab, shape.r)
+    B, k, V = 4, 4, shape.vocab
+    h = dev_tensor(W.step_hidden(B, k, shape.hidden, seed=5), "bf16")
+    buf = _buffers(B, k, V)
+    q0 = torch.zeros((B, k, V), dtype=torch.bfloat16, device="cuda")
+    d0 = torch.zeros((B, k), dtype=torch.int32, device="cuda")
+    ws = torch.empty(m.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
+    m.step(B, k, h, q0, d0, 1.0, 3, 0, buf["q_next"], buf["d_next"], buf["acc"], buf["tok"],
+           buf["cnt"], ws, logits_out=buf["logits"])
+    p = buf["logits"].reshape(B, k + 1, V)
+    np.testing.assert_array_equal(host_f64(p[:, 1:]), host_f64(buf["q_next"]))
+    acc, tok, cnt = U.psi_verify(p[:, 1:].contiguous(), buf["q_next"], buf["d_next"], 1.0, 3, 1)
+    assert np.all(acc.cpu().numpy() == k)
+    m.close()

@@ -1,0 +1,136 @@
+"""psi_verify on the GPU vs the fp64 oracle: identical accepted lengths and tokens
+except at logged near-ties (|u - p/q| < 1e-4, or a draw threshold within 1e-5 of
+a CDF edge), which must stay <= 1e-4 of all positions at full size."""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import sampling as S
+from gpu_util import (EXCUSED_CAP, check_verify_outputs_valid, compare_verify, dev_tensor)
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_verify(p, q, d, T, seed, step, seq_offset=0, dt="bf16", status=None):
+    import sampling_gated_lora_b200 as U
+    P = p if not isinstance(p, np.ndarray) else dev_tensor(p, dt)
+    Q = q if not isinstance(q, np.ndarray) else dev_tensor(q, dt)
+    acc, tok, cnt = U.psi_verify(P, Q, dev_tensor(d, "i32"), T, seed, step, seq_offset,
+                                 dev_status=status)
+    return acc.cpu().numpy(), tok.cpu().numpy(), cnt.cpu().numpy()
+
+
+def _case_check(case, T, seed, step, seq_offset=0, max_excused=1):
+    d = S.draft_sample(case.q_logits, T, seed + 1, step, seq_offset)   # inputs: drafts ~ q
+    gpu = _gpu_verify(case.p_logits, case.q_logits, d, T, seed, step, seq_offset, case.dtype)
+    ora = S.psi_verify(case.p_logits, case.q_logits, d, T, seed, step, seq_offset)
+    check_verify_outputs_valid(*gpu, d, case.k, case.k_p, case.V)
+    excused, bad = compare_verify(gpu, ora, case.k, range(case.B))
+    assert not bad, f"unexcused mismatches in sequences {bad}"
+    assert len(excused) <= max_excused
+    return gpu, ora
+
+
+def test_tiny_fp32_case():
+    case = W.tiny_logits_case()                      # B=2, k=4, V=1024, fp32
+    _case_check(case, 1.0, 0, 0)
+
+
+@pytest.mark.parametrize("T", [1.0, 0.7])
+@pytest.mark.parametrize("k,k_p", [(8, 8), (8, 9), (1, 1), (1, 2), (32, 32), (31, 32)])
+def test_medium_bf16(k, k_p, T):
+    case = W.logits_case(16, k, 20000, k_p=k_p, ar_std=3.0, sigma=1.0, seed=11)
+    _case_check(case, T, 5, 3)
+
+
+def test_ragged_vocab_unaligned_rows():
+    # V odd: rows are not 16-byte aligned; chunk edges are ragged
+    case = W.logits_case(6, 4, 1001, k_p=5, ar_std=2.0, sigma=1.5, seed=2)
+    _case_check(case, 1.0, 9, 1)
+    case = W.logits_case(3, 3, 2, ar_std=1.0, sigma=1.0, peak_frac=0.0, seed=4)   # V = 2
+    _case_check(case, 0.7, 1, 0)
+
+
+def test_fp32_logits_large_vocab():
+    case = W.logits_case(4, 6, 151936, k_p=7, ar_std=3.0, sigma=1.0, seed=7, dtype="f32")
+    _case_check(case, 1.0, 3, 2)
+
+
+def test_sequence_offset_reproduces_global_draws():
+    case = W.logits_case(8, 4, 5000, ar_std=3.0, sigma=1.0, seed=8)
+    d = S.draft_sample(case.q_logits, 1.0, 4, 0)
+    full = _gpu_verify(case.p_logits, case.q_logits, d, 1.0, 3, 0)
+    hi = _gpu_verify(case.p_logits[4:], case.q_logits[4:], d[4:], 1.0, 3, 0, seq_offset=4)
+    for a, b in zip(full, hi):
+        np.testing.assert_array_equal(a[4:], b)
+
+
+def test_zero_adapter_accepts_every_block():
+    """q == p (the adapter's B = 0): n = k for every sequence, with or without the bonus."""
+    case = W.logits_case(64, 8, 30000, k_p=9, ar_std=3.0, sigma=0.0, seed=12)
+    for T in (1.0, 0.7):
+        for seed in (0, 1, 2):
+            d = S.draft_sample(case.p_logits[:, :8], T, seed + 100, 0)
+            acc, tok, cnt = _gpu_verify(case.p_logits, case.p_logits[:, :8], d, T, seed, 0)
+            assert np.all(acc == 8) and np.all(cnt == 9)
+            np.testing.assert_array_equal(tok[:, :8], d)
+
+
+def test_bad_draft_and_nan_are_flagged_not_trapped():
+    import torch
+    import sampling_gated_lora_b200 as U
+    case = W.logits_case(4, 4, 4096, ar_std=3.0, sigma=1.0, seed=13)
+    d = S.draft_sample(case.q_logits, 1.0, 0, 0)
+    d_bad = d.copy()
+    d_bad[1, 2] = 4096            # out of range
+    p = case.p_logits.copy()
+    p[2, 1, 17] = 0x7FC0          # NaN
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    acc, tok, cnt = _gpu_verify(p, case.q_logits, d_bad, 1.0, 0, 0, status=status)
+    st = int(status.item())
+    assert st & U.DEV_BAD_DRAFT and st & U.DEV_NAN
+    assert acc[1] == -1 and cnt[1] == -1 and np.all(tok[1] == -1)
+    assert acc[2] == -1 and cnt[2] == -1 and np.all(tok[2] == -1)
+    ora = S.psi_verify(case.p_logits, case.q_logits, d, 1.0, 0, 0)
+    for b in (0, 3):
+        assert acc[b] == ora["accepted_len"][b]
+        np.testing.assert_array_equal(tok[b], ora["out_tokens"][b])
+    assert U.device_status(clear=True) & U.DEV_BAD_DRAFT
+
+
+def test_empty_batch():
+    import torch
+    import sampling_gated_lora_b200 as U
+    z = torch.empty((0, 4, 64), dtype=torch.bfloat16, device="cuda")
+    acc, tok, cnt = U.psi_verify(z, z, torch.empty((0, 4), dtype=torch.int32, device="cuda"),
+                                 1.0, 0, 0)
+    assert acc.numel() == 0
+
+
+@pytest.mark.parametrize("sigma", [0.25, 1.0])
+def test_full_size_sampled_parity(sigma):
+    """B=256, k=16, V=151936, AR std 3 with 5% peaked positions; T in {1, 0.7}.
+
+    The oracle recomputes 32 sampled sequences one by one; every sequence is
+    checked for validity; excused positions are logged and capped at 1e-4.
+    """
+    import torch
+    B, k, V = 256, 16, 151936
+    p, q = W.logits_case_torch(B, k, V, sigma=sigma, seed=1234)
+    p_h, q_h = W.from_torch_bf16(p), W.from_torch_bf16(q)
+    rng = np.random.default_rng(int(sigma * 100))
+    sample = np.sort(rng.choice(B, 32, replace=False))
+    total_excused = 0
+    for T in (1.0, 0.7):
+        d = S.draft_sample(q_h, T, 99, 0)
+        gpu = _gpu_verify(p, q, d, T, 1234, 0)
+        check_verify_outputs_valid(*gpu, d, k, k, V)
+        ora = S.psi_verify(p_h, q_h, d, T, 1234, 0, sequences=sample)
+        excused, bad = compare_verify(gpu, ora, k, sample)
+        assert not bad, f"sigma={sigma} T={T}: unexcused mismatches {bad}"
+        total_excused += len(excused)
+        print(f"sigma={sigma} T={T}: mean accepted {gpu[0].mean():.3f}, "
+              f"excused {len(excused)} of {len(sample) * k} positions")
+    assert total_excused <= max(EXCUSED_CAP * 2 * len(sample) * k, 0)
+    del p, q
+    torch.cuda.empty_cache()

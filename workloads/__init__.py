@@ -339,3 +339,32 @@ def step_hidden(B: int, k: int, hidden: int, seed=0) -> np.ndarray:
 def draft_ids(B: int, k: int, V: int, seed=0) -> np.ndarray:
     """Uniform draft token ids [B,k] int32 (for shape-only uses, e.g. the first step)."""
     return _rng(seed, B, k, V).integers(0, V, size=(B, k), dtype=np.int32)
+
+
+def logits_case_torch(B: int, k: int, V: int, *, k_p=None, ar_std=3.0, sigma=1.0,
+                      peak_frac=0.05, peak_add=12.0, seed=1234, device="cuda", chunk=32):
+    """Same recipe as `logits_case`, drawn by torch's seeded generator on `device`.
+
+    For full-size workloads (B=256, k=16, V=151936 is 1.24e9 normals), where
+    host generation takes minutes. Returns bf16 tensors (p [B,k_p,V], q [B,k,V]);
+    tests copy the rows they check back to the host.
+    """
+    import torch
+    k_p = k if k_p is None else k_p
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed) * 7919 + int(round(sigma * 1000)))
+    p = torch.empty((B, k_p, V), dtype=torch.bfloat16, device=device)
+    q = torch.empty((B, k, V), dtype=torch.bfloat16, device=device)
+    for b0 in range(0, B, chunk):
+        nb = min(chunk, B - b0)
+        ar = torch.randn((nb, k_p, V), generator=gen, device=device) * ar_std
+        if peak_frac > 0:
+            peaked = torch.rand((nb, k_p), generator=gen, device=device) < peak_frac
+            tok = torch.randint(0, V, (nb, k_p), generator=gen, device=device)
+            bump = torch.zeros((nb, k_p, V), device=device)
+            bump.scatter_(2, tok.unsqueeze(-1), (peaked.float() * peak_add).unsqueeze(-1))
+            ar += bump
+        noise = torch.randn((nb, k, V), generator=gen, device=device) * sigma
+        p[b0:b0 + nb] = ar.to(torch.bfloat16)
+        q[b0:b0 + nb] = (ar[:, :k] + noise).to(torch.bfloat16)
+    return p, q
