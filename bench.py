@@ -1,0 +1,548 @@
+#!/usr/bin/env python
+"""Benchmark of the synthetic Psi-Spec linear decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--B 256] [--k 8] [--impl uno|reference]
+
+One step = uno_psi_step on Qwen3-8B-shaped gated-LoRA projections (36 layers of
+q/k/v/o/gate/up/down, rank 128, no attention) + the gated LM head
+4096 -> 151936 + psi_verify (bonus enabled) + the linear-sampler draft, for B
+sequences with block size k (M = B(2k+1) rows). Metric: verified tokens/s =
+tokens emitted by verification / step time, summed over ranks (each rank runs
+its own replica on its own B sequences: weak scaling, no collective on the
+data path). Rank 0 prints one JSON line.
+
+Timing: W untimed steps, then K steps between CUDA events on the launching
+stream, bracketed by a barrier and device synchronisation; max over ranks.
+Every step streams 15.1 GB of weights, far larger than the 126 MB L2.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Ψ-Spec verified tokens/s at B=1..256; gated-LoRA/verify GB/s vs HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--B", type=int, default=256)
+    ap.add_argument("--k", type=int, default=8)
+    ap.add_argument("--temperature", type=float, default=1.0)
+    ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
+    ap.add_argument("--no-kernels", action="store_true", help="skip the per-config kernel lines")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--profile", choices=["gemm_up", "gemm_small", "verify", "draft"],
+                    help="run a few launches of one kernel on a small case (for ncu) and exit")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(B, k, T):
+    return {"workload": f"psi_step Qwen3-8B-shaped: 36 layers q/k/v/o 4096->4096/1024/1024/4096, "
+                        f"gate/up 4096->12288, down 12288->4096, LM head 4096->151936, rank 128, "
+                        f"no attention; B={B}, k={k}, rows B(2k+1)={B * (2 * k + 1)}, T={T}",
+            "B": B, "k": k, "rows": B * (2 * k + 1), "vocab": 151936, "rank": 128,
+            "layers": 36, "temperature": T,
+            "l2": "inputs larger than L2 (15.1 GB of weights streamed per step)"}
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        self.f = tempfile.NamedTemporaryFile("w+", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), int(parts[3], 16)))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        mask = 0
+        for r in rows:
+            mask |= r[3]
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows),
+                "reasons": [n for b, n in REASONS.items() if mask & b and b != 0x1]}
+
+
+# ---------------------------------------------------------------- oracle sample
+
+HEAD_SLICE = 8   # the oracle's LM head is timed on 1/8 of the vocabulary rows and scaled x8
+
+
+def oracle_step_sample(k, layers_np, head_slice, T, seed=0):
+    """One sequence (2k+1 rows) through the fp64 oracle, timed piecewise:
+    `len(layers_np)` decoder layers (scaled to 36), the LM head on a 1/HEAD_SLICE
+    vocabulary slice (scaled x HEAD_SLICE), then the draft sampler and verify
+    over the full 151936-token vocabulary on seeded logits of the verify
+    workload. Returns (seconds per full step, tokens emitted)."""
+    import workloads as W
+    from oracle import sampling as S
+    from oracle import stack as O
+    h = W.step_hidden(1, k, 4096, seed=seed)
+    gate = O.step_gate(1, k)
+    t0 = time.perf_counter()
+    x = O.as_f64(h)
+    for lw in layers_np:
+        x = O.layer_forward(x, lw, gate, 1.0)
+    t1 = time.perf_counter()
+    O.round_bf16(O._lin(O.round_bf16(O.rmsnorm(x)), head_slice, gate, 1.0))
+    t2 = time.perf_counter()
+    p, q = W.logits_sequence(seed, k, k + 1, 151936, ar_std=3.0, sigma=1.0, peak_frac=0.05, seed=1234)
+    t3 = time.perf_counter()
+    d = S.draft_sample(q[None], T, seed, 0)
+    res = S.psi_verify(p[None], q[None], d, T, seed, 1)
+    t4 = time.perf_counter()
+    per_layer = (t1 - t0) / max(1, len(layers_np))
+    return per_layer * 36 + (t2 - t1) * HEAD_SLICE + (t4 - t3), int(res["out_count"][0])
+
+
+SAMPLE_TEXT = ("per step: one sequence (2k+1 rows) through the fp64 NumPy oracle; 1 of 36 layers "
+               "timed and scaled x36, the LM head on 1/8 of the vocabulary scaled x8, draft + "
+               "verify over the full vocabulary timed in full")
+
+
+def host_weights(layers, head, n_layers):
+    """Copy n_layers layers and a 1/HEAD_SLICE row slice of the head (torch bf16, device) to host bits."""
+    import workloads as W
+    tl = lambda wab: tuple(W.from_torch_bf16(t) for t in wab)
+    rows = head[0].shape[0] // HEAD_SLICE
+    sl = (head[0][:rows], head[1], head[2][:rows])
+    return [{k: tl(v) for k, v in lw.items()} for lw in layers[:n_layers]], tl(sl)
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ---------------------------------------------------------------- kernel lines
+
+def kernel_lines(U, torch, pk):
+    """Per-config kernel measurements (gated GEMM small M and M=2048, psi_verify)."""
+    import numpy as np
+    import workloads as W
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(fn, reps=20):
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(ts)
+
+    dev = lambda shape, std: (torch.randn(shape, device="cuda") * std).to(torch.bfloat16)
+    for B in (1, 8, 64):
+        M, K, N, r = B * 9, 4096, 4096, 128
+        x, Wt, A, Bl = dev((M, K), 1), dev((N, K), K ** -0.5), dev((r, K), K ** -0.5), dev((N, r), 0.01)
+        g = torch.from_numpy(W.decode_gate(B, 8)).cuda()
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(U.load().uno_gated_lora_linear_workspace(0, M, K, N, r), dtype=torch.uint8,
+                         device="cuda")
+        f = lambda: U.gated_lora_linear(x, Wt, A, Bl, g, 1.0, y=y, workspace=ws)
+        f()
+        us = timed(f)
+        Mg = int(g.sum())
+        byts = 2 * (N * K + r * K + N * r + M * K + M * N)
+        flops = 2 * M * K * N + 2 * Mg * r * (K + N)
+        t_roof = max(byts / (pk["hbm_gbs"] * 1e9), flops / (pk["bf16_tflops"] * 1e12)) * 1e6
+        out[f"gated_linear_4096x4096_M{M}"] = {
+            "us": round(us, 2), "GBps": round(byts / us / 1e3, 1), "TFLOPs": round(flops / us / 1e6, 1),
+            "roofline_us": round(t_roof, 2), "frac_of_roofline": round(t_roof / us, 3),
+            "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3)}
+    for name, K, N in (("up", 4096, 12288), ("down", 12288, 4096)):
+        M, r = 2048, 128
+        x, Wt, A, Bl = dev((M, K), 1), dev((N, K), K ** -0.5), dev((r, K), K ** -0.5), dev((N, r), 0.01)
+        g = torch.cat([torch.zeros(M // 2, dtype=torch.uint8), torch.ones(M // 2, dtype=torch.uint8)]).cuda()
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(U.load().uno_gated_lora_linear_workspace(0, M, K, N, r), dtype=torch.uint8,
+                         device="cuda")
+        f = lambda: U.gated_lora_linear(x, Wt, A, Bl, g, 1.0, y=y, workspace=ws)
+        f()
+        us = timed(f)
+        flops = 2 * M * K * N + 2 * (M // 2) * r * (K + N)
+        out[f"gated_linear_mlp_{name}_M2048"] = {
+            "us": round(us, 2), "TFLOPs": round(flops / us / 1e6, 1),
+            "tensor_frac": round(flops / us / 1e6 / pk["bf16_tflops"], 3)}
+    del x, Wt, A, Bl, y
+    # psi_verify at B=256, k=16, V=151936 (sigma 1.0 and 0.25, T = 1)
+    B, k, V = 256, 16, 151936
+    for sigma in (1.0, 0.25):
+        p, q = W.logits_case_torch(B, k, V, sigma=sigma, seed=1234)
+        d = U.draft_sample(q, 1.0, 99, 0)
+        ws = torch.empty(U.load().uno_psi_verify_workspace(B, k, k, V), dtype=torch.uint8, device="cuda")
+        outs = [torch.empty(B, dtype=torch.int32, device="cuda"),
+                torch.empty((B, k + 1), dtype=torch.int32, device="cuda"),
+                torch.empty(B, dtype=torch.int32, device="cuda")]
+        f = lambda: U.psi_verify(p, q, d, 1.0, 1234, 0, accepted_len=outs[0], out_tokens=outs[1],
+                                 out_count=outs[2], workspace=ws)
+        f()
+        us = timed(f, reps=10)
+        byts = 2 * B * k * V * 2
+        out[f"psi_verify_B256_k16_sigma{sigma}"] = {
+            "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
+            "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3),
+            "mean_accepted": round(float(outs[0].float().mean()), 3)}
+        del p, q
+    torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------- main arms
+
+def run_uno(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import sampling_gated_lora_b200 as U
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    U.load()
+    pk, pk_src = peaks()
+    shape = W.QWEN3_8B_SHAPE
+    B, k, T = args.B, args.k, args.temperature
+    V = shape.vocab
+    layers, head = W.model_weights_torch(shape, "cuda", seed=0)
+    model = U.Model(layers, head, shape.hidden, shape.q_out, shape.kv_out, shape.inter, V, shape.r,
+                    shape.scale)
+    M = B * (2 * k + 1)
+    h_host = torch.from_numpy(W.step_hidden(B, k, shape.hidden, seed=rank).view(np.int16)).view(
+        torch.bfloat16).pin_memory()
+    h = h_host.cuda()
+    i32 = dict(dtype=torch.int32, device="cuda")
+    qb = [torch.zeros((B, k, V), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    db = [torch.zeros((B, k), **i32) for _ in range(2)]
+    n_total = args.warmup + args.steps
+    acc = torch.empty((n_total, B), **i32)
+    tok = torch.empty((n_total, B, k + 1), **i32)
+    cnt = torch.empty((n_total, B), **i32)
+    status = torch.zeros(1, **i32)
+    ws = torch.empty(model.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
+    seq_off = rank * B
+
+    def step(t):
+        model.step(B, k, h, qb[t % 2], db[t % 2], T, 2026, t, qb[(t + 1) % 2], db[(t + 1) % 2],
+                   acc[t], tok[t], cnt[t], ws, dev_status=status, seq_offset=seq_off)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for t in range(args.warmup):
+        step(t)
+    barrier()
+    dev_idx = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]
+    with ClockSampler(dev_idx) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for t in range(args.warmup, n_total):
+            step(t)
+        e1.record()
+        e1.synchronize()
+        barrier()
+    clocks = clk.summary()
+    ms = e0.elapsed_time(e1)
+    tokens = int(cnt[args.warmup:].sum())
+    st = int(status.item())
+    stat = torch.tensor([ms, float(tokens), float(st)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        mx = stat.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = stat.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        ms_max, tokens_all = float(mx[0]), int(sm[1])
+    else:
+        ms_max, tokens_all = ms, tokens
+    value = tokens_all / (ms_max / 1e3)
+
+    # e2e: the public API with host buffers; H2D of the step's hidden states and
+    # D2H of its results inside the timed region, every step.
+    acc_h = torch.empty((args.steps, B), dtype=torch.int32).pin_memory()
+    tok_h = torch.empty((args.steps, B, k + 1), dtype=torch.int32).pin_memory()
+    cnt_h = torch.empty((args.steps, B), dtype=torch.int32).pin_memory()
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record()
+    for i in range(args.steps):
+        t = n_total + i
+        h.copy_(h_host, non_blocking=True)
+        model.step(B, k, h, qb[t % 2], db[t % 2], T, 2026, t, qb[(t + 1) % 2], db[(t + 1) % 2],
+                   acc[i], tok[i], cnt[i], ws, dev_status=status, seq_offset=seq_off)
+        acc_h[i].copy_(acc[i], non_blocking=True)
+        tok_h[i].copy_(tok[i], non_blocking=True)
+        cnt_h[i].copy_(cnt[i], non_blocking=True)
+    e3.record()
+    e3.synchronize()
+    e2e_ms = e2.elapsed_time(e3)
+    e2e_tokens = int(cnt_h.sum())
+    est = torch.tensor([e2e_ms, float(e2e_tokens)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        mx = est.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = est.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        e2e_ms_max, e2e_tok_all = float(mx[0]), int(sm[1])
+    else:
+        e2e_ms_max, e2e_tok_all = e2e_ms, e2e_tokens
+    e2e = {"value": round(e2e_tok_all / (e2e_ms_max / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": h_host.numel() * 2,
+           "d2h_bytes_per_step": (acc_h[0].numel() + tok_h[0].numel() + cnt_h[0].numel()) * 4}
+
+    # dominant kernel: the gated linear of the MLP up projection at this step's M
+    # (gate/up/down carry 78 % of the step's flops), timed alone with events.
+    roof = None
+    if rank == 0:
+        Kd, Nd, r = shape.hidden, shape.inter, shape.r
+        x = torch.randn((M, Kd), device="cuda").to(torch.bfloat16)
+        lw = layers[0]["up"]
+        g = torch.from_numpy(W.step_gate(B, k)).cuda()
+        y = torch.empty((M, Nd), dtype=torch.bfloat16, device="cuda")
+        wsl = torch.empty(U.load().uno_gated_lora_linear_workspace(0, M, Kd, Nd, r),
+                          dtype=torch.uint8, device="cuda")
+        f = lambda: U.gated_lora_linear(x, lw[0], lw[1], lw[2], g, 1.0, y=y, workspace=wsl)
+        for _ in range(3):
+            f()
+        reps = 20
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            f()
+        b.record()
+        b.synchronize()
+        us = a.elapsed_time(b) * 1e3 / reps
+        Mg = B * k
+        flops = 2 * M * Kd * Nd + 2 * Mg * r * (Kd + Nd)
+        byts = 2 * (Nd * Kd + r * Kd + Nd * r + M * Kd + M * Nd)
+        tensor_bound = flops / (pk["bf16_tflops"] * 1e12) > byts / (pk["hbm_gbs"] * 1e9)
+        if tensor_bound:
+            ach = flops / us / 1e6
+            roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 3), "traffic": None}
+        else:
+            ach = byts / us / 1e3
+            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(ach / pk["hbm_gbs"], 3), "traffic": None}
+        roof.update({"kernel": f"gated_lora_linear (LoRA down + fused GEMM) up 4096->12288, M={M}",
+                     "us_per_launch": round(us, 2), "peak_source": pk_src + " burst",
+                     "algorithmic_flops": flops, "algorithmic_bytes": byts})
+        del x, y
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and hidden states; no attention)",
+        "config": workload_config(B, k, T), "clocks": clocks,
+        "gpu_launches": model.kernel_count() * args.steps, "e2e": e2e, "roofline": roof,
+        "mean_accepted": round(float(acc[args.warmup:n_total].float().mean()), 3),
+        "device_status": st,
+    }
+    if world == 1 and rank == 0 and not args.no_kernels:
+        # kernel lines and the B sweep (N = 1 only)
+        sweep = {}
+        for Bs in (1, 32, 128):
+            sweep[f"B{Bs}"] = sweep_point(U, torch, W, model, Bs, k, T, V, shape)
+        result["sweep_tokens_per_s"] = sweep
+        del ws, qb, db
+        torch.cuda.empty_cache()
+        result["kernels"] = kernel_lines(U, torch, pk)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        lw_np, head_np = host_weights(layers, head, 1)
+        secs, toks = 0.0, 0
+        for i in range(3):
+            s_, n_ = oracle_step_sample(k, lw_np, head_np, T, seed=i)
+            secs, toks = secs + s_, toks + n_
+        result["cpu_baseline"] = {"value": round(toks / secs, 4), "unit": "tokens/s",
+                                  "cores": cpu_cores(), "kind": "oracle",
+                                  "sample": "3 steps; " + SAMPLE_TEXT}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    model.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def sweep_point(U, torch, W, model, B, k, T, V, shape):
+    import numpy as np
+    i32 = dict(dtype=torch.int32, device="cuda")
+    h = W.to_torch_bf16(W.step_hidden(B, k, shape.hidden, seed=7), "cuda")
+    qb = [torch.zeros((B, k, V), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    db = [torch.zeros((B, k), **i32) for _ in range(2)]
+    acc, tok, cnt = torch.empty(B, **i32), torch.empty((B, k + 1), **i32), torch.empty((8, B), **i32)
+    ws = torch.empty(model.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
+    step = lambda t, c: model.step(B, k, h, qb[t % 2], db[t % 2], T, 5, t, qb[(t + 1) % 2],
+                                   db[(t + 1) % 2], acc, tok, c, ws)
+    for t in range(3):
+        step(t, cnt[0])
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(8):
+        step(3 + i, cnt[i])
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b)
+    return {"tokens_per_s": round(int(cnt.sum()) / (ms / 1e3), 1), "ms_per_step": round(ms / 8, 3)}
+
+
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm, on bounded samples of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import workloads as W
+    shape = W.QWEN3_8B_SHAPE
+    # one layer of weights and the head, drawn by torch's seeded CPU generator
+    gen = torch.Generator().manual_seed(0)
+    mk = lambda n, k_, std: W.from_torch_bf16((torch.randn((n, k_), generator=gen) * std).to(torch.bfloat16))
+    lw = {}
+    for name, K, N in shape.linears():
+        lw[name] = (mk(N, K, K ** -0.5), mk(shape.r, K, K ** -0.5), mk(N, shape.r, 0.01))
+    rows = shape.vocab // HEAD_SLICE
+    head = (mk(rows, shape.hidden, shape.hidden ** -0.5), mk(shape.r, shape.hidden, shape.hidden ** -0.5),
+            mk(rows, shape.r, 0.01))
+    for t in range(args.warmup):
+        oracle_step_sample(args.k, [lw], head, args.temperature, seed=t)
+    secs, toks = 0.0, 0
+    for t in range(args.steps):
+        s, n = oracle_step_sample(args.k, [lw], head, args.temperature, seed=100 + t)
+        secs += s
+        toks += n
+    value = toks / secs
+    sample = SAMPLE_TEXT
+    print(json.dumps({
+        "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(args.B, args.k, args.temperature),
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cpu_cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def run_profile(args):
+    """A few launches of one hot kernel on a small case, for an ncu capture.
+
+    gemm_up:    gated linear 4096 -> 12288, M = B(2k+1) rows (the step's MLP shape)
+    gemm_small: gated linear 4096 -> 4096, M = 9 (split-K cluster path)
+    verify:     psi_verify B=32, k=16, V=151936 (311 MB of logits)
+    draft:      draft sampler B=32, k=8, V=151936
+    """
+    import torch
+    import sampling_gated_lora_b200 as U
+    import workloads as W
+    torch.cuda.set_device(0)
+    dev = lambda shape, std: (torch.randn(shape, device="cuda") * std).to(torch.bfloat16)
+    if args.profile in ("gemm_up", "gemm_small"):
+        M, K, N = ((args.B * (2 * args.k + 1), 4096, 12288) if args.profile == "gemm_up"
+                   else (9, 4096, 4096))
+        r = 128
+        x, Wt, A, Bl = dev((M, K), 1), dev((N, K), K ** -0.5), dev((r, K), K ** -0.5), dev((N, r), 0.01)
+        g = (torch.arange(M, device="cuda") % 2).to(torch.uint8)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        f = lambda: U.gated_lora_linear(x, Wt, A, Bl, g, 1.0, y=y)
+    elif args.profile == "verify":
+        p, q = W.logits_case_torch(32, 16, 151936, sigma=1.0, seed=1234)
+        d = U.draft_sample(q, 1.0, 99, 0)
+        f = lambda: U.psi_verify(p, q, d, 1.0, 1234, 0)
+    else:
+        _, q = W.logits_case_torch(32, 8, 151936, sigma=1.0, seed=1234)
+        f = lambda: U.draft_sample(q, 1.0, 99, 0)
+    for _ in range(4):
+        f()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "status": U.device_status()}))
+
+
+def main():
+    args = parse()
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
+        run_reference(args)
+    else:
+        run_uno(args)
+
+
+if __name__ == "__main__":
+    main()

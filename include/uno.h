@@ -180,8 +180,10 @@ void uno_model_destroy(uno_model* m);
  *     (gate 1) that produce the next block's draft distributions.
  *   Verifies the previous block (q_prev [B,k,V] bf16, d_prev [B,k] int32)
  *   against this step's AR rows p [B,k+1,V] (bonus enabled), as
- *   uno_psi_verify with k_p = k+1 and the same seed/step; then drafts the next
- *   block from the mask rows as uno_draft_sample (same seed/step) into
+ *   uno_psi_verify with k_p = k+1 and the same seed/step/seq_offset (global
+ *   sequence ids seq_offset + b: a batch split over ranks draws what the
+ *   whole batch would); then drafts the next block from the mask rows as
+ *   uno_draft_sample (same seed/step/seq_offset) into
  *   d_next [B,k], and writes their logits to q_next [B,k,V] bf16.
  *   logits_out: optional [B(k+1), V] bf16 copy target for the AR rows (NULL
  *   to skip). accepted_len [B], out_tokens [B,k+1], out_count [B] as in
@@ -190,9 +192,12 @@ size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k);
 
 uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, const void* q_prev,
                         const int32_t* d_prev, float temperature, uint64_t seed, uint64_t step,
-                        void* q_next, int32_t* d_next, void* logits_out, int32_t* accepted_len,
-                        int32_t* out_tokens, int32_t* out_count, int32_t* dev_status,
-                        void* workspace, size_t ws_bytes, void* stream);
+                        uint64_t seq_offset, void* q_next, int32_t* d_next, void* logits_out,
+                        int32_t* accepted_len, int32_t* out_tokens, int32_t* out_count,
+                        int32_t* dev_status, void* workspace, size_t ws_bytes, void* stream);
+
+/* Number of kernel launches one uno_psi_step call of this model issues. */
+int32_t uno_psi_step_kernel_count(const uno_model* m);
 
 /* ---------------------------------------------------------------------------
  * The step's glue operations, exposed for testing (all bf16, device):

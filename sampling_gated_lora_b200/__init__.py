@@ -32,6 +32,7 @@ EXPORTS = [
     "uno_draft_sample_workspace", "uno_draft_sample",
     "uno_philox_uniforms",
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
+    "uno_psi_step_kernel_count",
     "uno_rmsnorm", "uno_silu_mul",
 ]
 
@@ -73,8 +74,9 @@ def load():
         "uno_model_create": (i32, [vp, i32, i32, i32, i32, i32, i32, i32, f32, vp]),
         "uno_model_destroy": (None, [vp]),
         "uno_psi_step_workspace": (sz, [vp, i32, i32]),
-        "uno_psi_step": (i32, [vp, i32, i32, vp, vp, vp, f32, u64, u64, vp, vp, vp, vp, vp, vp, vp,
-                               vp, sz, vp]),
+        "uno_psi_step": (i32, [vp, i32, i32, vp, vp, vp, f32, u64, u64, u64, vp, vp, vp, vp, vp,
+                               vp, vp, vp, sz, vp]),
+        "uno_psi_step_kernel_count": (i32, [vp]),
         "uno_rmsnorm": (i32, [i64, i64, vp, vp, f32, vp]),
         "uno_silu_mul": (i32, [i64, vp, vp, vp, vp]),
     }
@@ -279,15 +281,20 @@ class Model:
     def workspace_bytes(self, B, k):
         return load().uno_psi_step_workspace(self._h, B, k)
 
+    def kernel_count(self):
+        """Kernel launches issued by one step."""
+        return load().uno_psi_step_kernel_count(self._h)
+
     def step(self, B, k, h_in, q_prev, d_prev, temperature, seed, step, q_next, d_next,
              accepted_len, out_tokens, out_count, workspace, logits_out=None, dev_status=None,
-             stream=None):
+             seq_offset=0, stream=None):
         """uno_psi_step on caller-provided device buffers (see include/uno.h)."""
         _dev(h_in, q_prev, d_prev, q_next, d_next, accepted_len, out_tokens, out_count, workspace,
              logits_out, dev_status)
         wsb = workspace.numel() * workspace.element_size()
         _check(load().uno_psi_step(self._h, B, k, _ptr(h_in), _ptr(q_prev), _ptr(d_prev),
-                                   float(temperature), int(seed), int(step), _ptr(q_next),
+                                   float(temperature), int(seed), int(step), int(seq_offset),
+                                   _ptr(q_next),
                                    _ptr(d_next), _ptr(logits_out), _ptr(accepted_len),
                                    _ptr(out_tokens), _ptr(out_count), _ptr(dev_status),
                                    _ptr(workspace), wsb, _stream(stream)))

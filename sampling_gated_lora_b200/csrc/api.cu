@@ -499,17 +499,25 @@ size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k) {
   return step_layout(m, B, k).total;
 }
 
+int32_t uno_psi_step_kernel_count(const uno_model* m) {
+  if (!m) return 0;
+  // per layer: 2 rmsnorm + 7 linears (down-projection + main GEMM each when
+  // r > 0) + silu*up; then rmsnorm + LM head; verify (2 kernels) + draft (1)
+  const int per_lin = m->r > 0 ? 2 : 1;
+  return m->n_layers * (3 + kLinPerLayer * per_lin) + 1 + per_lin + 3;
+}
+
 uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, const void* q_prev,
                         const int32_t* d_prev, float temperature, uint64_t seed, uint64_t step,
-                        void* q_next, int32_t* d_next, void* logits_out, int32_t* accepted_len,
-                        int32_t* out_tokens, int32_t* out_count, int32_t* dev_status,
-                        void* workspace, size_t ws_bytes, void* stream) {
+                        uint64_t seq_offset, void* q_next, int32_t* d_next, void* logits_out,
+                        int32_t* accepted_len, int32_t* out_tokens, int32_t* out_count,
+                        int32_t* dev_status, void* workspace, size_t ws_bytes, void* stream) {
   if (!m) return set_error(UNO_ERR_INVALID_ARG, "model is NULL");
   uno_status s = check_sampler(UNO_BF16, B, k, m->vocab, temperature);
   if (s != UNO_OK) return s;
   if (B < 1) return set_error(UNO_ERR_INVALID_ARG, "B must be >= 1");
-  if (static_cast<uint64_t>(B) * static_cast<uint64_t>(k + 1) > (1ull << 32))
-    return set_error(UNO_ERR_UNSUPPORTED, "B * (k + 1) must be <= 2^32");
+  if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k + 1) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * (k + 1) must be <= 2^32");
   if (static_cast<int64_t>(B) * (2 * k + 1) > (1ll << 30))
     return set_error(UNO_ERR_UNSUPPORTED, "too many rows");
   if (!h_in || !q_prev || !d_prev || !q_next || !d_next || !accepted_len || !out_tokens ||
@@ -564,7 +572,7 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   va.temperature = temperature;
   va.seed = seed;
   va.step = step;
-  va.seq_offset = 0;
+  va.seq_offset = seq_offset;
   va.accepted_len = accepted_len;
   va.out_tokens = out_tokens;
   va.out_count = out_count;
@@ -580,7 +588,7 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   da.temperature = temperature;
   da.seed = seed;
   da.step = step;
-  da.seq_offset = 0;
+  da.seq_offset = seq_offset;
   da.draft = d_next;
   da.dev_status = dev_status;
   return draft_launch(da, st);

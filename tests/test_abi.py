@@ -119,9 +119,10 @@ def test_model_create_validates():
     assert L.uno_model_create(ctypes.byref(h), 1, 16, 16, 16, 16, 16, 8, 1.0, ptrs) == 0
     assert h.value
     assert L.uno_psi_step_workspace(h, 2, 4) > 0
-    st = L.uno_psi_step(h, 2, 4, None, None, None, 1.0, 0, 0, None, None, None, None, None, None,
-                        None, None, 0, None)
+    st = L.uno_psi_step(h, 2, 4, None, None, None, 1.0, 0, 0, 0, None, None, None, None, None,
+                        None, None, None, 0, None)
     assert st == 1
+    assert L.uno_psi_step_kernel_count(h) == 1 * (3 + 14) + 1 + 2 + 3
     L.uno_model_destroy(h)
 
 
