@@ -62,6 +62,25 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def csrc_hash():
+    import glob
+    import hashlib
+    srcs = sorted(glob.glob(os.path.join(ROOT, "sampling_gated_lora_b200", "csrc", "*")))
+    return hashlib.sha256(b"".join(open(f, "rb").read() for f in srcs)).hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
+    the kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    if d.get("kernel") != kernel or d.get("csrc_sha256_16") != csrc_hash():
+        return None
+    return d["traffic_bytes"]
+
+
 def workload_config(B, k, T):
     return {"workload": f"psi_step Qwen3-8B-shaped: 36 layers q/k/v/o 4096->4096/1024/1024/4096, "
                         f"gate/up 4096->12288, down 12288->4096, LM head 4096->151936, rank 128, "
@@ -397,7 +416,9 @@ def run_uno(args):
             ach = byts / us / 1e3
             roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": round(ach / pk["hbm_gbs"], 3), "traffic": None}
-        roof.update({"kernel": f"gated_lora_linear (LoRA down + fused GEMM) up 4096->12288, M={M}",
+        kname = f"gated_lora_linear up 4096->12288 M={M} (LoRA down + fused GEMM)"
+        roof["traffic"] = recorded_traffic(kname)
+        roof.update({"kernel": kname,
                      "us_per_launch": round(us, 2), "peak_source": pk_src + " burst",
                      "algorithmic_flops": flops, "algorithmic_bytes": byts})
         del x, y

@@ -1,7 +1,11 @@
 """One synthetic decode step (uno_psi_step) on a small model.
 
-Logits of every row are compared with the fp64 oracle stack (bf16 storage at
-the same points). The step's tokens are checked by composition: they must
+Logits of every row are compared with the fp64 oracle stack. The stack stores
+bf16 between operations, so its logits carry bf16 rounding noise whose size
+depends on where each side rounds; the bound is derived from the oracle itself:
+the GPU's logits must lie within twice the distance between the oracle with
+bf16 storage and the oracle in fp64 throughout (that distance, ~6e-3
+relative on the small model, is the noise floor of the storage format). The step's tokens are checked by composition: they must
 equal uno_psi_verify / uno_draft_sample run on the step's own logits (those
 two kernels have their own oracle parity tests)."""
 import numpy as np
@@ -10,7 +14,7 @@ import pytest
 import workloads as W
 from oracle import sampling as S
 from oracle import stack as O
-from gpu_util import check_close, dev_tensor, host_f64
+from gpu_util import dev_tensor, host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -57,9 +61,15 @@ def test_tiny_step(B, k, T):
     torch.cuda.synchronize()
     assert int(buf["status"].item()) == 0
     # logits of every row vs the oracle stack
-    ref = O.stack_logits(h, layers_np, head_np, O.step_gate(B, k), shape.scale)
+    gate = O.step_gate(B, k)
+    ref = O.stack_logits(h, layers_np, head_np, gate, shape.scale, store="bf16")
+    exact = O.stack_logits(h, layers_np, head_np, gate, shape.scale, store=None)
     got = np.concatenate([host_f64(buf["logits"]), host_f64(buf["q_next"]).reshape(B * k, V)])
-    check_close(got, ref, what="step logits")
+    rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)
+    floor = rel(ref, exact)
+    assert rel(got, exact) <= 2 * floor, (rel(got, exact), floor)
+    assert rel(got, ref) <= 2 * floor, (rel(got, ref), floor)
+    assert np.abs(got - exact).max() <= 2 * np.abs(ref - exact).max() + 2.0 ** -7 * np.abs(exact).max()
     # tokens: same as the verify / draft kernels on the step's own logits
     acc, tok, cnt = U.psi_verify(buf["logits"].reshape(B, k + 1, V), Q_prev, D_prev, T, 7, 5)
     np.testing.assert_array_equal(buf["acc"].cpu().numpy(), acc.cpu().numpy())
