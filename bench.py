@@ -62,6 +62,23 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def shard(B_per_rank, rank):
+    """Sequences of one rank under weak scaling: (count, global offset of its first sequence)."""
+    return B_per_rank, rank * B_per_rank
+
+
+def combine_over_ranks(ms, tokens, dist=None, device="cpu"):
+    """(max over ranks of the timed milliseconds, sum over ranks of the tokens)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms), int(tokens)
+    mx = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    sm = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+    return float(mx.item()), int(round(sm.item()))
+
+
 def csrc_hash():
     import glob
     import hashlib
@@ -311,7 +328,7 @@ def run_uno(args):
     cnt = torch.empty((n_total, B), **i32)
     status = torch.zeros(1, **i32)
     ws = torch.empty(model.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
-    seq_off = rank * B
+    B, seq_off = shard(B, rank)
 
     def step(t):
         model.step(B, k, h, qb[t % 2], db[t % 2], T, 2026, t, qb[(t + 1) % 2], db[(t + 1) % 2],
@@ -338,15 +355,7 @@ def run_uno(args):
     ms = e0.elapsed_time(e1)
     tokens = int(cnt[args.warmup:].sum())
     st = int(status.item())
-    stat = torch.tensor([ms, float(tokens), float(st)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        mx = stat.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = stat.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        ms_max, tokens_all = float(mx[0]), int(sm[1])
-    else:
-        ms_max, tokens_all = ms, tokens
+    ms_max, tokens_all = combine_over_ranks(ms, tokens, dist if world > 1 else None, "cuda")
     value = tokens_all / (ms_max / 1e3)
 
     # e2e: the public API with host buffers; H2D of the step's hidden states and
@@ -369,15 +378,8 @@ def run_uno(args):
     e3.synchronize()
     e2e_ms = e2.elapsed_time(e3)
     e2e_tokens = int(cnt_h.sum())
-    est = torch.tensor([e2e_ms, float(e2e_tokens)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        mx = est.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = est.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        e2e_ms_max, e2e_tok_all = float(mx[0]), int(sm[1])
-    else:
-        e2e_ms_max, e2e_tok_all = e2e_ms, e2e_tokens
+    e2e_ms_max, e2e_tok_all = combine_over_ranks(e2e_ms, e2e_tokens, dist if world > 1 else None,
+                                                  "cuda")
     e2e = {"value": round(e2e_tok_all / (e2e_ms_max / 1e3), 1), "unit": "tokens/s",
            "h2d_bytes_per_step": h_host.numel() * 2,
            "d2h_bytes_per_step": (acc_h[0].numel() + tok_h[0].numel() + cnt_h[0].numel()) * 4}

@@ -37,7 +37,11 @@ constexpr int kGemmThreads = 192;
 constexpr int kTileP = 128;         // MMA M
 constexpr int kRowBytes = 128;      // one K-block row of either operand (64 bf16 / 32 f32)
 constexpr int kMaxStages = 12;
-constexpr int kPartStride = 129;    // floats per column of a split-K partial tile (padded)
+// Split-K partial tiles in shared memory (fp32, padded rows):
+//   non-swapped: part[i][bn + 4]   (one row per accumulator lane = token)
+//   swapped:     part[j][128 + 4]  (one row per token column; lanes = features)
+// so the reduction reads 16-byte groups of 4 consecutive output features.
+constexpr int kPartPad = 4;
 
 struct GemmParams {
   int M, N;
@@ -80,6 +84,34 @@ __device__ __forceinline__ void epi_store1(const GemmParams& p, int p_row0, int 
   if (p.mode == kEpiRowScale) v *= p.scale * row_gate(p, m);
   if (p.mode == kEpiAdd) v += to_f32<T>(*dst);
   *dst = from_f32<T>(v);
+}
+
+// 4 consecutive features n..n+3 of token row m (n a multiple of 4, N % 4 == 0).
+template <typename T>
+__device__ __forceinline__ void epi_store4(const GemmParams& p, int m, int n, float4 a) {
+  T* base = static_cast<T*>(m < p.M0 ? p.y : p.y1);
+  const long long row = m < p.M0 ? m : m - p.M0;
+  T* dst = base + row * p.ldy + n;
+  if (p.mode == kEpiRowScale) {
+    const float rs = p.scale * row_gate(p, m);
+    a.x *= rs; a.y *= rs; a.z *= rs; a.w *= rs;
+  }
+  if constexpr (std::is_same<T, float>::value) {
+    float4* d = reinterpret_cast<float4*>(dst);
+    if (p.mode == kEpiAdd) {
+      const float4 o = *d;
+      a.x += o.x; a.y += o.y; a.z += o.z; a.w += o.w;
+    }
+    *d = a;
+  } else {
+    uint2* d = reinterpret_cast<uint2*>(dst);
+    if (p.mode == kEpiAdd) {
+      const uint2 o = *d;
+      a.x += bf16_lo(o.x); a.y += bf16_hi(o.x); a.z += bf16_lo(o.y); a.w += bf16_hi(o.y);
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+    *d = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+  }
 }
 
 // 16 consecutive features of one token row (non-swapped layout), vectorised.
@@ -279,42 +311,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-        float* part = reinterpret_cast<float*>(smem);   // [bn][kPartStride], stages are free now
+        float* part = reinterpret_cast<float*>(smem);   // the stage ring is free now
         for (int c = 0; c < bn; c += 16) {
           float v[16];
           tmem_ld16(trow + c, v);
+          if (kSwap) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) part[(c + j) * kPartStride + i] = v[j];
+            for (int j = 0; j < 16; ++j) part[(c + j) * (kTileP + kPartPad) + i] = v[j];
+          } else {
+            float4* row = reinterpret_cast<float4*>(part + i * (bn + kPartPad) + c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
         }
       }
     }
   }
 
   if (p.splits > 1) {
-    // Sum the cluster's partial tiles; CTA `rank` owns a contiguous slice of
-    // the tile's elements (ordered so that consecutive threads write
-    // consecutive output addresses).
+    // Sum the cluster's partial tiles. The tile is cut into groups of 4
+    // consecutive output features; CTA `rank` reduces a contiguous range of
+    // groups, reading the same group from every CTA of the cluster.
     cluster_sync();
     const uint32_t rank = cluster_ctarank();
     const int S = p.splits;
-    const int E = kTileP * bn;
-    const int chunk = (E + S - 1) / S;
-    const int e0 = static_cast<int>(rank) * chunk;
-    const int e1 = min(E, e0 + chunk);
+    const int groups = kTileP * bn / 4;
+    const int chunk = (groups + S - 1) / S;
+    const int g0 = static_cast<int>(rank) * chunk;
+    const int g1 = min(groups, g0 + chunk);
     const uint32_t part0 = smem_u32(smem);
-    for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += kGemmThreads) {
-      int i, j;
+    uint32_t peer[8];
+    for (int r = 0; r < S; ++r) peer[r] = map_shared_rank(part0, r);
+    for (int g = g0 + static_cast<int>(threadIdx.x); g < g1; g += kGemmThreads) {
+      int m, n;
+      uint32_t off;
       if (kSwap) {
-        i = e % kTileP;
-        j = e / kTileP;
+        const int j = g / (kTileP / 4), i4 = g % (kTileP / 4);
+        off = static_cast<uint32_t>((j * (kTileP + kPartPad) + 4 * i4) * 4);
+        m = q_row0 + j;
+        n = p_row0 + 4 * i4;
       } else {
-        i = e / bn;
-        j = e % bn;
+        const int i = g / (bn / 4), j4 = g % (bn / 4);
+        off = static_cast<uint32_t>((i * (bn + kPartPad) + 4 * j4) * 4);
+        m = p_row0 + i;
+        n = q_row0 + 4 * j4;
       }
-      const uint32_t off = static_cast<uint32_t>((j * kPartStride + i) * 4);
-      float acc = 0.f;
-      for (int r = 0; r < S; ++r) acc += ld_cluster_f32(map_shared_rank(part0 + off, r));
-      epi_store1<T, kSwap>(p, p_row0, q_row0, i, j, acc);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int r = 0; r < S; ++r) {
+        const float4 v = ld_cluster_f32x4(peer[r] + off);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      if (m < p.M && n < p.N) epi_store4<T>(p, m, n, acc);
     }
     cluster_sync();
   }
@@ -452,7 +500,9 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   int kb_per = (nkb + splits - 1) / splits;
   splits = (nkb + kb_per - 1) / kb_per;   // every split gets >= 1 K-block
   // the split-K partial tile must fit in the stage ring
-  if (splits > 1 && static_cast<uint32_t>(kPartStride * bn * 4) > stages * st) {
+  const uint32_t part_bytes = static_cast<uint32_t>(
+      (swap ? bn * (kTileP + kPartPad) : kTileP * (bn + kPartPad)) * 4);
+  if (splits > 1 && part_bytes > stages * st) {
     splits = 1;
     kb_per = nkb;
   }

@@ -171,18 +171,71 @@ __device__ __forceinline__ float2 row_stat(const float2* stats, int row, int chu
 
 // Shared state of one draw (per CTA).
 struct DrawSmem {
-  double segsum[kDrawThreads];
-  double seg_prefix[kDrawThreads + 1];
+  double prefix[kDrawThreads + 1];   // exclusive prefix of the per-thread segment sums
+  double warp_tot[kDrawThreads / 32];
   double chunk_total;
+  int owner[kDrawThreads / 32];
   int token;
 };
 
-// Inverse-CDF draw over the cluster: this CTA holds `len` weights w(i) of
-// vocab ids [lo, lo + len) (computed on demand by wfn, deterministic). Returns
-// in every CTA: the drawn vocab id if this CTA owns it, -1 otherwise; sets
-// *zero_total when the cluster-wide total is 0. All threads of all CTAs of the
-// cluster must call it (it contains cluster barriers). No CTA reads another
-// CTA's shared memory after the last barrier inside, so callers may exit.
+// Block-wide exclusive scan of one double per thread (kDrawThreads threads).
+// Writes sh.prefix[t] and sh.prefix[kDrawThreads] = sh.chunk_total = the total.
+__device__ __forceinline__ void block_scan(DrawSmem& sh, double v) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  double incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  if (lane == 31) sh.warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    double w = lane < kDrawThreads / 32 ? sh.warp_tot[lane] : 0.0;
+#pragma unroll
+    for (int o = 1; o < kDrawThreads / 32; o <<= 1) {
+      const double n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    if (lane < kDrawThreads / 32) sh.warp_tot[lane] = w;   // inclusive over warps
+  }
+  __syncthreads();
+  const double base = warp ? sh.warp_tot[warp - 1] : 0.0;
+  sh.prefix[t] = base + excl;
+  if (t == 0) {
+    sh.prefix[kDrawThreads] = sh.warp_tot[kDrawThreads / 32 - 1];
+    sh.chunk_total = sh.warp_tot[kDrawThreads / 32 - 1];
+  }
+  __syncthreads();
+}
+
+// Largest index t in [0, kDrawThreads) with `ok` true, over the block (-1 if none).
+__device__ __forceinline__ int block_max_index(DrawSmem& sh, bool ok) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int w = __reduce_max_sync(0xffffffffu, ok ? t : -1);
+  if (lane == 0) sh.owner[warp] = w;
+  __syncthreads();
+  int best = -1;
+#pragma unroll
+  for (int i = 0; i < kDrawThreads / 32; ++i) best = max(best, sh.owner[i]);
+  __syncthreads();
+  return best;
+}
+
+// Inverse-CDF draw over the cluster. This CTA holds `len` weights w(i) of
+// vocab ids [lo, lo + len), computed on demand by `wfn` (deterministic: the
+// same call returns the same bits). Thread t owns the contiguous segment
+// [t*seg, (t+1)*seg) of the chunk. The draw picks the smallest id whose
+// inclusive cumulative weight exceeds u * Z (Z = cluster total): the owning
+// CTA is the last one with prefix <= u*Z and positive mass, the owning
+// segment likewise, and the segment is scanned in ascending id. These rules
+// pick exactly one owner even when rounding makes prefixes of nested sums
+// disagree in the last bit. Returns the drawn id in the owning CTA, -1
+// elsewhere; *zero_total reports Z == 0. Every thread of every CTA of the
+// cluster must call it. No CTA reads another's shared memory after the last
+// cluster barrier inside, so callers may exit right after.
 template <typename WFn>
 __device__ int cluster_draw(DrawSmem& sh, const WFn& wfn, int lo, int len, double u,
                             bool* zero_total) {
@@ -191,31 +244,19 @@ __device__ int cluster_draw(DrawSmem& sh, const WFn& wfn, int lo, int len, doubl
   const int s0 = min(len, t * seg), s1 = min(len, s0 + seg);
   double my = 0.0;
   for (int i = s0; i < s1; ++i) my += static_cast<double>(wfn(i));
-  // exclusive prefix of the segment sums, sequential (one thread), so that the
-  // search below sees exactly the same partial sums
-  sh.segsum[t] = my;
-  __syncthreads();
-  if (t == 0) {
-    double run = 0.0;
-    for (int i = 0; i < kDrawThreads; ++i) {
-      sh.seg_prefix[i] = run;
-      run += sh.segsum[i];
-    }
-    sh.seg_prefix[kDrawThreads] = run;
-    sh.chunk_total = run;
-    sh.token = -1;
-  }
+  block_scan(sh, my);
+  if (t == 0) sh.token = -1;
   cluster_sync();
   // every CTA reads the chunk totals in rank order -> identical prefixes
   const uint32_t nrank = cluster_nctarank();
   const uint32_t myrank = cluster_ctarank();
   const uint32_t tot_addr = smem_u32(&sh.chunk_total);
-  double Z = 0.0, my_prefix = 0.0;
-  bool later_mass = false;
+  double Z = 0.0, thr_prefix[8];
+  double tots[8];
   for (uint32_t r = 0; r < nrank; ++r) {
     const double v = ld_cluster_f64(map_shared_rank(tot_addr, r));
-    if (r == myrank) my_prefix = Z;
-    if (r > myrank && v > 0.0) later_mass = true;
+    thr_prefix[r] = Z;
+    tots[r] = v;
     Z += v;
   }
   cluster_sync();   // totals read everywhere before anyone reuses the slot or exits
@@ -225,41 +266,29 @@ __device__ int cluster_draw(DrawSmem& sh, const WFn& wfn, int lo, int len, doubl
   }
   *zero_total = false;
   const double thr = u * Z;
-  const double mine = sh.chunk_total;
-  // owning CTA: my_prefix <= thr < my_prefix + mine (the last CTA with
-  // positive mass also owns thresholds that rounding pushed past the end)
-  bool own = (mine > 0.0) && (thr >= my_prefix) && (thr < my_prefix + mine);
-  if (!own && mine > 0.0 && thr >= my_prefix + mine && !later_mass) own = true;
-  if (own) {
-    const double tl = thr - my_prefix;
-    const double lo_s = sh.seg_prefix[t], hi_s = sh.seg_prefix[t + 1];
-    bool mine_seg = hi_s > lo_s && tl >= lo_s && tl < hi_s;
-    if (!mine_seg && hi_s > lo_s && tl >= hi_s) {
-      // rounding past the chunk total: the last segment with mass owns it
-      bool last = true;
-      for (int i = t + 1; i < kDrawThreads && last; ++i)
-        last = !(sh.seg_prefix[i + 1] > sh.seg_prefix[i]);
-      mine_seg = last;
-    }
-    if (mine_seg) {
-      const double tt = tl - lo_s;
-      double run = 0.0;
-      int pick = -1, last_nz = -1;
-      for (int i = s0; i < s1; ++i) {
-        const float w = wfn(i);
-        if (w > 0.f) last_nz = i;
-        run += static_cast<double>(w);
-        if (run > tt) {
-          pick = i;
-          break;
-        }
+  int owner_rank = -1;
+  for (uint32_t r = 0; r < nrank; ++r)
+    if (tots[r] > 0.0 && thr_prefix[r] <= thr) owner_rank = static_cast<int>(r);
+  if (owner_rank != static_cast<int>(myrank)) return -1;   // uniform over this CTA
+  const double tl = thr - thr_prefix[myrank];
+  const int own = block_max_index(sh, my > 0.0 && sh.prefix[t] <= tl);
+  if (t == own) {
+    const double tt = tl - sh.prefix[t];
+    double run = 0.0;
+    int pick = -1, last_nz = -1;
+    for (int i = s0; i < s1; ++i) {
+      const float w = wfn(i);
+      if (w > 0.f) last_nz = i;
+      run += static_cast<double>(w);
+      if (run > tt) {
+        pick = i;
+        break;
       }
-      if (pick < 0) pick = last_nz;
-      sh.token = lo + pick;
     }
+    sh.token = lo + (pick >= 0 ? pick : last_nz);
   }
   __syncthreads();
-  return own ? sh.token : -1;
+  return sh.token;
 }
 
 // Vocab range of CTA `rank` among `n`: chunks are multiples of 8 ids.
@@ -271,9 +300,30 @@ __device__ __forceinline__ void chunk_range(int V, int n, int rank, int* lo, int
   *len = min(V, a + per) - a;
 }
 
+// Stage `len` logits into shared memory: 16-byte streaming loads, four in
+// flight per thread, when the source is 16-byte aligned; scalar otherwise.
 template <typename T>
 __device__ __forceinline__ void load_chunk(T* dst, const T* src, int len) {
-  for (int i = threadIdx.x; i < len; i += blockDim.x) dst[i] = src[i];
+  constexpr int kN = 16 / static_cast<int>(sizeof(T));
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+    const int nv = len / kN;
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    int i = threadIdx.x;
+    const int step = blockDim.x;
+    for (; i + 3 * step < nv; i += 4 * step) {
+      const uint4 a = __ldcs(s4 + i), b = __ldcs(s4 + i + step);
+      const uint4 c = __ldcs(s4 + i + 2 * step), d = __ldcs(s4 + i + 3 * step);
+      d4[i] = a;
+      d4[i + step] = b;
+      d4[i + 2 * step] = c;
+      d4[i + 3 * step] = d;
+    }
+    for (; i < nv; i += step) d4[i] = __ldcs(s4 + i);
+    for (int j = nv * kN + threadIdx.x; j < len; j += step) dst[j] = src[j];
+  } else {
+    for (int j = threadIdx.x; j < len; j += blockDim.x) dst[j] = src[j];
+  }
 }
 
 struct FinalizeParams {
@@ -435,13 +485,12 @@ __global__ void __launch_bounds__(kDrawThreads)
   int lo, len;
   chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
   T* z = reinterpret_cast<T*>(dyn);
-  const T* src = q_logits + static_cast<size_t>(row) * V + lo;
+  load_chunk(z, q_logits + static_cast<size_t>(row) * V + lo, len);
+  __syncthreads();
   float mx = -INFINITY;
   bool nan = false;
   for (int i = threadIdx.x; i < len; i += blockDim.x) {
-    const T v = src[i];
-    z[i] = v;
-    const float f = to_f32<T>(v);
+    const float f = to_f32<T>(z[i]);
     nan |= isnan(f);
     mx = fmaxf(mx, f);
   }
