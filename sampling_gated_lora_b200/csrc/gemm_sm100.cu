@@ -27,6 +27,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "internal.h"
 
 namespace uno {
@@ -44,123 +45,17 @@ constexpr int kMaxStages = 12;
 constexpr int kPartPad = 4;
 
 struct GemmParams {
-  int M, N;
+  EpiArgs e;
   int bn;                 // Q rows per tile (multiple of 16, <= 256)
   int stages;
   int tmem_cols;
   int nkb_main, nkb_lora, kb_per_split, splits;
-  int mode;
-  int M0;
-  long long ldy;
-  void* y;
-  void* y1;
-  const uint8_t* gate;
-  int gate_row0;
-  float scale;
   int32_t* status;
 };
 static_assert(sizeof(GemmParams) <= 128, "GemmParams must fit GemmLaunch::params");
 
 __host__ __device__ constexpr uint32_t stage_bytes_for(int bn) {
   return ((kTileP + bn) * kRowBytes + 1023u) & ~1023u;
-}
-
-// Adapter gate of token row m: the gate vector, or (m >= gate_row0) without one.
-__device__ __forceinline__ float row_gate(const GemmParams& p, int m) {
-  return p.gate ? static_cast<float>(p.gate[m]) : (m >= p.gate_row0 ? 1.0f : 0.0f);
-}
-
-// Store one output element (accumulator row i, column j of this tile).
-template <typename T, bool kSwap>
-__device__ __forceinline__ void epi_store1(const GemmParams& p, int p_row0, int q_row0, int i,
-                                           int j, float acc) {
-  const int m = kSwap ? q_row0 + j : p_row0 + i;
-  const int n = kSwap ? p_row0 + i : q_row0 + j;
-  if (m >= p.M || n >= p.N) return;
-  T* base = static_cast<T*>(m < p.M0 ? p.y : p.y1);
-  const long long row = m < p.M0 ? m : m - p.M0;
-  T* dst = base + row * p.ldy + n;
-  float v = acc;
-  if (p.mode == kEpiRowScale) v *= p.scale * row_gate(p, m);
-  if (p.mode == kEpiAdd) v += to_f32<T>(*dst);
-  *dst = from_f32<T>(v);
-}
-
-// 4 consecutive features n..n+3 of token row m (n a multiple of 4, N % 4 == 0).
-template <typename T>
-__device__ __forceinline__ void epi_store4(const GemmParams& p, int m, int n, float4 a) {
-  T* base = static_cast<T*>(m < p.M0 ? p.y : p.y1);
-  const long long row = m < p.M0 ? m : m - p.M0;
-  T* dst = base + row * p.ldy + n;
-  if (p.mode == kEpiRowScale) {
-    const float rs = p.scale * row_gate(p, m);
-    a.x *= rs; a.y *= rs; a.z *= rs; a.w *= rs;
-  }
-  if constexpr (std::is_same<T, float>::value) {
-    float4* d = reinterpret_cast<float4*>(dst);
-    if (p.mode == kEpiAdd) {
-      const float4 o = *d;
-      a.x += o.x; a.y += o.y; a.z += o.z; a.w += o.w;
-    }
-    *d = a;
-  } else {
-    uint2* d = reinterpret_cast<uint2*>(dst);
-    if (p.mode == kEpiAdd) {
-      const uint2 o = *d;
-      a.x += bf16_lo(o.x); a.y += bf16_hi(o.x); a.z += bf16_lo(o.y); a.w += bf16_hi(o.y);
-    }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
-    *d = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-  }
-}
-
-// 16 consecutive features of one token row (non-swapped layout), vectorised.
-template <typename T>
-__device__ __forceinline__ void epi_store16_row(const GemmParams& p, int m, int n0,
-                                                const float (&v)[16]) {
-  T* base = static_cast<T*>(m < p.M0 ? p.y : p.y1);
-  const long long row = m < p.M0 ? m : m - p.M0;
-  T* dst = base + row * p.ldy + n0;
-  float w[16];
-  const float rs = (p.mode == kEpiRowScale) ? p.scale * row_gate(p, m) : 1.0f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) w[j] = v[j] * rs;
-  if constexpr (std::is_same<T, float>::value) {
-    float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float4 o = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-      if (p.mode == kEpiAdd) {
-        const float4 old = d4[q];
-        o.x += old.x; o.y += old.y; o.z += old.z; o.w += old.w;
-      }
-      d4[q] = o;
-    }
-  } else {
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      float a[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) a[e] = w[8 * q + e];
-      if (p.mode == kEpiAdd) {
-        const uint4 old = d4[q];
-        const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          a[2 * e] += bf16_lo(ow[e]);
-          a[2 * e + 1] += bf16_hi(ow[e]);
-        }
-      }
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * e], a[2 * e + 1]);
-        pk[e] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      d4[q] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-  }
 }
 
 template <typename T, bool kSwap>
@@ -297,17 +192,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld16(trow + c, v);
           if (!kSwap) {
             const int m = p_row0 + i, n0 = q_row0 + c;
-            if (m < p.M) {
-              if (n0 + 16 <= p.N) {
-                epi_store16_row<T>(p, m, n0, v);
+            if (m < p.e.M) {
+              if (n0 + 16 <= p.e.N) {
+                epi_store16_row<T>(p.e, m, n0, v);
               } else {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) epi_store1<T, kSwap>(p, p_row0, q_row0, i, c + j, v[j]);
+                for (int j = 0; j < 16; ++j) epi_store1<T, kSwap>(p.e, p_row0, q_row0, i, c + j, v[j]);
               }
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) epi_store1<T, kSwap>(p, p_row0, q_row0, i, c + j, v[j]);
+            for (int j = 0; j < 16; ++j) epi_store1<T, kSwap>(p.e, p_row0, q_row0, i, c + j, v[j]);
           }
         }
       } else {
@@ -362,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const float4 v = ld_cluster_f32x4(peer[r] + off);
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      if (m < p.M && n < p.N) epi_store4<T>(p, m, n, acc);
+      if (m < p.e.M && n < p.e.N) epi_store4<T>(p.e, m, n, acc);
     }
     cluster_sync();
   }
@@ -382,6 +277,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
+
+template <typename T, bool kSwap>
+void* kernel_ptr() {
+  return reinterpret_cast<void*>(&gated_gemm_kernel<T, kSwap>);
+}
+
+void* pick_kernel(uno_dtype dt, bool swap) {
+  if (dt == UNO_F32) return swap ? kernel_ptr<float, true>() : kernel_ptr<float, false>();
+  return swap ? kernel_ptr<__nv_bfloat16, true>() : kernel_ptr<__nv_bfloat16, false>();
+}
+
+int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+int pow2_at_least(int v) {
+  int c = 32;
+  while (c < v) c <<= 1;
+  return c;
+}
+
+}  // namespace
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -423,26 +338,6 @@ uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t in
   return UNO_OK;
 }
 
-template <typename T, bool kSwap>
-void* kernel_ptr() {
-  return reinterpret_cast<void*>(&gated_gemm_kernel<T, kSwap>);
-}
-
-void* pick_kernel(uno_dtype dt, bool swap) {
-  if (dt == UNO_F32) return swap ? kernel_ptr<float, true>() : kernel_ptr<float, false>();
-  return swap ? kernel_ptr<__nv_bfloat16, true>() : kernel_ptr<__nv_bfloat16, false>();
-}
-
-int round_up(int v, int m) { return (v + m - 1) / m * m; }
-
-int pow2_at_least(int v) {
-  int c = 32;
-  while (c < v) c <<= 1;
-  return c;
-}
-
-}  // namespace
-
 int device_sm_count() {
   static int n = [] {
     int dev = 0, v = 148;
@@ -454,6 +349,7 @@ int device_sm_count() {
 }
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
+  if (gemm_pair_suits(pb)) return gemm_pair_prepare(pb, out);
   const int esz = pb.dt == UNO_F32 ? 4 : 2;
   const int bke = kRowBytes / esz;
   const int sms = device_sm_count();
@@ -508,8 +404,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   }
 
   GemmParams gp{};
-  gp.M = static_cast<int>(M);
-  gp.N = static_cast<int>(N);
+  gp.e = epi_args(pb);
   gp.bn = bn;
   gp.stages = stages;
   gp.tmem_cols = pow2_at_least(bn);
@@ -517,14 +412,6 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   gp.nkb_lora = nkb_lora;
   gp.kb_per_split = kb_per;
   gp.splits = splits;
-  gp.mode = pb.mode;
-  gp.M0 = static_cast<int>(std::min<int64_t>(pb.M0, M));
-  gp.ldy = pb.ldy;
-  gp.y = pb.y;
-  gp.y1 = pb.y1;
-  gp.gate = pb.gate;
-  gp.gate_row0 = static_cast<int>(std::min<int64_t>(pb.gate_row0, M));
-  gp.scale = pb.scale;
   gp.status = nullptr;
 
   const uint32_t tok_box = swap ? static_cast<uint32_t>(bn) : kTileP;
@@ -540,6 +427,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
     out->tm[3] = out->tm[1];
   }
   std::memcpy(out->params, &gp, sizeof(gp));
+  out->kind = 0;
   out->swap = swap;
   out->grid_x = grid_x;
   out->grid_y = grid_y;
@@ -550,6 +438,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
 }
 
 uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream) {
+  if (l.kind == 1) return gemm_pair_run(l, stream);
   void* fn = pick_kernel(static_cast<uno_dtype>(l.dtype), l.swap != 0);
   cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, l.smem_bytes);

@@ -48,6 +48,7 @@ struct GemmProblem {
 struct GemmLaunch {
   CUtensorMap tm[4];
   alignas(8) unsigned char params[128];
+  int kind;               // 0: one-CTA kernel, 1: persistent CTA-pair kernel
   int swap;
   int grid_x, grid_y, splits;
   int smem_bytes;
@@ -55,6 +56,14 @@ struct GemmLaunch {
 };
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out);
+// Row-major [rows, inner] tensor map: box = 128 bytes of K x box_rows rows, 128-byte swizzle.
+uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t inner, uint64_t rows,
+                    uint32_t box_rows);
+// The persistent CTA-pair kernel (bf16, 256x256 tiles): whether it takes the
+// problem, its preparation and its launch.
+bool gemm_pair_suits(const GemmProblem& pb);
+uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out);
+uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
 uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sampler

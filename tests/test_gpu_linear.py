@@ -53,6 +53,8 @@ def test_mlp_concatenated_batch(which):
     (257, 256, 384, 0, "bf16"),
     (300, 4096, 136, 256, "bf16"),
     (1000, 200, 520, 32, "bf16"),
+    (1024, 264, 520, 24, "bf16"),      # CTA-pair kernel: ragged N, K
+    (1500, 1024, 1000, 128, "bf16"),   # CTA-pair kernel: ragged M and N
     (5, 36, 100, 4, "f32"),
     (300, 260, 132, 8, "f32"),
 ])
@@ -61,6 +63,17 @@ def test_ragged_shapes(M, K, N, r, dt):
     gate = (rng.random(M) < 0.5).astype(np.uint8)
     case = W.gated_linear_case(M, K, N, r, gate, dtype=dt, b_std=0.05, scale=0.75, seed=3)
     check_close(_run(case), _oracle(case), what=f"{M}x{K}x{N} r={r} {dt}")
+
+
+def test_pair_kernel_step_shapes():
+    """Large-M shapes of the decode step at B=256 (M=4352) on the CTA-pair kernel, sampled rows."""
+    for K, N in ((4096, 1024), (12288, 4096)):
+        rng = np.random.default_rng(N)
+        gate = W.step_gate(256, 8)
+        case = W.gated_linear_case(4352, K, N, 128, gate, seed=9)
+        y = _run(case)
+        rows = np.concatenate([np.arange(0, 4352, 97), [2303, 2304, 4351]])
+        check_close(y[rows], _oracle(case, rows), what=f"M=4352 {K}->{N} sampled rows")
 
 
 def test_gate_zero_matches_base_product_and_scale_zero():

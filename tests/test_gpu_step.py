@@ -40,7 +40,7 @@ def _buffers(B, k, V, dev="cuda"):
                 status=torch.zeros(1, **i32))
 
 
-@pytest.mark.parametrize("B,k,T", [(2, 4, 1.0), (3, 8, 0.7), (1, 1, 1.0)])
+@pytest.mark.parametrize("B,k,T", [(2, 4, 1.0), (3, 8, 0.7), (1, 1, 1.0), (64, 8, 1.0)])
 def test_tiny_step(B, k, T):
     import torch
     import sampling_gated_lora_b200 as U
