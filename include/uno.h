@@ -92,6 +92,28 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
                                  size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Grouped gated-LoRA linears sharing one input x [M,K] (one launch for the
+ * down-projections, one for the products; hyper.ai page, section "方法": the
+ * adapter is attached to every AR matrix, so the q, k, v projections of a
+ * layer, or its gate and up projections, read the same gated input):
+ *
+ *   mode 0:  y[i] = x W[i]^T + scale * g (.) ((x A[i]^T) Bl[i]^T),  i < G
+ *   mode 1:  G = 2, N[0] = N[1]:  y[0] = silu(lin_0(x)) * lin_1(x)   (silu(a) = a/(1+e^-a))
+ *
+ *   W[i] [N[i],K], A[i] [r,K], Bl[i] [N[i],r], y[i] [M,N[i]], all `dt`
+ *   (mode 1: bf16 only); gate [M] uint8; 1 <= G <= 3. Sizes as for
+ *   uno_gated_lora_linear. workspace: >= uno_gated_lora_linear_group_workspace.
+ * ------------------------------------------------------------------------- */
+size_t uno_gated_lora_linear_group_workspace(uno_dtype dt, int64_t M, int32_t r, int32_t G);
+
+uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32_t r, int32_t G,
+                                       const int64_t* N, const void* x, const void* const* W,
+                                       const void* const* A, const void* const* Bl,
+                                       const uint8_t* gate, float scale, int32_t mode,
+                                       void* const* y, void* workspace, size_t ws_bytes,
+                                       void* stream);
+
+/* ---------------------------------------------------------------------------
  * Psi-Spec verification of one drafted block per sequence (hyper.ai page,
  * section "方法", the Psi-Spec paragraph: rejection sampling against the base
  * AR distribution, longest valid prefix; ainews page: lossless).

@@ -28,6 +28,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIME
 EXPORTS = [
     "uno_last_error", "uno_version", "uno_device_status",
     "uno_gated_lora_linear_workspace", "uno_gated_lora_linear",
+    "uno_gated_lora_linear_group_workspace", "uno_gated_lora_linear_group",
     "uno_psi_verify_workspace", "uno_psi_verify",
     "uno_draft_sample_workspace", "uno_draft_sample",
     "uno_philox_uniforms",
@@ -65,6 +66,9 @@ def load():
         "uno_gated_lora_linear_workspace": (sz, [i32, i64, i64, i64, i32]),
         "uno_gated_lora_linear": (i32, [i32, i64, i64, i64, i32, vp, vp, vp, vp, vp, f32, vp, vp,
                                         sz, vp]),
+        "uno_gated_lora_linear_group_workspace": (sz, [i32, i64, i32, i32]),
+        "uno_gated_lora_linear_group": (i32, [i32, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, f32,
+                                              i32, vp, vp, sz, vp]),
         "uno_psi_verify_workspace": (sz, [i32, i32, i32, i32]),
         "uno_psi_verify": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, f32, u64, u64, u64, vp, vp,
                                  vp, vp, vp, sz, vp]),
@@ -161,6 +165,33 @@ def gated_lora_linear(x, W, A, Bl, gate, scale=1.0, y=None, workspace=None, stre
                                    _ptr(gate), float(scale), _ptr(y), _ptr(ws), wsb,
                                    _stream(stream)))
     return y
+
+
+def gated_lora_linear_group(x, Ws, As, Bls, gate, scale=1.0, silu_pair=False, ys=None,
+                            workspace=None, stream=None):
+    """Up to three gated linears on one input x; silu_pair: y = silu(lin_0(x)) * lin_1(x).
+
+    Returns the list of outputs ([y] in silu-pair mode).
+    """
+    torch = _torch()
+    L = load()
+    M, K = x.shape
+    G = len(Ws)
+    r = As[0].shape[0] if As else 0
+    Ns = [w.shape[0] for w in Ws]
+    if ys is None:
+        ys = [torch.empty((M, n), dtype=x.dtype, device=x.device) for n in (Ns[:1] if silu_pair else Ns)]
+    _dev(x, gate, *Ws, *As, *Bls, *ys)
+    dt = _dtype(x)
+    need = L.uno_gated_lora_linear_group_workspace(dt, M, r, G)
+    ws, wsb = _workspace(need, x.device, workspace)
+    arr = lambda ts: (ctypes.c_void_p * G)(*[t.data_ptr() for t in ts])
+    yarr = (ctypes.c_void_p * G)(*[ys[min(i, len(ys) - 1)].data_ptr() for i in range(G)])
+    Narr = (ctypes.c_int64 * G)(*Ns)
+    _check(L.uno_gated_lora_linear_group(dt, M, K, r, G, Narr, _ptr(x), arr(Ws), arr(As), arr(Bls),
+                                         _ptr(gate), float(scale), 1 if silu_pair else 0, yarr,
+                                         _ptr(ws), wsb, _stream(stream)))
+    return ys
 
 
 def psi_verify(p_logits, q_logits, draft, temperature, seed, step, seq_offset=0,

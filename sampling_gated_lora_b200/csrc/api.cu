@@ -72,50 +72,28 @@ uno_status check_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r
   return UNO_OK;
 }
 
-// Two launches: the gated down-projection t = scale * g * (x A^T), then the
-// base product with t folded in as extra K-blocks.
-uno_status linear_prepare(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r,
-                          const void* x, const void* W, const void* A, const void* Bl,
-                          const uint8_t* gate, int64_t gate_row0, float scale, void* t_buf,
-                          int mode, void* y, void* y1, int64_t M0, GemmLaunch* down,
-                          GemmLaunch* main, bool* has_down) {
-  *has_down = r > 0;
-  if (r > 0) {
-    GemmProblem d{};
-    d.dt = dt;
-    d.M = M;
-    d.N = r;
-    d.K = K;
-    d.r = 0;
-    d.x = x;
-    d.W = A;
-    d.mode = kEpiRowScale;
-    d.y = t_buf;
-    d.y1 = t_buf;
-    d.M0 = M;
-    d.ldy = r;
-    d.gate = gate;
-    d.gate_row0 = gate_row0;
-    d.scale = scale;
-    uno_status s = gemm_prepare(d, down);
-    if (s != UNO_OK) return s;
-  }
-  GemmProblem p{};
-  p.dt = dt;
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.r = r;
-  p.x = x;
-  p.W = W;
-  p.t = t_buf;
-  p.Bl = Bl;
-  p.mode = mode;
-  p.y = y;
-  p.y1 = y1 ? y1 : y;
-  p.M0 = y1 ? M0 : M;
-  p.ldy = N;
-  return gemm_prepare(p, main);
+// The rank-r down-projections t_g = scale * gate * (x A_g^T) of up to three
+// linears that share x, written side by side into t [M, G r].
+GemmProblem down_problem(uno_dtype dt, int64_t M, int64_t K, int32_t r, const void* x,
+                         const void* const* A, int G, const uint8_t* gate, int64_t gate_row0,
+                         float scale, void* t) {
+  GemmProblem d{};
+  d.dt = dt;
+  d.M = M;
+  d.K = K;
+  d.r = 0;
+  d.x = x;
+  d.ngroups = G;
+  const size_t esz = dt_size(dt);
+  for (int i = 0; i < G; ++i)
+    d.g[i] = GemmGroup{A[i], nullptr, r, static_cast<char*>(t) + i * r * esz,
+                       static_cast<int64_t>(G) * r, 0};
+  d.mode = kEpiRowScale;
+  d.M0 = M;
+  d.gate = gate;
+  d.gate_row0 = gate_row0;
+  d.scale = scale;
+  return d;
 }
 
 }  // namespace
@@ -173,11 +151,81 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
                      ws_bytes);
   void* t_buf = r > 0 ? static_cast<char*>(workspace) + L.t_off : nullptr;
   GemmLaunch down, main;
-  bool has_down = false;
-  s = linear_prepare(dt, M, K, N, r, x, W, A, Bl, gate, 0, scale, t_buf, kEpiStore, y, nullptr,
-                     M, &down, &main, &has_down);
-  if (s != UNO_OK) return s;
-  if (has_down && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
+  if (r > 0) {
+    const void* As[1] = {A};
+    if ((s = gemm_prepare(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), &down)) !=
+        UNO_OK)
+      return s;
+  }
+  GemmProblem pm{};
+  pm.dt = dt;
+  pm.M = M;
+  pm.K = K;
+  pm.r = r;
+  pm.x = x;
+  pm.t = t_buf;
+  pm.ldt = r;
+  pm.ngroups = 1;
+  pm.g[0] = GemmGroup{W, Bl, N, y, N, 0};
+  pm.mode = kEpiStore;
+  pm.M0 = M;
+  if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
+  if (r > 0 && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
+  return gemm_run(main, as_stream(stream));
+}
+
+size_t uno_gated_lora_linear_group_workspace(uno_dtype dt, int64_t M, int32_t r, int32_t G) {
+  if (M < 0 || r < 0 || G < 1 || G > kMaxGroups) return 0;
+  return align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * G * dt_size(dt));
+}
+
+uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32_t r, int32_t G,
+                                       const int64_t* N, const void* x, const void* const* W,
+                                       const void* const* A, const void* const* Bl,
+                                       const uint8_t* gate, float scale, int32_t mode,
+                                       void* const* y, void* workspace, size_t ws_bytes,
+                                       void* stream) {
+  if (G < 1 || G > kMaxGroups) return set_error(UNO_ERR_INVALID_ARG, "G=%d outside [1, 3]", G);
+  if (!N || !W || !y || (r > 0 && (!A || !Bl)))
+    return set_error(UNO_ERR_INVALID_ARG, "NULL array argument");
+  if (mode != 0 && mode != 1) return set_error(UNO_ERR_INVALID_ARG, "mode must be 0 or 1");
+  if (mode == 1 && (G != 2 || N[0] != N[1] || dt != UNO_BF16))
+    return set_error(UNO_ERR_INVALID_ARG, "mode 1 needs G = 2, N[0] = N[1] and bf16");
+  uno_status s;
+  for (int i = 0; i < G; ++i)
+    if ((s = check_linear(dt, M, K, N[i], r)) != UNO_OK) return s;
+  if (M == 0) return UNO_OK;
+  if (!x || !aligned16(x)) return set_error(UNO_ERR_INVALID_ARG, "x must be non-NULL and 16-byte aligned");
+  if (r > 0 && !gate) return set_error(UNO_ERR_INVALID_ARG, "gate must be non-NULL when r > 0");
+  for (int i = 0; i < G; ++i) {
+    if (!W[i] || !aligned16(W[i]) || (r > 0 && (!A[i] || !Bl[i] || !aligned16(A[i]) || !aligned16(Bl[i]))))
+      return set_error(UNO_ERR_INVALID_ARG, "group %d: NULL or unaligned weight", i);
+    if ((mode == 0 || i == 0) && (!y[i] || !aligned16(y[i])))
+      return set_error(UNO_ERR_INVALID_ARG, "group %d: NULL or unaligned output", i);
+  }
+  const size_t need = uno_gated_lora_linear_group_workspace(dt, M, r, G);
+  if (r > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
+  GemmLaunch down, main;
+  if (r > 0 && (s = gemm_prepare(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, workspace),
+                                 &down)) != UNO_OK)
+    return s;
+  GemmProblem pm{};
+  pm.dt = dt;
+  pm.M = M;
+  pm.K = K;
+  pm.r = r;
+  pm.x = x;
+  pm.t = workspace;
+  pm.ldt = static_cast<int64_t>(G) * r;
+  pm.ngroups = G;
+  for (int i = 0; i < G; ++i)
+    pm.g[i] = GemmGroup{W[i], r > 0 ? Bl[i] : nullptr, N[i], mode == 1 ? y[0] : y[i],
+                        mode == 1 ? N[0] : N[i], static_cast<int64_t>(i) * r};
+  pm.mode = mode == 1 ? kEpiSiluPair : kEpiStore;
+  pm.M0 = M;
+  if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
+  if (r > 0 && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
   return gemm_run(main, as_stream(stream));
 }
 
@@ -304,7 +352,15 @@ constexpr int kLinPerLayer = 7;   // q, k, v, o, gate, up, down
 enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
 
 struct StepLayout {
-  size_t h, n, q, kv, g, u, t, logits, vstat, total;
+  size_t h, n, q, k, v, act, t, logits, vstat, total;
+};
+
+// One operation of a step plan.
+struct StepOp {
+  int kind;            // 0 GEMM, 1 rmsnorm
+  GemmLaunch gemm;
+  const void* x;
+  void* y;
 };
 
 }  // namespace
@@ -315,29 +371,17 @@ struct uno_model {
   float scale;
   std::vector<const void*> w;   // 21 * n_layers + 3
 
-  // Launch descriptors of one (B, k, buffers) combination, in step order.
+  // The launches of one (B, k, buffers) combination, in step order.
   struct Plan {
     int32_t B, k;
     const void* ws;
     const void* q_next;
     const void* logits_out;
-    std::vector<GemmLaunch> down, main;
-    std::vector<char> has_down;
+    std::vector<uno::StepOp> ops;
   };
   std::mutex mu;
   std::vector<std::unique_ptr<Plan>> plans;   // most recently used last
 
-  int lin_in(int i) const { return i == uno::kO ? q_out : (i == uno::kDown ? inter : hidden); }
-  int lin_out(int i) const {
-    switch (i) {
-      case uno::kQ: return q_out;
-      case uno::kK:
-      case uno::kV: return kv_out;
-      case uno::kGate:
-      case uno::kUp: return inter;
-      default: return hidden;
-    }
-  }
   const void* wp(int layer, int i, int part) const {
     return w[static_cast<size_t>(layer * uno::kLinPerLayer + i) * 3 + part];
   }
@@ -362,74 +406,131 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
   L.h = take(M * m->hidden * 2);
   L.n = take(M * m->hidden * 2);
   L.q = take(M * m->q_out * 2);
-  L.kv = take(M * m->kv_out * 2);
-  L.g = take(M * m->inter * 2);
-  L.u = take(M * m->inter * 2);
-  L.t = take(M * m->r * 2);
+  L.k = take(M * m->kv_out * 2);
+  L.v = take(M * m->kv_out * 2);
+  L.act = take(M * m->inter * 2);
+  L.t = take(M * 3 * static_cast<size_t>(m->r) * 2);
   L.logits = take(Mv * static_cast<size_t>(m->vocab) * 2);
   L.vstat = take(verify_workspace(B, k, k + 1, m->vocab));
   L.total = off;
   return L;
 }
 
-// Input and output buffers of linear i of a layer, within the workspace.
-void lin_io(const uno_model* m, const StepLayout& L, char* base, int i, const void** x, void** y,
-            int* mode) {
-  *mode = kEpiStore;
-  switch (i) {
-    case kQ: *x = base + L.n; *y = base + L.q; break;
-    case kK:
-    case kV: *x = base + L.n; *y = base + L.kv; break;
-    case kO: *x = base + L.q; *y = base + L.h; *mode = kEpiAdd; break;
-    case kGate: *x = base + L.n; *y = base + L.g; break;
-    case kUp: *x = base + L.n; *y = base + L.u; break;
-    default: *x = base + L.g; *y = base + L.h; *mode = kEpiAdd; break;
-  }
-  (void)m;
-}
-
+// Plan of one step: per layer
+//   rmsnorm(h) -> n; down(n; A_q, A_k, A_v) -> t; gemm(n, t; q, k, v)
+//   down(q; A_o) -> t; gemm(q, t; o) += h
+//   rmsnorm(h) -> n; down(n; A_gate, A_up) -> t; gemm(n, t; silu(gate) * up) -> act
+//   down(act; A_down) -> t; gemm(act, t; down) += h
+// then rmsnorm(h) -> n, the LM head's down-projection and GEMM (AR rows ->
+// logits, mask rows -> q_next). Rows >= B(k+1) carry the adapter (gate 1).
 uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
                       void* logits_out, uno_model::Plan* P) {
   const StepLayout L = step_layout(m, B, k);
   char* base = static_cast<char*>(ws);
   const int64_t M = static_cast<int64_t>(B) * (2 * k + 1);
   const int64_t Mv = static_cast<int64_t>(B) * (k + 1);
-  const size_t n_lin = static_cast<size_t>(m->n_layers) * kLinPerLayer + 1;
+  const int32_t r = m->r;
   P->B = B;
   P->k = k;
   P->ws = ws;
   P->q_next = q_next;
   P->logits_out = logits_out;
-  P->down.assign(n_lin, GemmLaunch{});
-  P->main.assign(n_lin, GemmLaunch{});
-  P->has_down.assign(n_lin, 0);
-  void* t_buf = base + L.t;
+  P->ops.clear();
+  void* t = base + L.t;
+  auto norm = [&](const void* x, void* y) {
+    StepOp op{};
+    op.kind = 1;
+    op.x = x;
+    op.y = y;
+    P->ops.push_back(op);
+  };
+  auto gemm = [&](const GemmProblem& pb) -> uno_status {
+    StepOp op{};
+    op.kind = 0;
+    const uno_status s = gemm_prepare(pb, &op.gemm);
+    if (s == UNO_OK) P->ops.push_back(op);
+    return s;
+  };
+  // gated linear(s) on input x (width K): down-projections then the main GEMM
+  auto linear = [&](const void* x, int64_t K, int G, const int* which, int layer, void* const* y,
+                    const int64_t* ldy, int mode, void* y1, int64_t M0) -> uno_status {
+    uno_status s;
+    const void* As[kMaxGroups];
+    for (int i = 0; i < G; ++i)
+      As[i] = layer >= 0 ? m->wp(layer, which[i], 1) : m->head(1);
+    if (r > 0 && (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) !=
+                     UNO_OK)
+      return s;
+    GemmProblem pm{};
+    pm.dt = UNO_BF16;
+    pm.M = M;
+    pm.K = K;
+    pm.r = r;
+    pm.x = x;
+    pm.t = t;
+    pm.ldt = static_cast<int64_t>(G) * r;
+    pm.ngroups = G;
+    for (int i = 0; i < G; ++i) {
+      const void* W = layer >= 0 ? m->wp(layer, which[i], 0) : m->head(0);
+      const void* Bl = layer >= 0 ? m->wp(layer, which[i], 2) : m->head(2);
+      const int64_t N = layer >= 0 ? 0 : m->vocab;
+      pm.g[i] = GemmGroup{W, Bl, N, y[i], ldy[i], static_cast<int64_t>(i) * r};
+    }
+    for (int i = 0; i < G && layer >= 0; ++i) {
+      switch (which[i]) {
+        case kQ: pm.g[i].N = m->q_out; break;
+        case kK:
+        case kV: pm.g[i].N = m->kv_out; break;
+        case kGate:
+        case kUp: pm.g[i].N = m->inter; break;
+        default: pm.g[i].N = m->hidden; break;
+      }
+    }
+    pm.mode = mode;
+    pm.y1 = y1;
+    pm.M0 = M0;
+    return gemm(pm);
+  };
+  uno_status s;
   for (int l = 0; l < m->n_layers; ++l) {
-    for (int i = 0; i < kLinPerLayer; ++i) {
-      const void* x;
-      void* y;
-      int mode;
-      lin_io(m, L, base, i, &x, &y, &mode);
-      const size_t idx = static_cast<size_t>(l) * kLinPerLayer + i;
-      bool hd = false;
-      const uno_status s = linear_prepare(
-          UNO_BF16, M, m->lin_in(i), m->lin_out(i), m->r, x, m->wp(l, i, 0), m->wp(l, i, 1),
-          m->wp(l, i, 2), nullptr, Mv, m->scale, t_buf, mode, y, nullptr, M, &P->down[idx],
-          &P->main[idx], &hd);
-      if (s != UNO_OK) return s;
-      P->has_down[idx] = hd;
+    norm(base + L.h, base + L.n);
+    {
+      const int which[3] = {kQ, kK, kV};
+      void* y[3] = {base + L.q, base + L.k, base + L.v};
+      const int64_t ld[3] = {m->q_out, m->kv_out, m->kv_out};
+      if ((s = linear(base + L.n, m->hidden, 3, which, l, y, ld, kEpiStore, nullptr, M)) != UNO_OK)
+        return s;
+    }
+    {
+      const int which[1] = {kO};
+      void* y[1] = {base + L.h};
+      const int64_t ld[1] = {m->hidden};
+      if ((s = linear(base + L.q, m->q_out, 1, which, l, y, ld, kEpiAdd, nullptr, M)) != UNO_OK)
+        return s;
+    }
+    norm(base + L.h, base + L.n);
+    {
+      const int which[2] = {kGate, kUp};
+      void* y[2] = {base + L.act, base + L.act};
+      const int64_t ld[2] = {m->inter, m->inter};
+      if ((s = linear(base + L.n, m->hidden, 2, which, l, y, ld, kEpiSiluPair, nullptr, M)) !=
+          UNO_OK)
+        return s;
+    }
+    {
+      const int which[1] = {kDown};
+      void* y[1] = {base + L.h};
+      const int64_t ld[1] = {m->hidden};
+      if ((s = linear(base + L.act, m->inter, 1, which, l, y, ld, kEpiAdd, nullptr, M)) != UNO_OK)
+        return s;
     }
   }
-  // LM head: AR rows -> logits (caller's buffer or the workspace), mask rows -> q_next
+  norm(base + L.h, base + L.n);
   void* p_dst = logits_out ? logits_out : base + L.logits;
-  bool hd = false;
-  const uno_status s = linear_prepare(UNO_BF16, M, m->hidden, m->vocab, m->r, base + L.n,
-                                      m->head(0), m->head(1), m->head(2), nullptr, Mv, m->scale,
-                                      t_buf, kEpiStore, p_dst, q_next, Mv, &P->down[n_lin - 1],
-                                      &P->main[n_lin - 1], &hd);
-  if (s != UNO_OK) return s;
-  P->has_down[n_lin - 1] = hd;
-  return UNO_OK;
+  const int which[1] = {0};
+  void* y[1] = {p_dst};
+  const int64_t ld[1] = {m->vocab};
+  return linear(base + L.n, m->hidden, 1, which, -1, y, ld, kEpiStore, q_next, Mv);
 }
 
 uno_model::Plan* find_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
@@ -501,10 +602,10 @@ size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k) {
 
 int32_t uno_psi_step_kernel_count(const uno_model* m) {
   if (!m) return 0;
-  // per layer: 2 rmsnorm + 7 linears (down-projection + main GEMM each when
-  // r > 0) + silu*up; then rmsnorm + LM head; verify (2 kernels) + draft (1)
-  const int per_lin = m->r > 0 ? 2 : 1;
-  return m->n_layers * (3 + kLinPerLayer * per_lin) + 1 + per_lin + 3;
+  // per layer: 2 rmsnorm + 4 GEMM launches (+ 4 down-projections when r > 0);
+  // then rmsnorm + LM head (+ its down-projection); verify (2 kernels) + draft (1)
+  const int per_gemm = m->r > 0 ? 2 : 1;
+  return m->n_layers * (2 + 4 * per_gemm) + 1 + per_gemm + 3;
 }
 
 uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, const void* q_prev,
@@ -540,25 +641,10 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   cudaError_t e = cudaMemcpyAsync(base + L.h, h_in, static_cast<size_t>(M) * m->hidden * 2,
                                   cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_error(e, "copying h_in");
-  auto lin = [&](size_t idx) -> uno_status {
-    uno_status r2;
-    if (P->has_down[idx] && (r2 = gemm_run(P->down[idx], st)) != UNO_OK) return r2;
-    return gemm_run(P->main[idx], st);
-  };
-  for (int l = 0; l < m->n_layers; ++l) {
-    const size_t b0 = static_cast<size_t>(l) * kLinPerLayer;
-    if ((s = rmsnorm_launch(M, m->hidden, base + L.h, base + L.n, 1e-6f, st)) != UNO_OK) return s;
-    for (int i = kQ; i <= kO; ++i)
-      if ((s = lin(b0 + i)) != UNO_OK) return s;
-    if ((s = rmsnorm_launch(M, m->hidden, base + L.h, base + L.n, 1e-6f, st)) != UNO_OK) return s;
-    if ((s = lin(b0 + kGate)) != UNO_OK) return s;
-    if ((s = lin(b0 + kUp)) != UNO_OK) return s;
-    if ((s = silu_mul_launch(M * m->inter, base + L.g, base + L.u, base + L.g, st)) != UNO_OK)
-      return s;
-    if ((s = lin(b0 + kDown)) != UNO_OK) return s;
+  for (const StepOp& op : P->ops) {
+    s = op.kind == 0 ? gemm_run(op.gemm, st) : rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st);
+    if (s != UNO_OK) return s;
   }
-  if ((s = rmsnorm_launch(M, m->hidden, base + L.h, base + L.n, 1e-6f, st)) != UNO_OK) return s;
-  if ((s = lin(static_cast<size_t>(m->n_layers) * kLinPerLayer)) != UNO_OK) return s;
 
   VerifyArgs va{};
   va.dt = UNO_BF16;

@@ -1,8 +1,11 @@
 // Persistent CTA-pair gated GEMM for large M (bf16, sm_100a).
 //
-//   y = x W^T + t Bl^T   (t = the gated LoRA down-projection, folded in as
-//   extra K-blocks, so W streams once — the gated adapter of hyper.ai,
-//   section "方法")
+//   y_g = x W_g^T + t_g Bl_g^T   (t_g = the gated LoRA down-projection, folded
+//   in as extra K-blocks, so W streams once — the gated adapter of hyper.ai,
+//   section "方法"); up to three groups share x. In silu-pair tiles the 256
+//   B rows are 128 gate rows (CTA 0's half) and the same 128 up rows (CTA 1's
+//   half), so every CTA's accumulator holds gate and up side by side and the
+//   epilogue writes silu(gate) * up.
 //
 // One cluster of two CTAs on one TPC computes 256 x 256 output tiles with
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): CTA r of the pair
@@ -42,19 +45,14 @@ constexpr uint32_t kStageBytes = 2 * kHalfBytes;
 constexpr int kAccCols = 256;
 
 struct PairParams {
-  EpiArgs e;
-  int nkb_main, nkb_lora;
+  GemmArgs a;
   int tiles_m, num_tiles;
   int stages;
-  int32_t* status;
 };
-static_assert(sizeof(PairParams) <= 128, "PairParams must fit GemmLaunch::params");
+static_assert(sizeof(PairParams) <= 256, "PairParams must fit GemmLaunch::params");
 
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
-                     const __grid_constant__ CUtensorMap tm_w,
-                     const __grid_constant__ CUtensorMap tm_t,
-                     const __grid_constant__ CUtensorMap tm_b, const PairParams p) {
+    gemm_pair_kernel(const __grid_constant__ TensorMaps tm, const PairParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~static_cast<uintptr_t>(1023u));
@@ -71,7 +69,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int num_pairs = gridDim.x >> 1;
-  const int nkb = p.nkb_main + p.nkb_lora;
+  const GemmArgs& a = p.a;
+  const bool silu = a.mode == kEpiSiluPair;
+  const int nkb = a.nkb_main + (silu ? 2 : 1) * a.nkb_r;
+  const int tile_n = silu ? kHalf : kTile;   // output features per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -90,12 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish_pair();
   }
   if (warp == 1 && lane == 0) {
-    tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_w);
-    if (p.nkb_lora) {
-      tma_prefetch_desc(&tm_t);
-      tma_prefetch_desc(&tm_b);
-    }
+    tma_prefetch_desc(&tm.x);
+    tma_prefetch_desc(&tm.w[0]);
   }
   tc_fence_before();
   cluster_sync();   // barriers of both CTAs initialised, TMEM allocated in both
@@ -104,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   auto fail = [&]() {
     *abort_flag = 1;
-    raise_status(p.status, kDevTimeout);
+    raise_status(a.status, kDevTimeout);
   };
 
   if (warp == 0 && lane == 0) {
@@ -112,9 +109,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool ok = true;
     for (int tile = pair; ok && tile < p.num_tiles; tile += num_pairs) {
-      const int mb = tile % p.tiles_m, nb = tile / p.tiles_m;
+      const int mb = tile % p.tiles_m, ft = tile / p.tiles_m;
+      const int g = group_of(a, ft);
       const int m0 = mb * kTile + static_cast<int>(rank) * kHalf;
-      const int n0 = nb * kTile + static_cast<int>(rank) * kHalf;
+      // B rows of this CTA's half: its 128 features of group g, or (silu) the
+      // tile's 128 features of group `rank` (gate for CTA 0, up for CTA 1)
+      const int gb = silu ? static_cast<int>(rank) : g;
+      const int n0 = silu ? ft * kHalf : (ft - a.g[g].tile0) * kTile + static_cast<int>(rank) * kHalf;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1u;
@@ -125,11 +126,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t fb = map_shared_rank(smem_u32(&full[s]), 0);
         if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * kStageBytes);
-        const bool lora = kb >= p.nkb_main;
-        const int kc = (lora ? kb - p.nkb_main : kb) * 64;
         const uint32_t sa = smem_u32(smem + s * kStageBytes);
-        tma_load_2d_pair(sa, lora ? &tm_t : &tm_x, kc, m0, fb);
-        tma_load_2d_pair(sa + kHalfBytes, lora ? &tm_b : &tm_w, kc, n0, fb);
+        if (kb < a.nkb_main) {
+          tma_load_2d_pair(sa, &tm.x, kb * 64, m0, fb);
+          tma_load_2d_pair(sa + kHalfBytes, &tm.w[gb], kb * 64, n0, fb);
+        } else {
+          const int l = kb - a.nkb_main;
+          const int h = silu ? l / a.nkb_r : 0;
+          const int j = silu ? l % a.nkb_r : l;
+          tma_load_2d_pair(sa, &tm.t, a.g[silu ? h : g].t_col + j * 64, m0, fb);
+          // silu: the other group's adapter rows are read past the end (zeros)
+          const int row = (silu && h != static_cast<int>(rank)) ? a.g[gb].b_rows : n0;
+          tma_load_2d_pair(sa + kHalfBytes, &tm.b[gb], j * 64, row, fb);
+        }
       }
     }
   } else if (warp == 1 && lane == 0 && leader) {
@@ -184,23 +193,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int mb = tile % p.tiles_m, nb = tile / p.tiles_m;
+      const int mb = tile % p.tiles_m, ft = tile / p.tiles_m;
+      const int g = group_of(a, ft);
       const int m = mb * kTile + static_cast<int>(rank) * kHalf + i;
       const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                             static_cast<uint32_t>(b * kAccCols);
-      for (int c = 0; c < kTile; c += 16) {
-        float v[16];
-        tmem_ld16(trow + c, v);
-        const int n0 = nb * kTile + c;
-        if (m < p.e.M && n0 < p.e.N) {
-          if (n0 + 16 <= p.e.N) {
-            epi_store16_row<__nv_bfloat16>(p.e, m, n0, v);
-          } else {
+      if (!silu) {
+        const int nb0 = (ft - a.g[g].tile0) * kTile;
+        for (int c = 0; c < kTile; c += 16) {
+          float v[16];
+          tmem_ld16(trow + c, v);
+          if (nb0 + c < a.g[g].N) epi_store16<__nv_bfloat16>(a, g, m, nb0 + c, v);
+        }
+      } else {
+        const int f0 = ft * kHalf;
+        for (int c = 0; c < kHalf; c += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(trow + c, gv);
+          tmem_ld16(trow + kHalf + c, uv);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              epi_store1<__nv_bfloat16, false>(p.e, mb * kTile + static_cast<int>(rank) * kHalf,
-                                               n0, i, j, v[j]);
-          }
+          for (int j = 0; j < 16; ++j) gv[j] = silu_f(gv[j]) * uv[j];
+          if (f0 + c < a.g[0].N) epi_store16<__nv_bfloat16>(a, 0, m, f0 + c, gv);
         }
       }
       tc_fence_before();
@@ -224,32 +237,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 bool gemm_pair_suits(const GemmProblem& pb) {
-  if (pb.dt != UNO_BF16 || pb.M <= 256 || pb.N < 256 || pb.mode == kEpiRowScale) return false;
-  const int64_t tiles = ((pb.M + kTile - 1) / kTile) * ((pb.N + kTile - 1) / kTile);
+  if (pb.dt != UNO_BF16 || pb.M <= 256 || pb.mode == kEpiRowScale) return false;
+  if (pb.mode == kEpiSiluPair) return true;
+  int64_t ntiles = 0;
+  for (int i = 0; i < pb.ngroups; ++i) ntiles += (pb.g[i].N + kTile - 1) / kTile;
+  const int64_t tiles = ((pb.M + kTile - 1) / kTile) * ntiles;
   return tiles >= device_sm_count() / 2 || pb.M >= 1024;
 }
 
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
+  const bool silu = pb.mode == kEpiSiluPair;
+  const int tile_n = silu ? kHalf : kTile;
   PairParams pp{};
-  pp.e = epi_args(pb);
-  pp.nkb_main = static_cast<int>((pb.K + 63) / 64);
-  pp.nkb_lora = pb.r > 0 ? (pb.r + 63) / 64 : 0;
+  pp.a = make_gemm_args(pb, tile_n, 128);
   pp.tiles_m = static_cast<int>((pb.M + kTile - 1) / kTile);
-  const int64_t tiles_n = (pb.N + kTile - 1) / kTile;
-  const int64_t tiles = pp.tiles_m * tiles_n;
+  const int64_t tiles = static_cast<int64_t>(pp.tiles_m) * feature_tiles(pp.a, tile_n);
   if (tiles > (1ll << 30)) return set_error(UNO_ERR_UNSUPPORTED, "too many tiles");
   pp.num_tiles = static_cast<int>(tiles);
   pp.stages = 6;
-  pp.status = nullptr;
   uno_status s;
-  if ((s = make_map(&out->tm[0], pb.dt, pb.x, pb.K, pb.M, kHalf)) != UNO_OK) return s;
-  if ((s = make_map(&out->tm[1], pb.dt, pb.W, pb.K, pb.N, kHalf)) != UNO_OK) return s;
+  TensorMaps& tm = out->tm;
+  if ((s = make_map(&tm.x, pb.dt, pb.x, pb.K, pb.M, pb.K, kHalf)) != UNO_OK) return s;
   if (pb.r > 0) {
-    if ((s = make_map(&out->tm[2], pb.dt, pb.t, pb.r, pb.M, kHalf)) != UNO_OK) return s;
-    if ((s = make_map(&out->tm[3], pb.dt, pb.Bl, pb.r, pb.N, kHalf)) != UNO_OK) return s;
+    if ((s = make_map(&tm.t, pb.dt, pb.t, pb.ldt, pb.M, pb.ldt, kHalf)) != UNO_OK) return s;
   } else {
-    out->tm[2] = out->tm[0];
-    out->tm[3] = out->tm[1];
+    tm.t = tm.x;
+  }
+  for (int i = 0; i < kMaxGroups; ++i) {
+    const GemmGroup& G = pb.g[i < pb.ngroups ? i : 0];
+    if ((s = make_map(&tm.w[i], pb.dt, G.W, pb.K, G.N, pb.K, kHalf)) != UNO_OK) return s;
+    if (pb.r > 0) {
+      if ((s = make_map(&tm.b[i], pb.dt, G.Bl, pb.r, G.N, pb.r, kHalf)) != UNO_OK) return s;
+    } else {
+      tm.b[i] = tm.w[i];
+    }
   }
   std::memcpy(out->params, &pp, sizeof(pp));
   const int pairs = std::max(1, std::min<int>(device_sm_count() / 2, pp.num_tiles));
@@ -282,8 +303,7 @@ uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream) {
   cfg.numAttrs = 1;
   PairParams pp;
   std::memcpy(&pp, l.params, sizeof(pp));
-  void* args[5] = {const_cast<CUtensorMap*>(&l.tm[0]), const_cast<CUtensorMap*>(&l.tm[1]),
-                   const_cast<CUtensorMap*>(&l.tm[2]), const_cast<CUtensorMap*>(&l.tm[3]), &pp};
+  void* args[2] = {const_cast<TensorMaps*>(&l.tm), &pp};
   e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e != cudaSuccess) return cuda_error(e, "pair GEMM launch");
   return UNO_OK;

@@ -1,12 +1,15 @@
-// Gated-LoRA GEMM on the 5th-generation tensor cores (sm_100a).
+// Gated-LoRA GEMM on the 5th-generation tensor cores (sm_100a), one CTA per tile.
 //
-//   y = x W^T + t Bl^T,   t = scale * g (.) (x A^T)   (the gated LoRA adapter:
-//   hyper.ai page, section "方法" — adapter on every AR matrix, gated per row)
+//   y_g = x W_g^T + t_g Bl_g^T,   t_g = scale * gate (.) (x A_g^T)
+//   (the gated LoRA adapter: hyper.ai page, section "方法" — an adapter on
+//   every AR matrix, switched per row)
 //
 // The adapter's up-projection is folded into the same accumulator as extra
 // K-steps: the K loop runs over [x | t] against [W | Bl], so W streams from
 // HBM exactly once and the LoRA term costs r/64 extra K-blocks. The gated
-// down-projection t is the same kernel with epilogue kEpiRowScale.
+// down-projection t is the same kernel with epilogue kEpiRowScale. One launch
+// covers up to three output groups that share x (q|k|v, or their
+// down-projections); kEpiSiluPair fuses silu(gate) * up.
 //
 // Structure of one CTA (192 threads):
 //   warp 0, one lane : TMA producer — 128-byte-swizzled K-major tiles of both
@@ -17,11 +20,12 @@
 //   warps 2..5       : epilogue — tcgen05.ld of the accumulator (each warp
 //                      reads its 32-lane quarter), convert, store.
 // Operand roles: the "P" operand fills the 128 MMA rows, the "Q" operand the
-// bn MMA columns. Large M: P = tokens (x), Q = features (W). Small M
-// ("swap"): P = features (W), Q = tokens (x), so a decode batch of 9..256
-// rows still fills the 128-row MMA. Small problems split K across a thread
-// block cluster; the partial tiles are summed through distributed shared
-// memory (no global scratch, no atomics, no spin waits).
+// bn MMA columns. Normal: P = tokens (x), Q = features (W). "Swap" (decode
+// batches and the down-projections): P = features, Q = tokens (16..256 per
+// tile). In swap silu-pair tiles the 128 feature rows are 64 gate rows then
+// the same 64 up rows. Small problems split K across a thread-block cluster;
+// the partial tiles are summed through distributed shared memory (no global
+// scratch, no atomics, no spin waits).
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -41,29 +45,28 @@ constexpr int kMaxStages = 12;
 // Split-K partial tiles in shared memory (fp32, padded rows):
 //   non-swapped: part[i][bn + 4]   (one row per accumulator lane = token)
 //   swapped:     part[j][128 + 4]  (one row per token column; lanes = features)
-// so the reduction reads 16-byte groups of 4 consecutive output features.
+// so the reduction reads 16-byte groups of 4 consecutive lanes or columns.
 constexpr int kPartPad = 4;
+constexpr int kHalfP = kTileP / 2;
 
-struct GemmParams {
-  EpiArgs e;
+struct Gemm1Params {
+  GemmArgs a;
   int bn;                 // Q rows per tile (multiple of 16, <= 256)
   int stages;
   int tmem_cols;
-  int nkb_main, nkb_lora, kb_per_split, splits;
-  int32_t* status;
+  int kb_per_split, splits;
 };
-static_assert(sizeof(GemmParams) <= 128, "GemmParams must fit GemmLaunch::params");
+static_assert(sizeof(Gemm1Params) <= 256, "Gemm1Params must fit GemmLaunch::params");
 
 __host__ __device__ constexpr uint32_t stage_bytes_for(int bn) {
   return ((kTileP + bn) * kRowBytes + 1023u) & ~1023u;
 }
 
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 template <typename T, bool kSwap>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gated_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
-                      const __grid_constant__ CUtensorMap tm_w,
-                      const __grid_constant__ CUtensorMap tm_t,
-                      const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
+    gemm1_kernel(const __grid_constant__ TensorMaps tm, const Gemm1Params p) {
   constexpr bool kTf32 = std::is_same<T, float>::value;
   constexpr int kBKe = kRowBytes / static_cast<int>(sizeof(T));  // elements per K-block
   constexpr int kKSteps = kRowBytes / 32;                          // MMAs per K-block (32 B of K each)
@@ -71,6 +74,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~static_cast<uintptr_t>(1023u));
+  const GemmArgs& a = p.a;
   const int bn = p.bn;
   const uint32_t p_bytes = kTileP * kRowBytes;
   const uint32_t q_bytes = static_cast<uint32_t>(bn) * kRowBytes;
@@ -85,9 +89,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tok_tile = blockIdx.x, feat_tile = blockIdx.y, split = blockIdx.z;
-  const int p_row0 = kSwap ? feat_tile * kTileP : tok_tile * kTileP;
-  const int q_row0 = kSwap ? tok_tile * bn : feat_tile * bn;
+  const bool silu = a.mode == kEpiSiluPair;   // swap tiles only
+  const int ft = blockIdx.y, split = blockIdx.z;
+  const int g = group_of(a, ft);
+  const int feat_rows = kSwap ? (silu ? kHalfP : kTileP) : bn;
+  const int feat0 = (ft - a.g[g].tile0) * feat_rows;        // first feature of the tile in group g
+  const int tok0 = blockIdx.x * (kSwap ? bn : kTileP);      // first token of the tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -103,20 +110,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), static_cast<uint32_t>(p.tmem_cols));
     tmem_relinquish();
   }
-  if (warp == 1 && lane == 0) {
-    tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_w);
-    if (p.nkb_lora) {
-      tma_prefetch_desc(&tm_t);
-      tma_prefetch_desc(&tm_b);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int nkb = p.nkb_main + p.nkb_lora;
+  const int nkb_lora = silu ? 2 * a.nkb_r : a.nkb_r;
+  const int nkb = a.nkb_main + nkb_lora;
   const int kb0 = split * p.kb_per_split;
   const int kb1 = min(nkb, kb0 + p.kb_per_split);
   int issued = 0;
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t ph = (issued / p.stages) & 1u;
       if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u)) {
         *abort_flag = 1;
-        raise_status(p.status, kDevTimeout);
+        raise_status(a.status, kDevTimeout);
         break;
       }
       if (*abort_flag) break;
@@ -136,16 +136,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t sq = sp + p_bytes;
       const uint32_t fb = smem_u32(&full[s]);
       mbar_arrive_expect_tx(fb, p_bytes + q_bytes);
-      const bool lora = kb >= p.nkb_main;
-      const int kc = (lora ? kb - p.nkb_main : kb) * kBKe;
-      const CUtensorMap* tok_map = lora ? &tm_t : &tm_x;
-      const CUtensorMap* feat_map = lora ? &tm_b : &tm_w;
-      if (kSwap) {
-        tma_load_2d(sp, feat_map, kc, p_row0, fb);
-        tma_load_2d(sq, tok_map, kc, q_row0, fb);
+      const uint32_t s_tok = kSwap ? sq : sp;
+      const uint32_t s_feat = kSwap ? sp : sq;
+      if (kb < a.nkb_main) {
+        const int kc = kb * kBKe;
+        tma_load_2d(s_tok, &tm.x, kc, tok0, fb);
+        if (silu) {
+          tma_load_2d(s_feat, &tm.w[0], kc, feat0, fb);
+          tma_load_2d(s_feat + kHalfP * kRowBytes, &tm.w[1], kc, feat0, fb);
+        } else {
+          tma_load_2d(s_feat, &tm.w[g], kc, feat0, fb);
+        }
       } else {
-        tma_load_2d(sp, tok_map, kc, p_row0, fb);
-        tma_load_2d(sq, feat_map, kc, q_row0, fb);
+        const int l = kb - a.nkb_main;
+        const int h = silu ? l / a.nkb_r : 0;           // silu: 0 = gate block, 1 = up block
+        const int j = silu ? l % a.nkb_r : l;
+        tma_load_2d(s_tok, &tm.t, a.g[silu ? h : g].t_col + j * kBKe, tok0, fb);
+        if (silu) {
+          // the other half's adapter rows are read past the end: zeros
+          tma_load_2d(s_feat, &tm.b[0], j * kBKe, h == 0 ? feat0 : a.g[0].b_rows, fb);
+          tma_load_2d(s_feat + kHalfP * kRowBytes, &tm.b[1], j * kBKe,
+                      h == 1 ? feat0 : a.g[1].b_rows, fb);
+        } else {
+          tma_load_2d(s_feat, &tm.b[g], j * kBKe, feat0, fb);
+        }
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -157,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t ph = (it / p.stages) & 1u;
       if (!mbar_wait(smem_u32(&full[s]), ph)) {
         *abort_flag = 1;
-        raise_status(p.status, kDevTimeout);
+        raise_status(a.status, kDevTimeout);
         break;
       }
       tc_fence_after();
@@ -181,83 +195,108 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(accum), 0));
     if (!ok && lane == 0) {
       *abort_flag = 1;
-      raise_status(p.status, kDevTimeout);
+      raise_status(a.status, kDevTimeout);
     }
     tc_fence_after();
-    if (ok) {
-      const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (p.splits == 1) {
-        for (int c = 0; c < bn; c += 16) {
-          float v[16];
-          tmem_ld16(trow + c, v);
-          if (!kSwap) {
-            const int m = p_row0 + i, n0 = q_row0 + c;
-            if (m < p.e.M) {
-              if (n0 + 16 <= p.e.N) {
-                epi_store16_row<T>(p.e, m, n0, v);
-              } else {
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    float* stage = reinterpret_cast<float*>(smem);   // the stage ring is free now
+    if (p.splits == 1) {
+      if (!kSwap) {
+        if (ok) {
+          for (int c = 0; c < bn; c += 16) {
+            float v[16];
+            tmem_ld16(trow + c, v);
+            epi_store16<T>(a, g, tok0 + i, feat0 + c, v);
+          }
+        }
+      } else if (!silu) {
+        if (ok) {
+          for (int c = 0; c < bn; c += 16) {
+            float v[16];
+            tmem_ld16(trow + c, v);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) epi_store1<T, kSwap>(p.e, p_row0, q_row0, i, c + j, v[j]);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) epi_store1<T, kSwap>(p.e, p_row0, q_row0, i, c + j, v[j]);
+            for (int j = 0; j < 16; ++j) epi_store1<T>(a, g, tok0 + c + j, feat0 + i, v[j]);
           }
         }
       } else {
-        float* part = reinterpret_cast<float*>(smem);   // the stage ring is free now
-        for (int c = 0; c < bn; c += 16) {
-          float v[16];
-          tmem_ld16(trow + c, v);
-          if (kSwap) {
+        // lanes 0..63 hold gate, 64..127 the matching up features: stage both
+        // through shared memory, then every thread forms silu(gate) * up
+        const int R = bn * (kHalfP + 1);
+        const int f = i & (kHalfP - 1);
+        float* dst = stage + (i < kHalfP ? 0 : R);
+        if (ok) {
+          for (int c = 0; c < bn; c += 16) {
+            float v[16];
+            tmem_ld16(trow + c, v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) part[(c + j) * (kTileP + kPartPad) + i] = v[j];
-          } else {
-            float4* row = reinterpret_cast<float4*>(part + i * (bn + kPartPad) + c);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int j = 0; j < 16; ++j) dst[(c + j) * (kHalfP + 1) + f] = v[j];
           }
+        }
+        epi_bar();
+        if (ok) {
+          for (int j = i >> 6; j < bn; j += 2) {
+            const float gv = stage[j * (kHalfP + 1) + f];
+            const float uv = stage[R + j * (kHalfP + 1) + f];
+            epi_store1<T>(a, 0, tok0 + j, feat0 + f, silu_f(gv) * uv);
+          }
+        }
+      }
+    } else if (ok) {
+      for (int c = 0; c < bn; c += 16) {
+        float v[16];
+        tmem_ld16(trow + c, v);
+        if (kSwap) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) stage[(c + j) * (kTileP + kPartPad) + i] = v[j];
+        } else {
+          float4* row = reinterpret_cast<float4*>(stage + i * (bn + kPartPad) + c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
       }
     }
   }
 
   if (p.splits > 1) {
-    // Sum the cluster's partial tiles. The tile is cut into groups of 4
-    // consecutive output features; CTA `rank` reduces a contiguous range of
-    // groups, reading the same group from every CTA of the cluster.
+    // Sum the cluster's partial tiles. CTA `rank` reduces a contiguous range
+    // of 4-element groups, reading the same group from every CTA.
     cluster_sync();
     const uint32_t rank = cluster_ctarank();
     const int S = p.splits;
-    const int groups = kTileP * bn / 4;
+    const int groups = kSwap ? (silu ? bn * (kTileP / 8) : bn * (kTileP / 4)) : kTileP * bn / 4;
     const int chunk = (groups + S - 1) / S;
-    const int g0 = static_cast<int>(rank) * chunk;
-    const int g1 = min(groups, g0 + chunk);
+    const int e0 = static_cast<int>(rank) * chunk;
+    const int e1 = min(groups, e0 + chunk);
     const uint32_t part0 = smem_u32(smem);
     uint32_t peer[8];
     for (int r = 0; r < S; ++r) peer[r] = map_shared_rank(part0, r);
-    for (int g = g0 + static_cast<int>(threadIdx.x); g < g1; g += kGemmThreads) {
-      int m, n;
-      uint32_t off;
-      if (kSwap) {
-        const int j = g / (kTileP / 4), i4 = g % (kTileP / 4);
-        off = static_cast<uint32_t>((j * (kTileP + kPartPad) + 4 * i4) * 4);
-        m = q_row0 + j;
-        n = p_row0 + 4 * i4;
-      } else {
-        const int i = g / (bn / 4), j4 = g % (bn / 4);
-        off = static_cast<uint32_t>((i * (bn + kPartPad) + 4 * j4) * 4);
-        m = p_row0 + i;
-        n = q_row0 + 4 * j4;
-      }
+    auto sum4 = [&](uint32_t off) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int r = 0; r < S; ++r) {
         const float4 v = ld_cluster_f32x4(peer[r] + off);
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      if (m < p.e.M && n < p.e.N) epi_store4<T>(p.e, m, n, acc);
+      return acc;
+    };
+    for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += kGemmThreads) {
+      if (!kSwap) {
+        const int i = e / (bn / 4), j4 = e % (bn / 4);
+        const float4 acc = sum4(static_cast<uint32_t>((i * (bn + kPartPad) + 4 * j4) * 4));
+        epi_store4<T>(a, g, tok0 + i, feat0 + 4 * j4, acc);
+      } else if (!silu) {
+        const int j = e / (kTileP / 4), i4 = e % (kTileP / 4);
+        const float4 acc = sum4(static_cast<uint32_t>((j * (kTileP + kPartPad) + 4 * i4) * 4));
+        epi_store4<T>(a, g, tok0 + j, feat0 + 4 * i4, acc);
+      } else {
+        const int j = e / (kTileP / 8), f4 = e % (kTileP / 8);
+        const uint32_t row = static_cast<uint32_t>(j * (kTileP + kPartPad));
+        const float4 gv = sum4((row + 4 * f4) * 4);
+        const float4 uv = sum4((row + kHalfP + 4 * f4) * 4);
+        epi_store4<T>(a, 0, tok0 + j, feat0 + 4 * f4,
+                      make_float4(silu_f(gv.x) * uv.x, silu_f(gv.y) * uv.y, silu_f(gv.z) * uv.z,
+                                  silu_f(gv.w) * uv.w));
+      }
     }
     cluster_sync();
   }
@@ -276,11 +315,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------- host side
-
 template <typename T, bool kSwap>
 void* kernel_ptr() {
-  return reinterpret_cast<void*>(&gated_gemm_kernel<T, kSwap>);
+  return reinterpret_cast<void*>(&gemm1_kernel<T, kSwap>);
 }
 
 void* pick_kernel(uno_dtype dt, bool swap) {
@@ -295,8 +332,6 @@ int pow2_at_least(int v) {
   while (c < v) c <<= 1;
   return c;
 }
-
-}  // namespace
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -316,14 +351,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major [rows, inner] tensor, box = 128 bytes of K x box_rows rows, 128-byte swizzle.
+}  // namespace
+
 uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t inner, uint64_t rows,
-                    uint32_t box_rows) {
+                    uint64_t row_stride_elems, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return set_error(UNO_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   const uint32_t esz = dt == UNO_F32 ? 4u : 2u;
   const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {inner * esz};
+  const cuuint64_t strides[1] = {row_stride_elems * esz};
   const cuuint32_t box[2] = {kRowBytes / esz, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r =
@@ -349,31 +385,39 @@ int device_sm_count() {
 }
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
+  if (pb.ngroups < 1 || pb.ngroups > kMaxGroups)
+    return set_error(UNO_ERR_INVALID_ARG, "1..3 output groups per GEMM launch");
+  if (pb.mode == kEpiSiluPair && (pb.ngroups != 2 || pb.g[0].N != pb.g[1].N))
+    return set_error(UNO_ERR_INVALID_ARG, "silu-pair needs two groups of equal width");
   if (gemm_pair_suits(pb)) return gemm_pair_prepare(pb, out);
+  if (pb.mode == kEpiSiluPair && pb.M > 256)
+    return set_error(UNO_ERR_UNSUPPORTED, "silu-pair with M > 256 needs the bf16 pair kernel");
   const int esz = pb.dt == UNO_F32 ? 4 : 2;
-  const int bke = kRowBytes / esz;
+  (void)esz;
   const int sms = device_sm_count();
-  const int64_t M = pb.M, N = pb.N;
-  if (M > (1ll << 30) || N > (1ll << 30)) return set_error(UNO_ERR_UNSUPPORTED, "M or N too large");
+  const int64_t M = pb.M;
+  if (M > (1ll << 30)) return set_error(UNO_ERR_UNSUPPORTED, "M too large");
+  const bool silu = pb.mode == kEpiSiluPair;
 
-  // Tile shape: small M puts the weight rows on the 128-row MMA side.
-  const bool swap = M <= 256;
-  int bn, grid_x, grid_y;
+  // Tile shape: decode batches and the rank-r down-projections put the
+  // weight rows on the 128-row MMA side ("swap").
+  const bool swap = M <= 256 || pb.mode == kEpiRowScale;
+  int bn, tok_tiles;
   if (swap) {
-    bn = round_up(static_cast<int>(M), 16);
-    grid_x = 1;
-    grid_y = static_cast<int>((N + kTileP - 1) / kTileP);
+    tok_tiles = static_cast<int>((M + 255) / 256);
+    bn = round_up(static_cast<int>((M + tok_tiles - 1) / tok_tiles), 16);
   } else {
-    const int64_t tiles_tok = (M + kTileP - 1) / kTileP;
-    bn = (tiles_tok * ((N + 255) / 256) >= sms) ? 256 : 128;
-    grid_x = static_cast<int>(tiles_tok);
-    grid_y = static_cast<int>((N + bn - 1) / bn);
+    tok_tiles = static_cast<int>((M + kTileP - 1) / kTileP);
+    int64_t ntiles256 = 0;
+    for (int i = 0; i < pb.ngroups; ++i) ntiles256 += (pb.g[i].N + 255) / 256;
+    bn = (tok_tiles * ntiles256 >= sms) ? 256 : 128;
   }
-  if (grid_y > 65535) return set_error(UNO_ERR_UNSUPPORTED, "N too large for the tile grid");
+  const int feat_tile = swap ? (silu ? kHalfP : kTileP) : bn;
+  GemmArgs ga = make_gemm_args(pb, feat_tile, kRowBytes);
+  const int feat_tiles = feature_tiles(ga, feat_tile);
+  if (feat_tiles > 65535) return set_error(UNO_ERR_UNSUPPORTED, "N too large for the tile grid");
 
-  const int nkb_main = static_cast<int>((pb.K + bke - 1) / bke);
-  const int nkb_lora = pb.r > 0 ? (pb.r + bke - 1) / bke : 0;
-  const int nkb = nkb_main + nkb_lora;
+  const int nkb = ga.nkb_main + (silu ? 2 : 1) * ga.nkb_r;
 
   // Shared memory: ~96 KB (two or three CTAs per SM) for narrow decode tiles,
   // ~200 KB otherwise.
@@ -386,7 +430,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
                             : 1;
 
   // Split K across a cluster when the tile grid cannot fill the GPU.
-  const int64_t tiles = static_cast<int64_t>(grid_x) * grid_y;
+  const int64_t tiles = static_cast<int64_t>(tok_tiles) * feat_tiles;
   int splits = 1;
   const int64_t capacity = static_cast<int64_t>(sms) * per_sm;
   if (tiles < capacity) {
@@ -395,42 +439,49 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   }
   int kb_per = (nkb + splits - 1) / splits;
   splits = (nkb + kb_per - 1) / kb_per;   // every split gets >= 1 K-block
-  // the split-K partial tile must fit in the stage ring
+  // the split-K partial tile (and the silu hand-over) must fit in the stage ring
   const uint32_t part_bytes = static_cast<uint32_t>(
       (swap ? bn * (kTileP + kPartPad) : kTileP * (bn + kPartPad)) * 4);
+  const uint32_t silu_bytes = static_cast<uint32_t>(2 * bn * (kHalfP + 1) * 4);
   if (splits > 1 && part_bytes > stages * st) {
     splits = 1;
     kb_per = nkb;
   }
+  if (silu && splits == 1 && silu_bytes > stages * st)
+    return set_error(UNO_ERR_UNSUPPORTED, "silu-pair tile does not fit shared memory");
 
-  GemmParams gp{};
-  gp.e = epi_args(pb);
+  Gemm1Params gp{};
+  gp.a = ga;
   gp.bn = bn;
   gp.stages = stages;
   gp.tmem_cols = pow2_at_least(bn);
-  gp.nkb_main = nkb_main;
-  gp.nkb_lora = nkb_lora;
   gp.kb_per_split = kb_per;
   gp.splits = splits;
-  gp.status = nullptr;
 
   const uint32_t tok_box = swap ? static_cast<uint32_t>(bn) : kTileP;
-  const uint32_t feat_box = swap ? kTileP : static_cast<uint32_t>(bn);
+  const uint32_t feat_box = swap ? static_cast<uint32_t>(feat_tile) : static_cast<uint32_t>(bn);
   uno_status s;
-  if ((s = make_map(&out->tm[0], pb.dt, pb.x, pb.K, M, tok_box)) != UNO_OK) return s;
-  if ((s = make_map(&out->tm[1], pb.dt, pb.W, pb.K, N, feat_box)) != UNO_OK) return s;
+  TensorMaps& tm = out->tm;
+  if ((s = make_map(&tm.x, pb.dt, pb.x, pb.K, M, pb.K, tok_box)) != UNO_OK) return s;
   if (pb.r > 0) {
-    if ((s = make_map(&out->tm[2], pb.dt, pb.t, pb.r, M, tok_box)) != UNO_OK) return s;
-    if ((s = make_map(&out->tm[3], pb.dt, pb.Bl, pb.r, N, feat_box)) != UNO_OK) return s;
+    if ((s = make_map(&tm.t, pb.dt, pb.t, pb.ldt, M, pb.ldt, tok_box)) != UNO_OK) return s;
   } else {
-    out->tm[2] = out->tm[0];
-    out->tm[3] = out->tm[1];
+    tm.t = tm.x;
+  }
+  for (int i = 0; i < kMaxGroups; ++i) {
+    const GemmGroup& G = pb.g[i < pb.ngroups ? i : 0];
+    if ((s = make_map(&tm.w[i], pb.dt, G.W, pb.K, G.N, pb.K, feat_box)) != UNO_OK) return s;
+    if (pb.r > 0) {
+      if ((s = make_map(&tm.b[i], pb.dt, G.Bl, pb.r, G.N, pb.r, feat_box)) != UNO_OK) return s;
+    } else {
+      tm.b[i] = tm.w[i];
+    }
   }
   std::memcpy(out->params, &gp, sizeof(gp));
   out->kind = 0;
   out->swap = swap;
-  out->grid_x = grid_x;
-  out->grid_y = grid_y;
+  out->grid_x = tok_tiles;
+  out->grid_y = feat_tiles;
   out->splits = splits;
   out->smem_bytes = static_cast<int>(stages * st + 1024 + 64 + 16 * (2 * stages + 1));
   out->dtype = pb.dt;
@@ -443,10 +494,6 @@ uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream) {
   cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, l.smem_bytes);
   if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute(gemm smem)");
-  if (l.splits > 1) {
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    (void)e;
-  }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(l.grid_x, l.grid_y, l.splits);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
@@ -461,10 +508,9 @@ uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  GemmParams gp;
+  Gemm1Params gp;
   std::memcpy(&gp, l.params, sizeof(gp));
-  void* args[5] = {const_cast<CUtensorMap*>(&l.tm[0]), const_cast<CUtensorMap*>(&l.tm[1]),
-                   const_cast<CUtensorMap*>(&l.tm[2]), const_cast<CUtensorMap*>(&l.tm[3]), &gp};
+  void* args[2] = {const_cast<TensorMaps*>(&l.tm), &gp};
   e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e != cudaSuccess) return cuda_error(e, "gated GEMM launch");
   return UNO_OK;

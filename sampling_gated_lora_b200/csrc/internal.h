@@ -18,36 +18,54 @@ uno_status cuda_error(cudaError_t e, const char* what);
 
 enum EpilogueMode : int {
   kEpiStore = 0,     // y = acc
-  kEpiAdd = 1,       // y = y + acc (in place)
+  kEpiAdd = 1,       // y = y + acc (in place: the residual add)
   kEpiRowScale = 2,  // y = scale * gate[m] * acc   (the gated LoRA down-projection)
+  kEpiSiluPair = 3,  // groups 0 (gate) and 1 (up): y0 = silu(acc_gate) * acc_up
 };
 
-// One launch of the gated-LoRA GEMM:
-//   y[m, n] = epi( sum_k x[m,k] W[n,k] + sum_j t[m,j] Bl[n,j] )
-// Rows m >= M0 are written to y1 (row m - M0) instead of y.
+constexpr int kMaxGroups = 3;
+
+// One output group of a GEMM launch: its weights, adapter and output.
+struct GemmGroup {
+  const void* W;          // [N, K]
+  const void* Bl;         // [N, r]  (unused when r == 0)
+  int64_t N;
+  void* y;                // [M, ldy], features [0, N)
+  int64_t ldy;
+  int64_t t_col;          // first column of this group's rank-r block in t
+};
+
+// One launch of the gated-LoRA GEMM over up to kMaxGroups linears that share
+// the input x (and its LoRA activations t):
+//   y_g[m, n] = epi( sum_k x[m,k] W_g[n,k] + sum_j t[m, t_col_g + j] Bl_g[n,j] )
+// Group 0 rows m >= M0 are written to y1 (row m - M0) instead of y_0.
 struct GemmProblem {
   uno_dtype dt;
-  int64_t M, N, K;
-  int32_t r;              // 0: no LoRA term
+  int64_t M, K;
+  int32_t r;              // LoRA rank per group (0: no LoRA term)
   const void* x;          // [M, K]
-  const void* W;          // [N, K]
-  const void* t;          // [M, r]  (rank-r activations, already gated and scaled)
-  const void* Bl;         // [N, r]
+  const void* t;          // [M, ldt] rank-r activations, already gated and scaled
+  int64_t ldt;
+  int ngroups;
+  GemmGroup g[kMaxGroups];
   int mode;
-  void* y;
   void* y1;
-  int64_t M0;             // rows >= M0 go to y1
-  int64_t ldy;
+  int64_t M0;
   const uint8_t* gate;    // kEpiRowScale; NULL: gate[m] = (m >= gate_row0)
   int64_t gate_row0;
   float scale;            // kEpiRowScale
 };
 
+// All tensor maps of one launch (passed to the kernel as one parameter).
+struct TensorMaps {
+  CUtensorMap x, t, w[kMaxGroups], b[kMaxGroups];
+};
+
 // Cached launch of a GemmProblem (tensor maps + grid); valid while the
 // pointers of the problem stay the same.
 struct GemmLaunch {
-  CUtensorMap tm[4];
-  alignas(8) unsigned char params[128];
+  TensorMaps tm;
+  alignas(8) unsigned char params[256];
   int kind;               // 0: one-CTA kernel, 1: persistent CTA-pair kernel
   int swap;
   int grid_x, grid_y, splits;
@@ -56,15 +74,15 @@ struct GemmLaunch {
 };
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out);
+uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream);
 // Row-major [rows, inner] tensor map: box = 128 bytes of K x box_rows rows, 128-byte swizzle.
 uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t inner, uint64_t rows,
-                    uint32_t box_rows);
+                    uint64_t row_stride_elems, uint32_t box_rows);
 // The persistent CTA-pair kernel (bf16, 256x256 tiles): whether it takes the
 // problem, its preparation and its launch.
 bool gemm_pair_suits(const GemmProblem& pb);
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
-uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sampler
 

@@ -97,3 +97,51 @@ def test_empty_batch_is_a_no_op():
     g = torch.empty((0,), dtype=torch.uint8, device="cuda")
     y = U.gated_lora_linear(x, W_, A, Bl, g)
     assert y.shape == (0, 128)
+
+
+def _group_case(M, K, Ns, r, seed, b_std=0.01):
+    rng = np.random.default_rng(seed)
+    gate = (rng.random(M) < 0.5).astype(np.uint8)
+    cases = [W.gated_linear_case(M, K, N, r, gate, b_std=b_std, seed=seed + i) for i, N in enumerate(Ns)]
+    x = cases[0].x
+    return x, gate, cases
+
+
+def _run_group(x, gate, cases, silu_pair):
+    import sampling_gated_lora_b200 as U
+    t = lambda a: dev_tensor(a, "bf16")
+    ys = U.gated_lora_linear_group(t(x), [t(c.W) for c in cases], [t(c.A) for c in cases],
+                                   [t(c.Bl) for c in cases], dev_tensor(gate, "u8"), 1.0,
+                                   silu_pair=silu_pair)
+    return [host_f64(y) for y in ys]
+
+
+def _oracle_group(x, gate, c, rows=None):
+    f = W.bf16_to_f64
+    xs = f(x) if rows is None else f(x[rows])
+    g = gate if rows is None else gate[rows]
+    return gated_linear(xs, f(c.W), f(c.A), f(c.Bl), g, 1.0)
+
+
+@pytest.mark.parametrize("M", [9, 72, 576, 1088])
+def test_grouped_qkv(M):
+    """q, k, v of one layer in one launch (4096 -> 4096 / 1024 / 1024, r = 128)."""
+    x, gate, cases = _group_case(M, 4096, (4096, 1024, 1024), 128, seed=M)
+    ys = _run_group(x, gate, cases, False)
+    rows = None if M <= 576 else np.arange(0, M, 7)
+    for y, c in zip(ys, cases):
+        ref = _oracle_group(x, gate, c, rows)
+        check_close(y if rows is None else y[rows], ref, what=f"group N={c.N} M={M}")
+
+
+@pytest.mark.parametrize("M,K,N,r", [(9, 4096, 12288, 128), (72, 4096, 1024, 128),
+                                     (17, 264, 200, 24), (300, 1024, 520, 64),
+                                     (2048, 4096, 12288, 128)])
+def test_silu_pair(M, K, N, r):
+    """y = silu(gate(x)) * up(x) in one launch."""
+    from oracle.stack import silu
+    x, gate, cases = _group_case(M, K, (N, N), r, seed=N + M)
+    y = _run_group(x, gate, cases, True)[0]
+    rows = None if M <= 300 else np.concatenate([np.arange(0, M, 37), [M // 2 - 1, M // 2, M - 1]])
+    ref = silu(_oracle_group(x, gate, cases[0], rows)) * _oracle_group(x, gate, cases[1], rows)
+    check_close(y if rows is None else y[rows], ref, what=f"silu-pair M={M} K={K} N={N}")
