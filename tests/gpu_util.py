@@ -49,12 +49,13 @@ def case_to_f64(a, dtype):
     return W.bf16_to_f64(a) if dtype == "bf16" else np.asarray(a, dtype=np.float64)
 
 
-def check_close(y, ref, rel=REL_FROB, max_abs=MAX_ABS, what=""):
+def check_close(y, ref, rel=REL_FROB, max_abs=MAX_ABS, what="", rel_elem=0.0):
+    """rel-Frobenius <= rel and |y - ref| <= max_abs + rel_elem |ref| elementwise."""
     err = y - ref
     rf = np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-30)
-    ma = np.abs(err).max() if err.size else 0.0
-    assert rf <= rel and ma <= max_abs, f"{what}: rel-Frobenius {rf:.3e}, max-abs {ma:.3e}"
-    return rf, ma
+    excess = (np.abs(err) - rel_elem * np.abs(ref)).max() if err.size else 0.0
+    assert rf <= rel and excess <= max_abs, f"{what}: rel-Frobenius {rf:.3e}, max-abs excess {excess:.3e}"
+    return rf, excess
 
 
 def compare_verify(gpu, ora, k, sequences):

@@ -138,10 +138,16 @@ def test_grouped_qkv(M):
                                      (17, 264, 200, 24), (300, 1024, 520, 64),
                                      (2048, 4096, 12288, 128)])
 def test_silu_pair(M, K, N, r):
-    """y = silu(gate(x)) * up(x) in one launch."""
+    """y = silu(gate(x)) * up(x) in one launch.
+
+    The product reaches |y| >= 8, where one bf16 rounding of the output alone
+    exceeds the single-linear max-abs bound: elements are held to
+    3e-2 + 2^-8 |ref| (that bound plus one bf16 rounding of the product).
+    """
     from oracle.stack import silu
     x, gate, cases = _group_case(M, K, (N, N), r, seed=N + M)
     y = _run_group(x, gate, cases, True)[0]
     rows = None if M <= 300 else np.concatenate([np.arange(0, M, 37), [M // 2 - 1, M // 2, M - 1]])
     ref = silu(_oracle_group(x, gate, cases[0], rows)) * _oracle_group(x, gate, cases[1], rows)
-    check_close(y if rows is None else y[rows], ref, what=f"silu-pair M={M} K={K} N={N}")
+    check_close(y if rows is None else y[rows], ref, what=f"silu-pair M={M} K={K} N={N}",
+                rel_elem=2.0 ** -8)
