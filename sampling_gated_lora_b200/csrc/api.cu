@@ -1,6 +1,7 @@
 // C ABI of the library (include/uno.h): argument validation, error reporting,
 // the model handle and the orchestration of one synthetic decode step.
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <memory>
@@ -33,6 +34,14 @@ uno_status set_error(uno_status st, const char* fmt, ...) {
   vsnprintf(g_err, sizeof(g_err), fmt, ap);
   va_end(ap);
   return st;
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("UNO_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 uno_status cuda_error(cudaError_t e, const char* what) {

@@ -40,6 +40,18 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Kernels of this library are launched so that the next kernel on the stream
+// may start its prologue while this one finishes. Each kernel triggers its
+// dependents once its own prologue is done, and touches no data written by
+// an earlier kernel before pdl_wait() returns (constant weights may be
+// prefetched before it).
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ smem / mbarrier
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();   // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_trigger();
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -106,8 +107,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
+    // The first stages' weight halves are constant: they are issued before
+    // waiting for the kernel that writes the activations.
     int it = 0;
     bool ok = true;
+    int pre = 0;   // k-blocks of the first tile whose W half went out early
     for (int tile = pair; ok && tile < p.num_tiles; tile += num_pairs) {
       const int mb = tile % p.tiles_m, ft = tile / p.tiles_m;
       const int g = group_of(a, ft);
@@ -116,7 +120,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tile's 128 features of group `rank` (gate for CTA 0, up for CTA 1)
       const int gb = silu ? static_cast<int>(rank) : g;
       const int n0 = silu ? ft * kHalf : (ft - a.g[g].tile0) * kTile + static_cast<int>(rank) * kHalf;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
+      auto load_b = [&](int kb, uint32_t sb, uint32_t fb) {
+        if (kb < a.nkb_main) {
+          tma_load_2d_pair(sb, &tm.w[gb], kb * 64, n0, fb);
+        } else {
+          const int l = kb - a.nkb_main;
+          const int h = silu ? l / a.nkb_r : 0;
+          const int j = silu ? l % a.nkb_r : l;
+          // silu: the other group's adapter rows are read past the end (zeros)
+          const int row = (silu && h != static_cast<int>(rank)) ? a.g[gb].b_rows : n0;
+          tma_load_2d_pair(sb, &tm.b[gb], j * 64, row, fb);
+        }
+      };
+      auto load_a = [&](int kb, uint32_t sa, uint32_t fb) {
+        if (kb < a.nkb_main) {
+          tma_load_2d_pair(sa, &tm.x, kb * 64, m0, fb);
+        } else {
+          const int l = kb - a.nkb_main;
+          const int h = silu ? l / a.nkb_r : 0;
+          const int j = silu ? l % a.nkb_r : l;
+          tma_load_2d_pair(sa, &tm.t, a.g[silu ? h : g].t_col + j * 64, m0, fb);
+        }
+      };
+      if (tile == pair) {
+        pre = min(S, nkb);
+        for (int q = 0; q < pre; ++q) {
+          const uint32_t sa = smem_u32(smem + q * kStageBytes);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[q]), 2 * kStageBytes);
+          load_b(q, sa + kHalfBytes, map_shared_rank(smem_u32(&full[q]), 0));
+        }
+        pdl_wait();
+        for (int q = 0; q < pre; ++q)
+          load_a(q, smem_u32(smem + q * kStageBytes), map_shared_rank(smem_u32(&full[q]), 0));
+        it = pre;
+      }
+      for (int kb = (tile == pair) ? pre : 0; kb < nkb; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1u;
         if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u) || *abort_flag) {
@@ -127,20 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = map_shared_rank(smem_u32(&full[s]), 0);
         if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * kStageBytes);
         const uint32_t sa = smem_u32(smem + s * kStageBytes);
-        if (kb < a.nkb_main) {
-          tma_load_2d_pair(sa, &tm.x, kb * 64, m0, fb);
-          tma_load_2d_pair(sa + kHalfBytes, &tm.w[gb], kb * 64, n0, fb);
-        } else {
-          const int l = kb - a.nkb_main;
-          const int h = silu ? l / a.nkb_r : 0;
-          const int j = silu ? l % a.nkb_r : l;
-          tma_load_2d_pair(sa, &tm.t, a.g[silu ? h : g].t_col + j * 64, m0, fb);
-          // silu: the other group's adapter rows are read past the end (zeros)
-          const int row = (silu && h != static_cast<int>(rank)) ? a.g[gb].b_rows : n0;
-          tma_load_2d_pair(sa + kHalfBytes, &tm.b[gb], j * 64, row, fb);
-        }
+        load_a(kb, sa, fb);
+        load_b(kb, sa + kHalfBytes, fb);
       }
     }
+    if (pre == 0) pdl_wait();   // no tile for this pair: still order after the writer
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer (leader)
     const uint32_t idesc = idesc_f32acc(kTile, kTile, false);
@@ -181,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    pdl_wait();
     const int quarter = warp & 3;
     const int i = quarter * 32 + lane;
     int lt = 0;
@@ -294,13 +324,9 @@ uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = l.smem_bytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  cfg.numAttrs = launch_attrs(attr, 2, 1, 1);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
   PairParams pp;
   std::memcpy(&pp, l.params, sizeof(pp));
   void* args[2] = {const_cast<TensorMaps*>(&l.tm), &pp};

@@ -28,6 +28,9 @@
 // scratch, no atomics, no spin waits).
 #include <algorithm>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
 #include <type_traits>
 
 #include "common.cuh"
@@ -114,6 +117,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_trigger();
 
   const int nkb_lora = silu ? 2 * a.nkb_r : a.nkb_r;
   const int nkb = a.nkb_main + nkb_lora;
@@ -123,24 +127,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
-    for (int kb = kb0; kb < kb1; ++kb, ++issued) {
-      const int s = issued % p.stages;
-      const uint32_t ph = (issued / p.stages) & 1u;
-      if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u)) {
-        *abort_flag = 1;
-        raise_status(a.status, kDevTimeout);
-        break;
-      }
-      if (*abort_flag) break;
-      const uint32_t sp = smem_u32(smem + s * st_bytes);
-      const uint32_t sq = sp + p_bytes;
-      const uint32_t fb = smem_u32(&full[s]);
-      mbar_arrive_expect_tx(fb, p_bytes + q_bytes);
-      const uint32_t s_tok = kSwap ? sq : sp;
-      const uint32_t s_feat = kSwap ? sp : sq;
+    // The weight (feature) operand of the first stages is constant: issue it
+    // before waiting for the kernel that writes the activations.
+    auto load_feat = [&](int kb, uint32_t s_feat, uint32_t fb) {
       if (kb < a.nkb_main) {
         const int kc = kb * kBKe;
-        tma_load_2d(s_tok, &tm.x, kc, tok0, fb);
         if (silu) {
           tma_load_2d(s_feat, &tm.w[0], kc, feat0, fb);
           tma_load_2d(s_feat + kHalfP * kRowBytes, &tm.w[1], kc, feat0, fb);
@@ -151,7 +142,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int l = kb - a.nkb_main;
         const int h = silu ? l / a.nkb_r : 0;           // silu: 0 = gate block, 1 = up block
         const int j = silu ? l % a.nkb_r : l;
-        tma_load_2d(s_tok, &tm.t, a.g[silu ? h : g].t_col + j * kBKe, tok0, fb);
         if (silu) {
           // the other half's adapter rows are read past the end: zeros
           tma_load_2d(s_feat, &tm.b[0], j * kBKe, h == 0 ? feat0 : a.g[0].b_rows, fb);
@@ -161,6 +151,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(s_feat, &tm.b[g], j * kBKe, feat0, fb);
         }
       }
+    };
+    auto load_tok = [&](int kb, uint32_t s_tok, uint32_t fb) {
+      if (kb < a.nkb_main) {
+        tma_load_2d(s_tok, &tm.x, kb * kBKe, tok0, fb);
+      } else {
+        const int l = kb - a.nkb_main;
+        const int h = silu ? l / a.nkb_r : 0;
+        const int j = silu ? l % a.nkb_r : l;
+        tma_load_2d(s_tok, &tm.t, a.g[silu ? h : g].t_col + j * kBKe, tok0, fb);
+      }
+    };
+    const int pre = min(p.stages, kb1 - kb0);
+    for (int q = 0; q < pre; ++q) {
+      const uint32_t sp = smem_u32(smem + q * st_bytes);
+      const uint32_t fb = smem_u32(&full[q]);
+      mbar_arrive_expect_tx(fb, p_bytes + q_bytes);
+      load_feat(kb0 + q, kSwap ? sp : sp + p_bytes, fb);
+    }
+    pdl_wait();
+    for (int q = 0; q < pre; ++q) {
+      const uint32_t sp = smem_u32(smem + q * st_bytes);
+      load_tok(kb0 + q, kSwap ? sp + p_bytes : sp, smem_u32(&full[q]));
+    }
+    issued = pre;
+    for (int kb = kb0 + pre; kb < kb1; ++kb, ++issued) {
+      const int s = issued % p.stages;
+      const uint32_t ph = (issued / p.stages) & 1u;
+      if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u)) {
+        *abort_flag = 1;
+        raise_status(a.status, kDevTimeout);
+        break;
+      }
+      if (*abort_flag) break;
+      const uint32_t sp = smem_u32(smem + s * st_bytes);
+      const uint32_t fb = smem_u32(&full[s]);
+      mbar_arrive_expect_tx(fb, p_bytes + q_bytes);
+      load_feat(kb, kSwap ? sp : sp + p_bytes, fb);
+      load_tok(kb, kSwap ? sp + p_bytes : sp, fb);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -192,6 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;            // TMEM lanes this warp may read
     const int i = quarter * 32 + lane;       // accumulator row
+    pdl_wait();
     const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(accum), 0));
     if (!ok && lane == 0) {
       *abort_flag = 1;
@@ -327,6 +356,37 @@ void* pick_kernel(uno_dtype dt, bool swap) {
 
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
+// How many clusters of `cluster` CTAs (cluster along z) of kernel `fn` with
+// `smem` bytes of dynamic shared memory the GPU can hold at once (cached).
+int64_t max_active_clusters(void* fn, int cluster, int smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<void*, int, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(fn, cluster, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(1, 1, cluster);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = cluster;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 1 << 20;   // unknown: do not restrict
+    }
+  }
+  cache[key] = n;
+  return n;
+}
+
 int pow2_at_least(int v) {
   int c = 32;
   while (c < v) c <<= 1;
@@ -404,7 +464,10 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   const bool swap = M <= 256 || pb.mode == kEpiRowScale;
   int bn, tok_tiles;
   if (swap) {
-    tok_tiles = static_cast<int>((M + 255) / 256);
+    // decode batches: one token tile of up to 256; down-projections of large
+    // batches: 128-token tiles (two CTAs per SM, more tiles to spread)
+    const int tile = M <= 256 ? 256 : 128;
+    tok_tiles = static_cast<int>((M + tile - 1) / tile);
     bn = round_up(static_cast<int>((M + tok_tiles - 1) / tok_tiles), 16);
   } else {
     tok_tiles = static_cast<int>((M + kTileP - 1) / kTileP);
@@ -422,7 +485,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   // Shared memory: ~96 KB (two or three CTAs per SM) for narrow decode tiles,
   // ~200 KB otherwise.
   const uint32_t st = stage_bytes_for(bn);
-  const bool narrow = bn <= 64;
+  const bool narrow = bn <= 64 || (swap && M > 256);
   const uint32_t budget = narrow ? 96u * 1024u : 200u * 1024u;
   int stages = std::min<int>(kMaxStages, static_cast<int>(budget / st));
   stages = std::max(stages, 2);
@@ -437,6 +500,13 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
     splits = static_cast<int>(std::min<int64_t>(8, capacity / tiles));
     splits = std::max(1, std::min(splits, nkb / 2));
   }
+  // every cluster of the launch must be resident at once: cap the split by
+  // the number of clusters of that size the GPU can hold
+  while (splits > 1 &&
+         max_active_clusters(pick_kernel(pb.dt, swap), splits,
+                             static_cast<int>(stages * st + 1024 + 64 + 16 * (2 * stages + 1))) <
+             tiles)
+    --splits;
   int kb_per = (nkb + splits - 1) / splits;
   splits = (nkb + kb_per - 1) / kb_per;   // every split gets >= 1 K-block
   // the split-K partial tile (and the silu hand-over) must fit in the stage ring
@@ -499,15 +569,9 @@ uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream) {
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = l.smem_bytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  if (l.splits > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = l.splits;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
+  cudaLaunchAttribute attr[2];
+  cfg.numAttrs = launch_attrs(attr, 1, 1, static_cast<unsigned>(l.splits));
+  cfg.attrs = attr;
   Gemm1Params gp;
   std::memcpy(&gp, l.params, sizeof(gp));
   void* args[2] = {const_cast<TensorMaps*>(&l.tm), &gp};

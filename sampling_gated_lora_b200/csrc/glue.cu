@@ -13,6 +13,8 @@ constexpr int kNormThreads = 256;
 __global__ void __launch_bounds__(kNormThreads)
     rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y, int D,
                    float eps) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
   const size_t row = blockIdx.x;
   const __nv_bfloat16* xr = x + row * D;
   __nv_bfloat16* yr = y + row * D;
@@ -69,6 +71,8 @@ __device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.0f +
 __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
                                 const __nv_bfloat16* __restrict__ b,
                                 __nv_bfloat16* __restrict__ y, int64_t n) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
   const int64_t nv = n / 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
@@ -95,10 +99,9 @@ __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
 uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
                           cudaStream_t s) {
   if (M == 0) return UNO_OK;
-  rmsnorm_kernel<<<static_cast<unsigned>(M), kNormThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), static_cast<int>(D),
-      eps);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_kernel(
+      rmsnorm_kernel, dim3(static_cast<unsigned>(M)), dim3(kNormThreads), 0, s, 1,
+      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), static_cast<int>(D), eps);
   return e == cudaSuccess ? UNO_OK : cuda_error(e, "rmsnorm launch");
 }
 
@@ -107,10 +110,10 @@ uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cud
   const int threads = 256;
   const int64_t want = (n / 8 + threads - 1) / threads + 1;
   const int blocks = static_cast<int>(std::min<int64_t>(want, 16 * device_sm_count()));
-  silu_mul_kernel<<<blocks, threads, 0, s>>>(static_cast<const __nv_bfloat16*>(a),
-                                             static_cast<const __nv_bfloat16*>(b),
-                                             static_cast<__nv_bfloat16*>(y), n);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_kernel(silu_mul_kernel, dim3(blocks), dim3(threads), 0, s, 1,
+                                      static_cast<const __nv_bfloat16*>(a),
+                                      static_cast<const __nv_bfloat16*>(b),
+                                      static_cast<__nv_bfloat16*>(y), n);
   return e == cudaSuccess ? UNO_OK : cuda_error(e, "silu_mul launch");
 }
 

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -122,5 +123,42 @@ uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float ep
 uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s);
 
 int device_sm_count();
+
+// Launch attributes shared by every kernel launch: programmatic stream
+// serialisation (unless UNO_PDL=0 in the environment) and, when cluster_x *
+// cluster_y * cluster_z > 1, the cluster shape. Returns the attribute count.
+bool pdl_enabled();
+inline int launch_attrs(cudaLaunchAttribute (&attr)[2], unsigned cluster_x = 1,
+                        unsigned cluster_y = 1, unsigned cluster_z = 1) {
+  int n = 0;
+  if (cluster_x * cluster_y * cluster_z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = cluster_y;
+    attr[n].val.clusterDim.z = cluster_z;
+    ++n;
+  }
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  return n;
+}
+
+// Launch a kernel on `s` with the library's launch attributes (see launch_attrs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  cfg.numAttrs = launch_attrs(attr, cluster_x, 1, 1);
+  cfg.attrs = attr;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 }  // namespace uno

@@ -98,6 +98,8 @@ template <typename T>
 __global__ void __launch_bounds__(kStatThreads)
     row_stats_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits, int rows_p,
                      int V, int chunk_len, float c, float2* __restrict__ stats) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.y;
   const T* z = row < rows_p ? p_logits + static_cast<size_t>(row) * V
                             : q_logits + static_cast<size_t>(row - rows_p) * V;
@@ -349,6 +351,8 @@ __global__ void __launch_bounds__(kDrawThreads)
   __shared__ int s_n, s_bad, s_nan;
   __shared__ float s_stat[4];   // Mp, Sp, Mq, Sq of the drawing row(s)
 
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
   const uint32_t nrank = cluster_nctarank();
   const uint32_t rank = cluster_ctarank();
   const int b = blockIdx.x / nrank;
@@ -478,6 +482,8 @@ __global__ void __launch_bounds__(kDrawThreads)
   __shared__ DrawSmem sh;
   __shared__ float s_max;
   __shared__ float s_cmax[kDrawThreads / 32];
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
   const uint32_t nrank = cluster_nctarank();
   const uint32_t rank = cluster_ctarank();
   const int row = blockIdx.x / nrank;
@@ -538,6 +544,8 @@ __global__ void __launch_bounds__(kDrawThreads)
 
 __global__ void philox_kernel(uint64_t seed, uint64_t step, uint32_t stream, uint32_t index0,
                               int64_t n, uint32_t* words, float* u) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint32_t w = philox_word0(seed, step, stream, index0 + static_cast<uint32_t>(i));
@@ -568,13 +576,9 @@ uno_status launch_cluster(Kern kern, int grid, int cluster, size_t smem, cudaStr
   cfg.blockDim = dim3(kDrawThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  cfg.numAttrs = launch_attrs(attr, static_cast<unsigned>(cluster), 1, 1);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, kern, args...);
   if (e != cudaSuccess) return cuda_error(e, "sampler launch");
   return UNO_OK;
@@ -623,16 +627,17 @@ uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s) {
   fp.chunk_elems = chunk_elems;
   const size_t smem = static_cast<size_t>(chunk_elems) * esz * 2;
   const dim3 grid(chunks, rows);
+  cudaError_t e;
   if (a.dt == UNO_F32) {
-    row_stats_kernel<float><<<grid, kStatThreads, 0, s>>>(
-        static_cast<const float*>(a.p_logits), static_cast<const float*>(a.q_logits),
-        a.B * a.k_p, a.V, chunk_len, c, stats);
+    e = launch_kernel(row_stats_kernel<float>, grid, dim3(kStatThreads), 0, s, 1,
+                      static_cast<const float*>(a.p_logits), static_cast<const float*>(a.q_logits),
+                      a.B * a.k_p, a.V, chunk_len, c, stats);
   } else {
-    row_stats_kernel<__nv_bfloat16><<<grid, kStatThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(a.p_logits),
-        static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.k_p, a.V, chunk_len, c, stats);
+    e = launch_kernel(row_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1,
+                      static_cast<const __nv_bfloat16*>(a.p_logits),
+                      static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.k_p, a.V, chunk_len,
+                      c, stats);
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_error(e, "row_stats launch");
   if (a.dt == UNO_F32)
     return launch_cluster(verify_finalize_kernel<float>, a.B * cl, cl, smem, s,
@@ -670,9 +675,9 @@ uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint3
   if (n == 0) return UNO_OK;
   const int threads = 256;
   const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 8 * device_sm_count());
-  philox_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(seed, step, stream_id, index0, n,
-                                                             words, u);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_kernel(philox_kernel, dim3(static_cast<unsigned>(blocks)),
+                                      dim3(threads), 0, s, 1, seed, step, stream_id, index0, n,
+                                      words, u);
   if (e != cudaSuccess) return cuda_error(e, "philox launch");
   return UNO_OK;
 }
