@@ -431,7 +431,7 @@ def run_uno(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded random-init weights and hidden states; no attention)",
         "config": workload_config(B, k, T), "clocks": clocks,
-        "gpu_launches": model.kernel_count() * args.steps, "e2e": e2e, "roofline": roof,
+        "gpu_launches": model.kernel_count(B, k) * args.steps, "e2e": e2e, "roofline": roof,
         "mean_accepted": round(float(acc[args.warmup:n_total].float().mean()), 3),
         "device_status": st,
     }

@@ -218,8 +218,9 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
                         int32_t* accepted_len, int32_t* out_tokens, int32_t* out_count,
                         int32_t* dev_status, void* workspace, size_t ws_bytes, void* stream);
 
-/* Number of kernel launches one uno_psi_step call of this model issues. */
-int32_t uno_psi_step_kernel_count(const uno_model* m);
+/* Number of kernel launches one uno_psi_step call with this (B, k) issues;
+ * 0 until such a step has been run (the launch plan is built on first use). */
+int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k);
 
 /* ---------------------------------------------------------------------------
  * The step's glue operations, exposed for testing (all bf16, device):

@@ -80,7 +80,7 @@ def load():
         "uno_psi_step_workspace": (sz, [vp, i32, i32]),
         "uno_psi_step": (i32, [vp, i32, i32, vp, vp, vp, f32, u64, u64, u64, vp, vp, vp, vp, vp,
                                vp, vp, vp, sz, vp]),
-        "uno_psi_step_kernel_count": (i32, [vp]),
+        "uno_psi_step_kernel_count": (i32, [vp, i32, i32]),
         "uno_rmsnorm": (i32, [i64, i64, vp, vp, f32, vp]),
         "uno_silu_mul": (i32, [i64, vp, vp, vp, vp]),
     }
@@ -312,9 +312,9 @@ class Model:
     def workspace_bytes(self, B, k):
         return load().uno_psi_step_workspace(self._h, B, k)
 
-    def kernel_count(self):
-        """Kernel launches issued by one step."""
-        return load().uno_psi_step_kernel_count(self._h)
+    def kernel_count(self, B, k):
+        """Kernel launches issued by one step for (B, k) (0 before the first such step)."""
+        return load().uno_psi_step_kernel_count(self._h, B, k)
 
     def step(self, B, k, h_in, q_prev, d_prev, temperature, seed, step, q_next, d_next,
              accepted_len, out_tokens, out_count, workspace, logits_out=None, dev_status=None,

@@ -160,12 +160,6 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
                      ws_bytes);
   void* t_buf = r > 0 ? static_cast<char*>(workspace) + L.t_off : nullptr;
   GemmLaunch down, main;
-  if (r > 0) {
-    const void* As[1] = {A};
-    if ((s = gemm_prepare(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), &down)) !=
-        UNO_OK)
-      return s;
-  }
   GemmProblem pm{};
   pm.dt = dt;
   pm.M = M;
@@ -176,10 +170,20 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   pm.ldt = r;
   pm.ngroups = 1;
   pm.g[0] = GemmGroup{W, Bl, N, y, N, 0};
+  pm.A[0] = A;
   pm.mode = kEpiStore;
   pm.M0 = M;
+  pm.gate = gate;
+  pm.scale = scale;
+  const bool fused = r > 0 && gemm_dec_suits(pm);
+  if (r > 0 && !fused) {
+    const void* As[1] = {A};
+    if ((s = gemm_prepare(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), &down)) !=
+        UNO_OK)
+      return s;
+  }
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
-  if (r > 0 && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
+  if (r > 0 && !fused && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
   return gemm_run(main, as_stream(stream));
 }
 
@@ -216,9 +220,6 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   if (r > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
     return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
   GemmLaunch down, main;
-  if (r > 0 && (s = gemm_prepare(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, workspace),
-                                 &down)) != UNO_OK)
-    return s;
   GemmProblem pm{};
   pm.dt = dt;
   pm.M = M;
@@ -231,10 +232,18 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   for (int i = 0; i < G; ++i)
     pm.g[i] = GemmGroup{W[i], r > 0 ? Bl[i] : nullptr, N[i], mode == 1 ? y[0] : y[i],
                         mode == 1 ? N[0] : N[i], static_cast<int64_t>(i) * r};
+  for (int i = 0; i < G; ++i) pm.A[i] = r > 0 ? A[i] : nullptr;
   pm.mode = mode == 1 ? kEpiSiluPair : kEpiStore;
   pm.M0 = M;
+  pm.gate = gate;
+  pm.scale = scale;
+  const bool fused = r > 0 && gemm_dec_suits(pm);
+  if (r > 0 && !fused &&
+      (s = gemm_prepare(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, workspace), &down)) !=
+          UNO_OK)
+    return s;
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
-  if (r > 0 && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
+  if (r > 0 && !fused && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
   return gemm_run(main, as_stream(stream));
 }
 
@@ -464,12 +473,9 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
   auto linear = [&](const void* x, int64_t K, int G, const int* which, int layer, void* const* y,
                     const int64_t* ldy, int mode, void* y1, int64_t M0) -> uno_status {
     uno_status s;
-    const void* As[kMaxGroups];
+    const void* As[kMaxGroups] = {nullptr, nullptr, nullptr};
     for (int i = 0; i < G; ++i)
       As[i] = layer >= 0 ? m->wp(layer, which[i], 1) : m->head(1);
-    if (r > 0 && (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) !=
-                     UNO_OK)
-      return s;
     GemmProblem pm{};
     pm.dt = UNO_BF16;
     pm.M = M;
@@ -498,6 +504,13 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     pm.mode = mode;
     pm.y1 = y1;
     pm.M0 = M0;
+    pm.gate = nullptr;
+    pm.gate_row0 = Mv;
+    pm.scale = m->scale;
+    for (int i = 0; i < G; ++i) pm.A[i] = r > 0 ? As[i] : nullptr;
+    if (r > 0 && !gemm_dec_suits(pm) &&
+        (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
+      return s;
     return gemm(pm);
   };
   uno_status s;
@@ -609,12 +622,15 @@ size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k) {
   return step_layout(m, B, k).total;
 }
 
-int32_t uno_psi_step_kernel_count(const uno_model* m) {
-  if (!m) return 0;
-  // per layer: 2 rmsnorm + 4 GEMM launches (+ 4 down-projections when r > 0);
-  // then rmsnorm + LM head (+ its down-projection); verify (2 kernels) + draft (1)
-  const int per_gemm = m->r > 0 ? 2 : 1;
-  return m->n_layers * (2 + 4 * per_gemm) + 1 + per_gemm + 3;
+int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k) {
+  if (!m || B < 1 || k < 1) return 0;
+  // per layer: 2 rmsnorm + 4 GEMM launches, each with a separate
+  // down-projection launch unless the fused decode kernel takes it; then
+  // rmsnorm + LM head; verify (2 kernels) + draft (1)
+  std::lock_guard<std::mutex> lock(const_cast<uno_model*>(m)->mu);
+  for (const auto& p : m->plans)
+    if (p->B == B && p->k == k) return static_cast<int32_t>(p->ops.size()) + 3;
+  return 0;
 }
 
 uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, const void* q_prev,

@@ -450,6 +450,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   if (pb.mode == kEpiSiluPair && (pb.ngroups != 2 || pb.g[0].N != pb.g[1].N))
     return set_error(UNO_ERR_INVALID_ARG, "silu-pair needs two groups of equal width");
   if (gemm_pair_suits(pb)) return gemm_pair_prepare(pb, out);
+  if (gemm_dec_suits(pb)) return gemm_dec_prepare(pb, out);
   if (pb.mode == kEpiSiluPair && pb.M > 256)
     return set_error(UNO_ERR_UNSUPPORTED, "silu-pair with M > 256 needs the bf16 pair kernel");
   const int esz = pb.dt == UNO_F32 ? 4 : 2;
@@ -560,6 +561,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
 
 uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream) {
   if (l.kind == 1) return gemm_pair_run(l, stream);
+  if (l.kind == 2) return gemm_dec_run(l, stream);
   void* fn = pick_kernel(static_cast<uno_dtype>(l.dtype), l.swap != 0);
   cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, l.smem_bytes);

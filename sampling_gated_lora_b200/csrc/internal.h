@@ -42,6 +42,7 @@ struct GemmGroup {
 // Group 0 rows m >= M0 are written to y1 (row m - M0) instead of y_0.
 struct GemmProblem {
   uno_dtype dt;
+  const void* A[kMaxGroups];   // adapters' A [r, K]: lets a decode-size launch fuse the down-projection
   int64_t M, K;
   int32_t r;              // LoRA rank per group (0: no LoRA term)
   const void* x;          // [M, K]
@@ -58,8 +59,9 @@ struct GemmProblem {
 };
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
+// a[] (the adapters' A matrices) is used by the fused decode kernel only.
 struct TensorMaps {
-  CUtensorMap x, t, w[kMaxGroups], b[kMaxGroups];
+  CUtensorMap x, t, w[kMaxGroups], b[kMaxGroups], a[kMaxGroups];
 };
 
 // Cached launch of a GemmProblem (tensor maps + grid); valid while the
@@ -84,6 +86,11 @@ uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t in
 bool gemm_pair_suits(const GemmProblem& pb);
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
+// The fused decode kernel (bf16, M <= 256, r <= 128): computes t = scale * gate
+// * (x A^T) in the same launch, so no separate down-projection is needed.
+bool gemm_dec_suits(const GemmProblem& pb);
+uno_status gemm_dec_prepare(const GemmProblem& pb, GemmLaunch* out);
+uno_status gemm_dec_run(const GemmLaunch& l, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sampler
 

@@ -122,7 +122,7 @@ def test_model_create_validates():
     st = L.uno_psi_step(h, 2, 4, None, None, None, 1.0, 0, 0, 0, None, None, None, None, None,
                         None, None, None, 0, None)
     assert st == 1
-    assert L.uno_psi_step_kernel_count(h) == 1 * (2 + 8) + 1 + 2 + 3
+    assert L.uno_psi_step_kernel_count(h, 2, 4) == 0      # no plan before a first step
     L.uno_model_destroy(h)
 
 
