@@ -176,6 +176,7 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   pm.gate = gate;
   pm.scale = scale;
   const bool fused = r > 0 && gemm_dec_suits(pm);
+  pm.x_ready = r > 0 && !fused;
   if (r > 0 && !fused) {
     const void* As[1] = {A};
     if ((s = gemm_prepare(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), &down)) !=
@@ -238,6 +239,7 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   pm.gate = gate;
   pm.scale = scale;
   const bool fused = r > 0 && gemm_dec_suits(pm);
+  pm.x_ready = r > 0 && !fused;
   if (r > 0 && !fused &&
       (s = gemm_prepare(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, workspace), &down)) !=
           UNO_OK)
@@ -508,7 +510,8 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     pm.gate_row0 = Mv;
     pm.scale = m->scale;
     for (int i = 0; i < G; ++i) pm.A[i] = r > 0 ? As[i] : nullptr;
-    if (r > 0 && !gemm_dec_suits(pm) &&
+    pm.x_ready = r > 0 && !gemm_dec_suits(pm);
+    if (pm.x_ready &&
         (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
       return s;
     return gemm(pm);

@@ -31,6 +31,7 @@ struct GemmArgs {
   void* y1;
   const uint8_t* gate;
   int32_t* status;
+  int x_ready;    // x complete at launch: wait for the predecessor only before reading t
   GroupArgs g[kMaxGroups];
 };
 
@@ -50,6 +51,7 @@ inline GemmArgs make_gemm_args(const GemmProblem& pb, int tile_n, int row_bytes)
   a.y1 = pb.y1;
   a.gate = pb.gate;
   a.status = nullptr;
+  a.x_ready = pb.x_ready ? 1 : 0;
   int tiles = 0;
   for (int i = 0; i < pb.ngroups; ++i) {
     a.g[i].y = pb.g[i].y;

@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool ok = true;
     int pre = 0;   // k-blocks of the first tile whose W half went out early
+    bool waited = false;
     for (int tile = pair; ok && tile < p.num_tiles; tile += num_pairs) {
       const int mb = tile % p.tiles_m, ft = tile / p.tiles_m;
       const int g = group_of(a, ft);
@@ -149,9 +150,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (leader) mbar_arrive_expect_tx(smem_u32(&full[q]), 2 * kStageBytes);
           load_b(q, sa + kHalfBytes, map_shared_rank(smem_u32(&full[q]), 0));
         }
-        pdl_wait();
-        for (int q = 0; q < pre; ++q)
+        if (!a.x_ready) {
+          pdl_wait();
+          waited = true;
+        }
+        for (int q = 0; q < pre; ++q) {
+          if (!waited && q >= a.nkb_main) {
+            pdl_wait();
+            waited = true;
+          }
           load_a(q, smem_u32(smem + q * kStageBytes), map_shared_rank(smem_u32(&full[q]), 0));
+        }
         it = pre;
       }
       for (int kb = (tile == pair) ? pre : 0; kb < nkb; ++kb, ++it) {
@@ -165,11 +174,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = map_shared_rank(smem_u32(&full[s]), 0);
         if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * kStageBytes);
         const uint32_t sa = smem_u32(smem + s * kStageBytes);
+        if (!waited && kb >= a.nkb_main) {
+          pdl_wait();
+          waited = true;
+        }
         load_a(kb, sa, fb);
         load_b(kb, sa + kHalfBytes, fb);
       }
     }
-    if (pre == 0) pdl_wait();   // no tile for this pair: still order after the writer
+    if (!waited) pdl_wait();
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer (leader)
     const uint32_t idesc = idesc_f32acc(kTile, kTile, false);
@@ -210,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    pdl_wait();
+    if (!a.x_ready) pdl_wait();
     const int quarter = warp & 3;
     const int i = quarter * 32 + lane;
     int lt = 0;

@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) pdl_trigger();
+  if (threadIdx.x == 0 && a.mode != kEpiRowScale) pdl_trigger();
 
   const int nkb_lora = silu ? 2 * a.nkb_r : a.nkb_r;
   const int nkb = a.nkb_main + nkb_lora;
@@ -162,6 +162,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_load_2d(s_tok, &tm.t, a.g[silu ? h : g].t_col + j * kBKe, tok0, fb);
       }
     };
+    // Down-projections (kEpiRowScale) let their dependent start only once
+    // they have waited for the writer of their own input; a main GEMM so
+    // launched (x_ready) reads x at once and waits only before reading t.
+    const bool down = a.mode == kEpiRowScale;
+    bool waited = false;
+    auto wait_pred = [&]() {
+      if (!waited) {
+        pdl_wait();
+        waited = true;
+        if (down) pdl_trigger();
+      }
+    };
     const int pre = min(p.stages, kb1 - kb0);
     for (int q = 0; q < pre; ++q) {
       const uint32_t sp = smem_u32(smem + q * st_bytes);
@@ -169,10 +181,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_arrive_expect_tx(fb, p_bytes + q_bytes);
       load_feat(kb0 + q, kSwap ? sp : sp + p_bytes, fb);
     }
-    pdl_wait();
     for (int q = 0; q < pre; ++q) {
+      const int kb = kb0 + q;
+      if (!a.x_ready || kb >= a.nkb_main) wait_pred();
       const uint32_t sp = smem_u32(smem + q * st_bytes);
-      load_tok(kb0 + q, kSwap ? sp + p_bytes : sp, smem_u32(&full[q]));
+      load_tok(kb, kSwap ? sp + p_bytes : sp, smem_u32(&full[q]));
     }
     issued = pre;
     for (int kb = kb0 + pre; kb < kb1; ++kb, ++issued) {
@@ -188,8 +201,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t fb = smem_u32(&full[s]);
       mbar_arrive_expect_tx(fb, p_bytes + q_bytes);
       load_feat(kb, kSwap ? sp : sp + p_bytes, fb);
+      if (kb >= a.nkb_main) wait_pred();
       load_tok(kb, kSwap ? sp + p_bytes : sp, fb);
     }
+    if (down) wait_pred();   // a CTA with no K-blocks still triggers
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_f32acc(kTileP, bn, kTf32);
@@ -220,7 +235,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;            // TMEM lanes this warp may read
     const int i = quarter * 32 + lane;       // accumulator row
-    pdl_wait();
+    if (!a.x_ready) pdl_wait();
     const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(accum), 0));
     if (!ok && lane == 0) {
       *abort_flag = 1;

@@ -56,6 +56,10 @@ struct GemmProblem {
   const uint8_t* gate;    // kEpiRowScale; NULL: gate[m] = (m >= gate_row0)
   int64_t gate_row0;
   float scale;            // kEpiRowScale
+  // The launch right before this one is the down-projection that writes t and
+  // only triggers its dependents once the writer of x has finished: x may be
+  // read at once, and only t must wait (so the two launches overlap).
+  bool x_ready;
 };
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
