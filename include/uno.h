@@ -145,6 +145,35 @@ uno_status uno_psi_verify(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32
                           int32_t* dev_status, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * uno_psi_verify without a workspace: a library addition, the pages have no
+ * counterpart. For callers that cannot allocate device memory where they
+ * verify (cudaMalloc/cudaFree may synchronise the whole device and stall a
+ * decode loop; some host runtimes own no device allocator).
+ *
+ *   Arguments, checks, kernels and results: those of uno_psi_verify, with the
+ *   stats scratch taken from a 2 MiB static device array inside the library
+ *   (one per device) instead of a workspace.
+ *   Limit: uno_psi_verify_workspace(B, k, k_p, V) <= 2 MiB, which holds
+ *     B * (k_p + k) <= 262144 logit rows; larger calls return
+ *     UNO_ERR_UNSUPPORTED and launch nothing.
+ *   Setup: the first call on a device (the current device, which must own
+ *     the buffers and the stream) looks up the array's device address, which
+ *     may load the library's module; make that first call before any stream
+ *     capture begins. Later calls do no setup.
+ *   Starting values: none needed; every entry a call reads it wrote itself.
+ *   Concurrency: all calls on one device share the array. Calls on one stream
+ *     are ordered and safe; calls whose kernels may overlap (other streams
+ *     without ordering, other host threads) race on it and give wrong results.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * ------------------------------------------------------------------------- */
+uno_status uno_psi_verify_noalloc(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32_t V,
+                                  const void* p_logits, const void* q_logits,
+                                  const int32_t* draft, float temperature, uint64_t seed,
+                                  uint64_t step, uint64_t seq_offset, int32_t* accepted_len,
+                                  int32_t* out_tokens, int32_t* out_count, int32_t* dev_status,
+                                  void* stream);
+
+/* ---------------------------------------------------------------------------
  * Linear-sampler draft (hyper.ai page, section "方法": the linear sampler
  * draws one candidate block from the per-position marginals):
  *   draft[b,j] = smallest v with C(v) > u0 * C(V-1), C the inclusive

@@ -29,7 +29,7 @@ EXPORTS = [
     "uno_last_error", "uno_version", "uno_device_status",
     "uno_gated_lora_linear_workspace", "uno_gated_lora_linear",
     "uno_gated_lora_linear_group_workspace", "uno_gated_lora_linear_group",
-    "uno_psi_verify_workspace", "uno_psi_verify",
+    "uno_psi_verify_workspace", "uno_psi_verify", "uno_psi_verify_noalloc",
     "uno_draft_sample_workspace", "uno_draft_sample",
     "uno_philox_uniforms",
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
@@ -72,6 +72,8 @@ def load():
         "uno_psi_verify_workspace": (sz, [i32, i32, i32, i32]),
         "uno_psi_verify": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, f32, u64, u64, u64, vp, vp,
                                  vp, vp, vp, sz, vp]),
+        "uno_psi_verify_noalloc": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, f32, u64, u64, u64,
+                                         vp, vp, vp, vp, vp]),
         "uno_draft_sample_workspace": (sz, [i32, i32, i32]),
         "uno_draft_sample": (i32, [i32, i32, i32, i32, vp, f32, u64, u64, u64, vp, vp, vp, sz, vp]),
         "uno_philox_uniforms": (i32, [u64, u64, u32, u32, i64, vp, vp, vp]),
@@ -214,6 +216,28 @@ def psi_verify(p_logits, q_logits, draft, temperature, seed, step, seq_offset=0,
                             _ptr(draft), float(temperature), int(seed), int(step), int(seq_offset),
                             _ptr(accepted_len), _ptr(out_tokens), _ptr(out_count),
                             _ptr(dev_status), _ptr(ws), wsb, _stream(stream)))
+    return accepted_len, out_tokens, out_count
+
+
+def psi_verify_noalloc(p_logits, q_logits, draft, temperature, seed, step, seq_offset=0,
+                       accepted_len=None, out_tokens=None, out_count=None, dev_status=None,
+                       stream=None):
+    """psi_verify with the library's static stats scratch (no workspace argument)."""
+    torch = _torch()
+    L = load()
+    B, k_p, V = p_logits.shape
+    k = q_logits.shape[1]
+    dev = p_logits.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    accepted_len = torch.empty(B, **i32) if accepted_len is None else accepted_len
+    out_tokens = torch.empty((B, k + 1), **i32) if out_tokens is None else out_tokens
+    out_count = torch.empty(B, **i32) if out_count is None else out_count
+    _dev(p_logits, q_logits, draft, accepted_len, out_tokens, out_count, dev_status)
+    _check(L.uno_psi_verify_noalloc(_dtype(p_logits), B, k, k_p, V, _ptr(p_logits),
+                                    _ptr(q_logits), _ptr(draft), float(temperature), int(seed),
+                                    int(step), int(seq_offset), _ptr(accepted_len),
+                                    _ptr(out_tokens), _ptr(out_count), _ptr(dev_status),
+                                    _stream(stream)))
     return accepted_len, out_tokens, out_count
 
 

@@ -25,6 +25,7 @@
 #include <algorithm>
 #include <cfloat>
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -683,3 +684,72 @@ uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint3
 }
 
 }  // namespace uno
+
+// ---------------------------------------------------------------- verify without allocation
+//
+// uno_psi_verify_noalloc keeps the per-(logit row, vocab chunk) stats in a
+// static device array of this file instead of a caller workspace. It serves
+// callers that cannot allocate device memory where they verify: a decode loop
+// that must not stall on the device-wide synchronisation cudaMalloc/cudaFree
+// may cause, or a host runtime that owns the logits and output buffers but no
+// device allocator. The pages describe no such variant.
+namespace uno {
+namespace {
+
+constexpr size_t kNoAllocStatsBytes = size_t{2} << 20;   // 2 MiB: 262,144 (m, s) pairs
+constexpr int kNoAllocMaxDevices = 64;
+
+// Every entry a call reads is written earlier in the same call (row stats
+// kernel before the finalize kernel, ordered on one stream), so the array
+// needs no starting value and is never cleared.
+static __device__ __align__(256) float2 g_noalloc_stats[kNoAllocStatsBytes / sizeof(float2)];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_stats on the current device; looked up once per
+// device (the lookup may load this library's module onto the device).
+uno_status noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return set_error(UNO_ERR_UNSUPPORTED, "device %d: the static verify scratch serves devices 0..%d",
+                     dev, kNoAllocMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_stats);
+    if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress of the static verify scratch");
+    if (!p) return set_error(UNO_ERR_CUDA, "static verify scratch has a NULL device address");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return UNO_OK;
+}
+
+}  // namespace
+}  // namespace uno
+
+extern "C" uno_status uno_psi_verify_noalloc(uno_dtype dt, int32_t B, int32_t k, int32_t k_p,
+                                             int32_t V, const void* p_logits,
+                                             const void* q_logits, const int32_t* draft,
+                                             float temperature, uint64_t seed, uint64_t step,
+                                             uint64_t seq_offset, int32_t* accepted_len,
+                                             int32_t* out_tokens, int32_t* out_count,
+                                             int32_t* dev_status, void* stream) {
+  using namespace uno;
+  const size_t need = uno_psi_verify_workspace(B, k, k_p, V);
+  if (need > kNoAllocStatsBytes)
+    return set_error(UNO_ERR_UNSUPPORTED,
+                     "uno_psi_verify_noalloc: B=%d k=%d k_p=%d V=%d needs %zu bytes of stats "
+                     "scratch, the static scratch holds %zu; call uno_psi_verify with a workspace",
+                     B, k, k_p, V, need, kNoAllocStatsBytes);
+  void* ws = nullptr;
+  const uno_status s = noalloc_scratch(&ws);
+  if (s != UNO_OK) return s;
+  // Argument checks, kernels and results are those of uno_psi_verify.
+  return uno_psi_verify(dt, B, k, k_p, V, p_logits, q_logits, draft, temperature, seed, step,
+                        seq_offset, accepted_len, out_tokens, out_count, dev_status, ws,
+                        kNoAllocStatsBytes, stream);
+}
