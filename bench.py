@@ -239,7 +239,7 @@ def kernel_lines(U, torch, pk):
         x, Wt, A, Bl = dev((M, K), 1), dev((N, K), K ** -0.5), dev((r, K), K ** -0.5), dev((N, r), 0.01)
         g = torch.from_numpy(W.decode_gate(B, 8)).cuda()
         y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        ws = torch.empty(U.load().uno_gated_lora_linear_workspace(0, M, K, N, r), dtype=torch.uint8,
+        ws = torch.zeros(U.load().uno_gated_lora_linear_workspace(0, M, K, N, r), dtype=torch.uint8,
                          device="cuda")
         f = lambda: U.gated_lora_linear(x, Wt, A, Bl, g, 1.0, y=y, workspace=ws)
         f()
@@ -257,7 +257,7 @@ def kernel_lines(U, torch, pk):
         x, Wt, A, Bl = dev((M, K), 1), dev((N, K), K ** -0.5), dev((r, K), K ** -0.5), dev((N, r), 0.01)
         g = torch.cat([torch.zeros(M // 2, dtype=torch.uint8), torch.ones(M // 2, dtype=torch.uint8)]).cuda()
         y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        ws = torch.empty(U.load().uno_gated_lora_linear_workspace(0, M, K, N, r), dtype=torch.uint8,
+        ws = torch.zeros(U.load().uno_gated_lora_linear_workspace(0, M, K, N, r), dtype=torch.uint8,
                          device="cuda")
         f = lambda: U.gated_lora_linear(x, Wt, A, Bl, g, 1.0, y=y, workspace=ws)
         f()
@@ -393,7 +393,7 @@ def run_uno(args):
         lw = layers[0]["up"]
         g = torch.from_numpy(W.step_gate(B, k)).cuda()
         y = torch.empty((M, Nd), dtype=torch.bfloat16, device="cuda")
-        wsl = torch.empty(U.load().uno_gated_lora_linear_workspace(0, M, Kd, Nd, r),
+        wsl = torch.zeros(U.load().uno_gated_lora_linear_workspace(0, M, Kd, Nd, r),
                           dtype=torch.uint8, device="cuda")
         f = lambda: U.gated_lora_linear(x, lw[0], lw[1], lw[2], g, 1.0, y=y, workspace=wsl)
         for _ in range(3):

@@ -78,11 +78,17 @@ uno_status uno_device_status(int32_t* bits_out, int32_t clear, void* stream);
  *   1 = adapter on: the draft path theta_AR + theta_Delta); y [M,N] `dt`.
  *   fp32 accumulation. The rank-r product x A^T is rounded to `dt` before the
  *   up-projection, which runs in the same tensor-core pass as x W^T, so W is
- *   read from HBM once.
+ *   read from HBM once. Decode-size bf16 batches (M <= 128, r <= 128) run in
+ *   one launch that splits K into slices and rounds each slice's x_s A_s^T.
  *   Sizes: M >= 0 (M = 0 launches nothing), K >= 1, N >= 1, 0 <= r <= 256.
  *   bf16: K, N, r multiples of 8; f32: multiples of 4 (16-byte row strides).
  *   f32 inputs run on the tf32 tensor-core path (10-bit mantissa products).
- *   workspace: >= uno_gated_lora_linear_workspace(...) bytes of device memory.
+ *   workspace: >= uno_gated_lora_linear_workspace(...) bytes of device
+ *   memory, 256-byte aligned, ZERO-FILLED before its first use: its first
+ *   64 KiB hold counters of the decode-size path, which every call leaves at
+ *   zero (zero them again after a call that raised a device status bit).
+ *   Required when r > 0; with r = 0 it may be NULL (no decode-size path).
+ *   Calls that share a workspace must not run at the same time.
  * ------------------------------------------------------------------------- */
 size_t uno_gated_lora_linear_workspace(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r);
 
@@ -102,7 +108,8 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
  *
  *   W[i] [N[i],K], A[i] [r,K], Bl[i] [N[i],r], y[i] [M,N[i]], all `dt`
  *   (mode 1: bf16 only); gate [M] uint8; 1 <= G <= 3. Sizes as for
- *   uno_gated_lora_linear. workspace: >= uno_gated_lora_linear_group_workspace.
+ *   uno_gated_lora_linear. workspace: >= uno_gated_lora_linear_group_workspace,
+ *   aligned and zero-filled as for uno_gated_lora_linear.
  * ------------------------------------------------------------------------- */
 size_t uno_gated_lora_linear_group_workspace(uno_dtype dt, int64_t M, int32_t r, int32_t G);
 

@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdlib>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <memory>
 #include <mutex>
@@ -56,10 +57,13 @@ struct LinearLayout {
   size_t t_off, total;
 };
 
-LinearLayout linear_layout(uno_dtype dt, int64_t M, int32_t r) {
+// Workspace of a gated linear: the decode kernel's counters, then t (when the
+// down-projection runs as its own launch) or the decode kernel's data.
+LinearLayout linear_layout(uno_dtype dt, int64_t M, int32_t r, int32_t G = 1) {
   LinearLayout l{};
-  l.t_off = 0;
-  l.total = align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * dt_size(dt));
+  l.t_off = kDecCounterBytes;
+  l.total = kDecCounterBytes + align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * G * dt_size(dt));
+  if (dt == UNO_BF16) l.total = std::max(l.total, gemm_dec_workspace_bound(M, r));
   return l;
 }
 
@@ -161,6 +165,8 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   void* t_buf = r > 0 ? static_cast<char*>(workspace) + L.t_off : nullptr;
   GemmLaunch down, main;
   GemmProblem pm{};
+  pm.scratch = workspace;
+  pm.scratch_bytes = workspace ? ws_bytes : 0;
   pm.dt = dt;
   pm.M = M;
   pm.K = K;
@@ -190,7 +196,7 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
 
 size_t uno_gated_lora_linear_group_workspace(uno_dtype dt, int64_t M, int32_t r, int32_t G) {
   if (M < 0 || r < 0 || G < 1 || G > kMaxGroups) return 0;
-  return align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * G * dt_size(dt));
+  return linear_layout(dt, M, r, G).total;
 }
 
 uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32_t r, int32_t G,
@@ -222,12 +228,15 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
     return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
   GemmLaunch down, main;
   GemmProblem pm{};
+  pm.scratch = workspace;
+  pm.scratch_bytes = workspace ? ws_bytes : 0;
+  void* t_buf = r > 0 ? static_cast<char*>(workspace) + kDecCounterBytes : nullptr;
   pm.dt = dt;
   pm.M = M;
   pm.K = K;
   pm.r = r;
   pm.x = x;
-  pm.t = workspace;
+  pm.t = t_buf;
   pm.ldt = static_cast<int64_t>(G) * r;
   pm.ngroups = G;
   for (int i = 0; i < G; ++i)
@@ -241,7 +250,7 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
   if (r > 0 && !fused &&
-      (s = gemm_prepare(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, workspace), &down)) !=
+      (s = gemm_prepare(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, t_buf), &down)) !=
           UNO_OK)
     return s;
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
@@ -372,7 +381,7 @@ constexpr int kLinPerLayer = 7;   // q, k, v, o, gate, up, down
 enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
 
 struct StepLayout {
-  size_t h, n, q, k, v, act, t, logits, vstat, total;
+  size_t h, n, q, k, v, act, t, dec, dec_bytes, logits, vstat, total;
 };
 
 // One operation of a step plan.
@@ -430,6 +439,8 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
   L.v = take(M * m->kv_out * 2);
   L.act = take(M * m->inter * 2);
   L.t = take(M * 3 * static_cast<size_t>(m->r) * 2);
+  L.dec_bytes = gemm_dec_workspace_bound(static_cast<int64_t>(M), m->r);
+  L.dec = take(L.dec_bytes);   // starts with the decode kernel's counters
   L.logits = take(Mv * static_cast<size_t>(m->vocab) * 2);
   L.vstat = take(verify_workspace(B, k, k + 1, m->vocab));
   L.total = off;
@@ -479,6 +490,8 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     for (int i = 0; i < G; ++i)
       As[i] = layer >= 0 ? m->wp(layer, which[i], 1) : m->head(1);
     GemmProblem pm{};
+    pm.scratch = base + L.dec;
+    pm.scratch_bytes = L.dec_bytes;
     pm.dt = UNO_BF16;
     pm.M = M;
     pm.K = K;
@@ -669,6 +682,9 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   cudaError_t e = cudaMemcpyAsync(base + L.h, h_in, static_cast<size_t>(M) * m->hidden * 2,
                                   cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_error(e, "copying h_in");
+  // the decode kernel's counters start every step at zero (its launches leave them so)
+  e = cudaMemsetAsync(base + L.dec, 0, kDecCounterBytes, st);
+  if (e != cudaSuccess) return cuda_error(e, "clearing the decode counters");
   for (const StepOp& op : P->ops) {
     s = op.kind == 0 ? gemm_run(op.gemm, st) : rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st);
     if (s != UNO_OK) return s;

@@ -122,6 +122,19 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order generic-proxy global-memory writes that this thread has observed
+// (through an acquire) before its later async-proxy (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Acquire load (gpu scope) of a flag or counter written by another CTA.
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -299,11 +312,22 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
 // All threads of all CTAs of the cluster; release our shared-memory writes,
 // acquire everyone else's. The warp is reconverged first (the barrier is
 // .aligned: every lane of a warp must execute the same instance).
+// The kernels give whole roles to single lanes (TMA producer, MMA issuer), so
+// a warp can reach a barrier split in time. The .aligned barrier forms assume
+// converged warps and were seen to complete early in that case; these
+// barriers use the per-thread (non-aligned) forms.
 __device__ __forceinline__ void cluster_sync() {
-  __syncwarp();
   asm volatile(
-      "barrier.cluster.arrive.release.aligned;\n\t"
-      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+      "barrier.cluster.arrive.release;\n\t"
+      "barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Barrier of all threads of the CTA (per-thread form, see cluster_sync).
+__device__ __forceinline__ void cta_sync() { asm volatile("barrier.sync 0;" ::: "memory"); }
+
+// Named barrier `id` of `n` threads (per-thread form).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t n) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 // Address of the same shared-memory offset in CTA `rank` of this cluster.
 __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t rank) {

@@ -48,7 +48,7 @@ struct DecParams {
 };
 static_assert(sizeof(DecParams) <= 256, "DecParams must fit GemmLaunch::params");
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { named_sync(1, 128); }
 
 template <bool kSilu>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) pdl_trigger();
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     __syncwarp();
     tc_fence_after();
@@ -395,6 +395,12 @@ int dec_stages(const GemmProblem& pb, int bn, uint32_t* stage_bytes, uint32_t* b
 }
 
 }  // namespace
+
+size_t gemm_dec_workspace_bound(int64_t M, int32_t r) {
+  (void)M;
+  (void)r;
+  return kDecCounterBytes;   // this kernel keeps its scratch on chip
+}
 
 bool gemm_dec_suits(const GemmProblem& pb) {
   if (pb.dt != UNO_BF16 || pb.M < 1 || pb.M > 256 || pb.r < 1 || pb.r > 128) return false;

@@ -65,7 +65,7 @@ __host__ __device__ constexpr uint32_t stage_bytes_for(int bn) {
   return ((kTileP + bn) * kRowBytes + 1023u) & ~1023u;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { named_sync(1, 128); }
 
 template <typename T, bool kSwap>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0 && a.mode != kEpiRowScale) pdl_trigger();
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_wait(smem_u32(&full[it % p.stages]), (it / p.stages) & 1u, kWaitLimitNs / 4);
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();   // every warp is done with TMEM before it is freed
   if (warp == 0) {
     __syncwarp();
     tc_fence_after();

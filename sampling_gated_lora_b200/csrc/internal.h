@@ -60,7 +60,17 @@ struct GemmProblem {
   // only triggers its dependents once the writer of x has finished: x may be
   // read at once, and only t must wait (so the two launches overlap).
   bool x_ready;
+  // Workspace of the decode kernel: kDecCounterBytes of counters (zero before
+  // the first call, left zero by every call), then its data. NULL: not used.
+  void* scratch;
+  size_t scratch_bytes;
 };
+
+// Counter region at the start of every gated-linear workspace.
+constexpr size_t kDecCounterBytes = size_t{64} << 10;
+// Decode-kernel workspace (counters included) that covers every problem with
+// M rows and rank r, whatever K, N and the number of groups.
+size_t gemm_dec_workspace_bound(int64_t M, int32_t r);
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
 // a[] (the adapters' A matrices) is used by the fused decode kernel only.
@@ -68,11 +78,13 @@ struct TensorMaps {
   CUtensorMap x, t, w[kMaxGroups], b[kMaxGroups], a[kMaxGroups];
 };
 
+constexpr size_t kLaunchParamBytes = 320;
+
 // Cached launch of a GemmProblem (tensor maps + grid); valid while the
 // pointers of the problem stay the same.
 struct GemmLaunch {
   TensorMaps tm;
-  alignas(8) unsigned char params[256];
+  alignas(8) unsigned char params[kLaunchParamBytes];
   int kind;               // 0: one-CTA kernel, 1: persistent CTA-pair kernel
   int swap;
   int grid_x, grid_y, splits;
@@ -90,8 +102,9 @@ uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t in
 bool gemm_pair_suits(const GemmProblem& pb);
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
-// The fused decode kernel (bf16, M <= 256, r <= 128): computes t = scale * gate
-// * (x A^T) in the same launch, so no separate down-projection is needed.
+// The decode kernel (bf16, M <= 128, r <= 128): computes t = scale * gate
+// * (x A^T) in the same launch, so no separate down-projection is needed;
+// needs GemmProblem::scratch.
 bool gemm_dec_suits(const GemmProblem& pb);
 uno_status gemm_dec_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_dec_run(const GemmLaunch& l, cudaStream_t stream);

@@ -49,6 +49,8 @@ def test_mlp_concatenated_batch(which):
     (1, 64, 128, 8, "bf16"),
     (3, 72, 200, 16, "bf16"),
     (17, 520, 264, 24, "bf16"),
+    (40, 512, 640, 0, "bf16"),          # decode-size path without an adapter
+    (24, 4096, 10240, 64, "bf16"),      # decode-size path: split tiles over two waves
     (130, 1024, 1000, 128, "bf16"),
     (257, 256, 384, 0, "bf16"),
     (300, 4096, 136, 256, "bf16"),
