@@ -285,7 +285,9 @@ bool gemm_pair_suits(const GemmProblem& pb) {
   int64_t ntiles = 0;
   for (int i = 0; i < pb.ngroups; ++i) ntiles += (pb.g[i].N + kTile - 1) / kTile;
   const int64_t tiles = ((pb.M + kTile - 1) / kTile) * ntiles;
-  return tiles >= device_sm_count() / 2 || pb.M >= 1024;
+  // two or more full token tiles already beat the one-CTA kernel (measured
+  // at M = 544..800); just above 256 rows the one-CTA kernel's split-K wins
+  return tiles >= device_sm_count() / 2 || pb.M >= 512;
 }
 
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
