@@ -84,10 +84,7 @@ uno_status uno_device_status(int32_t* bits_out, int32_t clear, void* stream);
  *   bf16: K, N, r multiples of 8; f32: multiples of 4 (16-byte row strides).
  *   f32 inputs run on the tf32 tensor-core path (10-bit mantissa products).
  *   workspace: >= uno_gated_lora_linear_workspace(...) bytes of device
- *   memory, 256-byte aligned, ZERO-FILLED before its first use: its first
- *   64 KiB hold counters of the decode-size path, which every call leaves at
- *   zero (zero them again after a call that raised a device status bit).
- *   Required when r > 0; with r = 0 it may be NULL (no decode-size path).
+ *   memory, 16-byte aligned; required when r > 0 (NULL allowed when r = 0).
  *   Calls that share a workspace must not run at the same time.
  * ------------------------------------------------------------------------- */
 size_t uno_gated_lora_linear_workspace(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r);
@@ -108,8 +105,7 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
  *
  *   W[i] [N[i],K], A[i] [r,K], Bl[i] [N[i],r], y[i] [M,N[i]], all `dt`
  *   (mode 1: bf16 only); gate [M] uint8; 1 <= G <= 3. Sizes as for
- *   uno_gated_lora_linear. workspace: >= uno_gated_lora_linear_group_workspace,
- *   aligned and zero-filled as for uno_gated_lora_linear.
+ *   uno_gated_lora_linear. workspace: >= uno_gated_lora_linear_group_workspace.
  * ------------------------------------------------------------------------- */
 size_t uno_gated_lora_linear_group_workspace(uno_dtype dt, int64_t M, int32_t r, int32_t G);
 

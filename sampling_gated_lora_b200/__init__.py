@@ -143,8 +143,8 @@ def _workspace(nbytes, device, workspace):
     torch = _torch()
     if nbytes == 0:
         return None, 0
-    if workspace is None:   # zero-filled: gated-linear workspaces start with counters
-        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
     return workspace, workspace.numel() * workspace.element_size()
 
 

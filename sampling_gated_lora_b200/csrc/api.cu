@@ -57,13 +57,11 @@ struct LinearLayout {
   size_t t_off, total;
 };
 
-// Workspace of a gated linear: the decode kernel's counters, then t (when the
-// down-projection runs as its own launch) or the decode kernel's data.
+// Workspace of a gated linear: t (used when the down-projection runs as its own launch).
 LinearLayout linear_layout(uno_dtype dt, int64_t M, int32_t r, int32_t G = 1) {
   LinearLayout l{};
-  l.t_off = kDecCounterBytes;
-  l.total = kDecCounterBytes + align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * G * dt_size(dt));
-  if (dt == UNO_BF16) l.total = std::max(l.total, gemm_dec_workspace_bound(M, r));
+  l.t_off = 0;
+  l.total = align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * G * dt_size(dt));
   return l;
 }
 
@@ -165,8 +163,6 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   void* t_buf = r > 0 ? static_cast<char*>(workspace) + L.t_off : nullptr;
   GemmLaunch down, main;
   GemmProblem pm{};
-  pm.scratch = workspace;
-  pm.scratch_bytes = workspace ? ws_bytes : 0;
   pm.dt = dt;
   pm.M = M;
   pm.K = K;
@@ -228,9 +224,7 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
     return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
   GemmLaunch down, main;
   GemmProblem pm{};
-  pm.scratch = workspace;
-  pm.scratch_bytes = workspace ? ws_bytes : 0;
-  void* t_buf = r > 0 ? static_cast<char*>(workspace) + kDecCounterBytes : nullptr;
+  void* t_buf = r > 0 ? workspace : nullptr;
   pm.dt = dt;
   pm.M = M;
   pm.K = K;
@@ -381,7 +375,7 @@ constexpr int kLinPerLayer = 7;   // q, k, v, o, gate, up, down
 enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
 
 struct StepLayout {
-  size_t h, n, q, k, v, act, t, dec, dec_bytes, logits, vstat, total;
+  size_t h, n, q, k, v, act, t, logits, vstat, total;
 };
 
 // One operation of a step plan.
@@ -439,8 +433,6 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
   L.v = take(M * m->kv_out * 2);
   L.act = take(M * m->inter * 2);
   L.t = take(M * 3 * static_cast<size_t>(m->r) * 2);
-  L.dec_bytes = gemm_dec_workspace_bound(static_cast<int64_t>(M), m->r);
-  L.dec = take(L.dec_bytes);   // starts with the decode kernel's counters
   L.logits = take(Mv * static_cast<size_t>(m->vocab) * 2);
   L.vstat = take(verify_workspace(B, k, k + 1, m->vocab));
   L.total = off;
@@ -490,8 +482,6 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     for (int i = 0; i < G; ++i)
       As[i] = layer >= 0 ? m->wp(layer, which[i], 1) : m->head(1);
     GemmProblem pm{};
-    pm.scratch = base + L.dec;
-    pm.scratch_bytes = L.dec_bytes;
     pm.dt = UNO_BF16;
     pm.M = M;
     pm.K = K;
@@ -682,9 +672,6 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   cudaError_t e = cudaMemcpyAsync(base + L.h, h_in, static_cast<size_t>(M) * m->hidden * 2,
                                   cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_error(e, "copying h_in");
-  // the decode kernel's counters start every step at zero (its launches leave them so)
-  e = cudaMemsetAsync(base + L.dec, 0, kDecCounterBytes, st);
-  if (e != cudaSuccess) return cuda_error(e, "clearing the decode counters");
   for (const StepOp& op : P->ops) {
     s = op.kind == 0 ? gemm_run(op.gemm, st) : rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st);
     if (s != UNO_OK) return s;

@@ -49,7 +49,7 @@ struct PairParams {
   int tiles_m, num_tiles;
   int stages;
 };
-static_assert(sizeof(PairParams) <= 256, "PairParams must fit GemmLaunch::params");
+static_assert(sizeof(PairParams) <= kLaunchParamBytes, "PairParams must fit GemmLaunch::params");
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ TensorMaps tm, const PairParams p) {

@@ -297,14 +297,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int e0 = static_cast<int>(rank) * chunk;
     const int e1 = min(groups, e0 + chunk);
     const uint32_t part0 = smem_u32(smem);
+    // unrolled to the largest cluster (8) with constant indices, so the peer
+    // addresses and partials stay in registers and all loads go out at once
     uint32_t peer[8];
-    for (int r = 0; r < Sp; ++r) peer[r] = map_shared_rank(part0, r);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) peer[r] = map_shared_rank(part0, r < Sp ? r : 0);
     auto sum4 = [&](uint32_t off) {
+      float4 v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < Sp) v[r] = ld_cluster_f32x4(peer[r] + off);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int r = 0; r < Sp; ++r) {
-        const float4 v = ld_cluster_f32x4(peer[r] + off);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < Sp) {
+          acc.x += v[r].x; acc.y += v[r].y; acc.z += v[r].z; acc.w += v[r].w;
+        }
       return acc;
     };
     for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += kThreads) {
@@ -395,12 +403,6 @@ int dec_stages(const GemmProblem& pb, int bn, uint32_t* stage_bytes, uint32_t* b
 }
 
 }  // namespace
-
-size_t gemm_dec_workspace_bound(int64_t M, int32_t r) {
-  (void)M;
-  (void)r;
-  return kDecCounterBytes;   // this kernel keeps its scratch on chip
-}
 
 bool gemm_dec_suits(const GemmProblem& pb) {
   if (pb.dt != UNO_BF16 || pb.M < 1 || pb.M > 256 || pb.r < 1 || pb.r > 128) return false;

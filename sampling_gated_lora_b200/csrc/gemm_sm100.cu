@@ -313,14 +313,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int e0 = static_cast<int>(rank) * chunk;
     const int e1 = min(groups, e0 + chunk);
     const uint32_t part0 = smem_u32(smem);
+    // unrolled to the largest cluster (8) with constant indices, so the peer
+    // addresses and partials stay in registers and all loads go out at once
     uint32_t peer[8];
-    for (int r = 0; r < S; ++r) peer[r] = map_shared_rank(part0, r);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) peer[r] = map_shared_rank(part0, r < S ? r : 0);
     auto sum4 = [&](uint32_t off) {
+      float4 v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < S) v[r] = ld_cluster_f32x4(peer[r] + off);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int r = 0; r < S; ++r) {
-        const float4 v = ld_cluster_f32x4(peer[r] + off);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < S) {
+          acc.x += v[r].x; acc.y += v[r].y; acc.z += v[r].z; acc.w += v[r].w;
+        }
       return acc;
     };
     for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += kGemmThreads) {

@@ -60,17 +60,7 @@ struct GemmProblem {
   // only triggers its dependents once the writer of x has finished: x may be
   // read at once, and only t must wait (so the two launches overlap).
   bool x_ready;
-  // Workspace of the decode kernel: kDecCounterBytes of counters (zero before
-  // the first call, left zero by every call), then its data. NULL: not used.
-  void* scratch;
-  size_t scratch_bytes;
 };
-
-// Counter region at the start of every gated-linear workspace.
-constexpr size_t kDecCounterBytes = size_t{64} << 10;
-// Decode-kernel workspace (counters included) that covers every problem with
-// M rows and rank r, whatever K, N and the number of groups.
-size_t gemm_dec_workspace_bound(int64_t M, int32_t r);
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
 // a[] (the adapters' A matrices) is used by the fused decode kernel only.
@@ -102,9 +92,8 @@ uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t in
 bool gemm_pair_suits(const GemmProblem& pb);
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
-// The decode kernel (bf16, M <= 128, r <= 128): computes t = scale * gate
-// * (x A^T) in the same launch, so no separate down-projection is needed;
-// needs GemmProblem::scratch.
+// The fused decode kernel (bf16, M <= 256, r <= 128): computes t = scale * gate
+// * (x A^T) in the same launch, so no separate down-projection is needed.
 bool gemm_dec_suits(const GemmProblem& pb);
 uno_status gemm_dec_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_dec_run(const GemmLaunch& l, cudaStream_t stream);

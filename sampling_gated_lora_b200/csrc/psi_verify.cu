@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kStatThreads)
     sm[warp] = m;
     ss[warp] = s;
   }
-  __syncthreads();
+  cta_sync();
   if (threadIdx.x == 0) {
     float M = sm[0], S = ss[0];
     for (int w = 1; w < kStatThreads / 32; ++w) merge_stat(M, S, sm[w], ss[w], c);
@@ -194,7 +194,7 @@ __device__ __forceinline__ void block_scan(DrawSmem& sh, double v) {
   double excl = __shfl_up_sync(0xffffffffu, incl, 1);
   if (lane == 0) excl = 0.0;
   if (lane == 31) sh.warp_tot[warp] = incl;
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     double w = lane < kDrawThreads / 32 ? sh.warp_tot[lane] : 0.0;
 #pragma unroll
@@ -204,14 +204,14 @@ __device__ __forceinline__ void block_scan(DrawSmem& sh, double v) {
     }
     if (lane < kDrawThreads / 32) sh.warp_tot[lane] = w;   // inclusive over warps
   }
-  __syncthreads();
+  cta_sync();
   const double base = warp ? sh.warp_tot[warp - 1] : 0.0;
   sh.prefix[t] = base + excl;
   if (t == 0) {
     sh.prefix[kDrawThreads] = sh.warp_tot[kDrawThreads / 32 - 1];
     sh.chunk_total = sh.warp_tot[kDrawThreads / 32 - 1];
   }
-  __syncthreads();
+  cta_sync();
 }
 
 // Largest index t in [0, kDrawThreads) with `ok` true, over the block (-1 if none).
@@ -219,11 +219,11 @@ __device__ __forceinline__ int block_max_index(DrawSmem& sh, bool ok) {
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int w = __reduce_max_sync(0xffffffffu, ok ? t : -1);
   if (lane == 0) sh.owner[warp] = w;
-  __syncthreads();
+  cta_sync();
   int best = -1;
 #pragma unroll
   for (int i = 0; i < kDrawThreads / 32; ++i) best = max(best, sh.owner[i]);
-  __syncthreads();
+  cta_sync();
   return best;
 }
 
@@ -254,13 +254,16 @@ __device__ int cluster_draw(DrawSmem& sh, const WFn& wfn, int lo, int len, doubl
   const uint32_t nrank = cluster_nctarank();
   const uint32_t myrank = cluster_ctarank();
   const uint32_t tot_addr = smem_u32(&sh.chunk_total);
-  double Z = 0.0, thr_prefix[8];
-  double tots[8];
-  for (uint32_t r = 0; r < nrank; ++r) {
-    const double v = ld_cluster_f64(map_shared_rank(tot_addr, r));
+  // (unrolled to the largest cluster with constant indices: registers, not stack)
+  double Z = 0.0, thr_prefix[8], tots[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
     thr_prefix[r] = Z;
-    tots[r] = v;
-    Z += v;
+    tots[r] = 0.0;
+    if (r < static_cast<int>(nrank)) {
+      tots[r] = ld_cluster_f64(map_shared_rank(tot_addr, static_cast<uint32_t>(r)));
+      Z += tots[r];
+    }
   }
   cluster_sync();   // totals read everywhere before anyone reuses the slot or exits
   if (!(Z > 0.0)) {
@@ -270,10 +273,14 @@ __device__ int cluster_draw(DrawSmem& sh, const WFn& wfn, int lo, int len, doubl
   *zero_total = false;
   const double thr = u * Z;
   int owner_rank = -1;
-  for (uint32_t r = 0; r < nrank; ++r)
-    if (tots[r] > 0.0 && thr_prefix[r] <= thr) owner_rank = static_cast<int>(r);
+  double my_prefix = 0.0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r < static_cast<int>(nrank) && tots[r] > 0.0 && thr_prefix[r] <= thr) owner_rank = r;
+    if (r == static_cast<int>(myrank)) my_prefix = thr_prefix[r];
+  }
   if (owner_rank != static_cast<int>(myrank)) return -1;   // uniform over this CTA
-  const double tl = thr - thr_prefix[myrank];
+  const double tl = thr - my_prefix;
   const int own = block_max_index(sh, my > 0.0 && sh.prefix[t] <= tl);
   if (t == own) {
     const double tt = tl - sh.prefix[t];
@@ -290,7 +297,7 @@ __device__ int cluster_draw(DrawSmem& sh, const WFn& wfn, int lo, int len, doubl
     }
     sh.token = lo + (pick >= 0 ? pick : last_nz);
   }
-  __syncthreads();
+  cta_sync();
   return sh.token;
 }
 
@@ -391,7 +398,7 @@ __global__ void __launch_bounds__(kDrawThreads)
       s_nan = nanm != 0;
     }
   }
-  __syncthreads();
+  cta_sync();
   const int n = s_n;
   int32_t* tok = a.out_tokens + static_cast<size_t>(b) * (k + 1);
   if (s_bad || s_nan) {
@@ -439,7 +446,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   T* zq = zp + a.chunk_elems;
   load_chunk(zp, p_logits + static_cast<size_t>(prow) * V + lo, len);
   if (residual) load_chunk(zq, q_logits + static_cast<size_t>(qrow_local) * V + lo, len);
-  __syncthreads();
+  cta_sync();
   const float Mp = s_stat[0], inv_sp = 1.f / s_stat[1];
   const float Mq = s_stat[2], inv_sq = residual ? 1.f / s_stat[3] : 0.f;
   const float c = a.c;
@@ -493,7 +500,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
   T* z = reinterpret_cast<T*>(dyn);
   load_chunk(z, q_logits + static_cast<size_t>(row) * V + lo, len);
-  __syncthreads();
+  cta_sync();
   float mx = -INFINITY;
   bool nan = false;
   for (int i = threadIdx.x; i < len; i += blockDim.x) {
@@ -504,7 +511,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   mx = warp_max(mx);
   nan = __any_sync(0xffffffffu, nan);
   if ((threadIdx.x & 31) == 0) s_cmax[threadIdx.x >> 5] = nan ? NAN : mx;
-  __syncthreads();
+  cta_sync();
   if (threadIdx.x == 0) {
     float m = -INFINITY;
     bool any_nan = false;
