@@ -72,7 +72,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const GemmArgs& a = p.a;
   const bool silu = a.mode == kEpiSiluPair;
   const int nkb = a.nkb_main + (silu ? 2 : 1) * a.nkb_r;
-  const int tile_n = silu ? kHalf : kTile;   // output features per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
