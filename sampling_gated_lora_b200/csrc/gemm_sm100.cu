@@ -489,7 +489,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   int bn, tok_tiles;
   if (swap) {
     // decode batches: one token tile of up to 256; down-projections of large
-    // batches: 128-token tiles (two CTAs per SM, more tiles to spread)
+    // batches: 128-token tiles (more tiles to spread over the SMs)
     const int tile = M <= 256 ? 256 : 128;
     tok_tiles = static_cast<int>((M + tile - 1) / tile);
     bn = round_up(static_cast<int>((M + tok_tiles - 1) / tok_tiles), 16);
@@ -508,8 +508,11 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
 
   // Shared memory: ~96 KB (two or three CTAs per SM) for narrow decode tiles,
   // ~200 KB otherwise.
+  // Down-projections of large batches take the full ring: their cluster grid
+  // is sized to one CTA per SM, and each CTA streams a long K-slice whose
+  // rate is set by the bytes it keeps in flight.
   const uint32_t st = stage_bytes_for(bn);
-  const bool narrow = bn <= 64 || (swap && M > 256);
+  const bool narrow = bn <= 64;
   const uint32_t budget = narrow ? 96u * 1024u : 200u * 1024u;
   int stages = std::min<int>(kMaxStages, static_cast<int>(budget / st));
   stages = std::max(stages, 2);
