@@ -84,7 +84,12 @@ uno_status uno_device_status(int32_t* bits_out, int32_t clear, void* stream);
  *   bf16: K, N, r multiples of 8; f32: multiples of 4 (16-byte row strides).
  *   f32 inputs run on the tf32 tensor-core path (10-bit mantissa products).
  *   workspace: >= uno_gated_lora_linear_workspace(...) bytes of device
- *   memory, 16-byte aligned; required when r > 0 (NULL allowed when r = 0).
+ *   memory, 16-byte aligned, any contents; required when r > 0. When r = 0 it
+ *   may be NULL (or smaller than the query): the call then runs without the
+ *   scratch below. bf16 batches with M > 256 (the CTA-pair kernel) also keep
+ *   in it the fp32 partial sums of tiles whose K range two pairs of SMs share
+ *   (stream-K over the last round of tiles) and the flags that order them;
+ *   the call clears those flags on `stream` before its first launch.
  *   Calls that share a workspace must not run at the same time.
  * ------------------------------------------------------------------------- */
 size_t uno_gated_lora_linear_workspace(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r);
@@ -241,7 +246,10 @@ void uno_model_destroy(uno_model* m);
  *   d_next [B,k], and writes their logits to q_next [B,k,V] bf16.
  *   logits_out: optional [B(k+1), V] bf16 copy target for the AR rows (NULL
  *   to skip). accepted_len [B], out_tokens [B,k+1], out_count [B] as in
- *   uno_psi_verify. q_next must not alias q_prev. */
+ *   uno_psi_verify. q_next must not alias q_prev.
+ *   workspace: >= uno_psi_step_workspace(m, B, k) bytes, 16-byte aligned,
+ *   any contents (the step clears the stream-K flags it holds on `stream`
+ *   first). Steps that share a workspace must not run at the same time. */
 size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k);
 
 uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, const void* q_prev,

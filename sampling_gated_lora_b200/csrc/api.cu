@@ -54,15 +54,46 @@ uno_status cuda_error(cudaError_t e, const char* what) {
 namespace {
 
 struct LinearLayout {
-  size_t t_off, total;
+  size_t t_off, sk_part_off, sk_flag_off, total;
+  bool sk;
 };
 
-// Workspace of a gated linear: t (used when the down-projection runs as its own launch).
+// Workspace of a gated linear: t (used when the down-projection runs as its
+// own launch), then, for batches the CTA-pair kernel takes (bf16, M > 256),
+// its stream-K partial sums and flags.
 LinearLayout linear_layout(uno_dtype dt, int64_t M, int32_t r, int32_t G = 1) {
   LinearLayout l{};
   l.t_off = 0;
-  l.total = align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * G * dt_size(dt));
+  size_t off = align_up(static_cast<size_t>(M) * static_cast<size_t>(r) * G * dt_size(dt));
+  l.sk = dt == UNO_BF16 && M > 256;
+  if (l.sk) {
+    l.sk_part_off = off;
+    off += align_up(pair_sk_part_bytes());
+    l.sk_flag_off = off;
+    off += align_up(pair_sk_flag_bytes());
+  }
+  l.total = off;
   return l;
+}
+
+// Points a problem at the stream-K scratch of a linear's workspace (when it has one).
+void attach_sk(GemmProblem* pm, const LinearLayout& L, void* workspace) {
+  if (!L.sk || !workspace) return;
+  pm->sk_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.sk_part_off);
+  pm->sk_flag = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + L.sk_flag_off);
+  pm->sk_slots = pair_sk_slots();
+}
+
+// Runs the down-projection (if any) and the main launch of a gated linear,
+// zeroing the main launch's stream-K flags first.
+uno_status run_linear(const GemmLaunch* down, const GemmLaunch& main, cudaStream_t st) {
+  if (main.sk_flag) {
+    const cudaError_t e = cudaMemsetAsync(main.sk_flag, 0, main.sk_flag_bytes, st);
+    if (e != cudaSuccess) return cuda_error(e, "clearing the stream-K flags");
+  }
+  uno_status s;
+  if (down && (s = gemm_run(*down, st)) != UNO_OK) return s;
+  return gemm_run(main, st);
 }
 
 uno_status check_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r) {
@@ -160,8 +191,9 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   if (r > 0 && (!workspace || ws_bytes < L.total || !aligned16(workspace)))
     return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", L.total,
                      ws_bytes);
+  const bool use_ws = workspace && ws_bytes >= L.total && aligned16(workspace);
   void* t_buf = r > 0 ? static_cast<char*>(workspace) + L.t_off : nullptr;
-  GemmLaunch down, main;
+  GemmLaunch down{}, main{};
   GemmProblem pm{};
   pm.dt = dt;
   pm.M = M;
@@ -177,6 +209,7 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   pm.M0 = M;
   pm.gate = gate;
   pm.scale = scale;
+  if (use_ws) attach_sk(&pm, L, workspace);
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
   if (r > 0 && !fused) {
@@ -186,8 +219,7 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
       return s;
   }
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
-  if (r > 0 && !fused && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
-  return gemm_run(main, as_stream(stream));
+  return run_linear(r > 0 && !fused ? &down : nullptr, main, as_stream(stream));
 }
 
 size_t uno_gated_lora_linear_group_workspace(uno_dtype dt, int64_t M, int32_t r, int32_t G) {
@@ -219,10 +251,12 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
     if ((mode == 0 || i == 0) && (!y[i] || !aligned16(y[i])))
       return set_error(UNO_ERR_INVALID_ARG, "group %d: NULL or unaligned output", i);
   }
-  const size_t need = uno_gated_lora_linear_group_workspace(dt, M, r, G);
+  const LinearLayout L = linear_layout(dt, M, r, G);
+  const size_t need = L.total;
   if (r > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
     return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
-  GemmLaunch down, main;
+  const bool use_ws = workspace && ws_bytes >= need && aligned16(workspace);
+  GemmLaunch down{}, main{};
   GemmProblem pm{};
   void* t_buf = r > 0 ? workspace : nullptr;
   pm.dt = dt;
@@ -241,6 +275,7 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   pm.M0 = M;
   pm.gate = gate;
   pm.scale = scale;
+  if (use_ws) attach_sk(&pm, L, workspace);
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
   if (r > 0 && !fused &&
@@ -248,8 +283,7 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
           UNO_OK)
     return s;
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
-  if (r > 0 && !fused && (s = gemm_run(down, as_stream(stream))) != UNO_OK) return s;
-  return gemm_run(main, as_stream(stream));
+  return run_linear(r > 0 && !fused ? &down : nullptr, main, as_stream(stream));
 }
 
 // ---------------------------------------------------------------- sampler
@@ -375,7 +409,7 @@ constexpr int kLinPerLayer = 7;   // q, k, v, o, gate, up, down
 enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
 
 struct StepLayout {
-  size_t h, n, q, k, v, act, t, logits, vstat, total;
+  size_t h, n, q, k, v, act, t, logits, vstat, sk_part, sk_flag, sk_flag_bytes, total;
 };
 
 // One operation of a step plan.
@@ -435,6 +469,13 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
   L.t = take(M * 3 * static_cast<size_t>(m->r) * 2);
   L.logits = take(Mv * static_cast<size_t>(m->vocab) * 2);
   L.vstat = take(verify_workspace(B, k, k + 1, m->vocab));
+  // stream-K scratch of the CTA-pair GEMMs (M > 256): partial sums shared by
+  // the step's launches, one block of flags per launch (4 per layer + head)
+  if (M > 256) {
+    L.sk_part = take(pair_sk_part_bytes());
+    L.sk_flag_bytes = (static_cast<size_t>(m->n_layers) * 4 + 1) * align_up(pair_sk_flag_bytes());
+    L.sk_flag = take(L.sk_flag_bytes);
+  }
   L.total = off;
   return L;
 }
@@ -460,6 +501,7 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
   P->logits_out = logits_out;
   P->ops.clear();
   void* t = base + L.t;
+  int main_launches = 0;   // stream-K flag block of the next main GEMM
   auto norm = [&](const void* x, void* y) {
     StepOp op{};
     op.kind = 1;
@@ -513,6 +555,13 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     pm.gate_row0 = Mv;
     pm.scale = m->scale;
     for (int i = 0; i < G; ++i) pm.A[i] = r > 0 ? As[i] : nullptr;
+    if (L.sk_flag_bytes) {
+      pm.sk_part = reinterpret_cast<float*>(base + L.sk_part);
+      pm.sk_flag = reinterpret_cast<int32_t*>(
+          base + L.sk_flag + static_cast<size_t>(main_launches) * align_up(pair_sk_flag_bytes()));
+      pm.sk_slots = pair_sk_slots();
+      ++main_launches;
+    }
     pm.x_ready = r > 0 && !gemm_dec_suits(pm);
     if (pm.x_ready &&
         (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
@@ -672,6 +721,8 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   cudaError_t e = cudaMemcpyAsync(base + L.h, h_in, static_cast<size_t>(M) * m->hidden * 2,
                                   cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_error(e, "copying h_in");
+  if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
+    return cuda_error(e, "clearing the stream-K flags");
   for (const StepOp& op : P->ops) {
     s = op.kind == 0 ? gemm_run(op.gemm, st) : rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st);
     if (s != UNO_OK) return s;

@@ -40,6 +40,27 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ flags between CTAs
+// A word in global memory that one CTA raises after writing data and another
+// CTA of the same grid waits for before reading it (waits are bounded).
+__device__ __forceinline__ void flag_release(int32_t* f, int32_t v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t flag_acquire(const int32_t* f) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool flag_wait(const int32_t* f, int32_t v,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  if (flag_acquire(f) == v) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (flag_acquire(f) == v) return true;
+    if ((i & 63u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // Kernels of this library are launched so that the next kernel on the stream
 // may start its prologue while this one finishes. Each kernel triggers its
@@ -225,6 +246,16 @@ __device__ __forceinline__ void tmem_relinquish_pair() {
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
+}
+
+// Contiguous copy global -> this CTA's shared memory (no tensor map),
+// completion counted on `bar`. dst, src and bytes: multiples of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 // 2D tiled load into this CTA's shared memory whose completion is counted on

@@ -25,7 +25,10 @@
 //     buffer to the leader's accumulator-empty barrier.
 // Two 256-column TMEM accumulators let the epilogue of tile i overlap the
 // mainloop of tile i+1. Tiles are visited token-block fastest so concurrent
-// pairs share W tiles (and x stays resident in L2).
+// pairs share W tiles (and x stays resident in L2). For deep tiles whose count
+// would leave the last round part-empty, the K-blocks of the last tiles are
+// shared out evenly (stream-K); the two pairs that cut a tile meet through
+// fp32 partial sums and flags in the caller's workspace.
 #include <algorithm>
 #include <cstring>
 
@@ -43,13 +46,64 @@ constexpr int kTile = 256;                  // tile edge (M and N) per pair
 constexpr uint32_t kHalfBytes = kHalf * 128;   // one 128-row, 128-byte K-block half
 constexpr uint32_t kStageBytes = 2 * kHalfBytes;
 constexpr int kAccCols = 256;
+// Stream-K partial sum of one epilogue warp: 32 accumulator rows x 256 columns,
+// column-major so that a warp's 32 lanes touch 128 contiguous bytes.
+constexpr uint32_t kSkWarpFloats = 32 * kAccCols;
+constexpr uint32_t kSkWarpBytes = kSkWarpFloats * 4;
 
 struct PairParams {
   GemmArgs a;
   int tiles_m, num_tiles;
   int stages;
+  // Tiles [0, dp_tiles) are visited whole, round-robin over the pairs. The
+  // K-block iterations of the remaining tiles (sk_iters in all, the tiles
+  // taken in order) are shared out evenly, stream-K style: pair p takes
+  // iterations [p I / P, (p + 1) I / P).
+  int dp_tiles;
+  long long sk_iters;
+  float* sk_part;       // [pairs][2 CTAs][4 epilogue warps][256 columns][32 rows] fp32
+  int32_t* sk_flag;     // [pairs][2 CTAs][4 epilogue warps], zero at launch
 };
 static_assert(sizeof(PairParams) <= kLaunchParamBytes, "PairParams must fit GemmLaunch::params");
+
+// The work of one pair: its whole tiles, then its stream-K share cut at tile
+// boundaries. Each share spans at least one tile's worth of K-blocks (the
+// stream-K tiles number at least as many as the pairs), so a tile that two
+// shares cut has exactly two parts: the first (kb0 = 0, kb1 < nkb) belongs
+// to pair p, which finishes the tile with the partial sum of the second
+// (kb0 > 0, kb1 = nkb), the first part of pair p + 1's share. Pair p reaches
+// its part last in its share, pair p + 1 first in its own.
+struct WorkCursor {
+  int tile;
+  long long it, it_end;
+};
+
+__device__ __forceinline__ WorkCursor work_begin(const PairParams& p, int pair, int pairs) {
+  WorkCursor c;
+  c.tile = pair;
+  c.it = p.sk_iters * pair / pairs;
+  c.it_end = p.sk_iters * (pair + 1) / pairs;
+  return c;
+}
+
+__device__ __forceinline__ bool work_next(const PairParams& p, int pairs, int nkb, WorkCursor& c,
+                                          int& tile, int& kb0, int& kb1) {
+  if (c.tile < p.dp_tiles) {
+    tile = c.tile;
+    kb0 = 0;
+    kb1 = nkb;
+    c.tile += pairs;
+    return true;
+  }
+  if (c.it >= c.it_end) return false;
+  const long long rel = c.it / nkb;
+  const long long end = min((rel + 1) * nkb, c.it_end);
+  tile = p.dp_tiles + static_cast<int>(rel);
+  kb0 = static_cast<int>(c.it - rel * nkb);
+  kb1 = static_cast<int>(end - rel * nkb);
+  c.it = end;
+  return true;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ TensorMaps tm, const PairParams p) {
@@ -61,7 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + S;
   uint64_t* accf = empty + S;     // [2]
   uint64_t* acce = accf + 2;      // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* skbar = acce + 2;     // [4] stream-K partial sums copied in, one per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(skbar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -82,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&accf[b]), 1);
       mbar_init(smem_u32(&acce[b]), 8);   // 4 epilogue warps x 2 CTAs
     }
+    for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&skbar[q]), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -110,9 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // waiting for the kernel that writes the activations.
     int it = 0;
     bool ok = true;
-    int pre = 0;   // k-blocks of the first tile whose W half went out early
+    bool first = true;
     bool waited = false;
-    for (int tile = pair; ok && tile < p.num_tiles; tile += num_pairs) {
+    WorkCursor wc = work_begin(p, pair, num_pairs);
+    int tile, kb0, kb1;
+    while (ok && work_next(p, num_pairs, nkb, wc, tile, kb0, kb1)) {
       const int mb = tile % p.tiles_m, ft = tile / p.tiles_m;
       const int g = group_of(a, ft);
       const int m0 = mb * kTile + static_cast<int>(rank) * kHalf;
@@ -142,27 +200,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d_pair(sa, &tm.t, a.g[silu ? h : g].t_col + j * 64, m0, fb);
         }
       };
-      if (tile == pair) {
-        pre = min(S, nkb);
+      int kb_next = kb0;
+      if (first) {
+        // k-blocks of the first work item whose W half goes out early
+        first = false;
+        const int pre = min(S, kb1 - kb0);
         for (int q = 0; q < pre; ++q) {
           const uint32_t sa = smem_u32(smem + q * kStageBytes);
           if (leader) mbar_arrive_expect_tx(smem_u32(&full[q]), 2 * kStageBytes);
-          load_b(q, sa + kHalfBytes, map_shared_rank(smem_u32(&full[q]), 0));
+          load_b(kb0 + q, sa + kHalfBytes, map_shared_rank(smem_u32(&full[q]), 0));
         }
         if (!a.x_ready) {
           pdl_wait();
           waited = true;
         }
         for (int q = 0; q < pre; ++q) {
-          if (!waited && q >= a.nkb_main) {
+          if (!waited && kb0 + q >= a.nkb_main) {
             pdl_wait();
             waited = true;
           }
-          load_a(q, smem_u32(smem + q * kStageBytes), map_shared_rank(smem_u32(&full[q]), 0));
+          load_a(kb0 + q, smem_u32(smem + q * kStageBytes), map_shared_rank(smem_u32(&full[q]), 0));
         }
         it = pre;
+        kb_next = kb0 + pre;
       }
-      for (int kb = (tile == pair) ? pre : 0; kb < nkb; ++kb, ++it) {
+      for (int kb = kb_next; kb < kb1; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1u;
         if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u) || *abort_flag) {
@@ -187,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t idesc = idesc_f32acc(kTile, kTile, false);
     int it = 0, lt = 0;
     bool ok = true;
-    for (int tile = pair; ok && tile < p.num_tiles; tile += num_pairs, ++lt) {
+    WorkCursor wc = work_begin(p, pair, num_pairs);
+    int tile, kb0, kb1;
+    for (; ok && work_next(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
       const int b = lt & 1;
       const uint32_t aph = (lt >> 1) & 1u;
       if (!mbar_wait_cluster(smem_u32(&acce[b]), aph ^ 1u)) {
@@ -196,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t dacc = tmem + static_cast<uint32_t>(b * kAccCols);
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1u;
         if (!mbar_wait(smem_u32(&full[s]), ph)) {
@@ -211,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_pair_bf16(dacc, ad + static_cast<uint64_t>(2 * kk), bd + static_cast<uint64_t>(2 * kk),
-                        idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
         const uint32_t eb = smem_u32(&empty[s]);
         mma_commit_pair(map_shared_rank(eb, 0));
         mma_commit_pair(map_shared_rank(eb, 1));
@@ -226,7 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int i = quarter * 32 + lane;
     int lt = 0;
-    for (int tile = pair; tile < p.num_tiles; tile += num_pairs, ++lt) {
+    WorkCursor wc = work_begin(p, pair, num_pairs);
+    int tile, kb0, kb1;
+    for (; work_next(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
       const int b = lt & 1;
       const uint32_t aph = (lt >> 1) & 1u;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&accf[b]), aph));
@@ -240,22 +306,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m = mb * kTile + static_cast<int>(rank) * kHalf + i;
       const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                             static_cast<uint32_t>(b * kAccCols);
-      if (!silu) {
-        const int nb0 = (ft - a.g[g].tile0) * kTile;
+      if (kb0 > 0) {
+        // second part of a stream-K tile: hand this warp's partial sum (its
+        // 32 rows, all 256 columns) to the pair that holds the first part
+        const int fi = ((pair - 1) * 2 + static_cast<int>(rank)) * 4 + quarter;
+        float* part = p.sk_part + static_cast<size_t>(fi) * kSkWarpFloats;
         for (int c = 0; c < kTile; c += 16) {
           float v[16];
           tmem_ld16(trow + c, v);
-          if (nb0 + c < a.g[g].N) epi_store16<__nv_bfloat16>(a, g, m, nb0 + c, v);
-        }
-      } else {
-        const int f0 = ft * kHalf;
-        for (int c = 0; c < kHalf; c += 16) {
-          float gv[16], uv[16];
-          tmem_ld16(trow + c, gv);
-          tmem_ld16(trow + kHalf + c, uv);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) gv[j] = silu_f(gv[j]) * uv[j];
-          if (f0 + c < a.g[0].N) epi_store16<__nv_bfloat16>(a, 0, m, f0 + c, gv);
+          for (int j = 0; j < 16; ++j) part[(c + j) * 32 + lane] = v[j];
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) flag_release(p.sk_flag + fi, 1);
+      } else {
+        // first part of a stream-K tile (the pair's last work item, so the
+        // stage ring is idle): copy the next pair's partial sum for this
+        // warp's rows into shared memory, then add it
+        const float* part = nullptr;
+        if (kb1 < nkb) {
+          const int fi = (pair * 2 + static_cast<int>(rank)) * 4 + quarter;
+          bool got = __all_sync(0xffffffffu, flag_wait(p.sk_flag + fi, 1));
+          const uint32_t dst = smem_u32(smem + static_cast<uint32_t>(quarter) * kSkWarpBytes);
+          if (got) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(smem_u32(&skbar[quarter]), kSkWarpBytes);
+              bulk_load(dst, p.sk_part + static_cast<size_t>(fi) * kSkWarpFloats, kSkWarpBytes,
+                        smem_u32(&skbar[quarter]));
+            }
+            got = __all_sync(0xffffffffu, mbar_wait(smem_u32(&skbar[quarter]), 0));
+          }
+          if (got)
+            part = reinterpret_cast<const float*>(smem + static_cast<uint32_t>(quarter) * kSkWarpBytes);
+          else if (lane == 0)
+            fail();
+        }
+        if (!silu) {
+          const int nb0 = (ft - a.g[g].tile0) * kTile;
+          for (int c = 0; c < kTile; c += 16) {
+            float v[16];
+            tmem_ld16(trow + c, v);
+            if (part) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] += part[(c + j) * 32 + lane];
+            }
+            if (nb0 + c < a.g[g].N) epi_store16<__nv_bfloat16>(a, g, m, nb0 + c, v);
+          }
+        } else {
+          const int f0 = ft * kHalf;
+          for (int c = 0; c < kHalf; c += 16) {
+            float gv[16], uv[16];
+            tmem_ld16(trow + c, gv);
+            tmem_ld16(trow + kHalf + c, uv);
+            if (part) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                gv[j] += part[(c + j) * 32 + lane];
+                uv[j] += part[(kHalf + c + j) * 32 + lane];
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) gv[j] = silu_f(gv[j]) * uv[j];
+            if (f0 + c < a.g[0].N) epi_store16<__nv_bfloat16>(a, 0, m, f0 + c, gv);
+          }
         }
       }
       tc_fence_before();
@@ -289,6 +403,14 @@ bool gemm_pair_suits(const GemmProblem& pb) {
   return tiles >= device_sm_count() / 2 || pb.M >= 512;
 }
 
+int pair_sk_slots() { return std::max(1, device_sm_count() / 2); }
+
+size_t pair_sk_part_bytes() {
+  return static_cast<size_t>(pair_sk_slots()) * 2 * kTile * kHalf * sizeof(float);
+}
+
+size_t pair_sk_flag_bytes() { return static_cast<size_t>(pair_sk_slots()) * 2 * 4 * sizeof(int32_t); }
+
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
   const bool silu = pb.mode == kEpiSiluPair;
   const int tile_n = silu ? kHalf : kTile;
@@ -316,8 +438,33 @@ uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
       tm.b[i] = tm.w[i];
     }
   }
-  std::memcpy(out->params, &pp, sizeof(pp));
   const int pairs = std::max(1, std::min<int>(device_sm_count() / 2, pp.num_tiles));
+  // Stream-K: when the whole tiles would leave the last round part-empty
+  // (rem of the pairs busy), the last `pairs + rem` tiles are shared out by
+  // K-blocks instead, so every pair ends at the same time. Taken for deep
+  // tiles only (>= 128 K-blocks, e.g. 12288 -> 4096 at M = 4352: 419 -> 396 us
+  // on one B200): with 64-block tiles a part-empty last round runs its tiles
+  // faster (fewer pairs share the L2), and splitting them measured no gain.
+  // Not worth the hand-over of partial sums when the last round is nearly full.
+  const int nkb = pp.a.nkb_main + (silu ? 2 : 1) * pp.a.nkb_r;
+  const int rem = pp.num_tiles % pairs;
+  // the finishing pair stages the partial sums in its idle stage ring
+  static_assert(4 * kSkWarpBytes <= 6 * kStageBytes, "partial sums must fit the stage ring");
+  pp.dp_tiles = pp.num_tiles;
+  pp.sk_iters = 0;
+  out->sk_flag = nullptr;
+  out->sk_flag_bytes = 0;
+  if (pb.sk_part && pb.sk_flag && pairs <= pb.sk_slots && rem > 0 && 5 * rem <= 4 * pairs &&
+      nkb >= 128) {
+    const int sk_tiles = pairs + rem;
+    pp.dp_tiles = pp.num_tiles - sk_tiles;
+    pp.sk_iters = static_cast<long long>(sk_tiles) * nkb;
+    pp.sk_part = pb.sk_part;
+    pp.sk_flag = pb.sk_flag;
+    out->sk_flag = pb.sk_flag;
+    out->sk_flag_bytes = pair_sk_flag_bytes();
+  }
+  std::memcpy(out->params, &pp, sizeof(pp));
   out->kind = 1;
   out->swap = 0;
   out->grid_x = 2 * pairs;

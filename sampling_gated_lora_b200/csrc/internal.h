@@ -60,6 +60,12 @@ struct GemmProblem {
   // only triggers its dependents once the writer of x has finished: x may be
   // read at once, and only t must wait (so the two launches overlap).
   bool x_ready;
+  // Stream-K scratch of the CTA-pair kernel (NULL: whole tiles only). The
+  // partial sums may be shared by launches of one stream; the flags are this
+  // launch's own and must be zero when it starts (see pair_sk_bytes).
+  float* sk_part;
+  int32_t* sk_flag;
+  int sk_slots;           // pairs the scratch serves
 };
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
@@ -80,6 +86,8 @@ struct GemmLaunch {
   int grid_x, grid_y, splits;
   int smem_bytes;
   int dtype;
+  int32_t* sk_flag;       // stream-K flags this launch reads: zero them before it runs (or NULL)
+  size_t sk_flag_bytes;
 };
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out);
@@ -90,6 +98,11 @@ uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t in
 // The persistent CTA-pair kernel (bf16, 256x256 tiles): whether it takes the
 // problem, its preparation and its launch.
 bool gemm_pair_suits(const GemmProblem& pb);
+// Stream-K scratch of the CTA-pair kernel on this device: the fp32 partial
+// tiles (one per pair) and one launch's flags (eight words per pair).
+size_t pair_sk_part_bytes();
+size_t pair_sk_flag_bytes();
+int pair_sk_slots();
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
 // The fused decode kernel (bf16, M <= 256, r <= 128): computes t = scale * gate

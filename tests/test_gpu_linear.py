@@ -78,6 +78,34 @@ def test_pair_kernel_step_shapes():
         check_close(y[rows], _oracle(case, rows), what=f"M=4352 {K}->{N} sampled rows")
 
 
+@pytest.mark.parametrize("M,K,N,r", [
+    (600, 8192, 8192, 8),     # 96 tiles of 129 K-blocks on 74 pairs
+    (700, 8200, 8000, 24),    # ragged M, N and K (130 K-blocks)
+])
+def test_stream_k_tiles(M, K, N, r):
+    """Deep tiles whose count would leave the last round of the CTA-pair kernel part-empty:
+    the last tiles are shared out by K-blocks and two pairs add up each cut tile."""
+    rng = np.random.default_rng(M + N)
+    gate = (rng.random(M) < 0.5).astype(np.uint8)
+    case = W.gated_linear_case(M, K, N, r, gate, b_std=0.05, scale=0.75, seed=5)
+    check_close(_run(case), _oracle(case), what=f"stream-K {M}x{K}x{N} r={r}")
+
+
+def test_stream_k_without_workspace_scratch():
+    """r = 0: with the workspace the size query asks for, the pair kernel cuts tiles; with
+    none it runs whole tiles only. Both match the oracle."""
+    import torch
+    import sampling_gated_lora_b200 as U
+    M, K, N = 600, 8192, 8192
+    case = W.gated_linear_case(M, K, N, 0, np.zeros(M, np.uint8), seed=6)
+    ref = _oracle(case)
+    args = [dev_tensor(a, "bf16") for a in (case.x, case.W, case.A, case.Bl)]
+    g = dev_tensor(case.gate, "u8")
+    for ws in (None, torch.zeros(16, dtype=torch.uint8, device="cuda")):
+        y = U.gated_lora_linear(*args, g, 1.0, workspace=ws)
+        check_close(host_f64(y), ref, what=f"r=0 workspace={'full' if ws is None else 'none'}")
+
+
 def test_gate_zero_matches_base_product_and_scale_zero():
     case = W.small_m_case(8)
     base = W.GatedLinearCase(case.dtype, case.x, case.W, case.A, case.Bl,
@@ -138,6 +166,7 @@ def test_grouped_qkv(M):
 
 @pytest.mark.parametrize("M,K,N,r", [(9, 4096, 12288, 128), (72, 4096, 1024, 128),
                                      (17, 264, 200, 24), (300, 1024, 520, 64),
+                                     (600, 8192, 4096, 64),   # 96 deep tiles: stream-K
                                      (2048, 4096, 12288, 128)])
 def test_silu_pair(M, K, N, r):
     """y = silu(gate(x)) * up(x) in one launch.
