@@ -89,7 +89,7 @@ uno_status uno_device_status(int32_t* bits_out, int32_t clear, void* stream);
  *   scratch below. bf16 batches with M > 256 (the CTA-pair kernel) also keep
  *   in it the fp32 partial sums of tiles whose K range two pairs of SMs share
  *   (stream-K over the last round of tiles) and the flags that order them;
- *   the call clears those flags on `stream` before its first launch.
+ *   the call clears those flags on `stream` before the pairs use them.
  *   Calls that share a workspace must not run at the same time.
  * ------------------------------------------------------------------------- */
 size_t uno_gated_lora_linear_workspace(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r);

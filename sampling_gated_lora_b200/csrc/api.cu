@@ -84,10 +84,21 @@ void attach_sk(GemmProblem* pm, const LinearLayout& L, void* workspace) {
   pm->sk_slots = pair_sk_slots();
 }
 
-// Runs the down-projection (if any) and the main launch of a gated linear,
-// zeroing the main launch's stream-K flags first.
-uno_status run_linear(const GemmLaunch* down, const GemmLaunch& main, cudaStream_t st) {
+// Prepares the down-projection launched right before `main`; it clears the
+// stream-K flags of `main` once it has waited for its own predecessor.
+uno_status prepare_down(GemmProblem d, const GemmLaunch& main, GemmLaunch* out) {
   if (main.sk_flag) {
+    d.zero_flags = main.sk_flag;
+    d.zero_words = static_cast<int>(main.sk_flag_bytes / sizeof(int32_t));
+  }
+  return gemm_prepare(d, out);
+}
+
+// Runs the down-projection (if any) and the main launch of a gated linear.
+// The main launch's stream-K flags are cleared by the down-projection (see
+// prepare_down); without one, by a memset first.
+uno_status run_linear(const GemmLaunch* down, const GemmLaunch& main, cudaStream_t st) {
+  if (main.sk_flag && !down) {
     const cudaError_t e = cudaMemsetAsync(main.sk_flag, 0, main.sk_flag_bytes, st);
     if (e != cudaSuccess) return cuda_error(e, "clearing the stream-K flags");
   }
@@ -212,13 +223,13 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   if (use_ws) attach_sk(&pm, L, workspace);
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
+  if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
   if (r > 0 && !fused) {
     const void* As[1] = {A};
-    if ((s = gemm_prepare(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), &down)) !=
-        UNO_OK)
+    if ((s = prepare_down(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), main,
+                          &down)) != UNO_OK)
       return s;
   }
-  if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
   return run_linear(r > 0 && !fused ? &down : nullptr, main, as_stream(stream));
 }
 
@@ -278,11 +289,11 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   if (use_ws) attach_sk(&pm, L, workspace);
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
+  if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
   if (r > 0 && !fused &&
-      (s = gemm_prepare(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, t_buf), &down)) !=
+      (s = prepare_down(down_problem(dt, M, K, r, x, A, G, gate, 0, scale, t_buf), main, &down)) !=
           UNO_OK)
     return s;
-  if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
   return run_linear(r > 0 && !fused ? &down : nullptr, main, as_stream(stream));
 }
 

@@ -62,7 +62,7 @@ struct PairParams {
   int dp_tiles;
   long long sk_iters;
   float* sk_part;       // [pairs][2 CTAs][4 epilogue warps][256 columns][32 rows] fp32
-  int32_t* sk_flag;     // [pairs][2 CTAs][4 epilogue warps], zero at launch
+  int32_t* sk_flag;     // [pairs][2 CTAs][4 epilogue warps], zero once the predecessor is done
 };
 static_assert(sizeof(PairParams) <= kLaunchParamBytes, "PairParams must fit GemmLaunch::params");
 
@@ -319,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __threadfence();
         __syncwarp();
+        pdl_wait();   // the flags were cleared by the preceding launch
         if (lane == 0) flag_release(p.sk_flag + fi, 1);
       } else {
         // first part of a stream-K tile (the pair's last work item, so the
@@ -327,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* part = nullptr;
         if (kb1 < nkb) {
           const int fi = (pair * 2 + static_cast<int>(rank)) * 4 + quarter;
+          pdl_wait();   // the flags were cleared by the preceding launch
           bool got = __all_sync(0xffffffffu, flag_wait(p.sk_flag + fi, 1));
           const uint32_t dst = smem_u32(smem + static_cast<uint32_t>(quarter) * kSkWarpBytes);
           if (got) {

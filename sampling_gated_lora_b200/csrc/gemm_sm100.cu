@@ -58,6 +58,8 @@ struct Gemm1Params {
   int stages;
   int tmem_cols;
   int kb_per_split, splits;
+  int32_t* zero_flags;    // cleared by CTA (0,0,0) after its wait (or NULL); 16-byte aligned
+  int zero_words;         // a multiple of 4
 };
 static_assert(sizeof(Gemm1Params) <= 256, "Gemm1Params must fit GemmLaunch::params");
 
@@ -171,6 +173,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!waited) {
         pdl_wait();
         waited = true;
+        if (p.zero_flags && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+          for (int w = 0; w < p.zero_words; w += 4)
+            *reinterpret_cast<int4*>(p.zero_flags + w) = make_int4(0, 0, 0, 0);
         if (down) pdl_trigger();
       }
     };
@@ -474,6 +479,9 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
     return set_error(UNO_ERR_INVALID_ARG, "1..3 output groups per GEMM launch");
   if (pb.mode == kEpiSiluPair && (pb.ngroups != 2 || pb.g[0].N != pb.g[1].N))
     return set_error(UNO_ERR_INVALID_ARG, "silu-pair needs two groups of equal width");
+  if (pb.zero_flags && (pb.mode != kEpiRowScale || pb.M <= 256 || pb.zero_words % 4 ||
+                        reinterpret_cast<uintptr_t>(pb.zero_flags) % 16))
+    return set_error(UNO_ERR_INVALID_ARG, "only a large-batch down-projection clears flags");
   if (gemm_pair_suits(pb)) return gemm_pair_prepare(pb, out);
   if (gemm_dec_suits(pb)) return gemm_dec_prepare(pb, out);
   if (pb.mode == kEpiSiluPair && pb.M > 256)
@@ -556,6 +564,8 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   gp.tmem_cols = pow2_at_least(bn);
   gp.kb_per_split = kb_per;
   gp.splits = splits;
+  gp.zero_flags = pb.zero_flags;
+  gp.zero_words = pb.zero_words;
 
   const uint32_t tok_box = swap ? static_cast<uint32_t>(bn) : kTileP;
   const uint32_t feat_box = swap ? static_cast<uint32_t>(feat_tile) : static_cast<uint32_t>(bn);

@@ -66,6 +66,10 @@ struct GemmProblem {
   float* sk_part;
   int32_t* sk_flag;
   int sk_slots;           // pairs the scratch serves
+  // Words this launch sets to zero once it has waited for its predecessor: a
+  // down-projection clears the stream-K flags of the GEMM launched behind it.
+  int32_t* zero_flags;
+  int zero_words;
 };
 
 // All tensor maps of one launch (passed to the kernel as one parameter).

@@ -91,6 +91,26 @@ def test_stream_k_tiles(M, K, N, r):
     check_close(_run(case), _oracle(case), what=f"stream-K {M}x{K}x{N} r={r}")
 
 
+@pytest.mark.parametrize("r", [16, 0])
+def test_stream_k_flags_cleared_by_the_call(r):
+    """A workspace whose every word already reads "ready" (1), used by two calls in a row:
+    each call clears its stream-K flags before the pairs use them (the down-projection
+    does it when r > 0, a memset when r = 0), so both match the oracle."""
+    import torch
+    import sampling_gated_lora_b200 as U
+    M, K, N = 600, 8192, 8192
+    gate = (np.arange(M) % 3 == 0).astype(np.uint8)
+    case = W.gated_linear_case(M, K, N, r, gate, b_std=0.05, seed=7)
+    ref = _oracle(case)
+    args = [dev_tensor(a, "bf16") for a in (case.x, case.W, case.A, case.Bl)]
+    g = dev_tensor(case.gate, "u8")
+    need = U.load().uno_gated_lora_linear_workspace(U.UNO_BF16, M, K, N, r)
+    ws = torch.ones(need // 4, dtype=torch.int32, device="cuda").view(torch.uint8)
+    for call in range(2):
+        y = U.gated_lora_linear(*args, g, 1.0, workspace=ws)
+        check_close(host_f64(y), ref, what=f"r={r} call {call}")
+
+
 def test_stream_k_without_workspace_scratch():
     """r = 0: with the workspace the size query asks for, the pair kernel cuts tiles; with
     none it runs whole tiles only. Both match the oracle."""
