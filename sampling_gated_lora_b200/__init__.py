@@ -139,6 +139,25 @@ def _dev(*ts):
                 raise ValueError("tensors must be contiguous")
 
 
+def _expect(t, shape, dtypes, name, optional=False):
+    """Check that tensor `t` has `shape` (None entries match any size) and one of
+    `dtypes` before any pointer reaches the library: the C ABI takes sizes from
+    a few arguments only, so a smaller buffer elsewhere would be read past its end."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if t.dim() != len(shape) or any(d is not None and t.shape[i] != d for i, d in enumerate(shape)):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {tuple(dtypes)}")
+
+
+def _floats():
+    torch = _torch()
+    return (torch.bfloat16, torch.float32)
+
+
 def _workspace(nbytes, device, workspace):
     torch = _torch()
     if nbytes == 0:
@@ -153,10 +172,16 @@ def _workspace(nbytes, device, workspace):
 def gated_lora_linear(x, W, A, Bl, gate, scale=1.0, y=None, workspace=None, stream=None):
     """y [M,N] = x W^T + scale * gate (x A^T) Bl^T (bf16 or f32 tensors, uint8 gate)."""
     torch = _torch()
-    L = load()
+    _expect(x, (None, None), _floats(), "x")
     M, K = x.shape
+    _expect(W, (None, K), (x.dtype,), "W")
     N = W.shape[0]
     r = A.shape[0] if A is not None else 0
+    _expect(A, (r, K), (x.dtype,), "A", optional=r == 0)
+    _expect(Bl, (N, r), (x.dtype,), "Bl", optional=r == 0)
+    _expect(gate, (M,), (torch.uint8,), "gate", optional=r == 0)
+    _expect(y, (M, N), (x.dtype,), "y", optional=True)
+    L = load()
     if y is None:
         y = torch.empty((M, N), dtype=x.dtype, device=x.device)
     _dev(x, W, A, Bl, gate, y)
@@ -176,11 +201,29 @@ def gated_lora_linear_group(x, Ws, As, Bls, gate, scale=1.0, silu_pair=False, ys
     Returns the list of outputs ([y] in silu-pair mode).
     """
     torch = _torch()
-    L = load()
+    _expect(x, (None, None), _floats(), "x")
     M, K = x.shape
     G = len(Ws)
+    if not 1 <= G <= 3:
+        raise ValueError(f"1 to 3 linears per call, got {G}")
     r = As[0].shape[0] if As else 0
-    Ns = [w.shape[0] for w in Ws]
+    if r > 0 and (len(As) != G or len(Bls) != G):
+        raise ValueError("As and Bls need one entry per linear")
+    Ns = []
+    for i, w in enumerate(Ws):
+        _expect(w, (None, K), (x.dtype,), f"Ws[{i}]")
+        Ns.append(w.shape[0])
+        if r > 0:
+            _expect(As[i], (r, K), (x.dtype,), f"As[{i}]")
+            _expect(Bls[i], (Ns[i], r), (x.dtype,), f"Bls[{i}]")
+    _expect(gate, (M,), (torch.uint8,), "gate", optional=r == 0)
+    if ys is not None:
+        outs = Ns[:1] if silu_pair else Ns
+        if len(ys) != len(outs):
+            raise ValueError(f"ys needs {len(outs)} outputs")
+        for i, (yt, n) in enumerate(zip(ys, outs)):
+            _expect(yt, (M, n), (x.dtype,), f"ys[{i}]")
+    L = load()
     if ys is None:
         ys = [torch.empty((M, n), dtype=x.dtype, device=x.device) for n in (Ns[:1] if silu_pair else Ns)]
     _dev(x, gate, *Ws, *As, *Bls, *ys)
@@ -196,14 +239,28 @@ def gated_lora_linear_group(x, Ws, As, Bls, gate, scale=1.0, silu_pair=False, ys
     return ys
 
 
+def _verify_shapes(p_logits, q_logits, draft, accepted_len, out_tokens, out_count, dev_status):
+    torch = _torch()
+    _expect(p_logits, (None, None, None), _floats(), "p_logits")
+    B, k_p, V = p_logits.shape
+    _expect(q_logits, (B, None, V), (p_logits.dtype,), "q_logits")
+    k = q_logits.shape[1]
+    _expect(draft, (B, k), (torch.int32,), "draft")
+    _expect(accepted_len, (B,), (torch.int32,), "accepted_len", optional=True)
+    _expect(out_tokens, (B, k + 1), (torch.int32,), "out_tokens", optional=True)
+    _expect(out_count, (B,), (torch.int32,), "out_count", optional=True)
+    _expect(dev_status, (1,), (torch.int32,), "dev_status", optional=True)
+    return B, k, k_p, V
+
+
 def psi_verify(p_logits, q_logits, draft, temperature, seed, step, seq_offset=0,
                accepted_len=None, out_tokens=None, out_count=None, dev_status=None,
                workspace=None, stream=None):
     """Verify one block per sequence; returns (accepted_len [B], out_tokens [B,k+1], out_count [B])."""
     torch = _torch()
+    B, k, k_p, V = _verify_shapes(p_logits, q_logits, draft, accepted_len, out_tokens, out_count,
+                                  dev_status)
     L = load()
-    B, k_p, V = p_logits.shape
-    k = q_logits.shape[1]
     dev = p_logits.device
     i32 = dict(dtype=torch.int32, device=dev)
     accepted_len = torch.empty(B, **i32) if accepted_len is None else accepted_len
@@ -224,9 +281,9 @@ def psi_verify_noalloc(p_logits, q_logits, draft, temperature, seed, step, seq_o
                        stream=None):
     """psi_verify with the library's static stats scratch (no workspace argument)."""
     torch = _torch()
+    B, k, k_p, V = _verify_shapes(p_logits, q_logits, draft, accepted_len, out_tokens, out_count,
+                                  dev_status)
     L = load()
-    B, k_p, V = p_logits.shape
-    k = q_logits.shape[1]
     dev = p_logits.device
     i32 = dict(dtype=torch.int32, device=dev)
     accepted_len = torch.empty(B, **i32) if accepted_len is None else accepted_len
@@ -245,8 +302,11 @@ def draft_sample(q_logits, temperature, seed, step, seq_offset=0, draft=None, de
                  stream=None):
     """Linear-sampler draft: draft [B,k] int32 from softmax(q_logits / T)."""
     torch = _torch()
-    L = load()
+    _expect(q_logits, (None, None, None), _floats(), "q_logits")
     B, k, V = q_logits.shape
+    _expect(draft, (B, k), (torch.int32,), "draft", optional=True)
+    _expect(dev_status, (1,), (torch.int32,), "dev_status", optional=True)
+    L = load()
     draft = torch.empty((B, k), dtype=torch.int32, device=q_logits.device) if draft is None else draft
     _dev(q_logits, draft, dev_status)
     _check(L.uno_draft_sample(_dtype(q_logits), B, k, V, _ptr(q_logits), float(temperature),
@@ -268,6 +328,8 @@ def philox_uniforms(seed, step, stream_id, index0, n, device="cuda", stream=None
 
 def rmsnorm(x, eps=1e-6, y=None, stream=None):
     torch = _torch()
+    _expect(x, (None, None), (torch.bfloat16,), "x")
+    _expect(y, tuple(x.shape), (torch.bfloat16,), "y", optional=True)
     L = load()
     y = torch.empty_like(x) if y is None else y
     _dev(x, y)
@@ -278,6 +340,9 @@ def rmsnorm(x, eps=1e-6, y=None, stream=None):
 
 def silu_mul(a, b, y=None, stream=None):
     torch = _torch()
+    _expect(a, tuple(a.shape), (torch.bfloat16,), "a")
+    _expect(b, tuple(a.shape), (torch.bfloat16,), "b")
+    _expect(y, tuple(a.shape), (torch.bfloat16,), "y", optional=True)
     L = load()
     y = torch.empty_like(a) if y is None else y
     _dev(a, b, y)
@@ -304,17 +369,31 @@ class Model:
     """
 
     def __init__(self, layers, head, hidden, q_out, kv_out, inter, vocab, r, scale=1.0):
+        torch = _torch()
+        # (out, in) of every linear, in LINEAR_NAMES order
+        dims = {"q": (q_out, hidden), "k": (kv_out, hidden), "v": (kv_out, hidden),
+                "o": (hidden, q_out), "gate": (inter, hidden), "up": (inter, hidden),
+                "down": (hidden, inter)}
+        bf16 = (torch.bfloat16,)
+
+        def check(parts, n_out, n_in, name):
+            if len(parts) != 3:
+                raise ValueError(f"{name}: expected (W, A, Bl)")
+            _expect(parts[0], (n_out, n_in), bf16, f"{name} W")
+            _expect(parts[1], (r, n_in), bf16, f"{name} A", optional=r == 0)
+            _expect(parts[2], (n_out, r), bf16, f"{name} Bl", optional=r == 0)
+
+        for li, lw in enumerate(layers):
+            for name in LINEAR_NAMES:
+                check(lw[name], *dims[name], f"layer {li} {name}")
+        check(head, vocab, hidden, "head")
         L = load()
         self._keep = (layers, head)
         ptrs = []
-        for lw in layers:
-            for name in LINEAR_NAMES:
-                for t in lw[name]:
-                    _dev(t)
-                    ptrs.append(t.data_ptr())
-        for t in head:
-            _dev(t)
-            ptrs.append(t.data_ptr())
+        for parts in [lw[name] for lw in layers for name in LINEAR_NAMES] + [head]:
+            for t in parts:
+                _dev(t)
+                ptrs.append(None if t is None else t.data_ptr())
         arr = (ctypes.c_void_p * len(ptrs))(*ptrs)
         h = ctypes.c_void_p()
         _check(L.uno_model_create(ctypes.byref(h), len(layers), hidden, q_out, kv_out, inter,
@@ -344,6 +423,21 @@ class Model:
              accepted_len, out_tokens, out_count, workspace, logits_out=None, dev_status=None,
              seq_offset=0, stream=None):
         """uno_psi_step on caller-provided device buffers (see include/uno.h)."""
+        torch = _torch()
+        bf16, i32 = (torch.bfloat16,), (torch.int32,)
+        V = self.vocab
+        _expect(h_in, (B * (2 * k + 1), self.hidden), bf16, "h_in")
+        _expect(q_prev, (B, k, V), bf16, "q_prev")
+        _expect(q_next, (B, k, V), bf16, "q_next")
+        _expect(d_prev, (B, k), i32, "d_prev")
+        _expect(d_next, (B, k), i32, "d_next")
+        _expect(accepted_len, (B,), i32, "accepted_len")
+        _expect(out_tokens, (B, k + 1), i32, "out_tokens")
+        _expect(out_count, (B,), i32, "out_count")
+        _expect(logits_out, (B * (k + 1), V), bf16, "logits_out", optional=True)
+        _expect(dev_status, (1,), i32, "dev_status", optional=True)
+        if workspace is None:
+            raise ValueError("workspace is required (Model.workspace_bytes(B, k) bytes)")
         _dev(h_in, q_prev, d_prev, q_next, d_next, accepted_len, out_tokens, out_count, workspace,
              logits_out, dev_status)
         wsb = workspace.numel() * workspace.element_size()
