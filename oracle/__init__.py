@@ -15,6 +15,8 @@ Modules
   sampling      softmax at temperature T, inverse-CDF draws, the draft
                 sampler, acceptance, first rejection, residual and bonus.
   stack         the synthetic decoder stack + LM head used by the step.
+  tree          the tree sampler: several drafted blocks verified as a prefix
+                tree (multi-candidate rejection sampling along the trie).
 
 Every function states the passage it follows. No function here is "parity
 unpinned": each has pins in tests/test_oracle_*.py.
