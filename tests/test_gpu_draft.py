@@ -79,7 +79,6 @@ def _positions():
 @pytest.mark.parametrize("which", [0, 1])
 def test_draft_chi_square_million(which):
     """10^6 GPU draft samples of one position against softmax(q / T)."""
-    import torch
     p, q, pos = _positions()
     j = pos[which]
     Q = _replicate(q[j], 1024)
