@@ -131,3 +131,29 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(U, "LIB_PATH", "/nonexistent/libuno.so")
     with pytest.raises(RuntimeError, match="missing"):
         U.load()
+
+
+def test_workspace_sizes_hold_the_stream_k_scratch():
+    """bf16 batches of more than 256 rows (the CTA-pair kernel) add the stream-K scratch:
+    one fp32 256 x 256 partial tile per pair of SMs and 32 bytes of flags per pair
+    (148 SMs assumed without a GPU); f32 and smaller batches do not."""
+    L = U.load()
+    pairs = 148 // 2
+    part, flags = pairs * 256 * 256 * 4, pairs * 32
+    ws = lambda dt, M, r: L.uno_gated_lora_linear_workspace(dt, M, 4096, 4096, r)
+    t_bytes = 300 * 128 * 2
+    assert ws(U.UNO_BF16, 256, 128) == 256 * 128 * 2
+    assert ws(U.UNO_BF16, 300, 128) >= t_bytes + part + flags
+    assert ws(U.UNO_BF16, 300, 0) >= part + flags            # r = 0: the scratch alone
+    assert ws(U.UNO_F32, 300, 128) == 300 * 128 * 4
+    g = L.uno_gated_lora_linear_group_workspace
+    assert g(U.UNO_BF16, 300, 128, 3) >= 3 * t_bytes + part + flags
+    assert g(U.UNO_BF16, 200, 128, 3) == 200 * 3 * 128 * 2
+    # the step: one partial-sum region and a flag block per main GEMM (4 a layer + head)
+    h = ctypes.c_void_p()
+    ptrs = (ctypes.c_void_p * 24)(*([0x10000] * 24))
+    assert L.uno_model_create(ctypes.byref(h), 1, 16, 16, 16, 16, 16, 8, 1.0, ptrs) == 0
+    small, big = L.uno_psi_step_workspace(h, 8, 8), L.uno_psi_step_workspace(h, 16, 8)
+    L.uno_model_destroy(h)
+    # 136 rows (no scratch) vs 272 rows: every other buffer only grows with the rows
+    assert big - small >= part + 5 * flags
