@@ -328,12 +328,12 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   return r;
 }
 // All threads of all CTAs of the cluster; release our shared-memory writes,
-// acquire everyone else's. The warp is reconverged first (the barrier is
-// .aligned: every lane of a warp must execute the same instance).
+// acquire everyone else's.
 // The kernels give whole roles to single lanes (TMA producer, MMA issuer), so
 // a warp can reach a barrier split in time. The .aligned barrier forms assume
 // converged warps and were seen to complete early in that case; these
-// barriers use the per-thread (non-aligned) forms.
+// barriers use the per-thread (non-aligned) forms, which any subset of a
+// warp's lanes may execute at different times.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile(
       "barrier.cluster.arrive.release;\n\t"
