@@ -17,6 +17,8 @@ Modules
   stack         the synthetic decoder stack + LM head used by the step.
   tree          the tree sampler: several drafted blocks verified as a prefix
                 tree (multi-candidate rejection sampling along the trie).
+  distill       the distillation objective alpha KL + beta TV between teacher
+                and student rows, and its gradient w.r.t. the student logits.
 
 Every function states the passage it follows. No function here is "parity
 unpinned": each has pins in tests/test_oracle_*.py.
