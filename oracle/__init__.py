@@ -11,7 +11,8 @@ path and never consumes a value the CUDA path produced.
 
 Modules
   philox        Philox4x32-10 counter-based generator and the uniform maps.
-  gated_linear  y = x W^T + s g (x A^T) Bl^T.
+  gated_linear  y = x W^T + s g (x A^T) Bl^T, and the adapter's gradients
+                (dA, dBl) with theta_AR frozen.
   sampling      softmax at temperature T, inverse-CDF draws, the draft
                 sampler, acceptance, first rejection, residual and bonus.
   stack         the synthetic decoder stack + LM head used by the step.

@@ -65,3 +65,48 @@ def test_gate_is_per_row():
     off = gated_linear(x, W, A, Bl, np.zeros(7, np.uint8), 0.5)
     for m in range(7):
         np.testing.assert_array_equal(y[m], (on if g[m] else off)[m])
+
+
+# ---------------------------------------------------------------- adapter backward (NEXT f4)
+
+def _bw_case(M=7, K=6, N=5, r=3, seed=0):
+    rng = np.random.default_rng(seed)
+    return (rng.normal(size=(M, K)), rng.normal(size=(N, K)), rng.normal(size=(r, K)),
+            rng.normal(size=(N, r)), (rng.random(M) < 0.5).astype(np.uint8), 0.8,
+            rng.normal(size=(M, N)))
+
+
+def test_adapter_grads_match_finite_differences():
+    from oracle.gated_linear import gated_linear_adapter_grads
+    x, W, A, Bl, g, s, dy = _bw_case()
+    dA, dBl = gated_linear_adapter_grads(x, A, Bl, g, s, dy)
+    f = lambda A_, Bl_: float((dy * gated_linear(x, W, A_, Bl_, g, s)).sum())
+    h = 1e-6
+    for P, G, name in ((A, dA, "A"), (Bl, dBl, "Bl")):
+        num = np.zeros_like(P)
+        for idx in np.ndindex(P.shape):
+            e = np.zeros_like(P)
+            e[idx] = h
+            num[idx] = ((f(A + e, Bl) - f(A - e, Bl)) if name == "A" else
+                        (f(A, Bl + e) - f(A, Bl - e))) / (2 * h)
+        np.testing.assert_allclose(G, num, rtol=1e-6, atol=1e-8)
+
+
+def test_adapter_grads_special_cases():
+    """Gate 0 everywhere or scale 0: no gradient; gate 1 everywhere: the merged-weight
+    form y = x (W + s Bl A)^T gives dBl = s dy^T x A^T and dA = s Bl^T dy^T x."""
+    from oracle.gated_linear import gated_linear_adapter_grads
+    x, W, A, Bl, g, s, dy = _bw_case(seed=1)
+    for gate, scale in ((np.zeros_like(g), s), (g, 0.0)):
+        dA, dBl = gated_linear_adapter_grads(x, A, Bl, gate, scale, dy)
+        assert not dA.any() and not dBl.any()
+    ones = np.ones_like(g)
+    dA, dBl = gated_linear_adapter_grads(x, A, Bl, ones, s, dy)
+    np.testing.assert_allclose(dBl, s * dy.T @ x @ A.T, rtol=1e-12)
+    np.testing.assert_allclose(dA, s * Bl.T @ dy.T @ x, rtol=1e-12)
+    # only gate-1 rows count: the gradient equals that of the gate-1 rows alone
+    keep = g.astype(bool)
+    dA1, dBl1 = gated_linear_adapter_grads(x[keep], A, Bl, ones[keep], s, dy[keep])
+    dA, dBl = gated_linear_adapter_grads(x, A, Bl, g, s, dy)
+    np.testing.assert_allclose(dA, dA1, rtol=1e-12)
+    np.testing.assert_allclose(dBl, dBl1, rtol=1e-12)
