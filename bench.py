@@ -447,7 +447,9 @@ def run_uno(args):
         if tensor_bound:
             ach = flops / us / 1e6
             roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 3), "traffic": None}
+                    "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 3), "traffic": None,
+                    "peak_sustained": pk["bf16_tflops_sustained"],
+                    "frac_sustained": round(ach / pk["bf16_tflops_sustained"], 3)}
         else:
             ach = byts / us / 1e3
             roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
