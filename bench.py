@@ -414,7 +414,10 @@ def run_uno(args):
     e2e_tokens = int(cnt_h.sum())
     e2e_ms_max, e2e_tok_all = combine_over_ranks(e2e_ms, e2e_tokens, dist if world > 1 else None,
                                                   "cuda")
+    # the e2e steps draw other tokens than the timed steps (other step indices), so their
+    # tokens/s also moves with the accepted counts; ms_per_step shows the copies' cost
     e2e = {"value": round(e2e_tok_all / (e2e_ms_max / 1e3), 1), "unit": "tokens/s",
+           "ms_per_step": round(e2e_ms_max / args.steps, 3),
            "h2d_bytes_per_step": h_host.numel() * 2,
            "d2h_bytes_per_step": (acc_h[0].numel() + tok_h[0].numel() + cnt_h[0].numel()) * 4}
 
