@@ -167,7 +167,10 @@ uno_status uno_psi_verify(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32
  *   Setup: the first call on a device (the current device, which must own
  *     the buffers and the stream) looks up the array's device address, which
  *     may load the library's module; make that first call before any stream
- *     capture begins. Later calls do no setup.
+ *     capture begins. Later calls do no setup and reuse that address, so a
+ *     device reset (cudaDeviceReset, or the primary context destroyed and
+ *     created again) leaves it stale: do not call this entry point on that
+ *     device again in the same process after one.
  *   Starting values: none needed; every entry a call reads it wrote itself.
  *   Concurrency: all calls on one device share the array. Calls on one stream
  *     are ordered and safe; calls whose kernels may overlap (other streams

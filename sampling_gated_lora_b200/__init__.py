@@ -114,11 +114,24 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, device=None):
+    """cudaStream_t of `stream` (default: the current stream of `device`); an
+    explicit stream must belong to `device`."""
     torch = _torch()
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _launch(device, stream, cfn, *args):
+    """Call library function `cfn(*args, stream)` with `device` current, so the
+    library's device queries and launches address the device that holds the
+    tensors; raise on a non-OK status."""
+    torch = _torch()
+    with torch.cuda.device(device):
+        _check(cfn(*args, _stream(stream, device)))
 
 
 def _dtype(t):
@@ -131,12 +144,19 @@ def _dtype(t):
 
 
 def _dev(*ts):
+    """Check that the tensors are contiguous and all on one CUDA device; return it."""
+    device = None
     for t in ts:
         if t is not None:
             if not t.is_cuda:
                 raise ValueError("tensors must be on a CUDA device")
             if not t.is_contiguous():
                 raise ValueError("tensors must be contiguous")
+            if device is None:
+                device = t.device
+            elif t.device != device:
+                raise ValueError(f"tensors on {device} and {t.device}: one device per call")
+    return device
 
 
 def _expect(t, shape, dtypes, name, optional=False):
@@ -184,13 +204,12 @@ def gated_lora_linear(x, W, A, Bl, gate, scale=1.0, y=None, workspace=None, stre
     L = load()
     if y is None:
         y = torch.empty((M, N), dtype=x.dtype, device=x.device)
-    _dev(x, W, A, Bl, gate, y)
+    dev = _dev(x, W, A, Bl, gate, y, workspace)
     dt = _dtype(x)
     need = L.uno_gated_lora_linear_workspace(dt, M, K, N, r)
-    ws, wsb = _workspace(need, x.device, workspace)
-    _check(L.uno_gated_lora_linear(dt, M, K, N, r, _ptr(x), _ptr(W), _ptr(A), _ptr(Bl),
-                                   _ptr(gate), float(scale), _ptr(y), _ptr(ws), wsb,
-                                   _stream(stream)))
+    ws, wsb = _workspace(need, dev, workspace)
+    _launch(dev, stream, L.uno_gated_lora_linear, dt, M, K, N, r, _ptr(x), _ptr(W), _ptr(A),
+            _ptr(Bl), _ptr(gate), float(scale), _ptr(y), _ptr(ws), wsb)
     return y
 
 
@@ -226,16 +245,16 @@ def gated_lora_linear_group(x, Ws, As, Bls, gate, scale=1.0, silu_pair=False, ys
     L = load()
     if ys is None:
         ys = [torch.empty((M, n), dtype=x.dtype, device=x.device) for n in (Ns[:1] if silu_pair else Ns)]
-    _dev(x, gate, *Ws, *As, *Bls, *ys)
+    dev = _dev(x, gate, *Ws, *As, *Bls, *ys, workspace)
     dt = _dtype(x)
     need = L.uno_gated_lora_linear_group_workspace(dt, M, r, G)
-    ws, wsb = _workspace(need, x.device, workspace)
+    ws, wsb = _workspace(need, dev, workspace)
     arr = lambda ts: (ctypes.c_void_p * G)(*[t.data_ptr() for t in ts])
     yarr = (ctypes.c_void_p * G)(*[ys[min(i, len(ys) - 1)].data_ptr() for i in range(G)])
     Narr = (ctypes.c_int64 * G)(*Ns)
-    _check(L.uno_gated_lora_linear_group(dt, M, K, r, G, Narr, _ptr(x), arr(Ws), arr(As), arr(Bls),
-                                         _ptr(gate), float(scale), 1 if silu_pair else 0, yarr,
-                                         _ptr(ws), wsb, _stream(stream)))
+    _launch(dev, stream, L.uno_gated_lora_linear_group, dt, M, K, r, G, Narr, _ptr(x), arr(Ws),
+            arr(As), arr(Bls), _ptr(gate), float(scale), 1 if silu_pair else 0, yarr, _ptr(ws),
+            wsb)
     return ys
 
 
@@ -266,13 +285,13 @@ def psi_verify(p_logits, q_logits, draft, temperature, seed, step, seq_offset=0,
     accepted_len = torch.empty(B, **i32) if accepted_len is None else accepted_len
     out_tokens = torch.empty((B, k + 1), **i32) if out_tokens is None else out_tokens
     out_count = torch.empty(B, **i32) if out_count is None else out_count
-    _dev(p_logits, q_logits, draft, accepted_len, out_tokens, out_count, dev_status)
+    _dev(p_logits, q_logits, draft, accepted_len, out_tokens, out_count, dev_status, workspace)
     need = L.uno_psi_verify_workspace(B, k, k_p, V)
     ws, wsb = _workspace(need, dev, workspace)
-    _check(L.uno_psi_verify(_dtype(p_logits), B, k, k_p, V, _ptr(p_logits), _ptr(q_logits),
-                            _ptr(draft), float(temperature), int(seed), int(step), int(seq_offset),
-                            _ptr(accepted_len), _ptr(out_tokens), _ptr(out_count),
-                            _ptr(dev_status), _ptr(ws), wsb, _stream(stream)))
+    _launch(dev, stream, L.uno_psi_verify, _dtype(p_logits), B, k, k_p, V, _ptr(p_logits),
+            _ptr(q_logits), _ptr(draft), float(temperature), int(seed), int(step),
+            int(seq_offset), _ptr(accepted_len), _ptr(out_tokens), _ptr(out_count),
+            _ptr(dev_status), _ptr(ws), wsb)
     return accepted_len, out_tokens, out_count
 
 
@@ -290,11 +309,10 @@ def psi_verify_noalloc(p_logits, q_logits, draft, temperature, seed, step, seq_o
     out_tokens = torch.empty((B, k + 1), **i32) if out_tokens is None else out_tokens
     out_count = torch.empty(B, **i32) if out_count is None else out_count
     _dev(p_logits, q_logits, draft, accepted_len, out_tokens, out_count, dev_status)
-    _check(L.uno_psi_verify_noalloc(_dtype(p_logits), B, k, k_p, V, _ptr(p_logits),
-                                    _ptr(q_logits), _ptr(draft), float(temperature), int(seed),
-                                    int(step), int(seq_offset), _ptr(accepted_len),
-                                    _ptr(out_tokens), _ptr(out_count), _ptr(dev_status),
-                                    _stream(stream)))
+    _launch(dev, stream, L.uno_psi_verify_noalloc, _dtype(p_logits), B, k, k_p, V,
+            _ptr(p_logits), _ptr(q_logits), _ptr(draft), float(temperature), int(seed),
+            int(step), int(seq_offset), _ptr(accepted_len), _ptr(out_tokens), _ptr(out_count),
+            _ptr(dev_status))
     return accepted_len, out_tokens, out_count
 
 
@@ -308,10 +326,10 @@ def draft_sample(q_logits, temperature, seed, step, seq_offset=0, draft=None, de
     _expect(dev_status, (1,), (torch.int32,), "dev_status", optional=True)
     L = load()
     draft = torch.empty((B, k), dtype=torch.int32, device=q_logits.device) if draft is None else draft
-    _dev(q_logits, draft, dev_status)
-    _check(L.uno_draft_sample(_dtype(q_logits), B, k, V, _ptr(q_logits), float(temperature),
-                              int(seed), int(step), int(seq_offset), _ptr(draft), _ptr(dev_status),
-                              None, 0, _stream(stream)))
+    dev = _dev(q_logits, draft, dev_status)
+    _launch(dev, stream, L.uno_draft_sample, _dtype(q_logits), B, k, V, _ptr(q_logits),
+            float(temperature), int(seed), int(step), int(seq_offset), _ptr(draft),
+            _ptr(dev_status), None, 0)
     return draft
 
 
@@ -321,8 +339,8 @@ def philox_uniforms(seed, step, stream_id, index0, n, device="cuda", stream=None
     L = load()
     words = torch.empty(n, dtype=torch.int32, device=device)
     u = torch.empty(n, dtype=torch.float32, device=device)
-    _check(L.uno_philox_uniforms(int(seed), int(step), int(stream_id), int(index0), int(n),
-                                 _ptr(words), _ptr(u), _stream(stream)))
+    _launch(words.device, stream, L.uno_philox_uniforms, int(seed), int(step), int(stream_id),
+            int(index0), int(n), _ptr(words), _ptr(u))
     return words.to(torch.int64) & 0xFFFFFFFF, u
 
 
@@ -332,9 +350,9 @@ def rmsnorm(x, eps=1e-6, y=None, stream=None):
     _expect(y, tuple(x.shape), (torch.bfloat16,), "y", optional=True)
     L = load()
     y = torch.empty_like(x) if y is None else y
-    _dev(x, y)
+    dev = _dev(x, y)
     M, D = x.shape
-    _check(L.uno_rmsnorm(M, D, _ptr(x), _ptr(y), float(eps), _stream(stream)))
+    _launch(dev, stream, L.uno_rmsnorm, M, D, _ptr(x), _ptr(y), float(eps))
     return y
 
 
@@ -345,16 +363,19 @@ def silu_mul(a, b, y=None, stream=None):
     _expect(y, tuple(a.shape), (torch.bfloat16,), "y", optional=True)
     L = load()
     y = torch.empty_like(a) if y is None else y
-    _dev(a, b, y)
-    _check(L.uno_silu_mul(a.numel(), _ptr(a), _ptr(b), _ptr(y), _stream(stream)))
+    dev = _dev(a, b, y)
+    _launch(dev, stream, L.uno_silu_mul, a.numel(), _ptr(a), _ptr(b), _ptr(y))
     return y
 
 
-def device_status(clear=True, stream=None) -> int:
-    """The library-wide device status bits (UNO_DEV_*), optionally cleared."""
+def device_status(clear=True, stream=None, device=None) -> int:
+    """The library-wide device status bits (UNO_DEV_*) of `device` (default: the
+    current device), optionally cleared."""
+    torch = _torch()
     L = load()
     v = ctypes.c_int32(0)
-    _check(L.uno_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _launch(dev, stream, L.uno_device_status, ctypes.byref(v), 1 if clear else 0)
     return v.value
 
 
@@ -390,10 +411,11 @@ class Model:
         L = load()
         self._keep = (layers, head)
         ptrs = []
-        for parts in [lw[name] for lw in layers for name in LINEAR_NAMES] + [head]:
-            for t in parts:
-                _dev(t)
-                ptrs.append(None if t is None else t.data_ptr())
+        tensors = [t for parts in [lw[name] for lw in layers for name in LINEAR_NAMES] + [head]
+                   for t in parts]
+        self.device = _dev(*tensors)
+        for t in tensors:
+            ptrs.append(None if t is None else t.data_ptr())
         arr = (ctypes.c_void_p * len(ptrs))(*ptrs)
         h = ctypes.c_void_p()
         _check(L.uno_model_create(ctypes.byref(h), len(layers), hidden, q_out, kv_out, inter,
@@ -438,12 +460,12 @@ class Model:
         _expect(dev_status, (1,), i32, "dev_status", optional=True)
         if workspace is None:
             raise ValueError("workspace is required (Model.workspace_bytes(B, k) bytes)")
-        _dev(h_in, q_prev, d_prev, q_next, d_next, accepted_len, out_tokens, out_count, workspace,
-             logits_out, dev_status)
+        dev = _dev(h_in, q_prev, d_prev, q_next, d_next, accepted_len, out_tokens, out_count,
+                   workspace, logits_out, dev_status)
+        if dev != self.device:
+            raise ValueError(f"step buffers on {dev}, the model's weights on {self.device}")
         wsb = workspace.numel() * workspace.element_size()
-        _check(load().uno_psi_step(self._h, B, k, _ptr(h_in), _ptr(q_prev), _ptr(d_prev),
-                                   float(temperature), int(seed), int(step), int(seq_offset),
-                                   _ptr(q_next),
-                                   _ptr(d_next), _ptr(logits_out), _ptr(accepted_len),
-                                   _ptr(out_tokens), _ptr(out_count), _ptr(dev_status),
-                                   _ptr(workspace), wsb, _stream(stream)))
+        _launch(dev, stream, load().uno_psi_step, self._h, B, k, _ptr(h_in), _ptr(q_prev),
+                _ptr(d_prev), float(temperature), int(seed), int(step), int(seq_offset),
+                _ptr(q_next), _ptr(d_next), _ptr(logits_out), _ptr(accepted_len),
+                _ptr(out_tokens), _ptr(out_count), _ptr(dev_status), _ptr(workspace), wsb)

@@ -143,6 +143,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order this thread's generic-proxy global-memory accesses (a flag acquired,
+// data stored) with its later async-proxy accesses (a bulk copy): acquire and
+// release order only the generic proxy, so a bulk copy of data another CTA
+// published behind a flag needs this between the acquire and the copy.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {

@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) part[(c + j) * 32 + lane] = v[j];
         }
+        fence_proxy_async_global();   // the reader copies them with the async proxy
         __threadfence();
         __syncwarp();
         pdl_wait();   // the flags were cleared by the preceding launch
@@ -333,6 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t dst = smem_u32(smem + static_cast<uint32_t>(quarter) * kSkWarpBytes);
           if (got) {
             if (lane == 0) {
+              // the partial sums were stored through the generic proxy; the
+              // bulk copy reads through the async proxy
+              fence_proxy_async_global();
               mbar_arrive_expect_tx(smem_u32(&skbar[quarter]), kSkWarpBytes);
               bulk_load(dst, p.sk_part + static_cast<size_t>(fi) * kSkWarpFloats, kSkWarpBytes,
                         smem_u32(&skbar[quarter]));

@@ -93,18 +93,21 @@ __device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s
   m = mx;
 }
 
-// Grid: (chunks, rows). Row r < rows_p reads p_logits row r, else q_logits
-// row r - rows_p. Writes stats[r * chunks + chunk] = (m, s).
+// Grid: rows * chunks blocks, one per (row, vocab chunk), chunk fastest (a
+// one-dimensional grid, so the row count is not held to gridDim.y's 65535).
+// Row r < rows_p reads p_logits row r, else q_logits row r - rows_p. Writes
+// stats[r * chunks + chunk] = (m, s).
 template <typename T>
 __global__ void __launch_bounds__(kStatThreads)
     row_stats_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits, int rows_p,
-                     int V, int chunk_len, float c, float2* __restrict__ stats) {
+                     int V, int chunks, int chunk_len, float c, float2* __restrict__ stats) {
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
-  const int row = blockIdx.y;
+  const int row = static_cast<int>(blockIdx.x / static_cast<unsigned>(chunks));
+  const int chunk = static_cast<int>(blockIdx.x - static_cast<unsigned>(row) * chunks);
   const T* z = row < rows_p ? p_logits + static_cast<size_t>(row) * V
                             : q_logits + static_cast<size_t>(row - rows_p) * V;
-  const int lo = blockIdx.x * chunk_len;
+  const int lo = chunk * chunk_len;
   const int hi = min(V, lo + chunk_len);
   constexpr int kN = Vec<T>::n;
   OnlineStat st;
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(kStatThreads)
     float M = sm[0], S = ss[0];
     for (int w = 1; w < kStatThreads / 32; ++w) merge_stat(M, S, sm[w], ss[w], c);
     // a NaN anywhere in the chunk makes S NaN (fmaxf skips it in the max)
-    stats[static_cast<size_t>(row) * gridDim.x + blockIdx.x] = make_float2(M, S);
+    stats[blockIdx.x] = make_float2(M, S);
   }
 }
 
@@ -634,17 +637,17 @@ uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s) {
   fp.status = a.dev_status;
   fp.chunk_elems = chunk_elems;
   const size_t smem = static_cast<size_t>(chunk_elems) * esz * 2;
-  const dim3 grid(chunks, rows);
+  const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(rows) * chunks));
   cudaError_t e;
   if (a.dt == UNO_F32) {
     e = launch_kernel(row_stats_kernel<float>, grid, dim3(kStatThreads), 0, s, 1,
                       static_cast<const float*>(a.p_logits), static_cast<const float*>(a.q_logits),
-                      a.B * a.k_p, a.V, chunk_len, c, stats);
+                      a.B * a.k_p, a.V, chunks, chunk_len, c, stats);
   } else {
     e = launch_kernel(row_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1,
                       static_cast<const __nv_bfloat16*>(a.p_logits),
-                      static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.k_p, a.V, chunk_len,
-                      c, stats);
+                      static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.k_p, a.V, chunks,
+                      chunk_len, c, stats);
   }
   if (e != cudaSuccess) return cuda_error(e, "row_stats launch");
   if (a.dt == UNO_F32)

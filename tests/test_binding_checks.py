@@ -139,3 +139,31 @@ def test_model_weight_mismatch_raises():
     with pytest.raises(ValueError, match="head W has shape"):
         U.Model(layers, (head[0][:-8], head[1], head[2]), s.hidden, s.q_out, s.kv_out, s.inter,
                 s.vocab, s.r)
+
+
+class _FakeCuda:
+    """Stands in for a contiguous CUDA tensor on device `cuda:<i>` (no GPU here)."""
+
+    def __init__(self, index):
+        self.is_cuda = True
+        self.device = torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return True
+
+
+def test_operands_on_two_devices_are_rejected():
+    """The library launches on the current device; tensors on another device would be
+    addressed from the wrong context, so the binding refuses mixed devices."""
+    a, b = _FakeCuda(0), _FakeCuda(1)
+    assert U._dev(a, None, _FakeCuda(0)) == torch.device("cuda", 0)
+    with pytest.raises(ValueError, match="one device per call"):
+        U._dev(a, b)
+
+
+def test_stream_of_another_device_is_rejected():
+    class _S:
+        device = torch.device("cuda", 1)
+        cuda_stream = 0
+    with pytest.raises(ValueError, match="stream is on"):
+        U._stream(_S(), torch.device("cuda", 0))

@@ -11,7 +11,7 @@ import pytest
 
 import workloads as W
 from oracle import sampling as S
-from gpu_util import check_verify_outputs_valid, dev_tensor
+from gpu_util import check_verify_outputs_valid, compare_verify, dev_tensor
 
 pytestmark = pytest.mark.gpu
 
@@ -54,6 +54,30 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
         np.testing.assert_array_equal(a, b)
 
 
+def test_noalloc_more_logit_rows_than_a_grid_dimension_holds():
+    """B (k_p + k) = 2048 * 33 = 67,584 logit rows, above 65,535 (the most one grid
+    dimension other than x takes); V = 64 keeps the stats (8 bytes a row) inside the
+    static scratch. The static-scratch call must match the workspace call exactly,
+    and both the oracle on sampled sequences."""
+    import sampling_gated_lora_b200 as U
+    B, k, k_p, V, T, seed, step = 2048, 16, 17, 64, 1.0, 31, 2
+    L = U.load()
+    assert B * (k_p + k) > 65535
+    assert L.uno_psi_verify_workspace(B, k, k_p, V) <= (2 << 20)
+    case = W.logits_case(B, k, V, k_p=k_p, ar_std=2.0, sigma=1.0, peak_frac=0.0, seed=seed)
+    d = S.draft_sample(case.q_logits, T, seed + 1, step)
+    P, Q, D = dev_tensor(case.p_logits, "bf16"), dev_tensor(case.q_logits, "bf16"), dev_tensor(d, "i32")
+    got = _host(U.psi_verify_noalloc(P, Q, D, T, seed, step))
+    want = _host(U.psi_verify(P, Q, D, T, seed, step))
+    for a, b in zip(got, want):
+        np.testing.assert_array_equal(a, b)
+    check_verify_outputs_valid(*got, d, k, k_p, V)
+    sample = list(range(0, B, 97)) + [B - 1]
+    ora = S.psi_verify(case.p_logits, case.q_logits, d, T, seed, step, sequences=sample)
+    excused, bad = compare_verify(got, ora, k, sample)
+    assert not bad and len(excused) <= 1
+
+
 def test_noalloc_rejects_sizes_beyond_the_static_scratch():
     import sampling_gated_lora_b200 as U
     L = U.load()
@@ -63,5 +87,6 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch():
                                   None, None, None, None, None)
     assert st == 2                               # UNO_ERR_UNSUPPORTED, nothing launched
     assert b"static scratch" in L.uno_last_error()
-    # the largest size that fits is accepted by the size check (k_p = k: 2k rows per sequence)
+    # the largest size that fits is accepted by the size check (k_p = k: 2k rows per
+    # sequence); the kernels' grids take any row count (one-dimensional)
     assert L.uno_psi_verify_workspace(8192, 16, 16, V) <= (2 << 20)
