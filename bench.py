@@ -320,6 +320,45 @@ def kernel_lines(U, torch, pk):
             "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3),
             "mean_accepted": round(float(outs[0].float().mean()), 3)}
         del p, q
+    # tree_verify at low batch: B=8 sequences, N=4 candidate blocks of k=8, V=151936.
+    # Candidates: the linear sampler on q repeated N times per sequence (Philox index
+    # (b N + i) k + j, the tree sampler's); AR row of each trie node = the draft row of
+    # its depth + N(0, 1) noise. Algorithmic bytes: one read of every node row and q row.
+    B, N, k, V = 8, 4, 8, 151936
+    _, q = W.logits_case_torch(B, k, V, sigma=1.0, seed=77)
+    cands = U.draft_sample(q.repeat_interleave(N, dim=0), 1.0, 5, 0).reshape(B, N, k).contiguous()
+    c_host = cands.cpu().numpy()
+    R = N * k + 1
+    depth_idx = torch.zeros((B, R), dtype=torch.long)
+    nodes = 0
+    for b in range(B):
+        ids = {(): 0}
+        for i in range(N):
+            for j in range(k):
+                pre = tuple(c_host[b, i, :j + 1])
+                if pre not in ids:
+                    ids[pre] = len(ids)
+                    depth_idx[b, ids[pre]] = min(j + 1, k - 1)
+        nodes += len(ids)
+    gen = torch.Generator(device="cuda").manual_seed(78)
+    qf = q.float()
+    p_nodes = (torch.gather(qf, 1, depth_idx.cuda()[:, :, None].expand(B, R, V))
+               + torch.randn((B, R, V), device="cuda", generator=gen)).to(torch.bfloat16)
+    ws = torch.empty(U.load().uno_tree_verify_workspace(B, N, k, R, V), dtype=torch.uint8,
+                     device="cuda")
+    touts = [torch.empty(B, dtype=torch.int32, device="cuda"),
+             torch.empty((B, k + 1), dtype=torch.int32, device="cuda"),
+             torch.empty(B, dtype=torch.int32, device="cuda")]
+    f = lambda: U.tree_verify(p_nodes, q, cands, 1.0, 1234, 0, bonus=True, accepted_len=touts[0],
+                              out_tokens=touts[1], out_count=touts[2], workspace=ws)
+    f()
+    us = timed(f, reps=10)
+    byts = (nodes + B * k) * V * 2
+    out[f"tree_verify_B{B}_N{N}_k{k}"] = {
+        "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
+        "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3), "trie_nodes": nodes,
+        "mean_accepted": round(float(touts[0].float().mean()), 3)}
+    del p_nodes, q
     torch.cuda.empty_cache()
     return out
 

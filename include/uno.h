@@ -185,6 +185,48 @@ uno_status uno_psi_verify_noalloc(uno_dtype dt, int32_t B, int32_t k, int32_t k_
                                   void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Tree-sampler verification (hyper.ai page, section "方法": at low batch
+ * sizes several candidate blocks are drawn and verified at once as a prefix
+ * tree; lossless as the linear sampler). Per sequence b:
+ *   cands [B,N,k] int32: N candidate blocks, each drawn from the per-position
+ *     draft marginals (N independent linear-sampler blocks).
+ *   The trie of the candidates is numbered in order of first visit when the
+ *     candidates are walked from the root in index order; node 0 is the root.
+ *     p_logits [B,R,V] `dt`: row n holds the AR logits of the next token after
+ *     node n's prefix (row 0: the anchor's). R >= the node count (at most
+ *     N*k + 1); rows of depth-k nodes are read only when `bonus` != 0.
+ *   q_logits [B,k,V] `dt`: the draft logits of position j.
+ *   At a node of depth j the live candidates (prefix = accepted path) are
+ *   tested in index order: candidate i with token x is accepted iff
+ *   u1 * q_j(x) < r_i(x), u1 from Philox stream 1 at index
+ *   ((seq_offset + b)*k + j)*N + i, r_1 = softmax(p_logits[b,node] / T) and,
+ *   after each rejection, r_{i+1} = max(r_i - q_j, 0) normalised (unchanged
+ *   when its mass is 0). On acceptance the walk moves to the child with every
+ *   candidate holding that token; if all are rejected, a token is drawn from
+ *   the last residual (stream 2, index (seq_offset + b)*k + j) and the block
+ *   ends. With all k accepted and `bonus` != 0, a bonus token is drawn from
+ *   the leaf's AR row (stream 3, index (seq_offset + b)*k + k).
+ *   Outputs as uno_psi_verify: accepted_len [B], out_tokens [B,k+1] (-1
+ *   padded), out_count [B]. With N = 1 the results equal uno_psi_verify's
+ *   (k_p = k, or k + 1 with the bonus).
+ *   Sizes: 1 <= N <= 32, 1 <= k <= 32, 1 <= R <= N*k + 1, V as for
+ *   uno_psi_verify; B * (R + k) <= 65535; (seq_offset + B) * (k + 1) * N <= 2^32.
+ *   Device-detected: a candidate token outside [0, V), more trie nodes than
+ *   R (UNO_DEV_BAD_DRAFT) or a NaN logit in a row the walk reads
+ *   (UNO_DEV_NAN) set the status bits; that sequence's outputs are -1.
+ *   workspace: >= uno_tree_verify_workspace(B, N, k, R, V) bytes, 16-byte
+ *   aligned, any contents.
+ * ------------------------------------------------------------------------- */
+size_t uno_tree_verify_workspace(int32_t B, int32_t N, int32_t k, int32_t R, int32_t V);
+
+uno_status uno_tree_verify(uno_dtype dt, int32_t B, int32_t N, int32_t k, int32_t R, int32_t V,
+                           const void* p_logits, const void* q_logits, const int32_t* cands,
+                           int32_t bonus, float temperature, uint64_t seed, uint64_t step,
+                           uint64_t seq_offset, int32_t* accepted_len, int32_t* out_tokens,
+                           int32_t* out_count, int32_t* dev_status, void* workspace,
+                           size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Linear-sampler draft (hyper.ai page, section "方法": the linear sampler
  * draws one candidate block from the per-position marginals):
  *   draft[b,j] = smallest v with C(v) > u0 * C(V-1), C the inclusive

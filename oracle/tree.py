@@ -48,7 +48,8 @@ from __future__ import annotations
 import numpy as np
 
 from . import philox
-from .sampling import accept_threshold, as_f64, inverse_cdf, residual_weights, softmax_t
+from .sampling import (accept_threshold, as_f64, cdf_margin, inverse_cdf, residual_weights,
+                       softmax_t)
 
 
 def tree_candidates(q_logits, N: int, T: float, seed: int, step: int, seq_offset: int = 0):
@@ -133,7 +134,10 @@ def tree_verify_sequence(p_logits, q_logits, cands, T: float, seed: int, step: i
     p_logits [n_nodes, V]: AR logits of every trie node (numbering of `trie`);
     the rows of depth-k nodes are read only when `bonus`. q_logits [k,V],
     cands [N,k]. Returns a dict: accepted_len n, tokens (the n accepted ones
-    plus the residual or bonus token), path (trie nodes visited), draw kind.
+    plus the residual or bonus token), path (trie nodes visited), draw kind,
+    and for comparisons with a lower-precision implementation: test_margin
+    (smallest |u - threshold| over the tests taken) and draw_margin (distance
+    of the draw's threshold to the nearest CDF edge of the drawn token, / Z).
     """
     p_logits, q_logits = as_f64(p_logits), as_f64(q_logits)
     cands = np.asarray(cands)
@@ -143,16 +147,21 @@ def tree_verify_sequence(p_logits, q_logits, cands, T: float, seed: int, step: i
         raise ValueError(f"p_logits has {p_logits.shape[0]} rows, the trie {len(parent)} nodes")
     q = softmax_t(q_logits, T)
     node, live, tokens, path = 0, list(range(N)), [], [0]
+    margin = np.inf
     for j in range(k):
         r = softmax_t(p_logits[node], T)
         ths, resid = node_tests(r, q[j], [cands[i, j] for i in live])
         idx = (np.uint64(b_global * k + j) * np.uint64(N) + np.asarray(live, np.uint64))
         u1 = philox.uniforms(seed, step, philox.STREAM_ACCEPT, idx)
         hit = next((t for t in range(len(live)) if u1[t] < ths[t]), None)
+        taken = len(live) if hit is None else hit + 1
+        margin = min([margin] + [abs(float(u1[t]) - float(ths[t])) for t in range(taken)])
         if hit is None:
             u2 = philox.uniforms(seed, step, philox.STREAM_RESIDUAL, b_global * k + j)
-            tokens.append(inverse_cdf(resid, u2))
-            return dict(accepted_len=j, tokens=tokens, path=path, draw="residual")
+            v = inverse_cdf(resid, u2)
+            tokens.append(v)
+            return dict(accepted_len=j, tokens=tokens, path=path, draw="residual",
+                        test_margin=margin, draw_margin=cdf_margin(resid, u2, v))
         x = int(cands[live[hit], j])
         tokens.append(x)
         node = int(node_of[live[hit], j + 1])
@@ -160,6 +169,10 @@ def tree_verify_sequence(p_logits, q_logits, cands, T: float, seed: int, step: i
         live = [i for i in live if int(cands[i, j]) == x]
     if bonus:
         u3 = philox.uniforms(seed, step, philox.STREAM_BONUS, b_global * k + k)
-        tokens.append(inverse_cdf(softmax_t(p_logits[node], T), u3))
-        return dict(accepted_len=k, tokens=tokens, path=path, draw="bonus")
-    return dict(accepted_len=k, tokens=tokens, path=path, draw=None)
+        w = softmax_t(p_logits[node], T)
+        v = inverse_cdf(w, u3)
+        tokens.append(v)
+        return dict(accepted_len=k, tokens=tokens, path=path, draw="bonus",
+                    test_margin=margin, draw_margin=cdf_margin(w, u3, v))
+    return dict(accepted_len=k, tokens=tokens, path=path, draw=None, test_margin=margin,
+                draw_margin=np.inf)

@@ -31,6 +31,7 @@ EXPORTS = [
     "uno_gated_lora_linear_group_workspace", "uno_gated_lora_linear_group",
     "uno_psi_verify_workspace", "uno_psi_verify", "uno_psi_verify_noalloc",
     "uno_draft_sample_workspace", "uno_draft_sample",
+    "uno_tree_verify_workspace", "uno_tree_verify",
     "uno_philox_uniforms",
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
     "uno_psi_step_kernel_count",
@@ -75,6 +76,9 @@ def load():
         "uno_psi_verify_noalloc": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, f32, u64, u64, u64,
                                          vp, vp, vp, vp, vp]),
         "uno_draft_sample_workspace": (sz, [i32, i32, i32]),
+        "uno_tree_verify_workspace": (sz, [i32, i32, i32, i32, i32]),
+        "uno_tree_verify": (i32, [i32, i32, i32, i32, i32, i32, vp, vp, vp, i32, f32, u64, u64, u64,
+                                  vp, vp, vp, vp, vp, sz, vp]),
         "uno_draft_sample": (i32, [i32, i32, i32, i32, vp, f32, u64, u64, u64, vp, vp, vp, sz, vp]),
         "uno_philox_uniforms": (i32, [u64, u64, u32, u32, i64, vp, vp, vp]),
         "uno_model_create": (i32, [vp, i32, i32, i32, i32, i32, i32, i32, f32, vp]),
@@ -313,6 +317,42 @@ def psi_verify_noalloc(p_logits, q_logits, draft, temperature, seed, step, seq_o
             _ptr(p_logits), _ptr(q_logits), _ptr(draft), float(temperature), int(seed),
             int(step), int(seq_offset), _ptr(accepted_len), _ptr(out_tokens), _ptr(out_count),
             _ptr(dev_status))
+    return accepted_len, out_tokens, out_count
+
+
+def tree_verify(p_nodes, q_logits, cands, temperature, seed, step, seq_offset=0, bonus=False,
+                accepted_len=None, out_tokens=None, out_count=None, dev_status=None,
+                workspace=None, stream=None):
+    """Tree-sampler verification; returns (accepted_len [B], out_tokens [B,k+1], out_count [B]).
+
+    p_nodes [B,R,V]: AR logits of every trie node of each sequence's candidates
+    (numbered in order of first visit, candidates walked in index order);
+    q_logits [B,k,V]; cands [B,N,k] int32.
+    """
+    torch = _torch()
+    _expect(p_nodes, (None, None, None), _floats(), "p_nodes")
+    B, R, V = p_nodes.shape
+    _expect(q_logits, (B, None, V), (p_nodes.dtype,), "q_logits")
+    k = q_logits.shape[1]
+    _expect(cands, (B, None, k), (torch.int32,), "cands")
+    N = cands.shape[1]
+    _expect(accepted_len, (B,), (torch.int32,), "accepted_len", optional=True)
+    _expect(out_tokens, (B, k + 1), (torch.int32,), "out_tokens", optional=True)
+    _expect(out_count, (B,), (torch.int32,), "out_count", optional=True)
+    _expect(dev_status, (1,), (torch.int32,), "dev_status", optional=True)
+    L = load()
+    dev = p_nodes.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    accepted_len = torch.empty(B, **i32) if accepted_len is None else accepted_len
+    out_tokens = torch.empty((B, k + 1), **i32) if out_tokens is None else out_tokens
+    out_count = torch.empty(B, **i32) if out_count is None else out_count
+    _dev(p_nodes, q_logits, cands, accepted_len, out_tokens, out_count, dev_status)
+    need = L.uno_tree_verify_workspace(B, N, k, R, V)
+    ws, wsb = _workspace(need, dev, workspace)
+    _check(L.uno_tree_verify(_dtype(p_nodes), B, N, k, R, V, _ptr(p_nodes), _ptr(q_logits),
+                             _ptr(cands), 1 if bonus else 0, float(temperature), int(seed),
+                             int(step), int(seq_offset), _ptr(accepted_len), _ptr(out_tokens),
+                             _ptr(out_count), _ptr(dev_status), _ptr(ws), wsb, _stream(stream)))
     return accepted_len, out_tokens, out_count
 
 

@@ -351,6 +351,58 @@ uno_status uno_psi_verify(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32
   return verify_launch(a, workspace, as_stream(stream));
 }
 
+size_t uno_tree_verify_workspace(int32_t B, int32_t N, int32_t k, int32_t R, int32_t V) {
+  if (B < 0 || N < 1 || N > 32 || k < 1 || k > 32 || R < 1 || V < 1) return 0;
+  return align_up(tree_verify_workspace(B, k, R, V));
+}
+
+uno_status uno_tree_verify(uno_dtype dt, int32_t B, int32_t N, int32_t k, int32_t R, int32_t V,
+                           const void* p_logits, const void* q_logits, const int32_t* cands,
+                           int32_t bonus, float temperature, uint64_t seed, uint64_t step,
+                           uint64_t seq_offset, int32_t* accepted_len, int32_t* out_tokens,
+                           int32_t* out_count, int32_t* dev_status, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  uno_status s = check_sampler(dt, B, k, V, temperature);
+  if (s != UNO_OK) return s;
+  if (N < 1 || N > 32) return set_error(UNO_ERR_UNSUPPORTED, "candidates N=%d outside [1, 32]", N);
+  if (R < 1 || static_cast<int64_t>(R) > static_cast<int64_t>(N) * k + 1)
+    return set_error(UNO_ERR_INVALID_ARG, "node rows R=%d outside [1, N*k+1]", R);
+  if (B == 0) return UNO_OK;
+  if (static_cast<int64_t>(B) * (R + k) > 65535)   // one grid row of the stats pass per logit row
+    return set_error(UNO_ERR_UNSUPPORTED, "B * (R + k) = %lld logit rows > 65535",
+                     static_cast<long long>(B) * (R + k));
+  if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k + 1) *
+          static_cast<uint64_t>(N) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * (k + 1) * N must be <= 2^32");
+  if (!p_logits || !q_logits || !cands || !accepted_len || !out_tokens || !out_count)
+    return set_error(UNO_ERR_INVALID_ARG, "NULL input or output pointer");
+  if (!aligned16(p_logits) || !aligned16(q_logits))
+    return set_error(UNO_ERR_INVALID_ARG, "logits must be 16-byte aligned");
+  const size_t need = uno_tree_verify_workspace(B, N, k, R, V);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
+  TreeVerifyArgs a{};
+  a.dt = dt;
+  a.B = B;
+  a.N = N;
+  a.k = k;
+  a.R = R;
+  a.V = V;
+  a.bonus = bonus ? 1 : 0;
+  a.p_logits = p_logits;
+  a.q_logits = q_logits;
+  a.cands = cands;
+  a.temperature = temperature;
+  a.seed = seed;
+  a.step = step;
+  a.seq_offset = seq_offset;
+  a.accepted_len = accepted_len;
+  a.out_tokens = out_tokens;
+  a.out_count = out_count;
+  a.dev_status = dev_status;
+  return tree_verify_launch(a, workspace, as_stream(stream));
+}
+
 size_t uno_draft_sample_workspace(int32_t B, int32_t k, int32_t V) {
   (void)B;
   (void)k;

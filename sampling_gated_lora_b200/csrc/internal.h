@@ -133,6 +133,22 @@ struct VerifyArgs {
 size_t verify_workspace(int32_t B, int32_t k, int32_t k_p, int32_t V);
 uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s);
 
+struct TreeVerifyArgs {
+  uno_dtype dt;
+  int32_t B, N, k, R, V, bonus;
+  const void* p_logits;   // [B, R, V]: AR logits of the trie nodes
+  const void* q_logits;   // [B, k, V]
+  const int32_t* cands;   // [B, N, k]
+  float temperature;
+  uint64_t seed, step, seq_offset;
+  int32_t* accepted_len;
+  int32_t* out_tokens;
+  int32_t* out_count;
+  int32_t* dev_status;
+};
+size_t tree_verify_workspace(int32_t B, int32_t k, int32_t R, int32_t V);
+uno_status tree_verify_launch(const TreeVerifyArgs& a, void* ws, cudaStream_t s);
+
 struct DraftArgs {
   uno_dtype dt;
   int32_t B, k, V;

@@ -477,6 +477,288 @@ __global__ void __launch_bounds__(kDrawThreads)
   if (token >= 0 && threadIdx.x == 0) tok[n] = token;
 }
 
+// ------------------------------------------------------------------ tree sampler
+//
+// Several drafted blocks per sequence, verified as a prefix tree (hyper.ai
+// page, section "方法", the tree sampler; lossless as for the linear sampler).
+// The candidates form a trie, numbered in order of first visit when they are
+// walked from the root in index order (node 0 = root). At a node of depth j
+// the live candidates (prefix = the accepted path) are tested in index order:
+// candidate i with token x is accepted iff u * q_j(x) < r_i(x), where r_1 = p
+// of the node and r_{i+1} = max(r_i - q_j, 0) / Z_i after each rejection
+// (Z_i its mass; the target stays when Z_i = 0). On acceptance the walk moves
+// to the child x with every candidate that has token x there; if all are
+// rejected, a token is drawn from the last residual. With one candidate this
+// is exactly the linear verification above.
+
+constexpr int kTreeMaxN = 32;   // candidate blocks per sequence
+constexpr int kTreeMaxK = 32;   // block length
+
+struct TreeParams {
+  int B, N, k, R, V, chunks, bonus;
+  float c;   // log2(e) / T
+  uint64_t seed, step, seq_offset;
+  const int32_t* cands;   // [B, N, k]
+  const float2* stats;    // chunk stats of node rows b*R + n, then q rows B*R + b*k + j
+  int32_t* accepted_len;
+  int32_t* out_tokens;
+  int32_t* out_count;
+  int32_t* status;
+  int chunk_elems;
+};
+
+// Sum of one double per thread over the block and then over the cluster, the
+// CTAs' sums added in rank order so that every CTA gets the same bits. Every
+// thread of every CTA of the cluster must call it.
+__device__ double cluster_sum(double* part_slot, double* warp_slots, double v) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) warp_slots[warp] = v;
+  cta_sync();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kDrawThreads / 32; ++w) t += warp_slots[w];
+    *part_slot = t;
+  }
+  cluster_sync();
+  const uint32_t nrank = cluster_nctarank();
+  const uint32_t addr = smem_u32(part_slot);
+  double total = 0.0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    if (r < static_cast<int>(nrank)) total += ld_cluster_f64(map_shared_rank(addr, static_cast<uint32_t>(r)));
+  cluster_sync();   // every CTA has read the slots before they are written again
+  return total;
+}
+
+// Target of a test at one vocab entry after `n` rejections at the node:
+// r_1 = p, r_{t+1} = max(r_t - q, 0) / Z_t (unchanged when Z_t = 0).
+__device__ __forceinline__ double tree_target(float p, float q, const double* Z, int n) {
+  double r = p;
+  for (int t = 0; t < n; ++t)
+    if (Z[t] > 0.0) r = fmax(r - static_cast<double>(q), 0.0) / Z[t];
+  return r;
+}
+
+// One cluster per sequence; blockDim = kDrawThreads.
+template <typename T>
+__global__ void __launch_bounds__(kDrawThreads)
+    tree_finalize_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits,
+                         const TreeParams a) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ DrawSmem sh;
+  __shared__ int s_node[kTreeMaxN][kTreeMaxK + 1];   // trie node after j tokens of candidate i
+  __shared__ int s_id[kTreeMaxN * kTreeMaxK];
+  __shared__ int s_tok[kTreeMaxK];
+  __shared__ double s_Z[kTreeMaxN];
+  __shared__ double s_part, s_warp[kDrawThreads / 32];
+  __shared__ float s_stat[4];
+  __shared__ int s_flag[4];   // [0] decision, [1] bad candidate, [2] trie nodes, [3] NaN
+
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const uint32_t nrank = cluster_nctarank();
+  const uint32_t rank = cluster_ctarank();
+  const int b = blockIdx.x / nrank;
+  const int N = a.N, k = a.k, V = a.V, R = a.R;
+  const int nk = N * k;
+  const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
+  const int32_t* cand = a.cands + static_cast<size_t>(b) * nk;
+  int32_t* tok = a.out_tokens + static_cast<size_t>(b) * (k + 1);
+  const float c = a.c;
+
+  // 1. Trie numbering. rep(i, j) = the first candidate with the same j+1
+  //    tokens; the first visits, in walk order (i, then j), get ids 1, 2, ...
+  if (threadIdx.x == 0) {
+    s_flag[1] = 0;
+    s_flag[3] = 0;
+  }
+  cta_sync();
+  for (int t = threadIdx.x; t < nk; t += blockDim.x) {
+    const int i = t / k, j = t - i * k;
+    const int x = cand[t];
+    if (x < 0 || x >= V) atomicOr(&s_flag[1], 1);
+    int rep = i;
+    for (int i2 = 0; i2 < i && rep == i; ++i2) {
+      bool same = true;
+      for (int jj = 0; jj <= j && same; ++jj) same = cand[i2 * k + jj] == cand[i * k + jj];
+      if (same) rep = i2;
+    }
+    s_node[i][j + 1] = rep;   // the representative for now
+    s_id[t] = rep == i ? 1 : 0;
+  }
+  cta_sync();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int t = 0; t < nk; ++t) s_id[t] = s_id[t] ? ++run : 0;
+    s_flag[2] = run + 1;   // nodes, the root included
+  }
+  cta_sync();
+  for (int t = threadIdx.x; t < nk; t += blockDim.x) {
+    const int i = t / k, j = t - i * k;
+    s_node[i][j + 1] = s_id[s_node[i][j + 1] * k + j];
+  }
+  for (int i = threadIdx.x; i < N; i += blockDim.x) s_node[i][0] = 0;
+  cta_sync();
+
+  // a candidate token outside [0, V), or more trie nodes than the R logit rows
+  // given per sequence: flagged, outputs -1 (uniform over the cluster)
+  auto give_up = [&](int32_t bits) {
+    if (rank == 0) {
+      if (threadIdx.x == 0) {
+        a.accepted_len[b] = -1;
+        a.out_count[b] = -1;
+        raise_status(a.status, bits);
+      }
+      for (int i = threadIdx.x; i <= k; i += blockDim.x) tok[i] = -1;
+    }
+  };
+  if (s_flag[1] || s_flag[2] > R) {
+    give_up(kDevBadDraft);
+    return;
+  }
+
+  int lo, len;
+  chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
+  T* zp = reinterpret_cast<T*>(dyn);
+  T* zq = zp + a.chunk_elems;
+  const size_t q_row0 = static_cast<size_t>(a.B) * R;
+  int node = 0, n = 0;
+  uint32_t live = N >= 32 ? 0xffffffffu : ((1u << N) - 1u);
+
+  // 2. The walk, one depth at a time. Thread 0 of every CTA takes the same
+  //    decisions from the same data; the residual masses are summed over the
+  //    cluster in a fixed order, so every CTA follows the same path.
+  for (int j = 0; j < k; ++j) {
+    if (threadIdx.x == 0) {
+      const float2 sp = row_stat(a.stats, b * R + node, a.chunks, c);
+      const float2 sq = row_stat(a.stats, static_cast<int>(q_row0) + b * k + j, a.chunks, c);
+      s_stat[0] = sp.x;
+      s_stat[1] = sp.y;
+      s_stat[2] = sq.x;
+      s_stat[3] = sq.y;
+      s_flag[3] = isnan(sp.y) || isnan(sq.y);
+    }
+    cta_sync();
+    if (s_flag[3]) {
+      give_up(kDevNaN);
+      return;
+    }
+    const float Mp = s_stat[0], inv_sp = 1.f / s_stat[1];
+    const float Mq = s_stat[2], inv_sq = 1.f / s_stat[3];
+    const T* prow = p_logits + (static_cast<size_t>(b) * R + node) * V;
+    const T* qrow = q_logits + (static_cast<size_t>(b) * k + j) * V;
+    int nz = 0, accepted = -1;
+    bool staged = false;
+    for (int i = 0; i < N; ++i) {
+      if (!((live >> i) & 1u)) continue;
+      if (threadIdx.x == 0) {
+        const int x = cand[i * k + j];
+        const float px = fast_exp2((to_f32<T>(prow[x]) - Mp) * c) * inv_sp;
+        const float qx = fast_exp2((to_f32<T>(qrow[x]) - Mq) * c) * inv_sq;
+        const float r = static_cast<float>(tree_target(px, qx, s_Z, nz));
+        const uint32_t idx = static_cast<uint32_t>(
+            (bg * static_cast<uint64_t>(k) + static_cast<uint64_t>(j)) * static_cast<uint64_t>(N) +
+            static_cast<uint64_t>(i));
+        const float u1 = uniform24(philox_word0(a.seed, a.step, kStreamAccept, idx));
+        s_flag[0] = (qx == 0.f) || (u1 * qx < r);
+      }
+      cta_sync();
+      const bool acc = s_flag[0] != 0;
+      cta_sync();   // read everywhere before thread 0 writes the next decision
+      if (acc) {
+        accepted = i;
+        break;
+      }
+      // rejected: the residual mass Z of this test, over the whole vocabulary
+      if (!staged) {
+        load_chunk(zp, prow + lo, len);
+        load_chunk(zq, qrow + lo, len);
+        cta_sync();
+        staged = true;
+      }
+      double part = 0.0;
+      for (int v = threadIdx.x; v < len; v += blockDim.x) {
+        const float p = fast_exp2((to_f32<T>(zp[v]) - Mp) * c) * inv_sp;
+        const float q = fast_exp2((to_f32<T>(zq[v]) - Mq) * c) * inv_sq;
+        part += fmax(tree_target(p, q, s_Z, nz) - static_cast<double>(q), 0.0);
+      }
+      const double Z = cluster_sum(&s_part, s_warp, part);
+      if (threadIdx.x == 0) s_Z[nz] = Z;
+      ++nz;
+      cta_sync();
+    }
+    if (accepted >= 0) {
+      const int x = cand[accepted * k + j];
+      if (threadIdx.x == 0) s_tok[n] = x;
+      ++n;
+      node = s_node[accepted][j + 1];
+      uint32_t next = 0;
+      for (int i = 0; i < N; ++i)
+        if (((live >> i) & 1u) && cand[i * k + j] == x) next |= 1u << i;
+      live = next;
+      cta_sync();
+      continue;
+    }
+    // every live candidate rejected: draw from the last residual (stream 2)
+    if (rank == 0) {
+      if (threadIdx.x == 0) {
+        a.accepted_len[b] = n;
+        a.out_count[b] = n + 1;
+      }
+      for (int i = threadIdx.x; i <= k; i += blockDim.x)
+        if (i != n) tok[i] = i < n ? s_tok[i] : -1;
+    }
+    const uint32_t idx2 = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + static_cast<uint64_t>(j));
+    const double u = static_cast<double>(uniform24(philox_word0(a.seed, a.step, kStreamResidual, idx2)));
+    const int last = nz - 1;
+    auto w_res = [&](int v) {
+      const float p = fast_exp2((to_f32<T>(zp[v]) - Mp) * c) * inv_sp;
+      const float q = fast_exp2((to_f32<T>(zq[v]) - Mq) * c) * inv_sq;
+      const double r = tree_target(p, q, s_Z, last);
+      return static_cast<float>(s_Z[last] > 0.0 ? fmax(r - static_cast<double>(q), 0.0) : r);
+    };
+    bool zero = false;
+    int token = cluster_draw(sh, w_res, lo, len, u, &zero);
+    if (zero) {   // residual mass lost to rounding: draw from p of the node
+      auto w_p = [&](int v) { return fast_exp2((to_f32<T>(zp[v]) - Mp) * c); };
+      token = cluster_draw(sh, w_p, lo, len, u, &zero);
+    }
+    if (token >= 0 && threadIdx.x == 0) tok[n] = token;
+    return;
+  }
+
+  // 3. All k positions accepted: the bonus token from p of the leaf (stream 3).
+  if (rank == 0) {
+    if (threadIdx.x == 0) {
+      a.accepted_len[b] = k;
+      a.out_count[b] = k + (a.bonus ? 1 : 0);
+    }
+    for (int i = threadIdx.x; i <= k; i += blockDim.x)
+      if (i < k || !a.bonus) tok[i] = i < k ? s_tok[i] : -1;
+  }
+  if (!a.bonus) return;
+  if (threadIdx.x == 0) {
+    const float2 sp = row_stat(a.stats, b * R + node, a.chunks, c);
+    s_stat[0] = sp.x;
+    s_flag[3] = isnan(sp.y);
+  }
+  cta_sync();
+  if (s_flag[3]) {
+    give_up(kDevNaN);
+    return;
+  }
+  const float Mp = s_stat[0];
+  load_chunk(zp, p_logits + (static_cast<size_t>(b) * R + node) * V + lo, len);
+  cta_sync();
+  const uint32_t idx3 = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + static_cast<uint64_t>(k));
+  const double u = static_cast<double>(uniform24(philox_word0(a.seed, a.step, kStreamBonus, idx3)));
+  auto w_p = [&](int v) { return fast_exp2((to_f32<T>(zp[v]) - Mp) * c); };
+  bool zero = false;
+  const int token = cluster_draw(sh, w_p, lo, len, u, &zero);
+  if (token >= 0 && threadIdx.x == 0) tok[k] = token;
+}
+
 struct DraftParams {
   int k, V;
   float c;
@@ -657,6 +939,63 @@ uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s) {
   return launch_cluster(verify_finalize_kernel<__nv_bfloat16>, a.B * cl, cl, smem, s,
                         static_cast<const __nv_bfloat16*>(a.p_logits),
                         static_cast<const __nv_bfloat16*>(a.q_logits), fp);
+}
+
+size_t tree_verify_workspace(int32_t B, int32_t k, int32_t R, int32_t V) {
+  const int rows = B * R + B * k;
+  const int chunks = stat_chunks(rows, V);
+  return static_cast<size_t>(rows) * chunks * sizeof(float2);
+}
+
+uno_status tree_verify_launch(const TreeVerifyArgs& a, void* ws, cudaStream_t s) {
+  const int rows = a.B * a.R + a.B * a.k;
+  const int chunks = stat_chunks(rows, a.V);
+  const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
+  const float c = kLog2e / a.temperature;
+  float2* stats = static_cast<float2*>(ws);
+  const int esz = a.dt == UNO_F32 ? 4 : 2;
+  int chunk_elems = 0;
+  const int cl = draw_cluster(a.V, esz, &chunk_elems);
+  TreeParams tp{};
+  tp.B = a.B;
+  tp.N = a.N;
+  tp.k = a.k;
+  tp.R = a.R;
+  tp.V = a.V;
+  tp.chunks = chunks;
+  tp.bonus = a.bonus ? 1 : 0;
+  tp.c = c;
+  tp.seed = a.seed;
+  tp.step = a.step;
+  tp.seq_offset = a.seq_offset;
+  tp.cands = a.cands;
+  tp.stats = stats;
+  tp.accepted_len = a.accepted_len;
+  tp.out_tokens = a.out_tokens;
+  tp.out_count = a.out_count;
+  tp.status = a.dev_status;
+  tp.chunk_elems = chunk_elems;
+  const size_t smem = static_cast<size_t>(chunk_elems) * esz * 2;
+  const dim3 grid(chunks, rows);
+  cudaError_t e;
+  if (a.dt == UNO_F32) {
+    e = launch_kernel(row_stats_kernel<float>, grid, dim3(kStatThreads), 0, s, 1,
+                      static_cast<const float*>(a.p_logits), static_cast<const float*>(a.q_logits),
+                      a.B * a.R, a.V, chunk_len, c, stats);
+  } else {
+    e = launch_kernel(row_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1,
+                      static_cast<const __nv_bfloat16*>(a.p_logits),
+                      static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.R, a.V, chunk_len,
+                      c, stats);
+  }
+  if (e != cudaSuccess) return cuda_error(e, "row_stats launch");
+  if (a.dt == UNO_F32)
+    return launch_cluster(tree_finalize_kernel<float>, a.B * cl, cl, smem, s,
+                          static_cast<const float*>(a.p_logits),
+                          static_cast<const float*>(a.q_logits), tp);
+  return launch_cluster(tree_finalize_kernel<__nv_bfloat16>, a.B * cl, cl, smem, s,
+                        static_cast<const __nv_bfloat16*>(a.p_logits),
+                        static_cast<const __nv_bfloat16*>(a.q_logits), tp);
 }
 
 uno_status draft_launch(const DraftArgs& a, cudaStream_t s) {

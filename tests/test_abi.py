@@ -157,3 +157,25 @@ def test_workspace_sizes_hold_the_stream_k_scratch():
     L.uno_model_destroy(h)
     # 136 rows (no scratch) vs 272 rows: every other buffer only grows with the rows
     assert big - small >= part + 5 * flags
+
+
+def test_tree_verify_rejects_bad_arguments():
+    L = U.load()
+    ok = ctypes.c_void_p(0x10000)
+    null = None
+
+    def call(B=2, N=2, k=4, R=9, V=1024, T=1.0, ws_bytes=1 << 30, off=0):
+        st = L.uno_tree_verify(U.UNO_BF16, B, N, k, R, V, ok, ok, ok, 0, T, 0, 0, off, ok, ok, ok,
+                               null, ok, ws_bytes, null)
+        return st, L.uno_last_error().decode()
+
+    assert call(N=0)[0] == 2 and call(N=33)[0] == 2
+    assert call(R=0)[0] == 1 and call(R=10)[0] == 1           # R <= N*k + 1
+    assert call(k=33)[0] == 2 and call(T=0.0)[0] == 1
+    st, msg = call(B=4000, N=32, k=16, R=400)
+    assert st == 2 and "65535" in msg
+    assert call(off=1 << 32)[0] == 2                          # Philox index range
+    assert call(ws_bytes=1)[0] == 6
+    assert call(B=0)[0] == 0
+    assert L.uno_tree_verify_workspace(2, 2, 4, 9, 1024) > 0
+    assert L.uno_tree_verify_workspace(2, 0, 4, 9, 1024) == 0
