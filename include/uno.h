@@ -210,7 +210,7 @@ uno_status uno_psi_verify_noalloc(uno_dtype dt, int32_t B, int32_t k, int32_t k_
  *   padded), out_count [B]. With N = 1 the results equal uno_psi_verify's
  *   (k_p = k, or k + 1 with the bonus).
  *   Sizes: 1 <= N <= 32, 1 <= k <= 32, 1 <= R <= N*k + 1, V as for
- *   uno_psi_verify; B * (R + k) <= 65535; (seq_offset + B) * (k + 1) * N <= 2^32.
+ *   uno_psi_verify; B * (R + k) <= 2^30; (seq_offset + B) * (k + 1) * N <= 2^32.
  *   Device-detected: a candidate token outside [0, V), more trie nodes than
  *   R (UNO_DEV_BAD_DRAFT) or a NaN logit in a row the walk reads
  *   (UNO_DEV_NAN) set the status bits; that sequence's outputs are -1.

@@ -368,8 +368,8 @@ uno_status uno_tree_verify(uno_dtype dt, int32_t B, int32_t N, int32_t k, int32_
   if (R < 1 || static_cast<int64_t>(R) > static_cast<int64_t>(N) * k + 1)
     return set_error(UNO_ERR_INVALID_ARG, "node rows R=%d outside [1, N*k+1]", R);
   if (B == 0) return UNO_OK;
-  if (static_cast<int64_t>(B) * (R + k) > 65535)   // one grid row of the stats pass per logit row
-    return set_error(UNO_ERR_UNSUPPORTED, "B * (R + k) = %lld logit rows > 65535",
+  if (static_cast<int64_t>(B) * (R + k) > (1ll << 30))
+    return set_error(UNO_ERR_UNSUPPORTED, "B * (R + k) = %lld logit rows > 2^30",
                      static_cast<long long>(B) * (R + k));
   if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k + 1) *
           static_cast<uint64_t>(N) > (1ull << 32))

@@ -976,17 +976,17 @@ uno_status tree_verify_launch(const TreeVerifyArgs& a, void* ws, cudaStream_t s)
   tp.status = a.dev_status;
   tp.chunk_elems = chunk_elems;
   const size_t smem = static_cast<size_t>(chunk_elems) * esz * 2;
-  const dim3 grid(chunks, rows);
+  const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(rows) * chunks));
   cudaError_t e;
   if (a.dt == UNO_F32) {
     e = launch_kernel(row_stats_kernel<float>, grid, dim3(kStatThreads), 0, s, 1,
                       static_cast<const float*>(a.p_logits), static_cast<const float*>(a.q_logits),
-                      a.B * a.R, a.V, chunk_len, c, stats);
+                      a.B * a.R, a.V, chunks, chunk_len, c, stats);
   } else {
     e = launch_kernel(row_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1,
                       static_cast<const __nv_bfloat16*>(a.p_logits),
-                      static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.R, a.V, chunk_len,
-                      c, stats);
+                      static_cast<const __nv_bfloat16*>(a.q_logits), a.B * a.R, a.V, chunks,
+                      chunk_len, c, stats);
   }
   if (e != cudaSuccess) return cuda_error(e, "row_stats launch");
   if (a.dt == UNO_F32)
