@@ -157,3 +157,14 @@ def test_workspace_sizes_hold_the_stream_k_scratch():
     L.uno_model_destroy(h)
     # 136 rows (no scratch) vs 272 rows: every other buffer only grows with the rows
     assert big - small >= part + 5 * flags
+
+
+def test_distill_rejects_bad_arguments():
+    L = U.load()
+    ok = ctypes.c_void_p(0x10000)
+    call = lambda rows=4, V=64, T=1.0, zt=ok, loss=ok: L.uno_distill(
+        U.UNO_BF16, rows, V, zt, ok, 1.0, 1.0, T, loss, None, None, None)
+    assert call(rows=-1) == 1 and call(V=1) == 2 and call(V=196609) == 2
+    assert call(T=0.0) == 1 and call(zt=None) == 1 and call(loss=None) == 1
+    assert call(zt=ctypes.c_void_p(0x10008)) == 1
+    assert call(rows=0) == 0
