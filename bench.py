@@ -359,6 +359,23 @@ def kernel_lines(U, torch, pk):
         "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3), "trie_nodes": nodes,
         "mean_accepted": round(float(touts[0].float().mean()), 3)}
     del p_nodes, q
+    # distillation losses + gradient on the MLP batch layout: 1024 clean (teacher) rows
+    # against 1024 noisy (student) rows, V=151936, bf16 logits, fp32 gradient.
+    # Algorithmic bytes: one read of both logit rows and one write of the gradient.
+    rows, V = 1024, 151936
+    gen = torch.Generator(device="cuda").manual_seed(91)
+    zt = (torch.randn((rows, V), device="cuda", generator=gen) * 3).to(torch.bfloat16)
+    zs = (zt.float() + torch.randn((rows, V), device="cuda", generator=gen)).to(torch.bfloat16)
+    dl = torch.empty((rows, 2), dtype=torch.float32, device="cuda")
+    dg = torch.empty((rows, V), dtype=torch.float32, device="cuda")
+    f = lambda: U.distill(zt, zs, 1.0, 1.0, 1.0, losses=dl, grad_out=dg)
+    f()
+    us = timed(f, reps=10)
+    byts = rows * V * (2 + 2 + 4)
+    out[f"distill_rows{rows}_V{V}"] = {
+        "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
+        "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3)}
+    del zt, zs, dg
     torch.cuda.empty_cache()
     return out
 

@@ -227,6 +227,24 @@ uno_status uno_tree_verify(uno_dtype dt, int32_t B, int32_t N, int32_t k, int32_
                            size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Distillation losses (hyper.ai page, section "方法": the adapter is trained
+ * with alpha * L_DCD + beta * L_TV on one gated forward pass, the clean rows
+ * (gate 0) giving the teacher logits, the noisy rows (gate 1) the student's):
+ *   per row i: p = softmax(z_teacher[i] / T), q = softmax(z_student[i] / T),
+ *     losses[i] = (KL(p || q), TV(p, q) = 1/2 sum |p - q|);
+ *   grad[i] (optional) = d(alpha * mean KL + beta * mean TV) / d z_student[i]
+ *     = (alpha (q - p) + beta q (s - sum_v s_v q_v) / 2) / (T rows),
+ *     s = sign(q - p) (0 where p = q).
+ *   z_teacher, z_student [rows, V] `dt`, 16-byte aligned; losses [rows, 2]
+ *   float; grad [rows, V] float or NULL (losses only). No workspace.
+ *   A NaN logit in a row pair: that pair's losses (and gradient) are NaN and
+ *   UNO_DEV_NAN is set in dev_status (may be NULL).
+ * ------------------------------------------------------------------------- */
+uno_status uno_distill(uno_dtype dt, int32_t rows, int32_t V, const void* z_teacher,
+                       const void* z_student, float alpha, float beta, float temperature,
+                       float* losses, float* grad, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Linear-sampler draft (hyper.ai page, section "方法": the linear sampler
  * draws one candidate block from the per-position marginals):
  *   draft[b,j] = smallest v with C(v) > u0 * C(V-1), C the inclusive

@@ -30,7 +30,7 @@ EXPORTS = [
     "uno_gated_lora_linear_workspace", "uno_gated_lora_linear",
     "uno_gated_lora_linear_group_workspace", "uno_gated_lora_linear_group",
     "uno_psi_verify_workspace", "uno_psi_verify", "uno_psi_verify_noalloc",
-    "uno_draft_sample_workspace", "uno_draft_sample",
+    "uno_draft_sample_workspace", "uno_draft_sample", "uno_distill",
     "uno_tree_verify_workspace", "uno_tree_verify",
     "uno_philox_uniforms",
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
@@ -79,6 +79,7 @@ def load():
         "uno_tree_verify_workspace": (sz, [i32, i32, i32, i32, i32]),
         "uno_tree_verify": (i32, [i32, i32, i32, i32, i32, i32, vp, vp, vp, i32, f32, u64, u64, u64,
                                   vp, vp, vp, vp, vp, sz, vp]),
+        "uno_distill": (i32, [i32, i32, i32, vp, vp, f32, f32, f32, vp, vp, vp, vp]),
         "uno_draft_sample": (i32, [i32, i32, i32, i32, vp, f32, u64, u64, u64, vp, vp, vp, sz, vp]),
         "uno_philox_uniforms": (i32, [u64, u64, u32, u32, i64, vp, vp, vp]),
         "uno_model_create": (i32, [vp, i32, i32, i32, i32, i32, i32, i32, f32, vp]),
@@ -354,6 +355,32 @@ def tree_verify(p_nodes, q_logits, cands, temperature, seed, step, seq_offset=0,
                              int(step), int(seq_offset), _ptr(accepted_len), _ptr(out_tokens),
                              _ptr(out_count), _ptr(dev_status), _ptr(ws), wsb, _stream(stream)))
     return accepted_len, out_tokens, out_count
+
+
+def distill(z_teacher, z_student, alpha=1.0, beta=1.0, temperature=1.0, grad=True, losses=None,
+            grad_out=None, dev_status=None, stream=None):
+    """Per-row (KL(p||q), TV(p,q)) [rows,2] and, if `grad`, d(alpha mean KL + beta mean TV)/d z_student.
+
+    Returns (losses, grad or None).
+    """
+    torch = _torch()
+    _expect(z_teacher, (None, None), _floats(), "z_teacher")
+    rows, V = z_teacher.shape
+    _expect(z_student, (rows, V), (z_teacher.dtype,), "z_student")
+    _expect(losses, (rows, 2), (torch.float32,), "losses", optional=True)
+    _expect(grad_out, (rows, V), (torch.float32,), "grad_out", optional=True)
+    _expect(dev_status, (1,), (torch.int32,), "dev_status", optional=True)
+    L = load()
+    dev = z_teacher.device
+    losses = torch.empty((rows, 2), dtype=torch.float32, device=dev) if losses is None else losses
+    if grad and grad_out is None:
+        grad_out = torch.empty((rows, V), dtype=torch.float32, device=dev)
+    g = grad_out if grad else None
+    _dev(z_teacher, z_student, losses, g, dev_status)
+    _check(L.uno_distill(_dtype(z_teacher), rows, V, _ptr(z_teacher), _ptr(z_student),
+                         float(alpha), float(beta), float(temperature), _ptr(losses), _ptr(g),
+                         _ptr(dev_status), _stream(stream)))
+    return losses, g
 
 
 def draft_sample(q_logits, temperature, seed, step, seq_offset=0, draft=None, dev_status=None,

@@ -403,6 +403,34 @@ uno_status uno_tree_verify(uno_dtype dt, int32_t B, int32_t N, int32_t k, int32_
   return tree_verify_launch(a, workspace, as_stream(stream));
 }
 
+uno_status uno_distill(uno_dtype dt, int32_t rows, int32_t V, const void* z_teacher,
+                       const void* z_student, float alpha, float beta, float temperature,
+                       float* losses, float* grad, int32_t* dev_status, void* stream) {
+  if (!valid_dtype(dt)) return set_error(UNO_ERR_INVALID_ARG, "unknown dtype %d", dt);
+  if (rows < 0) return set_error(UNO_ERR_INVALID_ARG, "rows=%d < 0", rows);
+  if (V < 2 || V > 196608) return set_error(UNO_ERR_UNSUPPORTED, "vocabulary V=%d outside [2, 196608]", V);
+  if (!(temperature > 0.f) || !(temperature < 1e30f))
+    return set_error(UNO_ERR_INVALID_ARG, "temperature must be > 0 (got %g)", temperature);
+  if (rows == 0) return UNO_OK;
+  if (!z_teacher || !z_student || !losses)
+    return set_error(UNO_ERR_INVALID_ARG, "NULL logits or losses pointer");
+  if (!aligned16(z_teacher) || !aligned16(z_student))
+    return set_error(UNO_ERR_INVALID_ARG, "logits must be 16-byte aligned");
+  DistillArgs a{};
+  a.dt = dt;
+  a.rows = rows;
+  a.V = V;
+  a.z_teacher = z_teacher;
+  a.z_student = z_student;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.temperature = temperature;
+  a.losses = losses;
+  a.grad = grad;
+  a.dev_status = dev_status;
+  return distill_launch(a, as_stream(stream));
+}
+
 size_t uno_draft_sample_workspace(int32_t B, int32_t k, int32_t V) {
   (void)B;
   (void)k;

@@ -130,6 +130,18 @@ struct VerifyArgs {
   int32_t* out_count;
   int32_t* dev_status;
 };
+struct DistillArgs {
+  uno_dtype dt;
+  int32_t rows, V;
+  const void* z_teacher;   // [rows, V]
+  const void* z_student;   // [rows, V]
+  float alpha, beta, temperature;
+  float* losses;           // [rows, 2]
+  float* grad;             // [rows, V] or NULL
+  int32_t* dev_status;
+};
+uno_status distill_launch(const DistillArgs& a, cudaStream_t s);
+
 size_t verify_workspace(int32_t B, int32_t k, int32_t k_p, int32_t V);
 uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s);
 

@@ -759,6 +759,174 @@ __global__ void __launch_bounds__(kDrawThreads)
   if (token >= 0 && threadIdx.x == 0) tok[k] = token;
 }
 
+// ------------------------------------------------------------------ distillation losses
+//
+// alpha * KL(p || q) + beta * TV(p, q) per row pair, p = softmax(z_teacher / T)
+// (the clean, gate-0 rows), q = softmax(z_student / T) (the noisy, gate-1 rows)
+// (hyper.ai page, section "方法": the distillation and total-variation
+// losses), and the gradient w.r.t. the student logits:
+//   (alpha (q - p) + beta q (s - sum_v s_v q_v) / 2) / (T rows),  s = sign(q - p).
+// One cluster per row pair; each CTA stages its vocab chunk of both rows.
+
+struct DistillParams {
+  int V, chunk_elems;
+  float c;            // log2(e) / T
+  float inv_t;        // 1 / T
+  float alpha, beta;
+  float grad_scale;   // 1 / (T rows)
+  float* losses;      // [rows, 2]: KL, TV
+  float* grad;        // [rows, V] or NULL
+  int32_t* status;
+};
+
+// Cluster-wide sums of kN doubles per thread; the CTAs' block sums are added
+// in rank order, so every CTA gets the same bits. Every thread of every CTA
+// of the cluster must call it.
+template <int kN>
+__device__ void cluster_sums(double (&v)[kN], double (*warp_slots)[kN], double* cta_slot) {
+#pragma unroll
+  for (int i = 0; i < kN; ++i) v[i] = warp_sum(v[i]);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < kN; ++i) warp_slots[warp][i] = v[i];
+  }
+  cta_sync();
+  if (threadIdx.x < kN) {
+    double t = 0.0;
+    for (int w = 0; w < kDrawThreads / 32; ++w) t += warp_slots[w][threadIdx.x];
+    cta_slot[threadIdx.x] = t;
+  }
+  cluster_sync();
+  const uint32_t nrank = cluster_nctarank();
+#pragma unroll
+  for (int i = 0; i < kN; ++i) {
+    const uint32_t addr = smem_u32(&cta_slot[i]);
+    double total = 0.0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < static_cast<int>(nrank)) total += ld_cluster_f64(map_shared_rank(addr, static_cast<uint32_t>(r)));
+    v[i] = total;
+  }
+  cluster_sync();   // every CTA has read the slots before they are written again
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDrawThreads)
+    distill_kernel(const T* __restrict__ z_teacher, const T* __restrict__ z_student,
+                   const DistillParams a) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ double s_warp[kDrawThreads / 32][3];
+  __shared__ double s_cta[3];
+  __shared__ float s_wmax[kDrawThreads / 32][2];
+  __shared__ float s_max[2];
+
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const uint32_t nrank = cluster_nctarank();
+  const uint32_t rank = cluster_ctarank();
+  const int row = blockIdx.x / nrank;
+  const int V = a.V;
+  int lo, len;
+  chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
+  T* zt = reinterpret_cast<T*>(dyn);
+  T* zs = zt + a.chunk_elems;
+  load_chunk(zt, z_teacher + static_cast<size_t>(row) * V + lo, len);
+  load_chunk(zs, z_student + static_cast<size_t>(row) * V + lo, len);
+  cta_sync();
+
+  // 1. the rows' maxima over the cluster (NaN kept)
+  float mt = -INFINITY, ms = -INFINITY;
+  bool nan = false;
+  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+    const float x = to_f32<T>(zt[i]), y = to_f32<T>(zs[i]);
+    nan |= isnan(x) || isnan(y);
+    mt = fmaxf(mt, x);
+    ms = fmaxf(ms, y);
+  }
+  mt = warp_max(mt);
+  ms = warp_max(ms);
+  nan = __any_sync(0xffffffffu, nan);
+  if ((threadIdx.x & 31) == 0) {
+    s_wmax[threadIdx.x >> 5][0] = nan ? NAN : mt;
+    s_wmax[threadIdx.x >> 5][1] = ms;
+  }
+  cta_sync();
+  if (threadIdx.x < 2) {
+    float m = -INFINITY;
+    bool any = false;
+    for (int w = 0; w < kDrawThreads / 32; ++w) {
+      any |= isnan(s_wmax[w][threadIdx.x]);
+      m = fmaxf(m, s_wmax[w][threadIdx.x]);
+    }
+    s_max[threadIdx.x] = any ? NAN : m;
+  }
+  cluster_sync();
+  float Mt = -INFINITY, Ms = -INFINITY;
+  bool any_nan = false;
+  for (uint32_t r = 0; r < nrank; ++r) {
+    const float x = ld_cluster_f32(map_shared_rank(smem_u32(&s_max[0]), r));
+    const float y = ld_cluster_f32(map_shared_rank(smem_u32(&s_max[1]), r));
+    any_nan |= isnan(x);
+    Mt = fmaxf(Mt, x);
+    Ms = fmaxf(Ms, y);
+  }
+  cluster_sync();
+  if (any_nan) {   // uniform over the cluster
+    if (rank == 0 && threadIdx.x == 0) {
+      a.losses[2 * row] = NAN;
+      a.losses[2 * row + 1] = NAN;
+      raise_status(a.status, kDevNaN);
+    }
+    if (a.grad)
+      for (int i = threadIdx.x; i < len; i += blockDim.x)
+        a.grad[static_cast<size_t>(row) * V + lo + i] = NAN;
+    return;
+  }
+
+  // 2. the partition sums, then KL, TV and sum(sign(q - p) q)
+  const float c = a.c;
+  double sums[3] = {0.0, 0.0, 0.0};
+  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+    sums[0] += static_cast<double>(fast_exp2((to_f32<T>(zt[i]) - Mt) * c));
+    sums[1] += static_cast<double>(fast_exp2((to_f32<T>(zs[i]) - Ms) * c));
+  }
+  cluster_sums<3>(sums, s_warp, s_cta);
+  const double St = sums[0], Ss = sums[1];
+  const double ln_st = log(St), ln_ss = log(Ss);
+  const double inv_st = 1.0 / St, inv_ss = 1.0 / Ss;
+  const double inv_t = a.inv_t;
+  double acc[3] = {0.0, 0.0, 0.0};   // KL, sum |p - q|, sum s q
+  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+    const float x = to_f32<T>(zt[i]), y = to_f32<T>(zs[i]);
+    const double p = fast_exp2((x - Mt) * c) * inv_st;
+    const double q = fast_exp2((y - Ms) * c) * inv_ss;
+    const double lp = (static_cast<double>(x) - Mt) * inv_t - ln_st;
+    const double lq = (static_cast<double>(y) - Ms) * inv_t - ln_ss;
+    if (p > 0.0) acc[0] += p * (lp - lq);
+    acc[1] += fabs(p - q);
+    acc[2] += q > p ? q : (q < p ? -q : 0.0);
+  }
+  cluster_sums<3>(acc, s_warp, s_cta);
+  if (rank == 0 && threadIdx.x == 0) {
+    a.losses[2 * row] = static_cast<float>(acc[0]);
+    a.losses[2 * row + 1] = static_cast<float>(0.5 * acc[1]);
+  }
+  if (!a.grad) return;
+
+  // 3. the gradient w.r.t. the student logits, this CTA's chunk
+  const double sq = acc[2];
+  const double ka = static_cast<double>(a.alpha) * a.grad_scale;
+  const double kb = 0.5 * static_cast<double>(a.beta) * a.grad_scale;
+  float* g = a.grad + static_cast<size_t>(row) * V + lo;
+  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+    const double p = fast_exp2((to_f32<T>(zt[i]) - Mt) * c) * inv_st;
+    const double q = fast_exp2((to_f32<T>(zs[i]) - Ms) * c) * inv_ss;
+    const double s = q > p ? 1.0 : (q < p ? -1.0 : 0.0);
+    g[i] = static_cast<float>(ka * (q - p) + kb * q * (s - sq));
+  }
+}
+
 struct DraftParams {
   int k, V;
   float c;
@@ -996,6 +1164,31 @@ uno_status tree_verify_launch(const TreeVerifyArgs& a, void* ws, cudaStream_t s)
   return launch_cluster(tree_finalize_kernel<__nv_bfloat16>, a.B * cl, cl, smem, s,
                         static_cast<const __nv_bfloat16*>(a.p_logits),
                         static_cast<const __nv_bfloat16*>(a.q_logits), tp);
+}
+
+uno_status distill_launch(const DistillArgs& a, cudaStream_t s) {
+  const int esz = a.dt == UNO_F32 ? 4 : 2;
+  int chunk_elems = 0;
+  const int cl = draw_cluster(a.V, esz, &chunk_elems);
+  DistillParams dp{};
+  dp.V = a.V;
+  dp.chunk_elems = chunk_elems;
+  dp.c = kLog2e / a.temperature;
+  dp.inv_t = 1.f / a.temperature;
+  dp.alpha = a.alpha;
+  dp.beta = a.beta;
+  dp.grad_scale = 1.f / (a.temperature * static_cast<float>(a.rows));
+  dp.losses = a.losses;
+  dp.grad = a.grad;
+  dp.status = a.dev_status;
+  const size_t smem = static_cast<size_t>(chunk_elems) * esz * 2;
+  if (a.dt == UNO_F32)
+    return launch_cluster(distill_kernel<float>, a.rows * cl, cl, smem, s,
+                          static_cast<const float*>(a.z_teacher),
+                          static_cast<const float*>(a.z_student), dp);
+  return launch_cluster(distill_kernel<__nv_bfloat16>, a.rows * cl, cl, smem, s,
+                        static_cast<const __nv_bfloat16*>(a.z_teacher),
+                        static_cast<const __nv_bfloat16*>(a.z_student), dp);
 }
 
 uno_status draft_launch(const DraftArgs& a, cudaStream_t s) {

@@ -180,3 +180,14 @@ def test_tree_verify_rejects_bad_arguments():
     assert call(B=0)[0] == 0
     assert L.uno_tree_verify_workspace(2, 2, 4, 9, 1024) > 0
     assert L.uno_tree_verify_workspace(2, 0, 4, 9, 1024) == 0
+
+
+def test_distill_rejects_bad_arguments():
+    L = U.load()
+    ok = ctypes.c_void_p(0x10000)
+    call = lambda rows=4, V=64, T=1.0, zt=ok, loss=ok: L.uno_distill(
+        U.UNO_BF16, rows, V, zt, ok, 1.0, 1.0, T, loss, None, None, None)
+    assert call(rows=-1) == 1 and call(V=1) == 2 and call(V=196609) == 2
+    assert call(T=0.0) == 1 and call(zt=None) == 1 and call(loss=None) == 1
+    assert call(zt=ctypes.c_void_p(0x10008)) == 1
+    assert call(rows=0) == 0
