@@ -505,11 +505,16 @@ struct StepLayout {
 
 // One operation of a step plan.
 struct StepOp {
-  int kind;            // 0 GEMM, 1 rmsnorm
+  int kind;            // 0 GEMM, 1 rmsnorm, 2 rmsnorm + LoRA down-projection
   GemmLaunch gemm;
   const void* x;
   void* y;
+  NormDownArgs nd;
 };
+
+// Decode-size batches fold the LoRA down-projection of an input that an
+// RMSNorm produces into that RMSNorm's launch (one launch instead of two).
+constexpr int64_t kNormDownMaxRows = 32;
 
 }  // namespace
 }  // namespace uno
@@ -607,9 +612,11 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     if (s == UNO_OK) P->ops.push_back(op);
     return s;
   };
-  // gated linear(s) on input x (width K): down-projections then the main GEMM
+  // gated linear(s) on input x (width K): down-projections then the main GEMM.
+  // t_ready: the preceding launch wrote t as well as x (no down-projection here).
   auto linear = [&](const void* x, int64_t K, int G, const int* which, int layer, void* const* y,
-                    const int64_t* ldy, int mode, void* y1, int64_t M0) -> uno_status {
+                    const int64_t* ldy, int mode, void* y1, int64_t M0,
+                    bool t_ready = false) -> uno_status {
     uno_status s;
     const void* As[kMaxGroups] = {nullptr, nullptr, nullptr};
     for (int i = 0; i < G; ++i)
@@ -653,7 +660,7 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       pm.sk_slots = pair_sk_slots();
       ++main_launches;
     }
-    pm.x_ready = r > 0 && !gemm_dec_suits(pm);
+    pm.x_ready = r > 0 && !gemm_dec_suits(pm) && !t_ready;
     if (pm.x_ready &&
         (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
       return s;
@@ -676,13 +683,46 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       if ((s = linear(base + L.q, m->q_out, 1, which, l, y, ld, kEpiAdd, nullptr, M)) != UNO_OK)
         return s;
     }
-    norm(base + L.h, base + L.n);
     {
       const int which[2] = {kGate, kUp};
       void* y[2] = {base + L.act, base + L.act};
       const int64_t ld[2] = {m->inter, m->inter};
-      if ((s = linear(base + L.n, m->hidden, 2, which, l, y, ld, kEpiSiluPair, nullptr, M)) !=
-          UNO_OK)
+      // the silu pair never fits the fused decode kernel (2 * inter rows > one wave): at
+      // decode sizes its down-projection rides in the RMSNorm launch
+      GemmProblem probe{};   // would the silu pair take the fused decode kernel?
+      probe.dt = UNO_BF16;
+      probe.M = M;
+      probe.K = m->hidden;
+      probe.r = r;
+      probe.ngroups = 2;
+      probe.mode = kEpiSiluPair;
+      probe.A[0] = m->wp(l, kGate, 1);
+      probe.A[1] = m->wp(l, kUp, 1);
+      probe.g[0].N = probe.g[1].N = m->inter;
+      const bool fold = r > 0 && M <= kNormDownMaxRows && m->hidden % 8 == 0 &&
+                        !gemm_dec_suits(probe);
+      if (fold) {
+        StepOp op{};
+        op.kind = 2;
+        op.nd.x = base + L.h;
+        op.nd.y = base + L.n;
+        op.nd.D = m->hidden;
+        op.nd.eps = 1e-6f;
+        op.nd.A[0] = m->wp(l, kGate, 1);
+        op.nd.A[1] = m->wp(l, kUp, 1);
+        op.nd.A[2] = op.nd.A[1];
+        op.nd.G = 2;
+        op.nd.r = r;
+        op.nd.t = t;
+        op.nd.ldt = 2 * r;
+        op.nd.scale = m->scale;
+        op.nd.gate_row0 = Mv;
+        P->ops.push_back(op);
+      } else {
+        norm(base + L.h, base + L.n);
+      }
+      if ((s = linear(base + L.n, m->hidden, 2, which, l, y, ld, kEpiSiluPair, nullptr, M,
+                      fold)) != UNO_OK)
         return s;
     }
     {
@@ -815,7 +855,9 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
     return cuda_error(e, "clearing the stream-K flags");
   for (const StepOp& op : P->ops) {
-    s = op.kind == 0 ? gemm_run(op.gemm, st) : rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st);
+    s = op.kind == 0 ? gemm_run(op.gemm, st)
+        : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st)
+                       : norm_down_launch(op.nd, M, st);
     if (s != UNO_OK) return s;
   }
 

@@ -66,6 +66,95 @@ __global__ void __launch_bounds__(kNormThreads)
   }
 }
 
+// RMSNorm of row blockIdx.x, with rmsnorm_kernel's arithmetic, and the gated
+// LoRA down-projection of the normalised (bf16-rounded) row for 32 rows of the
+// adapters' concatenated A (rows [32 blockIdx.y, +32)):
+//   t[m, j] = bf16(scale * g_m * sum_k y[m, k] A[j, k]),  g_m = (m >= gate_row0)
+// (the gated LoRA of hyper.ai page, section "方法"). Block y = 0 writes the
+// normalised row. For decode-size batches, where it replaces a separate
+// down-projection launch. D must be a multiple of 8.
+constexpr int kNdRows = 32;
+
+__global__ void __launch_bounds__(kNormThreads)
+    rmsnorm_down_kernel(const NormDownArgs a) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const size_t row = blockIdx.x;
+  const int D = a.D;
+  const int nv = D / 8;
+  const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(a.x) + row * D;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < nv; i += kNormThreads) {
+    const uint4 w = reinterpret_cast<const uint4*>(xr)[i];
+    const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = bf16_lo(q[e]), hi = bf16_hi(q[e]);
+      ss += lo * lo + hi * hi;
+    }
+  }
+  ss = warp_sum(ss);
+  __shared__ float red[kNormThreads / 32];
+  __shared__ float s_inv;
+  __shared__ float s_dot[kNormThreads / 32][kNdRows];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  cta_sync();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kNormThreads / 32; ++w) t += red[w];
+    s_inv = 1.0f / sqrtf(t / static_cast<float>(D) + a.eps);
+  }
+  cta_sync();
+  const float inv = s_inv;
+  const int j0 = blockIdx.y * kNdRows;
+  const int rows_a = a.G * a.r;
+  const __nv_bfloat16* arow[kNdRows];
+#pragma unroll
+  for (int jj = 0; jj < kNdRows; ++jj) {
+    const int j = min(j0 + jj, rows_a - 1);   // rows past the end repeat the last; not stored
+    arow[jj] = static_cast<const __nv_bfloat16*>(a.A[j / a.r == 0 ? 0 : (j / a.r == 1 ? 1 : 2)]) +
+               static_cast<size_t>(j % a.r) * D;
+  }
+  float acc[kNdRows];
+#pragma unroll
+  for (int jj = 0; jj < kNdRows; ++jj) acc[jj] = 0.f;
+  __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(a.y) + row * D;
+  for (int i = threadIdx.x; i < nv; i += kNormThreads) {
+    const uint4 w = reinterpret_cast<const uint4*>(xr)[i];
+    const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[4];
+    float n[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(bf16_lo(q[e]) * inv, bf16_hi(q[e]) * inv);
+      o[e] = *reinterpret_cast<uint32_t*>(&h);
+      n[2 * e] = bf16_lo(o[e]);
+      n[2 * e + 1] = bf16_hi(o[e]);
+    }
+    if (blockIdx.y == 0) reinterpret_cast<uint4*>(yr)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int jj = 0; jj < kNdRows; ++jj) {
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(arow[jj]) + i);
+      acc[jj] += n[0] * bf16_lo(b.x) + n[1] * bf16_hi(b.x) + n[2] * bf16_lo(b.y) +
+                 n[3] * bf16_hi(b.y) + n[4] * bf16_lo(b.z) + n[5] * bf16_hi(b.z) +
+                 n[6] * bf16_lo(b.w) + n[7] * bf16_hi(b.w);
+    }
+  }
+#pragma unroll
+  for (int jj = 0; jj < kNdRows; ++jj) {
+    const float v = warp_sum(acc[jj]);
+    if ((threadIdx.x & 31) == 0) s_dot[threadIdx.x >> 5][jj] = v;
+  }
+  cta_sync();
+  if (threadIdx.x < kNdRows && j0 + static_cast<int>(threadIdx.x) < rows_a) {
+    float t = 0.f;
+    for (int w = 0; w < kNormThreads / 32; ++w) t += s_dot[w][threadIdx.x];
+    const float g = static_cast<int64_t>(row) >= a.gate_row0 ? 1.f : 0.f;
+    static_cast<__nv_bfloat16*>(a.t)[row * a.ldt + j0 + threadIdx.x] =
+        __float2bfloat16_rn(a.scale * g * t);
+  }
+}
+
 __device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.0f + expf(-a)) * b; }
 
 __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
@@ -103,6 +192,14 @@ uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float ep
       rmsnorm_kernel, dim3(static_cast<unsigned>(M)), dim3(kNormThreads), 0, s, 1,
       static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), static_cast<int>(D), eps);
   return e == cudaSuccess ? UNO_OK : cuda_error(e, "rmsnorm launch");
+}
+
+uno_status norm_down_launch(const NormDownArgs& a, int64_t M, cudaStream_t s) {
+  if (M == 0) return UNO_OK;
+  const unsigned blocks_y = static_cast<unsigned>((a.G * a.r + kNdRows - 1) / kNdRows);
+  const cudaError_t e = launch_kernel(rmsnorm_down_kernel, dim3(static_cast<unsigned>(M), blocks_y),
+                                     dim3(kNormThreads), 0, s, 1, a);
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "rmsnorm_down launch");
 }
 
 uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s) {

@@ -180,6 +180,22 @@ uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float ep
                           cudaStream_t s);
 uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s);
 
+// RMSNorm of x into y plus the gated LoRA down-projection of y for G adapters
+// into t (see rmsnorm_down_kernel); D % 8 == 0.
+struct NormDownArgs {   // bf16 tensors
+  const void* x;
+  void* y;
+  int D;
+  float eps;
+  const void* A[3];
+  int G, r;
+  void* t;
+  int ldt;
+  float scale;
+  int64_t gate_row0;
+};
+uno_status norm_down_launch(const NormDownArgs& a, int64_t M, cudaStream_t s);
+
 int device_sm_count();
 
 // Launch attributes shared by every kernel launch: programmatic stream

@@ -40,11 +40,19 @@ def _buffers(B, k, V, dev="cuda"):
                 status=torch.zeros(1, **i32))
 
 
-@pytest.mark.parametrize("B,k,T", [(2, 4, 1.0), (3, 8, 0.7), (1, 1, 1.0), (64, 8, 1.0)])
-def test_tiny_step(B, k, T):
+# One layer whose MLP is too wide for the fused decode kernel (2 * 9728 rows in
+# 152 silu tiles > 148 SMs): at decode sizes the step folds the silu pair's
+# down-projection into the RMSNorm launch.
+WIDE_MLP_SHAPE = W.ModelShape(n_layers=1, hidden=256, q_out=256, kv_out=64, inter=9728,
+                              vocab=1024, r=16)
+
+
+@pytest.mark.parametrize("shape,B,k,T", [(W.TINY_SHAPE, 2, 4, 1.0), (W.TINY_SHAPE, 3, 8, 0.7),
+                                         (W.TINY_SHAPE, 1, 1, 1.0), (W.TINY_SHAPE, 64, 8, 1.0),
+                                         (WIDE_MLP_SHAPE, 1, 8, 1.0), (WIDE_MLP_SHAPE, 2, 4, 0.7)])
+def test_tiny_step(shape, B, k, T):
     import torch
     import sampling_gated_lora_b200 as U
-    shape = W.TINY_SHAPE
     m, layers_np, head_np = _model(shape, seed=1)
     V = shape.vocab
     h = W.step_hidden(B, k, shape.hidden, seed=2)
