@@ -321,6 +321,23 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
                         int32_t* accepted_len, int32_t* out_tokens, int32_t* out_count,
                         int32_t* dev_status, void* workspace, size_t ws_bytes, void* stream);
 
+/* The decoder-layer part of uno_psi_step, for inspecting a step layer by
+ * layer. Each layer has two residual sub-blocks: 2l (rmsnorm, q/k/v, h += o(q))
+ * and 2l+1 (rmsnorm, h += down(silu(gate) * up)). This call runs the launches
+ * uno_psi_step issues for the first n_blocks sub-blocks (0 <= n_blocks <=
+ * 2 * layers; the same kernels, launch shapes and workspace layout as a step
+ * with this B and k) on h_in [M, hidden] bf16, M = B(2k+1), and writes the
+ * hidden state after them to h_out [M, hidden] (h_out may alias h_in).
+ * Optional outputs (NULL to skip), all [M, width] bf16: q_out [M, q_out],
+ * k_out and v_out [M, kv_out] of the last projection sub-block run
+ * (n_blocks >= 1), act_out = silu(gate) * up [M, inter] of the last MLP
+ * sub-block run (n_blocks >= 2). workspace: as for uno_psi_step. No LM head,
+ * verify or draft. */
+uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h_in,
+                               int32_t n_blocks, void* h_out, void* q_out, void* k_out,
+                               void* v_out, void* act_out, void* workspace, size_t ws_bytes,
+                               void* stream);
+
 /* Number of kernel launches one uno_psi_step call with this (B, k) issues;
  * 0 until such a step has been run (the launch plan is built on first use). */
 int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k);

@@ -34,7 +34,7 @@ EXPORTS = [
     "uno_tree_verify_workspace", "uno_tree_verify",
     "uno_philox_uniforms",
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
-    "uno_psi_step_kernel_count",
+    "uno_psi_step_hidden", "uno_psi_step_kernel_count",
     "uno_rmsnorm", "uno_silu_mul",
 ]
 
@@ -87,6 +87,7 @@ def load():
         "uno_psi_step_workspace": (sz, [vp, i32, i32]),
         "uno_psi_step": (i32, [vp, i32, i32, vp, vp, vp, f32, u64, u64, u64, vp, vp, vp, vp, vp,
                                vp, vp, vp, sz, vp]),
+        "uno_psi_step_hidden": (i32, [vp, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
         "uno_psi_step_kernel_count": (i32, [vp, i32, i32]),
         "uno_rmsnorm": (i32, [i64, i64, vp, vp, f32, vp]),
         "uno_silu_mul": (i32, [i64, vp, vp, vp, vp]),
@@ -489,6 +490,7 @@ class Model:
                                   vocab, r, float(scale), arr))
         self._h = h
         self.n_layers, self.hidden, self.vocab, self.r = len(layers), hidden, vocab, r
+        self.q_out, self.kv_out, self.inter = q_out, kv_out, inter
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
@@ -507,6 +509,33 @@ class Model:
     def kernel_count(self, B, k):
         """Kernel launches issued by one step for (B, k) (0 before the first such step)."""
         return load().uno_psi_step_kernel_count(self._h, B, k)
+
+    def hidden(self, B, k, h_in, n_blocks, workspace, h_out=None, inter=False, stream=None):
+        """uno_psi_step_hidden: the step's hidden state after its first n_blocks residual
+        sub-blocks (two per layer). With inter=True also returns the products of the last
+        sub-blocks run: dict q, k, v (n_blocks >= 1) and act = silu(gate) * up (n_blocks >= 2)."""
+        torch = _torch()
+        bf16 = (torch.bfloat16,)
+        M = B * (2 * k + 1)
+        _expect(h_in, (M, self.hidden), bf16, "h_in")
+        _expect(h_out, (M, self.hidden), bf16, "h_out", optional=True)
+        if workspace is None:
+            raise ValueError("workspace is required (Model.workspace_bytes(B, k) bytes)")
+        h_out = torch.empty_like(h_in) if h_out is None else h_out
+        mk = lambda n: torch.empty((M, n), dtype=torch.bfloat16, device=h_in.device)
+        outs = {}
+        if inter and n_blocks >= 1:
+            outs.update(q=mk(self.q_out), k=mk(self.kv_out), v=mk(self.kv_out))
+        if inter and n_blocks >= 2:
+            outs["act"] = mk(self.inter)
+        dev = _dev(h_in, h_out, workspace, *outs.values())
+        if dev != self.device:
+            raise ValueError(f"buffers on {dev}, the model's weights on {self.device}")
+        wsb = workspace.numel() * workspace.element_size()
+        _launch(dev, stream, load().uno_psi_step_hidden, self._h, B, k, _ptr(h_in), int(n_blocks),
+                _ptr(h_out), _ptr(outs.get("q")), _ptr(outs.get("k")), _ptr(outs.get("v")),
+                _ptr(outs.get("act")), _ptr(workspace), wsb)
+        return (h_out, outs) if inter else h_out
 
     def step(self, B, k, h_in, q_prev, d_prev, temperature, seed, step, q_next, d_next,
              accepted_len, out_tokens, out_count, workspace, logits_out=None, dev_status=None,

@@ -528,9 +528,10 @@ struct uno_model {
   struct Plan {
     int32_t B, k;
     const void* ws;
-    const void* q_next;
+    const void* q_next;       // NULL: the decoder layers only (no LM head)
     const void* logits_out;
     std::vector<uno::StepOp> ops;
+    std::vector<size_t> block_end;   // ops.size() after each residual sub-block
   };
   std::mutex mu;
   std::vector<std::unique_ptr<Plan>> plans;   // most recently used last
@@ -596,6 +597,7 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
   P->q_next = q_next;
   P->logits_out = logits_out;
   P->ops.clear();
+  P->block_end.clear();
   void* t = base + L.t;
   int main_launches = 0;   // stream-K flag block of the next main GEMM
   auto norm = [&](const void* x, void* y) {
@@ -683,6 +685,7 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       if ((s = linear(base + L.q, m->q_out, 1, which, l, y, ld, kEpiAdd, nullptr, M)) != UNO_OK)
         return s;
     }
+    P->block_end.push_back(P->ops.size());
     {
       const int which[2] = {kGate, kUp};
       void* y[2] = {base + L.act, base + L.act};
@@ -732,7 +735,9 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       if ((s = linear(base + L.act, m->inter, 1, which, l, y, ld, kEpiAdd, nullptr, M)) != UNO_OK)
         return s;
     }
+    P->block_end.push_back(P->ops.size());
   }
+  if (!q_next) return UNO_OK;   // decoder layers only
   norm(base + L.h, base + L.n);
   void* p_dst = logits_out ? logits_out : base + L.logits;
   const int which[1] = {0};
@@ -815,7 +820,7 @@ int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k) {
   // rmsnorm + LM head; verify (2 kernels) + draft (1)
   std::lock_guard<std::mutex> lock(const_cast<uno_model*>(m)->mu);
   for (const auto& p : m->plans)
-    if (p->B == B && p->k == k) return static_cast<int32_t>(p->ops.size()) + 3;
+    if (p->B == B && p->k == k && p->q_next) return static_cast<int32_t>(p->ops.size()) + 3;
   return 0;
 }
 
@@ -893,6 +898,59 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   da.draft = d_next;
   da.dev_status = dev_status;
   return draft_launch(da, st);
+}
+
+uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h_in,
+                               int32_t n_blocks, void* h_out, void* q_out, void* k_out,
+                               void* v_out, void* act_out, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  if (!m) return set_error(UNO_ERR_INVALID_ARG, "model is NULL");
+  if (B < 1 || k < 1 || k > 32)
+    return set_error(UNO_ERR_INVALID_ARG, "B=%d must be >= 1 and k=%d in [1, 32]", B, k);
+  if (n_blocks < 0 || n_blocks > 2 * m->n_layers)
+    return set_error(UNO_ERR_INVALID_ARG, "n_blocks=%d outside [0, %d]", n_blocks,
+                     2 * m->n_layers);
+  if ((q_out || k_out || v_out) && n_blocks < 1)
+    return set_error(UNO_ERR_INVALID_ARG, "q/k/v outputs need n_blocks >= 1");
+  if (act_out && n_blocks < 2) return set_error(UNO_ERR_INVALID_ARG, "act_out needs n_blocks >= 2");
+  if (static_cast<int64_t>(B) * (2 * k + 1) > (1ll << 30))
+    return set_error(UNO_ERR_UNSUPPORTED, "too many rows");
+  if (!h_in || !h_out) return set_error(UNO_ERR_INVALID_ARG, "NULL h_in or h_out");
+  if (!aligned16(h_in) || !aligned16(h_out))
+    return set_error(UNO_ERR_INVALID_ARG, "h_in and h_out must be 16-byte aligned");
+  const StepLayout L = step_layout(m, B, k);
+  if (!workspace || ws_bytes < L.total || !aligned16(workspace))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", L.total, ws_bytes);
+  std::lock_guard<std::mutex> lock(m->mu);
+  uno_status s;
+  uno_model::Plan* P = find_plan(m, B, k, workspace, nullptr, nullptr, &s);
+  if (!P) return s;
+  cudaStream_t st = as_stream(stream);
+  char* base = static_cast<char*>(workspace);
+  const size_t M = static_cast<size_t>(B) * (2 * k + 1);
+  cudaError_t e = cudaMemcpyAsync(base + L.h, h_in, M * m->hidden * 2, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return cuda_error(e, "copying h_in");
+  if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
+    return cuda_error(e, "clearing the stream-K flags");
+  const size_t n_ops = n_blocks > 0 ? P->block_end[static_cast<size_t>(n_blocks) - 1] : 0;
+  for (size_t i = 0; i < n_ops; ++i) {
+    const StepOp& op = P->ops[i];
+    s = op.kind == 0 ? gemm_run(op.gemm, st)
+        : op.kind == 1 ? rmsnorm_launch(static_cast<int64_t>(M), m->hidden, op.x, op.y, 1e-6f, st)
+                       : norm_down_launch(op.nd, static_cast<int64_t>(M), st);
+    if (s != UNO_OK) return s;
+  }
+  // the step's buffers still hold the last sub-blocks' products
+  const struct { void* dst; size_t off, width; } outs[] = {
+      {h_out, L.h, static_cast<size_t>(m->hidden)}, {q_out, L.q, static_cast<size_t>(m->q_out)},
+      {k_out, L.k, static_cast<size_t>(m->kv_out)}, {v_out, L.v, static_cast<size_t>(m->kv_out)},
+      {act_out, L.act, static_cast<size_t>(m->inter)}};
+  for (const auto& o : outs) {
+    if (!o.dst) continue;
+    e = cudaMemcpyAsync(o.dst, base + o.off, M * o.width * 2, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_error(e, "copying a hidden-state output");
+  }
+  return UNO_OK;
 }
 
 }  // extern "C"

@@ -123,6 +123,15 @@ def test_model_create_validates():
                         None, None, None, 0, None)
     assert st == 1
     assert L.uno_psi_step_kernel_count(h, 2, 4) == 0      # no plan before a first step
+    ok = ctypes.c_void_p(0x10000)
+    ws = 1 << 30
+    hid = lambda B=2, k=4, n=1, hi=ok, ho=ok, q=None, act=None, wsb=ws: L.uno_psi_step_hidden(
+        h, B, k, hi, n, ho, q, None, None, act, ok, wsb, None)
+    assert hid(n=-1) == 1 and hid(n=3) == 1                 # 0 <= n_blocks <= 2 per layer
+    assert hid(n=0, q=ok) == 1 and hid(n=1, act=ok) == 1    # outputs of sub-blocks not run
+    assert hid(B=0) == 1 and hid(k=33) == 1
+    assert hid(hi=None) == 1 and hid(ho=ctypes.c_void_p(0x10008)) == 1
+    assert hid(wsb=16) == 6
     L.uno_model_destroy(h)
 
 

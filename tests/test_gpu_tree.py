@@ -63,7 +63,9 @@ def test_parity_with_oracle(N, k, V, T, bonus):
     acc, tok, cnt = _gpu(P, Q, cands, T, 21, 5, bonus, seq_offset=2)
     excused = 0
     for b in range(B):
-        o = OT.tree_verify_sequence(p_b[b], q_b[b], cands[b], T, 21, 5, b + 2, bonus=bonus)
+        n_nodes = len(OT.trie(cands[b])[1])          # the kernel reads rows [0, n_nodes) of R
+        o = OT.tree_verify_sequence(p_b[b][:n_nodes], q_b[b], cands[b], T, 21, 5, b + 2,
+                                    bonus=bonus)
         ref = np.full(k + 1, -1)
         ref[:len(o["tokens"])] = o["tokens"]
         same = acc[b] == o["accepted_len"] and (tok[b] == ref).all() and cnt[b] == len(o["tokens"])

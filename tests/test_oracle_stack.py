@@ -1,6 +1,8 @@
 """Pins for the oracle's synthetic decode stack (CPU only)."""
 import math
 
+import pytest
+
 import numpy as np
 from scipy import special
 
@@ -111,3 +113,102 @@ def test_step_gate_changes_only_mask_rows():
     nv = B * (k + 1)
     np.testing.assert_array_equal(on[:nv], off[:nv])
     assert np.abs(on[nv:] - off[nv:]).max() > 1e-3
+
+
+# ---------------------------------------------------------------- psi_step pins
+#
+# psi_step composes the stack, the row layout of a step, verification and the
+# draft. The stack has no attention, so every row's logits depend on that row
+# alone: evaluating the verify rows (gate 0) and the mask rows (gate 1) as two
+# separate batches gives p and q_next independently of psi_step's row split.
+# The pins below check psi_step against that, against the special case where
+# the previous block's draft distributions equal this step's AR rows (every
+# block accepted, then the bonus draw: k + 1 tokens), and show that planted
+# wiring slips fail at least one of them.
+
+def _pin_model(seed=11, b_scale=40.0):
+    """Tiny model (float64) whose adapter moves the draft rows well away from the AR rows."""
+    shape = W.TINY_SHAPE
+    layers, head = W.model_weights_np(shape, seed=seed)
+    f = lambda wab: (W.bf16_to_f64(wab[0]), W.bf16_to_f64(wab[1]), W.bf16_to_f64(wab[2]) * b_scale)
+    return shape, [{k: f(v) for k, v in lw.items()} for lw in layers], f(head)
+
+
+def _rows_apart(h, layers, head, B, k, scale):
+    """(p [B,k+1,V], q [B,k,V]): the verify rows and the mask rows evaluated as separate batches."""
+    nv = B * (k + 1)
+    p = O.stack_logits(h[:nv], layers, head, np.zeros(nv, np.uint8), scale)
+    q = O.stack_logits(h[nv:], layers, head, np.ones(B * k, np.uint8), scale)
+    V = p.shape[1]
+    return p.reshape(B, k + 1, V), q.reshape(B, k, V)
+
+
+def _step_pin_failures(step_fn, B=3, k=4, T=1.0):
+    """Names of the psi_step pins that `step_fn` (psi_step's signature) fails."""
+    shape, layers, head = _pin_model()
+    h = W.step_hidden(B, k, shape.hidden, seed=12)
+    p, q = _rows_apart(h, layers, head, B, k, 1.0)
+    fails = []
+    # 1. a previous block drawn from other draft distributions: verification runs on
+    #    this step's AR rows (all k + 1 per sequence, bonus enabled), the draft on its
+    #    mask rows, with the step's seed and step index
+    q_prev = W.bf16_to_f64(W.logits_case(B, k, shape.vocab, ar_std=2.0, sigma=0.0,
+                                         peak_frac=0.0, seed=13).q_logits)
+    d_prev = draft_sample(q_prev, T, 21, 4)
+    ver, d_next, q_next, logits = step_fn(h, layers, head, B, k, q_prev, d_prev, T, 21, 5, 1.0)
+    want = psi_verify(p, q_prev, d_prev, T, 21, 5)
+    if not (np.array_equal(ver["accepted_len"], want["accepted_len"])
+            and np.array_equal(ver["out_tokens"], want["out_tokens"])
+            and np.array_equal(ver["out_count"], want["out_count"])):
+        fails.append("verify on the AR rows")
+    if not np.allclose(q_next, q, rtol=0, atol=1e-9):
+        fails.append("q_next = mask rows")
+    if not np.array_equal(d_next, draft_sample(q, T, 21, 5)):
+        fails.append("draft from the mask rows")
+    # 2. q_prev equal to this step's AR rows 0..k-1: every block is accepted and the
+    #    bonus is drawn (k + 1 tokens), whatever the seed
+    for seed in (0, 1, 2):
+        d_same = draft_sample(p[:, :k], T, seed + 50, 3)
+        ver, *_ = step_fn(h, layers, head, B, k, p[:, :k], d_same, T, seed, 3, 1.0)
+        if not (np.all(ver["accepted_len"] == k) and np.all(ver["out_count"] == k + 1)
+                and np.array_equal(ver["out_tokens"][:, :k], d_same)):
+            fails.append(f"full acceptance + bonus (seed {seed})")
+            break
+    return fails
+
+
+def test_psi_step_pins():
+    assert _step_pin_failures(O.psi_step) == []
+    # the pins do not depend on T
+    assert _step_pin_failures(O.psi_step, B=2, k=3, T=0.7) == []
+
+
+def _mutant(kind):
+    """psi_step with one planted wiring slip."""
+    def step(h_in, layers, head, B, k, q_prev_logits, d_prev, T, seed, step, scale):
+        gate = O.step_gate(B, k)
+        if kind == "gate_swapped":
+            gate = 1 - gate
+        logits = O.stack_logits(h_in, layers, head, gate, scale)
+        V = logits.shape[1]
+        nv = B * (k + 1)
+        p = logits[:nv].reshape(B, k + 1, V)
+        q_next = logits[nv:].reshape(B, k, V)
+        if kind == "blocks_swapped":                     # mask rows taken as the AR rows
+            q_next = logits[:B * k].reshape(B, k, V)
+            p = logits[B * k:].reshape(B, k + 1, V)
+        if kind == "no_bonus":                           # verify with k_p = k
+            p = p[:, :k]
+        if kind == "shifted":                            # AR rows 1..k instead of 0..k-1
+            p = np.concatenate([p[:, 1:], p[:, -1:]], axis=1)
+        ver = psi_verify(p, q_prev_logits, d_prev, T, seed, step)
+        d_src = p[:, :k] if kind == "draft_from_p" else q_next
+        d_next = draft_sample(d_src, T, seed, step + (1 if kind == "draft_step" else 0))
+        return ver, d_next, q_next, logits
+    return step
+
+
+@pytest.mark.parametrize("kind", ["gate_swapped", "blocks_swapped", "no_bonus", "shifted",
+                                  "draft_from_p", "draft_step"])
+def test_psi_step_pins_catch_planted_slips(kind):
+    assert _step_pin_failures(_mutant(kind)), f"planted slip {kind!r} passed every pin"
