@@ -94,3 +94,26 @@ def check_verify_outputs_valid(acc, tok, cnt, draft, k, k_p, V):
         np.testing.assert_array_equal(tok[b, :n], draft[b, :n])
         assert np.all(tok[b, c:] == -1)
         assert np.all((tok[b, :c] >= 0) & (tok[b, :c] < V))
+
+
+def compare_drafts(gpu, q_logits, T, seed, step, seq_offset=0):
+    """GPU drafts [B,k] against the oracle's draft sampler on the same logits.
+
+    A differing draw is excused only where the oracle's threshold u * Z lies within
+    TIE_CDF (relative to Z) of an edge of its token's CDF interval. Returns
+    (number excused, list of unexcused (b, j)).
+    """
+    from oracle import philox
+    from oracle import sampling as S
+    q = S.as_f64(q_logits)
+    o = S.draft_sample(q, T, seed, step, seq_offset)
+    bad, excused = [], 0
+    for b, j in np.argwhere(np.asarray(gpu) != o):
+        idx = (int(b) + seq_offset) * q.shape[1] + int(j)
+        u = philox.uniform_scalar(seed, step, philox.STREAM_DRAFT, idx)
+        margin = S.cdf_margin(S.softmax_t(q[b, j], T), u, int(o[b, j]))
+        if margin < TIE_CDF:
+            excused += 1
+        else:
+            bad.append((int(b), int(j)))
+    return excused, bad

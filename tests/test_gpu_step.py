@@ -5,16 +5,17 @@ bf16 between operations, so its logits carry bf16 rounding noise whose size
 depends on where each side rounds; the bound is derived from the oracle itself:
 the GPU's logits must lie within twice the distance between the oracle with
 bf16 storage and the oracle in fp64 throughout (that distance, ~6e-3
-relative on the small model, is the noise floor of the storage format). The step's tokens are checked by composition: they must
-equal uno_psi_verify / uno_draft_sample run on the step's own logits (those
-two kernels have their own oracle parity tests)."""
+relative on the small model, is the noise floor of the storage format). The
+step's tokens are checked against the oracle's verification and draft run on
+the step's own bf16 logits (decisions may differ only at logged near-ties).
+The Qwen3-8B-shaped step is checked layer by layer in test_gpu_step_qwen3.py."""
 import numpy as np
 import pytest
 
 import workloads as W
 from oracle import sampling as S
 from oracle import stack as O
-from gpu_util import dev_tensor, host_f64
+from gpu_util import compare_drafts, compare_verify, dev_tensor, host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -78,13 +79,15 @@ def test_tiny_step(shape, B, k, T):
     assert rel(got, exact) <= 2 * floor, (rel(got, exact), floor)
     assert rel(got, ref) <= 2 * floor, (rel(got, ref), floor)
     assert np.abs(got - exact).max() <= 2 * np.abs(ref - exact).max() + 2.0 ** -7 * np.abs(exact).max()
-    # tokens: same as the verify / draft kernels on the step's own logits
-    acc, tok, cnt = U.psi_verify(buf["logits"].reshape(B, k + 1, V), Q_prev, D_prev, T, 7, 5)
-    np.testing.assert_array_equal(buf["acc"].cpu().numpy(), acc.cpu().numpy())
-    np.testing.assert_array_equal(buf["tok"].cpu().numpy(), tok.cpu().numpy())
-    np.testing.assert_array_equal(buf["cnt"].cpu().numpy(), cnt.cpu().numpy())
-    d = U.draft_sample(buf["q_next"], T, 7, 5)
-    np.testing.assert_array_equal(buf["d_next"].cpu().numpy(), d.cpu().numpy())
+    # tokens: the oracle's verification of the previous block against the step's own
+    # (bf16) AR rows, and its draft from the step's mask rows, decide what is emitted
+    p_gpu = host_f64(buf["logits"]).reshape(B, k + 1, V)
+    ora = S.psi_verify(p_gpu, q_prev, d_prev, T, 7, 5)
+    gpu = tuple(buf[n].cpu().numpy() for n in ("acc", "tok", "cnt"))
+    excused, bad = compare_verify(gpu, ora, k, range(B))
+    assert not bad and len(excused) <= 1, (bad, excused)
+    excused, bad = compare_drafts(buf["d_next"].cpu().numpy(), host_f64(buf["q_next"]), T, 7, 5)
+    assert not bad and excused <= 1, (bad, excused)
     m.close()
 
 
