@@ -320,6 +320,21 @@ def kernel_lines(U, torch, pk):
             "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3),
             "mean_accepted": round(float(outs[0].float().mean()), 3)}
         del p, q
+    # linear-sampler draft of the step at B=256, k=8: 2048 rows of V=151936 bf16 logits.
+    # Algorithmic bytes: one read of every logit (the draw re-reads one vocab chunk a row).
+    Bd, kd = 256, 8
+    _, qd = W.logits_case_torch(Bd, kd, V, sigma=1.0, seed=4321)
+    dws = torch.empty(U.load().uno_draft_sample_workspace(Bd, kd, V), dtype=torch.uint8,
+                      device="cuda")
+    dout = torch.empty((Bd, kd), dtype=torch.int32, device="cuda")
+    f = lambda: U.draft_sample(qd, 1.0, 99, 0, draft=dout, workspace=dws)
+    f()
+    us = timed(f, reps=10)
+    byts = Bd * kd * V * 2
+    out[f"draft_sample_B{Bd}_k{kd}"] = {
+        "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
+        "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3)}
+    del qd
     # tree_verify at low batch: B=8 sequences, N=4 candidate blocks of k=8, V=151936.
     # Candidates: the linear sampler on q repeated N times per sequence (Philox index
     # (b N + i) k + j, the tree sampler's); AR row of each trie node = the draft row of

@@ -251,6 +251,9 @@ uno_status uno_distill(uno_dtype dt, int32_t rows, int32_t V, const void* z_teac
  *   cumulative sum of softmax(q_logits[b,j] / T) in ascending id; u0 from
  *   Philox stream 0 at index (seq_offset + b)*k + j.
  *   q_logits [B,k,V] `dt`; draft [B,k] int32 (device).
+ *   workspace: >= uno_draft_sample_workspace(B, k, V) bytes, 16-byte
+ *   aligned, any contents (per-row, per-vocab-chunk softmax statistics).
+ *   A row holding a NaN logit gets draft -1 and sets UNO_DEV_NAN.
  * ------------------------------------------------------------------------- */
 size_t uno_draft_sample_workspace(int32_t B, int32_t k, int32_t V);
 

@@ -385,7 +385,7 @@ def distill(z_teacher, z_student, alpha=1.0, beta=1.0, temperature=1.0, grad=Tru
 
 
 def draft_sample(q_logits, temperature, seed, step, seq_offset=0, draft=None, dev_status=None,
-                 stream=None):
+                 workspace=None, stream=None):
     """Linear-sampler draft: draft [B,k] int32 from softmax(q_logits / T)."""
     torch = _torch()
     _expect(q_logits, (None, None, None), _floats(), "q_logits")
@@ -394,10 +394,11 @@ def draft_sample(q_logits, temperature, seed, step, seq_offset=0, draft=None, de
     _expect(dev_status, (1,), (torch.int32,), "dev_status", optional=True)
     L = load()
     draft = torch.empty((B, k), dtype=torch.int32, device=q_logits.device) if draft is None else draft
-    dev = _dev(q_logits, draft, dev_status)
+    dev = _dev(q_logits, draft, dev_status, workspace)
+    ws, wsb = _workspace(L.uno_draft_sample_workspace(B, k, V), dev, workspace)
     _launch(dev, stream, L.uno_draft_sample, _dtype(q_logits), B, k, V, _ptr(q_logits),
             float(temperature), int(seed), int(step), int(seq_offset), _ptr(draft),
-            _ptr(dev_status), None, 0)
+            _ptr(dev_status), _ptr(ws), wsb)
     return draft
 
 
@@ -510,7 +511,7 @@ class Model:
         """Kernel launches issued by one step for (B, k) (0 before the first such step)."""
         return load().uno_psi_step_kernel_count(self._h, B, k)
 
-    def hidden(self, B, k, h_in, n_blocks, workspace, h_out=None, inter=False, stream=None):
+    def hidden_state(self, B, k, h_in, n_blocks, workspace, h_out=None, inter=False, stream=None):
         """uno_psi_step_hidden: the step's hidden state after its first n_blocks residual
         sub-blocks (two per layer). With inter=True also returns the products of the last
         sub-blocks run: dict q, k, v (n_blocks >= 1) and act = silu(gate) * up (n_blocks >= 2)."""

@@ -432,24 +432,24 @@ uno_status uno_distill(uno_dtype dt, int32_t rows, int32_t V, const void* z_teac
 }
 
 size_t uno_draft_sample_workspace(int32_t B, int32_t k, int32_t V) {
-  (void)B;
-  (void)k;
-  (void)V;
-  return 0;
+  if (B < 0 || k < 1 || V < 1) return 0;
+  return align_up(draft_workspace(B, k, V));
 }
 
 uno_status uno_draft_sample(uno_dtype dt, int32_t B, int32_t k, int32_t V, const void* q_logits,
                             float temperature, uint64_t seed, uint64_t step, uint64_t seq_offset,
                             int32_t* draft, int32_t* dev_status, void* workspace, size_t ws_bytes,
                             void* stream) {
-  (void)workspace;
-  (void)ws_bytes;
   uno_status s = check_sampler(dt, B, k, V, temperature);
   if (s != UNO_OK) return s;
   if (B == 0) return UNO_OK;
   if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k) > (1ull << 32))
     return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * k must be <= 2^32");
+  if (static_cast<int64_t>(B) * k > (1ll << 30)) return set_error(UNO_ERR_UNSUPPORTED, "B * k > 2^30");
   if (!q_logits || !draft) return set_error(UNO_ERR_INVALID_ARG, "NULL q_logits or draft");
+  const size_t need = uno_draft_sample_workspace(B, k, V);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
   DraftArgs a{};
   a.dt = dt;
   a.B = B;
@@ -462,7 +462,7 @@ uno_status uno_draft_sample(uno_dtype dt, int32_t B, int32_t k, int32_t V, const
   a.seq_offset = seq_offset;
   a.draft = draft;
   a.dev_status = dev_status;
-  return draft_launch(a, as_stream(stream));
+  return draft_launch(a, workspace, as_stream(stream));
 }
 
 uno_status uno_philox_uniforms(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,
@@ -500,7 +500,7 @@ constexpr int kLinPerLayer = 7;   // q, k, v, o, gate, up, down
 enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
 
 struct StepLayout {
-  size_t h, n, q, k, v, act, t, logits, vstat, sk_part, sk_flag, sk_flag_bytes, total;
+  size_t h, n, q, k, v, act, t, logits, vstat, dstat, sk_part, sk_flag, sk_flag_bytes, total;
 };
 
 // One operation of a step plan.
@@ -566,6 +566,7 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
   L.t = take(M * 3 * static_cast<size_t>(m->r) * 2);
   L.logits = take(Mv * static_cast<size_t>(m->vocab) * 2);
   L.vstat = take(verify_workspace(B, k, k + 1, m->vocab));
+  L.dstat = take(draft_workspace(B, k, m->vocab));
   // stream-K scratch of the CTA-pair GEMMs (M > 256): partial sums shared by
   // the step's launches, one block of flags per launch (4 per layer + head)
   if (M > 256) {
@@ -817,10 +818,10 @@ int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k) {
   if (!m || B < 1 || k < 1) return 0;
   // per layer: 2 rmsnorm + 4 GEMM launches, each with a separate
   // down-projection launch unless the fused decode kernel takes it; then
-  // rmsnorm + LM head; verify (2 kernels) + draft (1)
+  // rmsnorm + LM head; verify (2 kernels) + draft (2)
   std::lock_guard<std::mutex> lock(const_cast<uno_model*>(m)->mu);
   for (const auto& p : m->plans)
-    if (p->B == B && p->k == k && p->q_next) return static_cast<int32_t>(p->ops.size()) + 3;
+    if (p->B == B && p->k == k && p->q_next) return static_cast<int32_t>(p->ops.size()) + 4;
   return 0;
 }
 
@@ -897,7 +898,7 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   da.seq_offset = seq_offset;
   da.draft = d_next;
   da.dev_status = dev_status;
-  return draft_launch(da, st);
+  return draft_launch(da, base + L.dstat, st);
 }
 
 uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h_in,

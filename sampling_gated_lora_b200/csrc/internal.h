@@ -170,7 +170,8 @@ struct DraftArgs {
   int32_t* draft;
   int32_t* dev_status;
 };
-uno_status draft_launch(const DraftArgs& a, cudaStream_t s);
+size_t draft_workspace(int32_t B, int32_t k, int32_t V);
+uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s);
 
 uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,
                          int64_t n, uint32_t* words, float* u, cudaStream_t s);

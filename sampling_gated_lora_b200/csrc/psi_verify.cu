@@ -16,9 +16,10 @@
 //                        residual (or bonus) inverse-CDF draw split over the
 //                        cluster's CTAs (chunk totals exchanged through
 //                        distributed shared memory).
-//   draft_sample_kernel  one cluster per (sequence, position): chunk max ->
-//                        cluster max -> weights exp((z - max) / T) -> the same
-//                        inverse-CDF draw.
+//   draft_draw_kernel    after row_stats_kernel has streamed the q rows once:
+//                        one CTA per (sequence, position) finds the vocab
+//                        chunk holding the draw from the chunk totals and
+//                        reads only that chunk again for the inverse-CDF draw.
 // Uniforms: Philox4x32-10 word 0 at counter (index, step lo, step hi,
 // stream), key (seed lo, seed hi); u = (x >> 8) 2^-24. The counter depends on
 // (sequence, position, stream) only, never on the launch shape.
@@ -928,79 +929,124 @@ __global__ void __launch_bounds__(kDrawThreads)
 }
 
 struct DraftParams {
-  int k, V;
+  int k, V, chunks, chunk_len;
   float c;
   uint64_t seed, step, seq_offset;
+  const float2* stats;   // [rows, chunks]: (chunk max, sum exp2((z - max) c)) of the q rows
   int32_t* draft;
   int32_t* status;
 };
 
-// One cluster per (sequence, position) row of q; blockDim = kDrawThreads.
+constexpr int kDraftMaxChunks = 128;   // draft_chunks() never exceeds it
+
+// Linear-sampler draw of one row, after row_stats_kernel has streamed the row
+// once: the chunk totals w_c = s_c 2^((m_c - M) c) (M the row max) give the
+// chunk that holds the threshold u0 * Z, Z = sum w_c (the last chunk with
+// positive total whose exclusive prefix is <= u0 Z), and only that chunk is
+// read again: per-thread contiguous segments of weights 2^((z - M) c), a block
+// scan of the segment sums, then the owning thread walks its segment in
+// ascending id. Every sum is taken in double from float weights. One CTA per
+// row (B k rows); blockDim = kDrawThreads.
 template <typename T>
 __global__ void __launch_bounds__(kDrawThreads)
-    draft_sample_kernel(const T* __restrict__ q_logits, const DraftParams a) {
-  extern __shared__ __align__(16) uint8_t dyn[];
+    draft_draw_kernel(const T* __restrict__ q_logits, const DraftParams a) {
   __shared__ DrawSmem sh;
-  __shared__ float s_max;
-  __shared__ float s_cmax[kDrawThreads / 32];
+  __shared__ double s_tot[kDraftMaxChunks];
+  __shared__ float s_M;
+  __shared__ int s_bad, s_owner;
+  __shared__ double s_tl;
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
-  const uint32_t nrank = cluster_nctarank();
-  const uint32_t rank = cluster_ctarank();
-  const int row = blockIdx.x / nrank;
-  const int V = a.V;
-  int lo, len;
-  chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
-  T* z = reinterpret_cast<T*>(dyn);
-  load_chunk(z, q_logits + static_cast<size_t>(row) * V + lo, len);
-  cta_sync();
-  float mx = -INFINITY;
-  bool nan = false;
-  for (int i = threadIdx.x; i < len; i += blockDim.x) {
-    const float f = to_f32<T>(z[i]);
-    nan |= isnan(f);
-    mx = fmaxf(mx, f);
-  }
-  mx = warp_max(mx);
-  nan = __any_sync(0xffffffffu, nan);
-  if ((threadIdx.x & 31) == 0) s_cmax[threadIdx.x >> 5] = nan ? NAN : mx;
-  cta_sync();
-  if (threadIdx.x == 0) {
+  const int row = blockIdx.x;
+  const int chunks = a.chunks;
+  const float c = a.c;
+  const float2* st = a.stats + static_cast<size_t>(row) * chunks;
+  if (threadIdx.x < 32) {
     float m = -INFINITY;
-    bool any_nan = false;
-    for (int w = 0; w < kDrawThreads / 32; ++w) {
-      any_nan |= isnan(s_cmax[w]);
-      m = fmaxf(m, s_cmax[w]);
+    bool nan = false;
+    for (int i = threadIdx.x; i < chunks; i += 32) {
+      const float2 v = st[i];
+      nan |= isnan(v.y);
+      m = fmaxf(m, v.x);
     }
-    s_max = any_nan ? NAN : m;
+    m = warp_max(m);
+    nan = __any_sync(0xffffffffu, nan);
+    if (threadIdx.x == 0) {
+      s_M = m;
+      s_bad = nan || m == -INFINITY;
+    }
   }
-  cluster_sync();
-  // cluster-wide max (NaN if any chunk saw a NaN)
-  float M = -INFINITY;
-  bool any_nan = false;
-  const uint32_t addr = smem_u32(&s_max);
-  for (uint32_t r = 0; r < nrank; ++r) {
-    const float v = ld_cluster_f32(map_shared_rank(addr, r));
-    any_nan |= isnan(v);
-    M = fmaxf(M, v);
-  }
-  cluster_sync();
-  if (any_nan || M == -INFINITY) {
-    if (rank == 0 && threadIdx.x == 0) {
+  cta_sync();
+  if (s_bad) {
+    if (threadIdx.x == 0) {
       a.draft[row] = -1;
       raise_status(a.status, kDevNaN);
     }
     return;
   }
-  const int b = row / a.k, j = row % a.k;
+  const float M = s_M;
+  for (int i = threadIdx.x; i < chunks; i += blockDim.x) {
+    const float2 v = st[i];
+    s_tot[i] = static_cast<double>(v.y) * static_cast<double>(fast_exp2((v.x - M) * c));
+  }
+  cta_sync();
+  const int b = row / a.k, j = row - b * a.k;
   const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
   const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(a.k) + j);
-  const double u = static_cast<double>(uniform24(philox_word0(a.seed, a.step, kStreamDraft, idx)));
-  const float c = a.c;
-  auto w = [&](int i) { return fast_exp2((to_f32<T>(z[i]) - M) * c); };
-  bool zero = false;
-  const int token = cluster_draw(sh, w, lo, len, u, &zero);
-  if (token >= 0 && threadIdx.x == 0) a.draft[row] = token;
+  if (threadIdx.x == 0) {
+    double Z = 0.0;
+    for (int i = 0; i < chunks; ++i) Z += s_tot[i];
+    const double thr = static_cast<double>(uniform24(philox_word0(a.seed, a.step, kStreamDraft, idx))) * Z;
+    double pre = 0.0, own_pre = 0.0;
+    int own = -1;
+    for (int i = 0; i < chunks; ++i) {
+      if (s_tot[i] > 0.0 && pre <= thr) {
+        own = i;
+        own_pre = pre;
+      }
+      pre += s_tot[i];
+    }
+    s_owner = own;
+    s_tl = thr - own_pre;
+  }
+  cta_sync();
+  const int own_chunk = s_owner;   // >= 0: the chunk holding the row max has total >= 1
+  const int lo = own_chunk * a.chunk_len;
+  const int len = min(a.V, lo + a.chunk_len) - lo;
+  const T* z = q_logits + static_cast<size_t>(row) * a.V + lo;
+  const int t = threadIdx.x;
+  const int seg = (len + kDrawThreads - 1) / kDrawThreads;
+  const int s0 = min(len, t * seg), s1 = min(len, s0 + seg);
+  double my = 0.0;
+  for (int i = s0; i < s1; ++i) my += static_cast<double>(fast_exp2((to_f32<T>(z[i]) - M) * c));
+  block_scan(sh, my);
+  const double tl = s_tl;
+  const int own = block_max_index(sh, my > 0.0 && sh.prefix[t] <= tl);
+  if (t == own) {
+    const double tt = tl - sh.prefix[t];
+    double run = 0.0;
+    int pick = -1, last_nz = -1;
+    for (int i = s0; i < s1; ++i) {
+      const float w = fast_exp2((to_f32<T>(z[i]) - M) * c);
+      if (w > 0.f) last_nz = i;
+      run += static_cast<double>(w);
+      if (run > tt) {
+        pick = i;
+        break;
+      }
+    }
+    a.draft[row] = lo + (pick >= 0 ? pick : last_nz);
+  } else if (own < 0 && t == 0) {
+    // every recomputed weight of the chunk flushed to zero (its total is below
+    // the float range): the chunk's first id with the row max
+    int arg = 0;
+    for (int i = 0; i < len; ++i)
+      if (to_f32<T>(z[i]) == M) {
+        arg = i;
+        break;
+      }
+    a.draft[row] = lo + arg;
+  }
 }
 
 __global__ void philox_kernel(uint64_t seed, uint64_t step, uint32_t stream, uint32_t index0,
@@ -1191,26 +1237,56 @@ uno_status distill_launch(const DistillArgs& a, cudaStream_t s) {
                         static_cast<const __nv_bfloat16*>(a.z_student), dp);
 }
 
-uno_status draft_launch(const DraftArgs& a, cudaStream_t s) {
-  const int esz = a.dt == UNO_F32 ? 4 : 2;
-  int chunk_elems = 0;
-  const int cl = draw_cluster(a.V, esz, &chunk_elems);
+// Vocabulary chunks of the draft's stats pass: enough CTAs to cover the SMs
+// (as for verification), and chunks of at most kDraftChunk ids so that the
+// draw re-reads a small part of each row.
+constexpr int kDraftChunk = 8192;
+
+int draft_chunks(int rows, int V) {
+  return std::min(kDraftMaxChunks, std::max(stat_chunks(rows, V), (V + kDraftChunk - 1) / kDraftChunk));
+}
+
+size_t draft_workspace(int32_t B, int32_t k, int32_t V) {
+  const int rows = B * k;
+  return static_cast<size_t>(rows) * draft_chunks(rows, V) * sizeof(float2);
+}
+
+uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
+  const int rows = a.B * a.k;
+  const int chunks = draft_chunks(rows, a.V);
+  const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
+  const float c = kLog2e / a.temperature;
+  float2* stats = static_cast<float2*>(ws);
   DraftParams dp{};
   dp.k = a.k;
   dp.V = a.V;
-  dp.c = kLog2e / a.temperature;
+  dp.chunks = chunks;
+  dp.chunk_len = chunk_len;
+  dp.c = c;
   dp.seed = a.seed;
   dp.step = a.step;
   dp.seq_offset = a.seq_offset;
+  dp.stats = stats;
   dp.draft = a.draft;
   dp.status = a.dev_status;
-  const size_t smem = static_cast<size_t>(chunk_elems) * esz;
-  const int rows = a.B * a.k;
-  if (a.dt == UNO_F32)
-    return launch_cluster(draft_sample_kernel<float>, rows * cl, cl, smem, s,
-                          static_cast<const float*>(a.q_logits), dp);
-  return launch_cluster(draft_sample_kernel<__nv_bfloat16>, rows * cl, cl, smem, s,
-                        static_cast<const __nv_bfloat16*>(a.q_logits), dp);
+  const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(rows) * chunks));
+  cudaError_t e;
+  if (a.dt == UNO_F32) {
+    const float* q = static_cast<const float*>(a.q_logits);
+    e = launch_kernel(row_stats_kernel<float>, grid, dim3(kStatThreads), 0, s, 1, q, q, 0, a.V,
+                      chunks, chunk_len, c, stats);
+    if (e == cudaSuccess)
+      e = launch_kernel(draft_draw_kernel<float>, dim3(rows), dim3(kDrawThreads), 0, s, 1, q, dp);
+  } else {
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_logits);
+    e = launch_kernel(row_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1, q, q, 0,
+                      a.V, chunks, chunk_len, c, stats);
+    if (e == cudaSuccess)
+      e = launch_kernel(draft_draw_kernel<__nv_bfloat16>, dim3(rows), dim3(kDrawThreads), 0, s, 1,
+                        q, dp);
+  }
+  if (e != cudaSuccess) return cuda_error(e, "draft launch");
+  return UNO_OK;
 }
 
 uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,

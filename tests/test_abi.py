@@ -100,6 +100,13 @@ def test_draft_and_misc_reject_bad_arguments():
     ok = ctypes.c_void_p(0x10000)
     assert L.uno_draft_sample(U.UNO_BF16, 2, 4, 1024, ok, 0.0, 0, 0, 0, ok, null, null, 0, null) == 1
     assert L.uno_draft_sample(U.UNO_BF16, 2, 4, 1024, null, 1.0, 0, 0, 0, ok, null, null, 0, null) == 1
+    # the draft's stats pass needs its workspace: (rows, vocab chunks of <= 8192 ids) pairs
+    need = L.uno_draft_sample_workspace(2, 4, 151936)
+    assert need >= 2 * 4 * 19 * 8
+    assert L.uno_draft_sample(U.UNO_BF16, 2, 4, 151936, ok, 1.0, 0, 0, 0, ok, null, null, 0,
+                              null) == 6
+    assert L.uno_draft_sample(U.UNO_BF16, 2, 4, 151936, ok, 1.0, 0, 0, 0, ok, null, ok,
+                              need - 1, null) == 6
     assert L.uno_philox_uniforms(0, 0, 0, 0xFFFFFFFF, 2, ok, ok, null) == 1
     assert L.uno_philox_uniforms(0, 0, 0, 0, -1, ok, ok, null) == 1
     assert L.uno_rmsnorm(-1, 8, ok, ok, 1e-6, null) == 1

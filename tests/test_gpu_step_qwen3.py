@@ -106,9 +106,9 @@ def test_every_sub_block_and_linear_from_the_gpu_input(qwen3):
             rows = run["rows"]
             g = O.step_gate(B, k)[rows]
             what = f"B={B} layer {li}"
-            h_l = _take(m.hidden(B, k, run["h"], 2 * li, run["ws"]), rows)
-            h_mid_t, mid = m.hidden(B, k, run["h"], 2 * li + 1, run["ws"], inter=True)
-            h_next_t, nxt = m.hidden(B, k, run["h"], 2 * li + 2, run["ws"], inter=True)
+            h_l = _take(m.hidden_state(B, k, run["h"], 2 * li, run["ws"]), rows)
+            h_mid_t, mid = m.hidden_state(B, k, run["h"], 2 * li + 1, run["ws"], inter=True)
+            h_next_t, nxt = m.hidden_state(B, k, run["h"], 2 * li + 2, run["ws"], inter=True)
             h_mid, h_next = _take(h_mid_t, rows), _take(h_next_t, rows)
             # projection sub-block: q, k, v from rmsnorm(h_l); h_mid = h_l + o(q)
             n1 = O.round_bf16(O.rmsnorm(h_l))
@@ -134,7 +134,7 @@ def test_lm_head_rows_split_into_logits_and_q_next(qwen3):
     for B, run in runs.items():
         rows = run["rows"]
         g = O.step_gate(B, k)[rows]
-        h_final = _take(m.hidden(B, k, run["h"], 2 * SHAPE.n_layers, run["ws"]), rows)
+        h_final = _take(m.hidden_state(B, k, run["h"], 2 * SHAPE.n_layers, run["ws"]), rows)
         n_f = O.round_bf16(O.rmsnorm(h_final))
         nv = B * (k + 1)
         logits = _bits(run["out"]["logits"])
