@@ -346,6 +346,23 @@ uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h
 int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k);
 
 /* ---------------------------------------------------------------------------
+ * Self-test of the bounded waits (a library addition; the pages have no
+ * counterpart). Every spin in the library's kernels gives up after a time
+ * limit, ORs UNO_DEV_TIMEOUT into the status words and returns, so a lost
+ * arrival ends in a status the host reads, never in a hung GPU. This call
+ * runs one such wait on a condition nothing will satisfy, with no copy or
+ * tensor-core work in flight:
+ *   which 0: a global-memory flag that is never raised;
+ *         1: an mbarrier phase that gets no arrival;
+ *         2: the same through the cluster-scope wait (used between CTA pairs);
+ *         3: control: the expected arrival comes first and the wait succeeds.
+ *   limit_ns in [1e3, 1e8]; result: device int32, 1 if the wait was
+ *   satisfied, 0 if it gave up; dev_status: optional device int32 word.
+ * ------------------------------------------------------------------------- */
+uno_status uno_wait_selftest(int32_t which, uint64_t limit_ns, int32_t* result,
+                             int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * The step's glue operations, exposed for testing (all bf16, device):
  *   uno_rmsnorm:  y[m,:] = x[m,:] / sqrt(mean(x[m,:]^2) + eps)      x, y [M,D]
  *   uno_silu_mul: y = silu(a) * b = a / (1 + exp(-a)) * b           [n]

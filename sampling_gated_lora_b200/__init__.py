@@ -35,7 +35,7 @@ EXPORTS = [
     "uno_philox_uniforms",
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
     "uno_psi_step_hidden", "uno_psi_step_kernel_count",
-    "uno_rmsnorm", "uno_silu_mul",
+    "uno_rmsnorm", "uno_silu_mul", "uno_wait_selftest",
 ]
 
 
@@ -91,6 +91,7 @@ def load():
         "uno_psi_step_kernel_count": (i32, [vp, i32, i32]),
         "uno_rmsnorm": (i32, [i64, i64, vp, vp, f32, vp]),
         "uno_silu_mul": (i32, [i64, vp, vp, vp, vp]),
+        "uno_wait_selftest": (i32, [i32, u64, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -435,6 +436,19 @@ def silu_mul(a, b, y=None, stream=None):
     dev = _dev(a, b, y)
     _launch(dev, stream, L.uno_silu_mul, a.numel(), _ptr(a), _ptr(b), _ptr(y))
     return y
+
+
+def wait_selftest(which, limit_ns=1_000_000, dev_status=None, device="cuda", stream=None):
+    """uno_wait_selftest: one bounded wait (0 flag, 1 mbarrier, 2 cluster-scope mbarrier,
+    3 control) on a condition nothing satisfies; returns the device result word
+    (1 satisfied, 0 gave up)."""
+    torch = _torch()
+    L = load()
+    result = torch.full((1,), -1, dtype=torch.int32, device=device)
+    dev = _dev(result, dev_status)
+    _launch(dev, stream, L.uno_wait_selftest, int(which), int(limit_ns), _ptr(result),
+            _ptr(dev_status))
+    return result
 
 
 def device_status(clear=True, stream=None, device=None) -> int:

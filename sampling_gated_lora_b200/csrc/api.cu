@@ -473,6 +473,16 @@ uno_status uno_philox_uniforms(uint64_t seed, uint64_t step, uint32_t stream_id,
   return philox_launch(seed, step, stream_id, index0, n, words, u, as_stream(stream));
 }
 
+uno_status uno_wait_selftest(int32_t which, uint64_t limit_ns, int32_t* result,
+                             int32_t* dev_status, void* stream) {
+  if (which < 0 || which > 3) return set_error(UNO_ERR_INVALID_ARG, "which=%d outside [0, 3]", which);
+  if (limit_ns < 1000 || limit_ns > 100000000ull)
+    return set_error(UNO_ERR_INVALID_ARG, "limit_ns=%llu outside [1e3, 1e8]",
+                     static_cast<unsigned long long>(limit_ns));
+  if (!result) return set_error(UNO_ERR_INVALID_ARG, "result is NULL");
+  return wait_selftest_launch(which, limit_ns, result, dev_status, as_stream(stream));
+}
+
 uno_status uno_rmsnorm(int64_t M, int64_t D, const void* x, void* y, float eps, void* stream) {
   if (M < 0 || D < 1) return set_error(UNO_ERR_INVALID_ARG, "bad sizes");
   if (M > 0 && (!x || !y)) return set_error(UNO_ERR_INVALID_ARG, "NULL pointer");

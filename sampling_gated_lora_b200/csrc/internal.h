@@ -197,6 +197,10 @@ struct NormDownArgs {   // bf16 tensors
 };
 uno_status norm_down_launch(const NormDownArgs& a, int64_t M, cudaStream_t s);
 
+// The bounded-wait self-test (waits.cu).
+uno_status wait_selftest_launch(int32_t which, uint64_t limit_ns, int32_t* result,
+                                int32_t* status, cudaStream_t s);
+
 int device_sm_count();
 
 // Launch attributes shared by every kernel launch: programmatic stream

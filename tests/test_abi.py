@@ -112,6 +112,10 @@ def test_draft_and_misc_reject_bad_arguments():
     assert L.uno_rmsnorm(-1, 8, ok, ok, 1e-6, null) == 1
     assert L.uno_silu_mul(-1, ok, ok, ok, null) == 1
     assert L.uno_device_status(null, 0, null) == 1
+    assert L.uno_wait_selftest(4, 1000000, ok, null, null) == 1           # which in [0, 3]
+    assert L.uno_wait_selftest(0, 10, ok, null, null) == 1                # limit >= 1 us
+    assert L.uno_wait_selftest(0, 10 ** 9, ok, null, null) == 1           # limit <= 100 ms
+    assert L.uno_wait_selftest(0, 1000000, null, null, null) == 1
 
 
 def test_model_create_validates():
