@@ -39,7 +39,23 @@ namespace {
 
 constexpr int kStatThreads = 256;
 constexpr int kDrawThreads = 256;
-constexpr float kLog2e = 1.4426950408889634f;
+
+// The softmax weights are 2^((z - max) c) with c = log2(e) / T. c is held as
+// an unevaluated sum hi + lo of two floats and the exponent is formed with
+// one fused multiply-add: a single float c would carry a rounding error of up
+// to 6e-8 relative that scales every weight by 2^(-(max - z) err), a
+// distortion correlated with the logits. (z - max is exact for bf16 logits.)
+struct TScale {
+  float hi, lo;
+};
+__device__ __forceinline__ float operator*(float d, TScale c) { return fmaf(d, c.hi, d * c.lo); }
+TScale make_tscale(float temperature) {
+  const double cd = 1.4426950408889634073599 / static_cast<double>(temperature);
+  TScale t;
+  t.hi = static_cast<float>(cd);
+  t.lo = static_cast<float>(cd - static_cast<double>(t.hi));
+  return t;
+}
 
 template <typename T>
 struct Vec;   // 16-byte vector of logits
@@ -65,7 +81,7 @@ struct Vec<float> {
 struct OnlineStat {
   float m = -INFINITY;
   float s = 0.f;
-  __device__ __forceinline__ void add(const float* v, int n, float c) {
+  __device__ __forceinline__ void add(const float* v, int n, TScale c) {
     float mx = v[0];
     for (int e = 1; e < n; ++e) mx = fmaxf(mx, v[e]);
     if (mx > m) {
@@ -77,7 +93,7 @@ struct OnlineStat {
 };
 
 // Merge (m1, s1) with (m2, s2); s is relative to m, exp base 2 with scale c.
-__device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s2, float c) {
+__device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s2, TScale c) {
   if (isnan(s2) || isnan(s)) {   // keep a NaN seen anywhere
     s = NAN;
     m = fmaxf(m, m2);
@@ -101,7 +117,7 @@ __device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s
 template <typename T>
 __global__ void __launch_bounds__(kStatThreads)
     row_stats_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits, int rows_p,
-                     int V, int chunks, int chunk_len, float c, float2* __restrict__ stats) {
+                     int V, int chunks, int chunk_len, TScale c, float2* __restrict__ stats) {
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
   const int row = static_cast<int>(blockIdx.x / static_cast<unsigned>(chunks));
@@ -163,7 +179,7 @@ __global__ void __launch_bounds__(kStatThreads)
 }
 
 // Merge the chunk stats of one row.
-__device__ __forceinline__ float2 row_stat(const float2* stats, int row, int chunks, float c) {
+__device__ __forceinline__ float2 row_stat(const float2* stats, int row, int chunks, TScale c) {
   float m = -INFINITY, s = 0.f;
   bool nan = false;
   for (int i = 0; i < chunks; ++i) {
@@ -342,7 +358,7 @@ __device__ __forceinline__ void load_chunk(T* dst, const T* src, int len) {
 
 struct FinalizeParams {
   int B, k, k_p, V, chunks;
-  float c;   // log2(e) / T
+  TScale c;   // log2(e) / T
   uint64_t seed, step, seq_offset;
   const int32_t* draft;
   const float2* stats;
@@ -453,7 +469,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   cta_sync();
   const float Mp = s_stat[0], inv_sp = 1.f / s_stat[1];
   const float Mq = s_stat[2], inv_sq = residual ? 1.f / s_stat[3] : 0.f;
-  const float c = a.c;
+  const TScale c = a.c;
   const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + (residual ? n : k));
   const double u = static_cast<double>(uniform24(
       philox_word0(a.seed, a.step, residual ? kStreamResidual : kStreamBonus, idx)));
@@ -497,7 +513,7 @@ constexpr int kTreeMaxK = 32;   // block length
 
 struct TreeParams {
   int B, N, k, R, V, chunks, bonus;
-  float c;   // log2(e) / T
+  TScale c;   // log2(e) / T
   uint64_t seed, step, seq_offset;
   const int32_t* cands;   // [B, N, k]
   const float2* stats;    // chunk stats of node rows b*R + n, then q rows B*R + b*k + j
@@ -566,7 +582,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
   const int32_t* cand = a.cands + static_cast<size_t>(b) * nk;
   int32_t* tok = a.out_tokens + static_cast<size_t>(b) * (k + 1);
-  const float c = a.c;
+  const TScale c = a.c;
 
   // 1. Trie numbering. rep(i, j) = the first candidate with the same j+1
   //    tokens; the first visits, in walk order (i, then j), get ids 1, 2, ...
@@ -771,7 +787,7 @@ __global__ void __launch_bounds__(kDrawThreads)
 
 struct DistillParams {
   int V, chunk_elems;
-  float c;            // log2(e) / T
+  TScale c;           // log2(e) / T
   float inv_t;        // 1 / T
   float alpha, beta;
   float grad_scale;   // 1 / (T rows)
@@ -886,7 +902,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   }
 
   // 2. the partition sums, then KL, TV and sum(sign(q - p) q)
-  const float c = a.c;
+  const TScale c = a.c;
   double sums[3] = {0.0, 0.0, 0.0};
   for (int i = threadIdx.x; i < len; i += blockDim.x) {
     sums[0] += static_cast<double>(fast_exp2((to_f32<T>(zt[i]) - Mt) * c));
@@ -930,7 +946,7 @@ __global__ void __launch_bounds__(kDrawThreads)
 
 struct DraftParams {
   int k, V, chunks, chunk_len;
-  float c;
+  TScale c;
   uint64_t seed, step, seq_offset;
   const float2* stats;   // [rows, chunks]: (chunk max, sum exp2((z - max) c)) of the q rows
   int32_t* draft;
@@ -959,7 +975,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   pdl_wait();
   const int row = blockIdx.x;
   const int chunks = a.chunks;
-  const float c = a.c;
+  const TScale c = a.c;
   const float2* st = a.stats + static_cast<size_t>(row) * chunks;
   if (threadIdx.x < 32) {
     float m = -INFINITY;
@@ -1110,7 +1126,7 @@ uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s) {
   const int rows = a.B * a.k_p + a.B * a.k;
   const int chunks = stat_chunks(rows, a.V);
   const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
-  const float c = kLog2e / a.temperature;
+  const TScale c = make_tscale(a.temperature);
   float2* stats = static_cast<float2*>(ws);
   const int esz = a.dt == UNO_F32 ? 4 : 2;
   int chunk_elems = 0;
@@ -1165,7 +1181,7 @@ uno_status tree_verify_launch(const TreeVerifyArgs& a, void* ws, cudaStream_t s)
   const int rows = a.B * a.R + a.B * a.k;
   const int chunks = stat_chunks(rows, a.V);
   const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
-  const float c = kLog2e / a.temperature;
+  const TScale c = make_tscale(a.temperature);
   float2* stats = static_cast<float2*>(ws);
   const int esz = a.dt == UNO_F32 ? 4 : 2;
   int chunk_elems = 0;
@@ -1219,7 +1235,7 @@ uno_status distill_launch(const DistillArgs& a, cudaStream_t s) {
   DistillParams dp{};
   dp.V = a.V;
   dp.chunk_elems = chunk_elems;
-  dp.c = kLog2e / a.temperature;
+  dp.c = make_tscale(a.temperature);
   dp.inv_t = 1.f / a.temperature;
   dp.alpha = a.alpha;
   dp.beta = a.beta;
@@ -1255,7 +1271,7 @@ uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
   const int rows = a.B * a.k;
   const int chunks = draft_chunks(rows, a.V);
   const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
-  const float c = kLog2e / a.temperature;
+  const TScale c = make_tscale(a.temperature);
   float2* stats = static_cast<float2*>(ws);
   DraftParams dp{};
   dp.k = a.k;

@@ -19,6 +19,12 @@ TIE_CDF = 1e-5
 EXCUSED_CAP = 1e-4   # excused positions / all positions, at full size
 
 
+def api_T(T):
+    """The temperature as the library receives it: the C ABI takes an IEEE float32,
+    so the oracle is given that same value (0.7 becomes 0.699999988...)."""
+    return float(np.float32(T))
+
+
 def torch_mod():
     import torch
     return torch

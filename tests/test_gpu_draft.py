@@ -7,7 +7,7 @@ from scipy import stats
 
 import workloads as W
 from oracle import sampling as S
-from gpu_util import TIE_CDF, dev_tensor
+from gpu_util import TIE_CDF, api_T, dev_tensor
 
 pytestmark = pytest.mark.gpu
 
@@ -19,6 +19,7 @@ def _gpu_draft(q, T, seed, step, seq_offset=0, dt="bf16"):
 
 
 def _check_parity(q, T, seed, step, dt, seq_offset=0):
+    T = api_T(T)
     g = _gpu_draft(q, T, seed, step, seq_offset, dt)
     o = S.draft_sample(q, T, seed, step, seq_offset)
     diff = np.argwhere(g != o)
@@ -45,6 +46,17 @@ def test_tiny_fp32(T):
 def test_bf16_parity(V, T):
     case = W.logits_case(8, 8, V, ar_std=3.0, sigma=1.0, seed=21)
     _check_parity(case.q_logits, T, 17, 4, "bf16", seq_offset=3)
+
+
+@pytest.mark.parametrize("T", [1.0, 0.7])
+def test_flat_rows_full_vocabulary(T):
+    """1024 rows of N(0, 1) logits over V = 151936: near-flat rows whose tokens hold
+    CDF intervals of ~1e-5 of the total, so a systematic error of the weights in the
+    last digits of float precision shows up as differing draws."""
+    import torch
+    gen = torch.Generator().manual_seed(int(T * 100))
+    q = W.from_torch_bf16(torch.randn((128, 8, 151936), generator=gen).to(torch.bfloat16))
+    _check_parity(q, T, 23, 6, "bf16")
 
 
 def _replicate(row_bits, n):

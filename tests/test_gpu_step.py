@@ -15,7 +15,7 @@ import pytest
 import workloads as W
 from oracle import sampling as S
 from oracle import stack as O
-from gpu_util import compare_drafts, compare_verify, dev_tensor, host_f64
+from gpu_util import api_T, compare_drafts, compare_verify, dev_tensor, host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -54,6 +54,7 @@ WIDE_MLP_SHAPE = W.ModelShape(n_layers=1, hidden=256, q_out=256, kv_out=64, inte
 def test_tiny_step(shape, B, k, T):
     import torch
     import sampling_gated_lora_b200 as U
+    T = api_T(T)
     m, layers_np, head_np = _model(shape, seed=1)
     V = shape.vocab
     h = W.step_hidden(B, k, shape.hidden, seed=2)

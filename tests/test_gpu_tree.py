@@ -58,6 +58,7 @@ def test_one_candidate_equals_linear_verification(bonus):
                                            (8, 4, 32000, 1.0, True), (3, 1, 5003, 1.0, False),
                                            (32, 2, 512, 1.0, True)])
 def test_parity_with_oracle(N, k, V, T, bonus):
+    T = float(np.float32(T))      # the C ABI's float32 temperature, given to the oracle too
     B = 12
     P, Q, cands, p_b, q_b = _case(B, N, k, V, sigma=1.5, seed=N * 7 + k, T=T)
     acc, tok, cnt = _gpu(P, Q, cands, T, 21, 5, bonus, seq_offset=2)

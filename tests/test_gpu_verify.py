@@ -6,7 +6,7 @@ import pytest
 
 import workloads as W
 from oracle import sampling as S
-from gpu_util import (EXCUSED_CAP, check_verify_outputs_valid, compare_verify, dev_tensor)
+from gpu_util import (EXCUSED_CAP, api_T, check_verify_outputs_valid, compare_verify, dev_tensor)
 
 pytestmark = pytest.mark.gpu
 
@@ -21,6 +21,7 @@ def _gpu_verify(p, q, d, T, seed, step, seq_offset=0, dt="bf16", status=None):
 
 
 def _case_check(case, T, seed, step, seq_offset=0, max_excused=1):
+    T = api_T(T)
     d = S.draft_sample(case.q_logits, T, seed + 1, step, seq_offset)   # inputs: drafts ~ q
     gpu = _gpu_verify(case.p_logits, case.q_logits, d, T, seed, step, seq_offset, case.dtype)
     ora = S.psi_verify(case.p_logits, case.q_logits, d, T, seed, step, seq_offset)
@@ -68,7 +69,7 @@ def test_sequence_offset_reproduces_global_draws():
 def test_zero_adapter_accepts_every_block():
     """q == p (the adapter's B = 0): n = k for every sequence, with or without the bonus."""
     case = W.logits_case(64, 8, 30000, k_p=9, ar_std=3.0, sigma=0.0, seed=12)
-    for T in (1.0, 0.7):
+    for T in (1.0, api_T(0.7)):
         for seed in (0, 1, 2):
             d = S.draft_sample(case.p_logits[:, :8], T, seed + 100, 0)
             acc, tok, cnt = _gpu_verify(case.p_logits, case.p_logits[:, :8], d, T, seed, 0)
@@ -120,7 +121,7 @@ def test_full_size_parity(sigma):
     p_h, q_h = W.from_torch_bf16(p), W.from_torch_bf16(q)
     sample = np.arange(B)
     total_excused = 0
-    for T in (1.0, 0.7):
+    for T in (1.0, api_T(0.7)):
         d = S.draft_sample(q_h, T, 99, 0)
         gpu = _gpu_verify(p, q, d, T, 1234, 0)
         check_verify_outputs_valid(*gpu, d, k, k, V)
