@@ -16,7 +16,7 @@
 //                        residual (or bonus) inverse-CDF draw split over the
 //                        cluster's CTAs (chunk totals exchanged through
 //                        distributed shared memory).
-//   draft_draw_kernel    after row_stats_kernel has streamed the q rows once:
+//   draft_draw_kernel    after row_stats_warp_kernel has streamed the q rows once:
 //                        one CTA per (sequence, position) finds the vocab
 //                        chunk holding the draw from the chunk totals and
 //                        reads only that chunk again for the inverse-CDF draw.
@@ -45,6 +45,8 @@ constexpr int kDrawThreads = 256;
 // one fused multiply-add: a single float c would carry a rounding error of up
 // to 6e-8 relative that scales every weight by 2^(-(max - z) err), a
 // distortion correlated with the logits. (z - max is exact for bf16 logits.)
+// hi is taken strictly below c, so lo > 0 and an infinite d gives an infinite
+// exponent of its own sign (never inf - inf).
 struct TScale {
   float hi, lo;
 };
@@ -53,6 +55,7 @@ TScale make_tscale(float temperature) {
   const double cd = 1.4426950408889634073599 / static_cast<double>(temperature);
   TScale t;
   t.hi = static_cast<float>(cd);
+  if (static_cast<double>(t.hi) >= cd) t.hi = std::nextafter(t.hi, 0.f);
   t.lo = static_cast<float>(cd - static_cast<double>(t.hi));
   return t;
 }
@@ -176,6 +179,65 @@ __global__ void __launch_bounds__(kStatThreads)
     // a NaN anywhere in the chunk makes S NaN (fmaxf skips it in the max)
     stats[blockIdx.x] = make_float2(M, S);
   }
+}
+
+// Warp-granular form for the draft: warp w of the grid (8 per CTA) takes
+// (row w / nsub, sub-chunk w % nsub) of sub_len ids, keeps one online stat
+// per lane over its 16-byte vectors (all loads of a lane in flight at once)
+// and reduces with shuffles only, so small sub-chunks cost no block
+// barrier. Writes stats[w] = (m, s). Rows are read from `z` [rows, V].
+constexpr int kSubLen = 2048;   // ids per sub-chunk (multiple of 8)
+
+template <typename T>
+__global__ void __launch_bounds__(kStatThreads)
+    row_stats_warp_kernel(const T* __restrict__ z_all, int rows, int V, int nsub, TScale c,
+                          float2* __restrict__ stats) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * (kStatThreads / 32) + (threadIdx.x >> 5);
+  if (w >= static_cast<int64_t>(rows) * nsub) return;
+  const int row = static_cast<int>(w / nsub);
+  const int sc = static_cast<int>(w - static_cast<int64_t>(row) * nsub);
+  const T* z = z_all + static_cast<size_t>(row) * V;
+  const int lo = sc * kSubLen;
+  const int hi = min(V, lo + kSubLen);
+  constexpr int kN = Vec<T>::n;
+  constexpr int kPerLane = kSubLen / kN / 32;   // vectors per lane in a whole sub-chunk
+  OnlineStat st;
+  int a0 = lo;
+  while (a0 < hi && (reinterpret_cast<uintptr_t>(z + a0) & 15u)) ++a0;
+  const int nvec = (hi - a0) / kN;
+  const int a1 = a0 + nvec * kN;
+  for (int v = lo + lane; v < a0; v += 32) {
+    float x = to_f32<T>(z[v]);
+    st.add(&x, 1, c);
+  }
+  if (nvec == kPerLane * 32) {
+    float v[kPerLane][kN];
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) Vec<T>::load(z + a0 + (lane + u * 32) * kN, v[u]);
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) st.add(v[u], kN, c);
+  } else {
+    for (int i = lane; i < nvec; i += 32) {
+      float v[kN];
+      Vec<T>::load(z + a0 + i * kN, v);
+      st.add(v, kN, c);
+    }
+  }
+  for (int v = a1 + lane; v < hi; v += 32) {
+    float x = to_f32<T>(z[v]);
+    st.add(&x, 1, c);
+  }
+  float m = st.m, s = st.s;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    merge_stat(m, s, m2, s2, c);
+  }
+  if (lane == 0) stats[w] = make_float2(m, s);
 }
 
 // Merge the chunk stats of one row.
@@ -1253,13 +1315,11 @@ uno_status distill_launch(const DistillArgs& a, cudaStream_t s) {
                         static_cast<const __nv_bfloat16*>(a.z_student), dp);
 }
 
-// Vocabulary chunks of the draft's stats pass: enough CTAs to cover the SMs
-// (as for verification), and chunks of at most kDraftChunk ids so that the
-// draw re-reads a small part of each row.
-constexpr int kDraftChunk = 8192;
-
+// Vocabulary chunks of the draft's stats pass: kSubLen ids each, one warp
+// per chunk, so the draw re-reads 1 / chunks of each row.
 int draft_chunks(int rows, int V) {
-  return std::min(kDraftMaxChunks, std::max(stat_chunks(rows, V), (V + kDraftChunk - 1) / kDraftChunk));
+  (void)rows;
+  return (V + kSubLen - 1) / kSubLen;
 }
 
 size_t draft_workspace(int32_t B, int32_t k, int32_t V) {
@@ -1270,7 +1330,8 @@ size_t draft_workspace(int32_t B, int32_t k, int32_t V) {
 uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
   const int rows = a.B * a.k;
   const int chunks = draft_chunks(rows, a.V);
-  const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
+  if (chunks > kDraftMaxChunks) return set_error(UNO_ERR_UNSUPPORTED, "vocabulary too large for the draft");
+  const int chunk_len = kSubLen;
   const TScale c = make_tscale(a.temperature);
   float2* stats = static_cast<float2*>(ws);
   DraftParams dp{};
@@ -1285,18 +1346,19 @@ uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
   dp.stats = stats;
   dp.draft = a.draft;
   dp.status = a.dev_status;
-  const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(rows) * chunks));
+  const int64_t warps = static_cast<int64_t>(rows) * chunks;
+  const dim3 grid(static_cast<unsigned>((warps + kStatThreads / 32 - 1) / (kStatThreads / 32)));
   cudaError_t e;
   if (a.dt == UNO_F32) {
     const float* q = static_cast<const float*>(a.q_logits);
-    e = launch_kernel(row_stats_kernel<float>, grid, dim3(kStatThreads), 0, s, 1, q, q, 0, a.V,
-                      chunks, chunk_len, c, stats);
+    e = launch_kernel(row_stats_warp_kernel<float>, grid, dim3(kStatThreads), 0, s, 1, q, rows,
+                      a.V, chunks, c, stats);
     if (e == cudaSuccess)
       e = launch_kernel(draft_draw_kernel<float>, dim3(rows), dim3(kDrawThreads), 0, s, 1, q, dp);
   } else {
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_logits);
-    e = launch_kernel(row_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1, q, q, 0,
-                      a.V, chunks, chunk_len, c, stats);
+    e = launch_kernel(row_stats_warp_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1, q,
+                      rows, a.V, chunks, c, stats);
     if (e == cudaSuccess)
       e = launch_kernel(draft_draw_kernel<__nv_bfloat16>, dim3(rows), dim3(kDrawThreads), 0, s, 1,
                         q, dp);
