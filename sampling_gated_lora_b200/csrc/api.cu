@@ -520,7 +520,15 @@ struct StepOp {
   const void* x;
   void* y;
   NormDownArgs nd;
+  PrefetchRange w[kMaxPrefetch];    // the weights this op streams, cut into its K-slices
+  PrefetchRange pf[kMaxPrefetch];   // the next weight-streaming op's, asked into L2 by this one
 };
+
+// Decode-size steps (every launch streams its weights once) hand each launch
+// the next weight-streaming launch's weights to prefetch into L2, up to this
+// many bytes (a share of the 126 MB L2; the leading part of every K-slice).
+constexpr int64_t kPrefetchMaxRows = 256;
+constexpr double kPrefetchBudget = 48.0 * (1 << 20);
 
 // Decode-size batches fold the LoRA down-projection of an input that an
 // RMSNorm produces into that RMSNorm's launch (one launch instead of two).
@@ -595,6 +603,37 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
 //   down(act; A_down) -> t; gemm(act, t; down) += h
 // then rmsnorm(h) -> n, the LM head's down-projection and GEMM (AR rows ->
 // logits, mask rows -> q_next). Rows >= B(k+1) carry the adapter (gate 1).
+// Decode-size plans: every op asks L2 for the leading part of each K-slice
+// of the next op that streams at least 4 MB of weights, up to kPrefetchBudget
+// bytes in all (see PrefetchRange).
+void plan_prefetch(uno_model::Plan* P, int64_t M) {
+  if (M > kPrefetchMaxRows) return;
+  auto bytes_of = [](const StepOp& o) {
+    double b = 0;
+    for (const PrefetchRange& r : o.w) b += static_cast<double>(r.rows) * static_cast<double>(r.row_bytes);
+    return b;
+  };
+  const size_t n = P->ops.size();
+  for (size_t i = 0; i < n; ++i) {
+    StepOp& op = P->ops[i];
+    size_t j = i + 1;
+    while (j < n && bytes_of(P->ops[j]) < 4.0 * (1 << 20)) ++j;
+    if (j == n) continue;
+    const double f = std::min(1.0, kPrefetchBudget / bytes_of(P->ops[j]));
+    for (int r = 0; r < kMaxPrefetch; ++r) {
+      PrefetchRange pr = P->ops[j].w[r];
+      if (pr.rows) {
+        const double want = static_cast<double>(pr.seg_bytes) * f;
+        pr.seg_bytes = f >= 1.0 ? pr.seg_bytes : static_cast<unsigned>(want / 128.0) * 128u;
+      }
+      op.pf[r] = pr;
+    }
+    if (op.kind == 0) gemm_set_prefetch(&op.gemm, op.pf);
+    if (op.kind == 2)
+      for (int r = 0; r < kMaxPrefetch; ++r) op.nd.pf[r] = op.pf[r];
+  }
+}
+
 uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
                       void* logits_out, uno_model::Plan* P) {
   const StepLayout L = step_layout(m, B, k);
@@ -618,12 +657,26 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     op.y = y;
     P->ops.push_back(op);
   };
-  auto gemm = [&](const GemmProblem& pb) -> uno_status {
+  // a GEMM launch; `wts` / `rows`: the weight matrices it streams (K columns each)
+  auto gemm = [&](const GemmProblem& pb, const void* const* wts, const int64_t* rows,
+                  int nw) -> uno_status {
     StepOp op{};
     op.kind = 0;
     const uno_status s = gemm_prepare(pb, &op.gemm);
-    if (s == UNO_OK) P->ops.push_back(op);
-    return s;
+    if (s != UNO_OK) return s;
+    const unsigned long long row_bytes = static_cast<unsigned long long>(pb.K) * 2;
+    const unsigned long long seg =
+        std::min<unsigned long long>(row_bytes, static_cast<unsigned long long>(op.gemm.kb_per_split) * 128ull);
+    for (int i = 0; i < nw && i < kMaxPrefetch; ++i) {
+      op.w[i].p = wts[i];
+      op.w[i].row_bytes = row_bytes;
+      op.w[i].seg_stride = seg;
+      op.w[i].rows = static_cast<unsigned>(rows[i]);
+      op.w[i].nseg = static_cast<unsigned>((row_bytes + seg - 1) / seg);
+      op.w[i].seg_bytes = static_cast<unsigned>(seg);
+    }
+    P->ops.push_back(op);
+    return UNO_OK;
   };
   // gated linear(s) on input x (width K): down-projections then the main GEMM.
   // t_ready: the preceding launch wrote t as well as x (no down-projection here).
@@ -674,10 +727,18 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       ++main_launches;
     }
     pm.x_ready = r > 0 && !gemm_dec_suits(pm) && !t_ready;
+    const int64_t a_rows[kMaxGroups] = {r, r, r};
     if (pm.x_ready &&
-        (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
+        (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t), As, a_rows,
+                  G)) != UNO_OK)
       return s;
-    return gemm(pm);
+    const void* Ws[kMaxGroups];
+    int64_t w_rows[kMaxGroups];
+    for (int i = 0; i < G; ++i) {
+      Ws[i] = pm.g[i].W;
+      w_rows[i] = pm.g[i].N;
+    }
+    return gemm(pm, Ws, w_rows, G);
   };
   uno_status s;
   for (int l = 0; l < m->n_layers; ++l) {
@@ -748,13 +809,19 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     }
     P->block_end.push_back(P->ops.size());
   }
-  if (!q_next) return UNO_OK;   // decoder layers only
+  if (!q_next) {   // decoder layers only
+    plan_prefetch(P, M);
+    return UNO_OK;
+  }
   norm(base + L.h, base + L.n);
   void* p_dst = logits_out ? logits_out : base + L.logits;
   const int which[1] = {0};
   void* y[1] = {p_dst};
   const int64_t ld[1] = {m->vocab};
-  return linear(base + L.n, m->hidden, 1, which, -1, y, ld, kEpiStore, q_next, Mv);
+  if ((s = linear(base + L.n, m->hidden, 1, which, -1, y, ld, kEpiStore, q_next, Mv)) != UNO_OK)
+    return s;
+  plan_prefetch(P, M);
+  return UNO_OK;
 }
 
 uno_model::Plan* find_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
@@ -872,7 +939,7 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
     return cuda_error(e, "clearing the stream-K flags");
   for (const StepOp& op : P->ops) {
     s = op.kind == 0 ? gemm_run(op.gemm, st)
-        : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st)
+        : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st, op.pf)
                        : norm_down_launch(op.nd, M, st);
     if (s != UNO_OK) return s;
   }
@@ -947,7 +1014,8 @@ uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h
   for (size_t i = 0; i < n_ops; ++i) {
     const StepOp& op = P->ops[i];
     s = op.kind == 0 ? gemm_run(op.gemm, st)
-        : op.kind == 1 ? rmsnorm_launch(static_cast<int64_t>(M), m->hidden, op.x, op.y, 1e-6f, st)
+        : op.kind == 1 ? rmsnorm_launch(static_cast<int64_t>(M), m->hidden, op.x, op.y, 1e-6f, st,
+                                        op.pf)
                        : norm_down_launch(op.nd, static_cast<int64_t>(M), st);
     if (s != UNO_OK) return s;
   }

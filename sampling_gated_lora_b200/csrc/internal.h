@@ -26,6 +26,22 @@ enum EpilogueMode : int {
 
 constexpr int kMaxGroups = 3;
 
+// Constant weights that the launch after this one reads: a launch asks L2 to
+// fetch them once its own loads are issued, so the HBM keeps streaming while
+// this launch drains and the next one starts. The region is `rows` rows of
+// `row_bytes`, each cut into `nseg` segments `seg_stride` bytes apart (the
+// K-slices the next launch's CTAs stream, in order); the first `seg_bytes` of
+// every segment are fetched, so every consuming CTA finds the same leading
+// share of its slice in L2. Pointers and byte counts: multiples of 16;
+// rows == 0: no region.
+struct PrefetchRange {
+  const void* p;
+  unsigned long long row_bytes;
+  unsigned long long seg_stride;
+  unsigned rows, nseg, seg_bytes, pad;
+};
+constexpr int kMaxPrefetch = 3;
+
 // One output group of a GEMM launch: its weights, adapter and output.
 struct GemmGroup {
   const void* W;          // [N, K]
@@ -78,7 +94,7 @@ struct TensorMaps {
   CUtensorMap x, t, w[kMaxGroups], b[kMaxGroups], a[kMaxGroups];
 };
 
-constexpr size_t kLaunchParamBytes = 320;
+constexpr size_t kLaunchParamBytes = 512;
 
 // Cached launch of a GemmProblem (tensor maps + grid); valid while the
 // pointers of the problem stay the same.
@@ -92,9 +108,12 @@ struct GemmLaunch {
   int dtype;
   int32_t* sk_flag;       // stream-K flags this launch reads: zero them before it runs (or NULL)
   size_t sk_flag_bytes;
+  int kb_per_split;       // K-blocks of one split (the K-slice a CTA streams)
 };
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out);
+// Sets the ranges a prepared launch prefetches for its successor (NULL: none).
+void gemm_set_prefetch(GemmLaunch* l, const PrefetchRange* pf);
 uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream);
 // Row-major [rows, inner] tensor map: box = 128 bytes of K x box_rows rows, 128-byte swizzle.
 uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t inner, uint64_t rows,
@@ -178,7 +197,7 @@ uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint3
 
 // ---------------------------------------------------------------- glue
 uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
-                          cudaStream_t s);
+                          cudaStream_t s, const PrefetchRange* pf = nullptr);
 uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s);
 
 // RMSNorm of x into y plus the gated LoRA down-projection of y for G adapters
@@ -194,6 +213,7 @@ struct NormDownArgs {   // bf16 tensors
   int ldt;
   float scale;
   int64_t gate_row0;
+  PrefetchRange pf[kMaxPrefetch];   // weights of the next launch (L2 hint)
 };
 uno_status norm_down_launch(const NormDownArgs& a, int64_t M, cudaStream_t s);
 

@@ -16,7 +16,7 @@
 //                        residual (or bonus) inverse-CDF draw split over the
 //                        cluster's CTAs (chunk totals exchanged through
 //                        distributed shared memory).
-//   draft_draw_kernel    after row_stats_warp_kernel has streamed the q rows once:
+//   draft_draw_kernel    after draft_stats_kernel has streamed the q rows once:
 //                        one CTA per (sequence, position) finds the vocab
 //                        chunk holding the draw from the chunk totals and
 //                        reads only that chunk again for the inverse-CDF draw.
@@ -40,13 +40,14 @@ namespace {
 constexpr int kStatThreads = 256;
 constexpr int kDrawThreads = 256;
 
-// The softmax weights are 2^((z - max) c) with c = log2(e) / T. c is held as
-// an unevaluated sum hi + lo of two floats and the exponent is formed with
-// one fused multiply-add: a single float c would carry a rounding error of up
-// to 6e-8 relative that scales every weight by 2^(-(max - z) err), a
-// distortion correlated with the logits. (z - max is exact for bf16 logits.)
-// hi is taken strictly below c, so lo > 0 and an infinite d gives an infinite
-// exponent of its own sign (never inf - inf).
+// The softmax weights are 2^((z - max) c) with c = log2(e) / T.
+// Verification takes c as one float: its rounding (up to 6e-8 relative)
+// scales a weight by 2^(-(max - z) err), far below what the accept test
+// resolves. The draft sampler, whose draws on near-flat 151936-way rows must
+// land in token intervals ~1e-5 of the total wide, holds c as an unevaluated
+// sum hi + lo of two floats and forms the exponent with one fused multiply-add
+// (z - max is exact for bf16 logits). hi is taken strictly below c, so lo > 0
+// and an infinite d gives an infinite exponent of its own sign.
 struct TScale {
   float hi, lo;
 };
@@ -58,6 +59,9 @@ TScale make_tscale(float temperature) {
   if (static_cast<double>(t.hi) >= cd) t.hi = std::nextafter(t.hi, 0.f);
   t.lo = static_cast<float>(cd - static_cast<double>(t.hi));
   return t;
+}
+float make_scale(float temperature) {
+  return static_cast<float>(1.4426950408889634073599 / static_cast<double>(temperature));
 }
 
 template <typename T>
@@ -84,7 +88,7 @@ struct Vec<float> {
 struct OnlineStat {
   float m = -INFINITY;
   float s = 0.f;
-  __device__ __forceinline__ void add(const float* v, int n, TScale c) {
+  __device__ __forceinline__ void add(const float* v, int n, float c) {
     float mx = v[0];
     for (int e = 1; e < n; ++e) mx = fmaxf(mx, v[e]);
     if (mx > m) {
@@ -96,7 +100,7 @@ struct OnlineStat {
 };
 
 // Merge (m1, s1) with (m2, s2); s is relative to m, exp base 2 with scale c.
-__device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s2, TScale c) {
+__device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s2, float c) {
   if (isnan(s2) || isnan(s)) {   // keep a NaN seen anywhere
     s = NAN;
     m = fmaxf(m, m2);
@@ -120,7 +124,7 @@ __device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s
 template <typename T>
 __global__ void __launch_bounds__(kStatThreads)
     row_stats_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits, int rows_p,
-                     int V, int chunks, int chunk_len, TScale c, float2* __restrict__ stats) {
+                     int V, int chunks, int chunk_len, float c, float2* __restrict__ stats) {
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
   const int row = static_cast<int>(blockIdx.x / static_cast<unsigned>(chunks));
@@ -181,17 +185,25 @@ __global__ void __launch_bounds__(kStatThreads)
   }
 }
 
-// Warp-granular form for the draft: warp w of the grid (8 per CTA) takes
-// (row w / nsub, sub-chunk w % nsub) of sub_len ids, keeps one online stat
-// per lane over its 16-byte vectors (all loads of a lane in flight at once)
-// and reduces with shuffles only, so small sub-chunks cost no block
-// barrier. Writes stats[w] = (m, s). Rows are read from `z` [rows, V].
-constexpr int kSubLen = 2048;   // ids per sub-chunk (multiple of 8)
+// Statistics of one vocab chunk for the draft (see draft_stats_kernel).
+struct DraftStat {
+  float m;    // chunk max (NaN: a NaN logit in the chunk)
+  float pad;
+  double s;   // sum of 2^((z - m) c) over the chunk
+};
+
+// The draft's stats pass: warp w of the grid (8 per CTA) takes (row w / nsub,
+// chunk w % nsub) of kSubLen ids and holds the whole chunk in registers (all
+// 16-byte loads of a lane in flight at once). Two passes over the registers,
+// no online rescaling: the chunk max by shuffles, then the weights
+// 2^((z - m) c) summed per vector in float and across vectors and lanes in
+// double. Shuffles only, no block barrier.
+constexpr int kSubLen = 2048;   // ids per chunk (multiple of 8)
 
 template <typename T>
 __global__ void __launch_bounds__(kStatThreads)
-    row_stats_warp_kernel(const T* __restrict__ z_all, int rows, int V, int nsub, TScale c,
-                          float2* __restrict__ stats) {
+    draft_stats_kernel(const T* __restrict__ z_all, int rows, int V, int nsub, TScale c,
+                       DraftStat* __restrict__ stats) {
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -203,45 +215,54 @@ __global__ void __launch_bounds__(kStatThreads)
   const int lo = sc * kSubLen;
   const int hi = min(V, lo + kSubLen);
   constexpr int kN = Vec<T>::n;
-  constexpr int kPerLane = kSubLen / kN / 32;   // vectors per lane in a whole sub-chunk
-  OnlineStat st;
-  int a0 = lo;
-  while (a0 < hi && (reinterpret_cast<uintptr_t>(z + a0) & 15u)) ++a0;
-  const int nvec = (hi - a0) / kN;
-  const int a1 = a0 + nvec * kN;
-  for (int v = lo + lane; v < a0; v += 32) {
-    float x = to_f32<T>(z[v]);
-    st.add(&x, 1, c);
+  constexpr int kPerLane = kSubLen / kN / 32;   // vectors per lane
+  float v[kPerLane][kN];
+  const bool whole = hi - lo == kSubLen && (reinterpret_cast<uintptr_t>(z + lo) & 15u) == 0;
+  if (whole) {
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) Vec<T>::load(z + lo + (lane + u * 32) * kN, v[u]);
+  } else {   // a ragged last chunk or unaligned rows: element loads, -inf past the end
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u)
+#pragma unroll
+      for (int q = 0; q < kN; ++q) {
+        const int e = lo + (lane + u * 32) * kN + q;
+        v[u][q] = e < hi ? to_f32<T>(z[e]) : -INFINITY;
+      }
   }
-  if (nvec == kPerLane * 32) {
-    float v[kPerLane][kN];
+  float m = -INFINITY;
+  bool nan = false;
 #pragma unroll
-    for (int u = 0; u < kPerLane; ++u) Vec<T>::load(z + a0 + (lane + u * 32) * kN, v[u]);
+  for (int u = 0; u < kPerLane; ++u)
 #pragma unroll
-    for (int u = 0; u < kPerLane; ++u) st.add(v[u], kN, c);
-  } else {
-    for (int i = lane; i < nvec; i += 32) {
-      float v[kN];
-      Vec<T>::load(z + a0 + i * kN, v);
-      st.add(v, kN, c);
+    for (int q = 0; q < kN; ++q) {
+      nan |= isnan(v[u][q]);
+      m = fmaxf(m, v[u][q]);
+    }
+  m = warp_max(m);
+  nan = __any_sync(0xffffffffu, nan);
+  double acc = 0.0;
+  if (m != -INFINITY) {
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) {
+      float part = 0.f;
+#pragma unroll
+      for (int q = 0; q < kN; ++q) part += fast_exp2((v[u][q] - m) * c);
+      acc += static_cast<double>(part);
     }
   }
-  for (int v = a1 + lane; v < hi; v += 32) {
-    float x = to_f32<T>(z[v]);
-    st.add(&x, 1, c);
+  acc = warp_sum(acc);
+  if (lane == 0) {
+    DraftStat st;
+    st.m = nan ? NAN : m;
+    st.pad = 0.f;
+    st.s = acc;
+    stats[w] = st;
   }
-  float m = st.m, s = st.s;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-    merge_stat(m, s, m2, s2, c);
-  }
-  if (lane == 0) stats[w] = make_float2(m, s);
 }
 
 // Merge the chunk stats of one row.
-__device__ __forceinline__ float2 row_stat(const float2* stats, int row, int chunks, TScale c) {
+__device__ __forceinline__ float2 row_stat(const float2* stats, int row, int chunks, float c) {
   float m = -INFINITY, s = 0.f;
   bool nan = false;
   for (int i = 0; i < chunks; ++i) {
@@ -420,7 +441,7 @@ __device__ __forceinline__ void load_chunk(T* dst, const T* src, int len) {
 
 struct FinalizeParams {
   int B, k, k_p, V, chunks;
-  TScale c;   // log2(e) / T
+  float c;   // log2(e) / T
   uint64_t seed, step, seq_offset;
   const int32_t* draft;
   const float2* stats;
@@ -531,7 +552,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   cta_sync();
   const float Mp = s_stat[0], inv_sp = 1.f / s_stat[1];
   const float Mq = s_stat[2], inv_sq = residual ? 1.f / s_stat[3] : 0.f;
-  const TScale c = a.c;
+  const float c = a.c;
   const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + (residual ? n : k));
   const double u = static_cast<double>(uniform24(
       philox_word0(a.seed, a.step, residual ? kStreamResidual : kStreamBonus, idx)));
@@ -575,7 +596,7 @@ constexpr int kTreeMaxK = 32;   // block length
 
 struct TreeParams {
   int B, N, k, R, V, chunks, bonus;
-  TScale c;   // log2(e) / T
+  float c;   // log2(e) / T
   uint64_t seed, step, seq_offset;
   const int32_t* cands;   // [B, N, k]
   const float2* stats;    // chunk stats of node rows b*R + n, then q rows B*R + b*k + j
@@ -644,7 +665,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
   const int32_t* cand = a.cands + static_cast<size_t>(b) * nk;
   int32_t* tok = a.out_tokens + static_cast<size_t>(b) * (k + 1);
-  const TScale c = a.c;
+  const float c = a.c;
 
   // 1. Trie numbering. rep(i, j) = the first candidate with the same j+1
   //    tokens; the first visits, in walk order (i, then j), get ids 1, 2, ...
@@ -849,7 +870,7 @@ __global__ void __launch_bounds__(kDrawThreads)
 
 struct DistillParams {
   int V, chunk_elems;
-  TScale c;           // log2(e) / T
+  float c;            // log2(e) / T
   float inv_t;        // 1 / T
   float alpha, beta;
   float grad_scale;   // 1 / (T rows)
@@ -964,7 +985,7 @@ __global__ void __launch_bounds__(kDrawThreads)
   }
 
   // 2. the partition sums, then KL, TV and sum(sign(q - p) q)
-  const TScale c = a.c;
+  const float c = a.c;
   double sums[3] = {0.0, 0.0, 0.0};
   for (int i = threadIdx.x; i < len; i += blockDim.x) {
     sums[0] += static_cast<double>(fast_exp2((to_f32<T>(zt[i]) - Mt) * c));
@@ -1010,7 +1031,7 @@ struct DraftParams {
   int k, V, chunks, chunk_len;
   TScale c;
   uint64_t seed, step, seq_offset;
-  const float2* stats;   // [rows, chunks]: (chunk max, sum exp2((z - max) c)) of the q rows
+  const DraftStat* stats;   // [rows, chunks] of the q rows
   int32_t* draft;
   int32_t* status;
 };
@@ -1038,14 +1059,14 @@ __global__ void __launch_bounds__(kDrawThreads)
   const int row = blockIdx.x;
   const int chunks = a.chunks;
   const TScale c = a.c;
-  const float2* st = a.stats + static_cast<size_t>(row) * chunks;
+  const DraftStat* st = a.stats + static_cast<size_t>(row) * chunks;
   if (threadIdx.x < 32) {
     float m = -INFINITY;
     bool nan = false;
     for (int i = threadIdx.x; i < chunks; i += 32) {
-      const float2 v = st[i];
-      nan |= isnan(v.y);
-      m = fmaxf(m, v.x);
+      const DraftStat v = st[i];
+      nan |= isnan(v.m);
+      m = fmaxf(m, v.m);
     }
     m = warp_max(m);
     nan = __any_sync(0xffffffffu, nan);
@@ -1063,9 +1084,12 @@ __global__ void __launch_bounds__(kDrawThreads)
     return;
   }
   const float M = s_M;
+  // chunk totals relative to the row max: the rescale in double (exp2 of the
+  // exact bf16 difference times c), so it adds no error of float size
+  const double cd = static_cast<double>(c.hi) + static_cast<double>(c.lo);
   for (int i = threadIdx.x; i < chunks; i += blockDim.x) {
-    const float2 v = st[i];
-    s_tot[i] = static_cast<double>(v.y) * static_cast<double>(fast_exp2((v.x - M) * c));
+    const DraftStat v = st[i];
+    s_tot[i] = v.m == -INFINITY ? 0.0 : v.s * exp2(static_cast<double>(v.m - M) * cd);
   }
   cta_sync();
   const int b = row / a.k, j = row - b * a.k;
@@ -1188,7 +1212,7 @@ uno_status verify_launch(const VerifyArgs& a, void* ws, cudaStream_t s) {
   const int rows = a.B * a.k_p + a.B * a.k;
   const int chunks = stat_chunks(rows, a.V);
   const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
-  const TScale c = make_tscale(a.temperature);
+  const float c = make_scale(a.temperature);
   float2* stats = static_cast<float2*>(ws);
   const int esz = a.dt == UNO_F32 ? 4 : 2;
   int chunk_elems = 0;
@@ -1243,7 +1267,7 @@ uno_status tree_verify_launch(const TreeVerifyArgs& a, void* ws, cudaStream_t s)
   const int rows = a.B * a.R + a.B * a.k;
   const int chunks = stat_chunks(rows, a.V);
   const int chunk_len = ((a.V + chunks - 1) / chunks + 7) & ~7;
-  const TScale c = make_tscale(a.temperature);
+  const float c = make_scale(a.temperature);
   float2* stats = static_cast<float2*>(ws);
   const int esz = a.dt == UNO_F32 ? 4 : 2;
   int chunk_elems = 0;
@@ -1297,7 +1321,7 @@ uno_status distill_launch(const DistillArgs& a, cudaStream_t s) {
   DistillParams dp{};
   dp.V = a.V;
   dp.chunk_elems = chunk_elems;
-  dp.c = make_tscale(a.temperature);
+  dp.c = make_scale(a.temperature);
   dp.inv_t = 1.f / a.temperature;
   dp.alpha = a.alpha;
   dp.beta = a.beta;
@@ -1324,7 +1348,7 @@ int draft_chunks(int rows, int V) {
 
 size_t draft_workspace(int32_t B, int32_t k, int32_t V) {
   const int rows = B * k;
-  return static_cast<size_t>(rows) * draft_chunks(rows, V) * sizeof(float2);
+  return static_cast<size_t>(rows) * draft_chunks(rows, V) * sizeof(DraftStat);
 }
 
 uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
@@ -1333,7 +1357,7 @@ uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
   if (chunks > kDraftMaxChunks) return set_error(UNO_ERR_UNSUPPORTED, "vocabulary too large for the draft");
   const int chunk_len = kSubLen;
   const TScale c = make_tscale(a.temperature);
-  float2* stats = static_cast<float2*>(ws);
+  DraftStat* stats = static_cast<DraftStat*>(ws);
   DraftParams dp{};
   dp.k = a.k;
   dp.V = a.V;
@@ -1351,13 +1375,13 @@ uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
   cudaError_t e;
   if (a.dt == UNO_F32) {
     const float* q = static_cast<const float*>(a.q_logits);
-    e = launch_kernel(row_stats_warp_kernel<float>, grid, dim3(kStatThreads), 0, s, 1, q, rows,
-                      a.V, chunks, c, stats);
+    e = launch_kernel(draft_stats_kernel<float>, grid, dim3(kStatThreads), 0, s, 1, q, rows, a.V,
+                      chunks, c, stats);
     if (e == cudaSuccess)
       e = launch_kernel(draft_draw_kernel<float>, dim3(rows), dim3(kDrawThreads), 0, s, 1, q, dp);
   } else {
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_logits);
-    e = launch_kernel(row_stats_warp_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1, q,
+    e = launch_kernel(draft_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1, q,
                       rows, a.V, chunks, c, stats);
     if (e == cudaSuccess)
       e = launch_kernel(draft_draw_kernel<__nv_bfloat16>, dim3(rows), dim3(kDrawThreads), 0, s, 1,
