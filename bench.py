@@ -322,6 +322,29 @@ def kernel_lines(U, torch, pk):
             "tensor_frac": round(flops / us / 1e6 / pk["bf16_tflops"], 3)}
         del sets
     del x, y
+    # adapter gradients (the training layout, MLP up shape): M = 2048 rows, 1024 of them
+    # gated, 4096 -> 12288, r = 128. Algorithmic work counts the gated rows only (the
+    # others contribute nothing): flops 2 Mg r (2K + 2N); bytes: the gated rows of x and
+    # dy, A and Bl, and dA and dBl written.
+    M, K, N, r = 2048, 4096, 12288, 128
+    Mg = M // 2
+    x, dy = dev((M, K), 1), dev((M, N), 1)
+    A, Bl = dev((r, K), K ** -0.5), dev((N, r), 0.01)
+    g = torch.cat([torch.zeros(M - Mg, dtype=torch.uint8), torch.ones(Mg, dtype=torch.uint8)]).cuda()
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device="cuda")
+    dBl = torch.empty((N, r), dtype=torch.bfloat16, device="cuda")
+    bws = torch.empty(U.load().uno_gated_lora_backward_workspace(M, K, N, r), dtype=torch.uint8,
+                      device="cuda")
+    f = lambda: U.gated_lora_adapter_grads(x, dy, A, Bl, g, 1.0, dA=dA, dBl=dBl, workspace=bws)
+    f()
+    us = timed(f, reps=10)
+    flops = 2 * Mg * r * (2 * K + 2 * N)
+    byts = 2 * (Mg * K + Mg * N + 2 * (r * K + N * r))
+    t_roof = max(byts / (pk["hbm_gbs"] * 1e9), flops / (pk["bf16_tflops"] * 1e12)) * 1e6
+    out["adapter_grads_mlp_up_M2048"] = {
+        "us": round(us, 1), "TFLOPs": round(flops / us / 1e6, 1), "GBps": round(byts / us / 1e3, 1),
+        "roofline_us": round(t_roof, 2), "frac_of_roofline": round(t_roof / us, 3)}
+    del x, dy, A, Bl, bws
     # psi_verify at B=256, k=16, V=151936 (sigma 1.0 and 0.25, T = 1)
     B, k, V = 256, 16, 151936
     for sigma in (1.0, 0.25):

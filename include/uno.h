@@ -100,6 +100,30 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
                                  size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Gradients of the gated-LoRA adapter, the AR weights frozen (hyper.ai page,
+ * section "方法", the training-order paragraph: the AR weights stay fixed
+ * while the diffusion adapter trains). For the linear above and an output
+ * gradient dy [M,N], with t_u = x A^T:
+ *
+ *     dBl = (scale * g (.) dy)^T t_u      [N, r]
+ *     dA  = (dy Bl)^T (scale * g (.) x)   [r, K]
+ *
+ *   x [M,K], dy [M,N], A [r,K], Bl [N,r], gate [M] uint8: bf16 (the only
+ *   dtype); dA [r,K] and dBl [N,r] bf16 outputs. fp32 accumulation; t_u and
+ *   dy Bl are rounded to bf16 (tensor-core operands). Gate-0 rows contribute
+ *   nothing. Sizes: K, N multiples of 8, 8 <= r <= 256 (multiple of 8),
+ *   M >= 0 (M = 0 writes zero gradients). workspace: >=
+ *   uno_gated_lora_backward_workspace(M, K, N, r) bytes, 16-byte aligned, any
+ *   contents (x and dy transposed, and the rank-r products).
+ * ------------------------------------------------------------------------- */
+size_t uno_gated_lora_backward_workspace(int64_t M, int64_t K, int64_t N, int32_t r);
+
+uno_status uno_gated_lora_backward(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r,
+                                   const void* x, const void* dy, const void* A, const void* Bl,
+                                   const uint8_t* gate, float scale, void* dA, void* dBl,
+                                   void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Grouped gated-LoRA linears sharing one input x [M,K] (one launch for the
  * down-projections, one for the products; hyper.ai page, section "方法": the
  * adapter is attached to every AR matrix, so the q, k, v projections of a

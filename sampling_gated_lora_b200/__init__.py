@@ -29,6 +29,7 @@ EXPORTS = [
     "uno_last_error", "uno_version", "uno_device_status",
     "uno_gated_lora_linear_workspace", "uno_gated_lora_linear",
     "uno_gated_lora_linear_group_workspace", "uno_gated_lora_linear_group",
+    "uno_gated_lora_backward_workspace", "uno_gated_lora_backward",
     "uno_psi_verify_workspace", "uno_psi_verify", "uno_psi_verify_noalloc",
     "uno_draft_sample_workspace", "uno_draft_sample", "uno_distill",
     "uno_tree_verify_workspace", "uno_tree_verify",
@@ -70,6 +71,9 @@ def load():
         "uno_gated_lora_linear_group_workspace": (sz, [i32, i64, i32, i32]),
         "uno_gated_lora_linear_group": (i32, [i32, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, f32,
                                               i32, vp, vp, sz, vp]),
+        "uno_gated_lora_backward_workspace": (sz, [i64, i64, i64, i32]),
+        "uno_gated_lora_backward": (i32, [i32, i64, i64, i64, i32, vp, vp, vp, vp, vp, f32, vp,
+                                          vp, vp, sz, vp]),
         "uno_psi_verify_workspace": (sz, [i32, i32, i32, i32]),
         "uno_psi_verify": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, f32, u64, u64, u64, vp, vp,
                                  vp, vp, vp, sz, vp]),
@@ -263,6 +267,32 @@ def gated_lora_linear_group(x, Ws, As, Bls, gate, scale=1.0, silu_pair=False, ys
             arr(As), arr(Bls), _ptr(gate), float(scale), 1 if silu_pair else 0, yarr, _ptr(ws),
             wsb)
     return ys
+
+
+def gated_lora_adapter_grads(x, dy, A, Bl, gate, scale=1.0, dA=None, dBl=None, workspace=None,
+                             stream=None):
+    """(dA [r,K], dBl [N,r]) of sum(dy * y) for y = gated_lora_linear(x, W, A, Bl, gate, scale),
+    the AR weight W frozen (bf16 tensors, uint8 gate)."""
+    torch = _torch()
+    bf16 = (torch.bfloat16,)
+    _expect(x, (None, None), bf16, "x")
+    M, K = x.shape
+    _expect(A, (None, K), bf16, "A")
+    r = A.shape[0]
+    _expect(Bl, (None, r), bf16, "Bl")
+    N = Bl.shape[0]
+    _expect(dy, (M, N), bf16, "dy")
+    _expect(gate, (M,), (torch.uint8,), "gate")
+    _expect(dA, (r, K), bf16, "dA", optional=True)
+    _expect(dBl, (N, r), bf16, "dBl", optional=True)
+    L = load()
+    dA = torch.empty((r, K), dtype=torch.bfloat16, device=x.device) if dA is None else dA
+    dBl = torch.empty((N, r), dtype=torch.bfloat16, device=x.device) if dBl is None else dBl
+    dev = _dev(x, dy, A, Bl, gate, dA, dBl, workspace)
+    ws, wsb = _workspace(L.uno_gated_lora_backward_workspace(M, K, N, r), dev, workspace)
+    _launch(dev, stream, L.uno_gated_lora_backward, UNO_BF16, M, K, N, r, _ptr(x), _ptr(dy),
+            _ptr(A), _ptr(Bl), _ptr(gate), float(scale), _ptr(dA), _ptr(dBl), _ptr(ws), wsb)
+    return dA, dBl
 
 
 def _verify_shapes(p_logits, q_logits, draft, accepted_len, out_tokens, out_count, dev_status):

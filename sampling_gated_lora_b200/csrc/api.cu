@@ -297,6 +297,37 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   return run_linear(r > 0 && !fused ? &down : nullptr, main, as_stream(stream));
 }
 
+size_t uno_gated_lora_backward_workspace(int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (M < 0 || K < 1 || N < 1 || r < 1) return 0;
+  return align_up(adapter_backward_workspace(M, K, N, r));
+}
+
+uno_status uno_gated_lora_backward(uno_dtype dt, int64_t M, int64_t K, int64_t N, int32_t r,
+                                   const void* x, const void* dy, const void* A, const void* Bl,
+                                   const uint8_t* gate, float scale, void* dA, void* dBl,
+                                   void* workspace, size_t ws_bytes, void* stream) {
+  if (dt != UNO_BF16) return set_error(UNO_ERR_UNSUPPORTED, "the adapter backward takes bf16 only");
+  uno_status s = check_linear(dt, M, K, N, r);
+  if (s != UNO_OK) return s;
+  if (r < 8) return set_error(UNO_ERR_INVALID_ARG, "rank r=%d: the backward needs an adapter", r);
+  if (M > (1ll << 24)) return set_error(UNO_ERR_UNSUPPORTED, "M above 2^24 rows");
+  if (!dA || !dBl || !A || !Bl) return set_error(UNO_ERR_INVALID_ARG, "NULL adapter or gradient pointer");
+  if (!aligned16(dA) || !aligned16(dBl) || !aligned16(A) || !aligned16(Bl))
+    return set_error(UNO_ERR_INVALID_ARG, "A, Bl, dA and dBl must be 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  if (M == 0) {   // no rows: both gradients are zero
+    cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dBl, 0, static_cast<size_t>(N) * r * 2, st);
+    return e == cudaSuccess ? UNO_OK : cuda_error(e, "clearing the gradients");
+  }
+  if (!x || !dy || !gate) return set_error(UNO_ERR_INVALID_ARG, "x, dy and gate must be non-NULL");
+  if (!aligned16(x) || !aligned16(dy)) return set_error(UNO_ERR_INVALID_ARG, "x and dy must be 16-byte aligned");
+  const size_t need = uno_gated_lora_backward_workspace(M, K, N, r);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return set_error(UNO_ERR_WORKSPACE, "workspace must hold %zu bytes (got %zu)", need, ws_bytes);
+  return adapter_backward_launch(M, K, N, r, x, dy, A, Bl, gate, scale, dA, dBl, workspace, st);
+}
+
 // ---------------------------------------------------------------- sampler
 
 size_t uno_psi_verify_workspace(int32_t B, int32_t k, int32_t k_p, int32_t V) {

@@ -217,6 +217,13 @@ struct NormDownArgs {   // bf16 tensors
 };
 uno_status norm_down_launch(const NormDownArgs& a, int64_t M, cudaStream_t s);
 
+// Gradients of the gated-LoRA adapter (backward.cu): dA [r,K], dBl [N,r] bf16.
+size_t adapter_backward_workspace(int64_t M, int64_t K, int64_t N, int32_t r);
+uno_status adapter_backward_launch(int64_t M, int64_t K, int64_t N, int32_t r, const void* x,
+                                   const void* dy, const void* A, const void* Bl,
+                                   const uint8_t* gate, float scale, void* dA, void* dBl,
+                                   void* ws, cudaStream_t s);
+
 // The bounded-wait self-test (waits.cu).
 uno_status wait_selftest_launch(int32_t which, uint64_t limit_ns, int32_t* result,
                                 int32_t* status, cudaStream_t s);

@@ -118,6 +118,22 @@ def test_draft_and_misc_reject_bad_arguments():
     assert L.uno_wait_selftest(0, 1000000, null, null, null) == 1
 
 
+def test_adapter_backward_rejects_bad_arguments():
+    L = U.load()
+    ok = ctypes.c_void_p(0x10000)
+    null = None
+    call = lambda dt=U.UNO_BF16, M=64, K=64, N=128, r=8, x=ok, dA=ok, ws=1 << 30: L.uno_gated_lora_backward(
+        dt, M, K, N, r, x, ok, ok, ok, ok, 1.0, dA, ok, ok, ws, null)
+    assert call(dt=U.UNO_F32) == 2                # bf16 only
+    assert call(K=60) == 2 and call(r=0) == 1     # 16-byte rows; an adapter is needed
+    assert call(x=null) == 1 and call(dA=null) == 1
+    assert call(dA=ctypes.c_void_p(0x10008)) == 1
+    assert call(ws=16) == 6
+    need = L.uno_gated_lora_backward_workspace(2048, 4096, 12288, 128)
+    # x^T and dy^T at 2048 padded rows, Bl^T and the two rank-r products
+    assert need >= 2 * 2048 * (4096 + 12288) + 2 * 128 * 12288 + 2 * 2 * 128 * 2048
+
+
 def test_model_create_validates():
     L = U.load()
     h = ctypes.c_void_p()
