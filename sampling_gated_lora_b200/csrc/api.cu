@@ -556,10 +556,10 @@ struct StepOp {
 };
 
 // Decode-size steps (every launch streams its weights once) hand each launch
-// the next weight-streaming launch's weights to prefetch into L2, up to this
-// many bytes (a share of the 126 MB L2; the leading part of every K-slice).
+// the next weight-streaming launch's weights to prefetch into L2 when they
+// fit in this many bytes (half of the 126 MB L2).
 constexpr int64_t kPrefetchMaxRows = 256;
-constexpr double kPrefetchBudget = 48.0 * (1 << 20);
+constexpr double kPrefetchBudget = 64.0 * (1 << 20);
 
 // Decode-size batches fold the LoRA down-projection of an input that an
 // RMSNorm produces into that RMSNorm's launch (one launch instead of two).
@@ -650,15 +650,10 @@ void plan_prefetch(uno_model::Plan* P, int64_t M) {
     size_t j = i + 1;
     while (j < n && bytes_of(P->ops[j]) < 4.0 * (1 << 20)) ++j;
     if (j == n) continue;
-    const double f = std::min(1.0, kPrefetchBudget / bytes_of(P->ops[j]));
-    for (int r = 0; r < kMaxPrefetch; ++r) {
-      PrefetchRange pr = P->ops[j].w[r];
-      if (pr.rows) {
-        const double want = static_cast<double>(pr.seg_bytes) * f;
-        pr.seg_bytes = f >= 1.0 ? pr.seg_bytes : static_cast<unsigned>(want / 128.0) * 128u;
-      }
-      op.pf[r] = pr;
-    }
+    // whole weight matrices only: a partial prefetch needs one small request
+    // per row segment, and that many requests hold up the issuing thread
+    if (bytes_of(P->ops[j]) > kPrefetchBudget) continue;
+    for (int r = 0; r < kMaxPrefetch; ++r) op.pf[r] = P->ops[j].w[r];
     if (op.kind == 0) gemm_set_prefetch(&op.gemm, op.pf);
     if (op.kind == 2)
       for (int r = 0; r < kMaxPrefetch; ++r) op.nd.pf[r] = op.pf[r];

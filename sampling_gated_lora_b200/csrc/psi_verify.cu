@@ -88,7 +88,8 @@ struct Vec<float> {
 struct OnlineStat {
   float m = -INFINITY;
   float s = 0.f;
-  __device__ __forceinline__ void add(const float* v, int n, float c) {
+  template <typename C>
+  __device__ __forceinline__ void add(const float* v, int n, C c) {
     float mx = v[0];
     for (int e = 1; e < n; ++e) mx = fmaxf(mx, v[e]);
     if (mx > m) {
@@ -100,7 +101,8 @@ struct OnlineStat {
 };
 
 // Merge (m1, s1) with (m2, s2); s is relative to m, exp base 2 with scale c.
-__device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s2, float c) {
+template <typename C>
+__device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s2, C c) {
   if (isnan(s2) || isnan(s)) {   // keep a NaN seen anywhere
     s = NAN;
     m = fmaxf(m, m2);
@@ -117,22 +119,12 @@ __device__ __forceinline__ void merge_stat(float& m, float& s, float m2, float s
   m = mx;
 }
 
-// Grid: rows * chunks blocks, one per (row, vocab chunk), chunk fastest (a
-// one-dimensional grid, so the row count is not held to gridDim.y's 65535).
-// Row r < rows_p reads p_logits row r, else q_logits row r - rows_p. Writes
-// stats[r * chunks + chunk] = (m, s).
-template <typename T>
-__global__ void __launch_bounds__(kStatThreads)
-    row_stats_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits, int rows_p,
-                     int V, int chunks, int chunk_len, float c, float2* __restrict__ stats) {
-  if (threadIdx.x == 0) pdl_trigger();
-  pdl_wait();
-  const int row = static_cast<int>(blockIdx.x / static_cast<unsigned>(chunks));
-  const int chunk = static_cast<int>(blockIdx.x - static_cast<unsigned>(row) * chunks);
-  const T* z = row < rows_p ? p_logits + static_cast<size_t>(row) * V
-                            : q_logits + static_cast<size_t>(row - rows_p) * V;
-  const int lo = chunk * chunk_len;
-  const int hi = min(V, lo + chunk_len);
+// (max, sum of 2^((z - max) c)) of ids [lo, hi) of row z over the CTA
+// (kStatThreads threads, every one calls): 16-byte loads, four in flight per
+// thread, each thread an online stat, then shuffle and shared-memory merges.
+// The result is valid in thread 0. A NaN anywhere makes s NaN.
+template <typename T, typename C>
+__device__ __forceinline__ float2 block_row_stat(const T* z, int lo, int hi, C c) {
   constexpr int kN = Vec<T>::n;
   OnlineStat st;
   // aligned body [a0, a1) in whole 16-byte vectors; scalar head and tail
@@ -162,7 +154,6 @@ __global__ void __launch_bounds__(kStatThreads)
     float x = to_f32<T>(z[v]);
     st.add(&x, 1, c);
   }
-  // block reduction
   float m = st.m, s = st.s;
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -177,12 +168,29 @@ __global__ void __launch_bounds__(kStatThreads)
     ss[warp] = s;
   }
   cta_sync();
-  if (threadIdx.x == 0) {
-    float M = sm[0], S = ss[0];
+  float M = sm[0], S = ss[0];
+  if (threadIdx.x == 0)
     for (int w = 1; w < kStatThreads / 32; ++w) merge_stat(M, S, sm[w], ss[w], c);
-    // a NaN anywhere in the chunk makes S NaN (fmaxf skips it in the max)
-    stats[blockIdx.x] = make_float2(M, S);
-  }
+  return make_float2(M, S);
+}
+
+// Grid: rows * chunks blocks, one per (row, vocab chunk), chunk fastest (a
+// one-dimensional grid, so the row count is not held to gridDim.y's 65535).
+// Row r < rows_p reads p_logits row r, else q_logits row r - rows_p. Writes
+// stats[r * chunks + chunk] = (m, s).
+template <typename T>
+__global__ void __launch_bounds__(kStatThreads)
+    row_stats_kernel(const T* __restrict__ p_logits, const T* __restrict__ q_logits, int rows_p,
+                     int V, int chunks, int chunk_len, float c, float2* __restrict__ stats) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int row = static_cast<int>(blockIdx.x / static_cast<unsigned>(chunks));
+  const int chunk = static_cast<int>(blockIdx.x - static_cast<unsigned>(row) * chunks);
+  const T* z = row < rows_p ? p_logits + static_cast<size_t>(row) * V
+                            : q_logits + static_cast<size_t>(row - rows_p) * V;
+  const int lo = chunk * chunk_len;
+  const float2 st = block_row_stat<T>(z, lo, min(V, lo + chunk_len), c);
+  if (threadIdx.x == 0) stats[blockIdx.x] = st;
 }
 
 // Statistics of one vocab chunk for the draft (see draft_stats_kernel).
