@@ -269,6 +269,65 @@ uno_status uno_distill(uno_dtype dt, int32_t rows, int32_t V, const void* z_teac
                        float* losses, float* grad, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Verification and draft with the vocabulary split over G devices (the LM
+ * head's rows sharded; hyper.ai page, section "方法", the Psi-Spec
+ * paragraph: the test against the AR distribution needs its normaliser over
+ * the whole vocabulary, the residual and bonus draws cumulative mass in
+ * vocabulary order). Device `rank` holds the logits of its contiguous shard
+ * [v0, v0 + Vs) of the V ids, shards in rank order. Per step, on every device:
+ *   1. uno_vp_partials on its AR rows (id_kind 1) and draft rows (id_kind 2):
+ *      out [rows, 4] float = (m, s, z(d), 0) with m the row max over the
+ *      shard, s = sum 2^((z - m) log2(e) / T), z(d) the drafted token's logit
+ *      when the shard holds it (else -inf);
+ *   2. all-gather them ([G, rows, 4], rank order), then uno_vp_verify_decide:
+ *      the merged normalisers give p(d), q(d) and the same acceptance, first
+ *      rejection n and outputs as uno_psi_verify on every device, except the
+ *      drawn token: out_tokens[b, pos] = -1 at the draw position pos = draw[b]
+ *      (n < k residual, k bonus, -1 no draw); draw_stats [B, 4] float holds the
+ *      merged (Mp, Sp, Mq, Sq) of the draw row;
+ *   3. uno_vp_draw_masses: masses [B, 2] double = the draw row's residual mass
+ *      sum max(p - q, 0) (the bonus: p mass) and p mass over the shard;
+ *   4. all-gather them ([G, B, 2]), then uno_vp_draw: the shard holding
+ *      u * Z in rank order (u as in uno_psi_verify; a zero residual mass
+ *      falls back to p) writes the drawn global id at out_tokens[b, pos];
+ *      the others leave -1;
+ *   5. an all-reduce MAX of out_tokens over the devices gives every device
+ *      the tokens uno_psi_verify would emit.
+ * The next block's draft: uno_vp_partials on the shard's draft-logit rows
+ * (id_kind 0, precise 1: the float-pair scale of the single-device draft),
+ * all-gather, uno_vp_draft_draw (the owner writes the global id, the others
+ * -1), all-reduce MAX. Results equal the single-device calls up to the order
+ * of floating-point sums. Logits `dt`, 16-byte aligned rows (Vs a multiple of
+ * 8 for bf16); partial and mass buffers 16-byte aligned; 1 <= G <= 64.
+ * ------------------------------------------------------------------------- */
+uno_status uno_vp_partials(uno_dtype dt, int32_t rows, int32_t Vs, int32_t v0, const void* logits,
+                           const int32_t* draft, int32_t k, int32_t k_p, int32_t id_kind,
+                           int32_t precise, float temperature, float* out, void* stream);
+
+uno_status uno_vp_verify_decide(int32_t B, int32_t k, int32_t k_p, int32_t V, int32_t G,
+                                const float* parts_p, const float* parts_q, const int32_t* draft,
+                                float temperature, uint64_t seed, uint64_t step,
+                                uint64_t seq_offset, int32_t* accepted_len, int32_t* out_tokens,
+                                int32_t* out_count, int32_t* draw, float* draw_stats,
+                                int32_t* dev_status, void* stream);
+
+uno_status uno_vp_draw_masses(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32_t Vs,
+                              const void* p_shard, const void* q_shard, const int32_t* draw,
+                              const float* draw_stats, float temperature, double* masses,
+                              void* stream);
+
+uno_status uno_vp_draw(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32_t Vs, int32_t v0,
+                       int32_t V, int32_t G, int32_t rank, const void* p_shard,
+                       const void* q_shard, const int32_t* draw, const float* draw_stats,
+                       const double* masses_all, float temperature, uint64_t seed, uint64_t step,
+                       uint64_t seq_offset, int32_t* out_tokens, void* stream);
+
+uno_status uno_vp_draft_draw(uno_dtype dt, int32_t B, int32_t k, int32_t Vs, int32_t v0, int32_t V,
+                             int32_t G, int32_t rank, const void* q_shard, const float* parts_all,
+                             float temperature, uint64_t seed, uint64_t step, uint64_t seq_offset,
+                             int32_t* draft, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Linear-sampler draft (hyper.ai page, section "方法": the linear sampler
  * draws one candidate block from the per-position marginals):
  *   draft[b,j] = smallest v with C(v) > u0 * C(V-1), C the inclusive

@@ -37,6 +37,8 @@ EXPORTS = [
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
     "uno_psi_step_hidden", "uno_psi_step_kernel_count",
     "uno_rmsnorm", "uno_silu_mul", "uno_wait_selftest",
+    "uno_vp_partials", "uno_vp_verify_decide", "uno_vp_draw_masses", "uno_vp_draw",
+    "uno_vp_draft_draw",
 ]
 
 
@@ -96,6 +98,14 @@ def load():
         "uno_rmsnorm": (i32, [i64, i64, vp, vp, f32, vp]),
         "uno_silu_mul": (i32, [i64, vp, vp, vp, vp]),
         "uno_wait_selftest": (i32, [i32, u64, vp, vp, vp]),
+        "uno_vp_partials": (i32, [i32, i32, i32, i32, vp, vp, i32, i32, i32, i32, f32, vp, vp]),
+        "uno_vp_verify_decide": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, f32, u64, u64, u64,
+                                       vp, vp, vp, vp, vp, vp, vp]),
+        "uno_vp_draw_masses": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, vp, f32, vp, vp]),
+        "uno_vp_draw": (i32, [i32, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, f32,
+                              u64, u64, u64, vp, vp]),
+        "uno_vp_draft_draw": (i32, [i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, f32, u64, u64,
+                                    u64, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

@@ -462,6 +462,177 @@ uno_status uno_distill(uno_dtype dt, int32_t rows, int32_t V, const void* z_teac
   return distill_launch(a, as_stream(stream));
 }
 
+// ---------------------------------------------------------------- vocabulary shards
+
+namespace {
+uno_status check_vp(uno_dtype dt, int32_t B, int32_t k, int32_t Vs, int32_t v0, int32_t V,
+                    int32_t G, int32_t rank, float T) {
+  uno_status s = check_sampler(dt, B, k, V, T);
+  if (s != UNO_OK) return s;
+  if (G < 1 || G > 64) return set_error(UNO_ERR_UNSUPPORTED, "shards G=%d outside [1, 64]", G);
+  if (rank < 0 || rank >= G) return set_error(UNO_ERR_INVALID_ARG, "rank=%d outside [0, G)", rank);
+  if (Vs < 1 || v0 < 0 || static_cast<int64_t>(v0) + Vs > V)
+    return set_error(UNO_ERR_INVALID_ARG, "shard [v0, v0 + Vs) = [%d, %d) outside [0, V=%d)", v0,
+                     v0 + Vs, V);
+  return UNO_OK;
+}
+}  // namespace
+
+uno_status uno_vp_partials(uno_dtype dt, int32_t rows, int32_t Vs, int32_t v0, const void* logits,
+                           const int32_t* draft, int32_t k, int32_t k_p, int32_t id_kind,
+                           int32_t precise, float temperature, float* out, void* stream) {
+  if (!valid_dtype(dt)) return set_error(UNO_ERR_INVALID_ARG, "unknown dtype %d", dt);
+  if (rows < 0 || Vs < 1 || v0 < 0) return set_error(UNO_ERR_INVALID_ARG, "bad sizes");
+  if (id_kind < 0 || id_kind > 2) return set_error(UNO_ERR_INVALID_ARG, "id_kind=%d outside [0, 2]", id_kind);
+  if (id_kind != 0 && (k < 1 || k > 32 || (id_kind == 1 && k_p != k && k_p != k + 1)))
+    return set_error(UNO_ERR_INVALID_ARG, "k=%d, k_p=%d", k, k_p);
+  if (id_kind == 1 && rows % k_p) return set_error(UNO_ERR_INVALID_ARG, "rows not a multiple of k_p");
+  if (!(temperature > 0.f) || !(temperature < 1e30f))
+    return set_error(UNO_ERR_INVALID_ARG, "temperature must be > 0 (got %g)", temperature);
+  if (rows == 0) return UNO_OK;
+  if (!logits || !out || (id_kind != 0 && !draft))
+    return set_error(UNO_ERR_INVALID_ARG, "NULL logits, draft or out");
+  if (!aligned16(logits) || !aligned16(out))
+    return set_error(UNO_ERR_INVALID_ARG, "logits and out must be 16-byte aligned");
+  return vp_partials_launch(dt, rows, Vs, v0, logits, draft, k, k_p, id_kind, precise != 0,
+                            temperature, out, as_stream(stream));
+}
+
+uno_status uno_vp_verify_decide(int32_t B, int32_t k, int32_t k_p, int32_t V, int32_t G,
+                                const float* parts_p, const float* parts_q, const int32_t* draft,
+                                float temperature, uint64_t seed, uint64_t step,
+                                uint64_t seq_offset, int32_t* accepted_len, int32_t* out_tokens,
+                                int32_t* out_count, int32_t* draw, float* draw_stats,
+                                int32_t* dev_status, void* stream) {
+  uno_status s = check_vp(UNO_BF16, B, k, 1, 0, V, G, 0, temperature);
+  if (s != UNO_OK) return s;
+  if (k_p != k && k_p != k + 1) return set_error(UNO_ERR_INVALID_ARG, "k_p=%d must be k or k+1", k_p);
+  if (B == 0) return UNO_OK;
+  if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k + 1) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * (k + 1) must be <= 2^32");
+  if (!parts_p || !parts_q || !draft || !accepted_len || !out_tokens || !out_count || !draw ||
+      !draw_stats)
+    return set_error(UNO_ERR_INVALID_ARG, "NULL input or output pointer");
+  if (!aligned16(parts_p) || !aligned16(parts_q) || !aligned16(draw_stats))
+    return set_error(UNO_ERR_INVALID_ARG, "partials and draw_stats must be 16-byte aligned");
+  VpArgs a{};
+  a.B = B;
+  a.k = k;
+  a.k_p = k_p;
+  a.V = V;
+  a.G = G;
+  a.temperature = temperature;
+  a.seed = seed;
+  a.step = step;
+  a.seq_offset = seq_offset;
+  a.draft = draft;
+  a.parts_p = parts_p;
+  a.parts_q = parts_q;
+  a.accepted_len = accepted_len;
+  a.out_tokens = out_tokens;
+  a.out_count = out_count;
+  a.draw = draw;
+  a.draw_stats = draw_stats;
+  a.dev_status = dev_status;
+  return vp_decide_launch(a, as_stream(stream));
+}
+
+uno_status uno_vp_draw_masses(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32_t Vs,
+                              const void* p_shard, const void* q_shard, const int32_t* draw,
+                              const float* draw_stats, float temperature, double* masses,
+                              void* stream) {
+  uno_status s = check_vp(dt, B, k, Vs, 0, Vs, 1, 0, temperature);
+  if (s != UNO_OK) return s;
+  if (k_p != k && k_p != k + 1) return set_error(UNO_ERR_INVALID_ARG, "k_p=%d must be k or k+1", k_p);
+  if (B == 0) return UNO_OK;
+  if (!p_shard || !q_shard || !draw || !draw_stats || !masses)
+    return set_error(UNO_ERR_INVALID_ARG, "NULL input or output pointer");
+  if (!aligned16(draw_stats) || !aligned16(masses))
+    return set_error(UNO_ERR_INVALID_ARG, "draw_stats and masses must be 16-byte aligned");
+  VpArgs a{};
+  a.dt = dt;
+  a.B = B;
+  a.k = k;
+  a.k_p = k_p;
+  a.Vs = Vs;
+  a.temperature = temperature;
+  a.p = p_shard;
+  a.q = q_shard;
+  a.draw = const_cast<int32_t*>(draw);
+  a.draw_stats = const_cast<float*>(draw_stats);
+  a.masses = masses;
+  return vp_masses_launch(a, as_stream(stream));
+}
+
+uno_status uno_vp_draw(uno_dtype dt, int32_t B, int32_t k, int32_t k_p, int32_t Vs, int32_t v0,
+                       int32_t V, int32_t G, int32_t rank, const void* p_shard,
+                       const void* q_shard, const int32_t* draw, const float* draw_stats,
+                       const double* masses_all, float temperature, uint64_t seed, uint64_t step,
+                       uint64_t seq_offset, int32_t* out_tokens, void* stream) {
+  uno_status s = check_vp(dt, B, k, Vs, v0, V, G, rank, temperature);
+  if (s != UNO_OK) return s;
+  if (k_p != k && k_p != k + 1) return set_error(UNO_ERR_INVALID_ARG, "k_p=%d must be k or k+1", k_p);
+  if (B == 0) return UNO_OK;
+  if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k + 1) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * (k + 1) must be <= 2^32");
+  if (!p_shard || !q_shard || !draw || !draw_stats || !masses_all || !out_tokens)
+    return set_error(UNO_ERR_INVALID_ARG, "NULL input or output pointer");
+  if (!aligned16(draw_stats) || !aligned16(masses_all))
+    return set_error(UNO_ERR_INVALID_ARG, "draw_stats and masses must be 16-byte aligned");
+  VpArgs a{};
+  a.dt = dt;
+  a.B = B;
+  a.k = k;
+  a.k_p = k_p;
+  a.Vs = Vs;
+  a.v0 = v0;
+  a.V = V;
+  a.G = G;
+  a.rank = rank;
+  a.temperature = temperature;
+  a.seed = seed;
+  a.step = step;
+  a.seq_offset = seq_offset;
+  a.p = p_shard;
+  a.q = q_shard;
+  a.draw = const_cast<int32_t*>(draw);
+  a.draw_stats = const_cast<float*>(draw_stats);
+  a.masses = const_cast<double*>(masses_all);
+  a.out_tokens = out_tokens;
+  return vp_draw_launch(a, as_stream(stream));
+}
+
+uno_status uno_vp_draft_draw(uno_dtype dt, int32_t B, int32_t k, int32_t Vs, int32_t v0, int32_t V,
+                             int32_t G, int32_t rank, const void* q_shard, const float* parts_all,
+                             float temperature, uint64_t seed, uint64_t step, uint64_t seq_offset,
+                             int32_t* draft, int32_t* dev_status, void* stream) {
+  uno_status s = check_vp(dt, B, k, Vs, v0, V, G, rank, temperature);
+  if (s != UNO_OK) return s;
+  if (B == 0) return UNO_OK;
+  if ((seq_offset + static_cast<uint64_t>(B)) * static_cast<uint64_t>(k) > (1ull << 32))
+    return set_error(UNO_ERR_UNSUPPORTED, "(seq_offset + B) * k must be <= 2^32");
+  if (!q_shard || !parts_all || !draft) return set_error(UNO_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(parts_all)) return set_error(UNO_ERR_INVALID_ARG, "partials must be 16-byte aligned");
+  VpArgs a{};
+  a.dt = dt;
+  a.B = B;
+  a.k = k;
+  a.Vs = Vs;
+  a.v0 = v0;
+  a.V = V;
+  a.G = G;
+  a.rank = rank;
+  a.temperature = temperature;
+  a.seed = seed;
+  a.step = step;
+  a.seq_offset = seq_offset;
+  a.q = q_shard;
+  a.parts_q = parts_all;
+  a.draft_out = draft;
+  a.dev_status = dev_status;
+  return vp_draft_draw_launch(a, as_stream(stream));
+}
+
 size_t uno_draft_sample_workspace(int32_t B, int32_t k, int32_t V) {
   if (B < 0 || k < 1 || V < 1) return 0;
   return align_up(draft_workspace(B, k, V));

@@ -217,6 +217,35 @@ struct NormDownArgs {   // bf16 tensors
 };
 uno_status norm_down_launch(const NormDownArgs& a, int64_t M, cudaStream_t s);
 
+// Vocabulary-shard verification and draft (psi_verify.cu): the arguments of
+// the uno_vp_* entry points of one device's shard [v0, v0 + Vs).
+struct VpArgs {
+  uno_dtype dt;
+  int32_t B, k, k_p, Vs, v0, V, G, rank;
+  float temperature;
+  uint64_t seed, step, seq_offset;
+  const void* p;            // this shard's AR logits [B, k_p, Vs]
+  const void* q;            // this shard's draft logits [B, k, Vs]
+  const int32_t* draft;     // [B, k] global ids
+  const float* parts_p;     // [G, B k_p, 4]
+  const float* parts_q;     // [G, B k, 4]
+  int32_t* accepted_len;
+  int32_t* out_tokens;
+  int32_t* out_count;
+  int32_t* draw;            // [B]
+  float* draw_stats;        // [B, 4]
+  double* masses;           // [B, 2] (this shard) or [G, B, 2] (all shards)
+  int32_t* draft_out;       // [B k]
+  int32_t* dev_status;
+};
+uno_status vp_partials_launch(uno_dtype dt, int rows, int Vs, int v0, const void* z,
+                              const int32_t* draft, int k, int k_p, int id_kind, bool precise,
+                              float temperature, float* out, cudaStream_t s);
+uno_status vp_decide_launch(const VpArgs& a, cudaStream_t s);
+uno_status vp_masses_launch(const VpArgs& a, cudaStream_t s);
+uno_status vp_draw_launch(const VpArgs& a, cudaStream_t s);
+uno_status vp_draft_draw_launch(const VpArgs& a, cudaStream_t s);
+
 // Gradients of the gated-LoRA adapter (backward.cu): dA [r,K], dBl [N,r] bf16.
 size_t adapter_backward_workspace(int64_t M, int64_t K, int64_t N, int32_t r);
 uno_status adapter_backward_launch(int64_t M, int64_t K, int64_t N, int32_t r, const void* x,

@@ -1159,6 +1159,337 @@ __global__ void __launch_bounds__(kDrawThreads)
   }
 }
 
+// ------------------------------------------------------------------ vocabulary shards
+//
+// The vocabulary split over G devices, each holding the logits of its own
+// contiguous shard [v0, v0 + Vs) (hyper.ai page, section "方法": the
+// verification against the AR distribution needs the normaliser over the
+// whole vocabulary and, for the residual and bonus draws, cumulative mass in
+// vocabulary order). The kernels below compute each device's share; the
+// exchanges between devices (all-gathers of a few floats per row, a max over
+// the drawn token) are collectives issued by the caller:
+//   vp_partials   per row of the shard: (m, s, z(d)) — max, sum of
+//                 2^((z - m) c), and the drafted token's logit if held here;
+//   vp_decide     from all shards' partials: acceptance and the first
+//                 rejection n per sequence (the same on every device), the
+//                 draw row and its merged statistics;
+//   vp_masses     the draw row's residual mass and p mass over the shard;
+//   vp_draw       from all shards' masses: the shard holding u Z in shard
+//                 order draws inside its range (the others leave -1);
+//   vp_draft_draw the next block's draft, the same owner rule on the draft
+//                 rows' partials.
+
+// Inverse-CDF draw inside one CTA over local ids [0, len): the smallest id
+// whose inclusive cumulative weight (ascending id, summed in double) exceeds
+// tl; the last id with positive weight when the total falls short of tl; -1
+// when every weight is zero. Every thread calls it and gets the result.
+template <typename WFn>
+__device__ int block_draw(DrawSmem& sh, const WFn& wfn, int len, double tl) {
+  const int t = threadIdx.x;
+  const int seg = (len + kDrawThreads - 1) / kDrawThreads;
+  const int s0 = min(len, t * seg), s1 = min(len, s0 + seg);
+  double my = 0.0;
+  for (int i = s0; i < s1; ++i) my += static_cast<double>(wfn(i));
+  block_scan(sh, my);
+  const int own = block_max_index(sh, my > 0.0 && sh.prefix[t] <= tl);
+  if (t == 0) sh.token = -1;
+  cta_sync();
+  if (t == own) {
+    const double tt = tl - sh.prefix[t];
+    double run = 0.0;
+    int pick = -1, last_nz = -1;
+    for (int i = s0; i < s1; ++i) {
+      const float w = wfn(i);
+      if (w > 0.f) last_nz = i;
+      run += static_cast<double>(w);
+      if (run > tt) {
+        pick = i;
+        break;
+      }
+    }
+    sh.token = pick >= 0 ? pick : last_nz;
+  }
+  cta_sync();
+  return sh.token;
+}
+
+struct VpParams {
+  int B, k, k_p, Vs, v0, V, G, rank;
+  float c;      // log2(e) / T (verification)
+  TScale cd;    // the same as a float pair (draft)
+  uint64_t seed, step, seq_offset;
+  const int32_t* draft;     // [B, k] global ids
+  const float4* parts_p;    // [G, B k_p]: (m, s, z(d), 0) of the AR rows
+  const float4* parts_q;    // [G, rows]: of the draft rows (verify: B k; next draft: B k)
+  int32_t* accepted_len;
+  int32_t* out_tokens;      // [B, k + 1]
+  int32_t* out_count;
+  int32_t* draw;            // [B]: draw position (n < k: residual, k: bonus) or -1
+  float4* draw_stats;       // [B]: (Mp, Sp, Mq, Sq) of the draw row
+  double2* masses;          // vp_masses: [B] of this shard; vp_draw: [G, B] of all shards
+  int32_t* draft_out;       // vp_draft_draw: [rows]
+  int32_t* status;
+};
+
+// Per row of the shard: (m, s, z(id), 0). id_kind 1: AR rows (row b k_p + j
+// holds draft[b, j] for j < k, none for the bonus row); 2: draft rows (row i
+// holds draft[i]); 0: none. One CTA per row.
+template <typename T, typename C>
+__global__ void __launch_bounds__(kStatThreads)
+    vp_partials_kernel(const T* __restrict__ z, int Vs, int v0, const int32_t* __restrict__ draft,
+                       int k, int k_p, int id_kind, C c, float4* __restrict__ out) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x;
+  const T* zr = z + static_cast<size_t>(row) * Vs;
+  const float2 st = block_row_stat<T>(zr, 0, Vs, c);
+  if (threadIdx.x == 0) {
+    int id = -1;
+    if (id_kind == 1) {
+      const int b = row / k_p, j = row - b * k_p;
+      if (j < k) id = draft[b * k + j];
+    } else if (id_kind == 2) {
+      id = draft[row];
+    }
+    const float zid = (id >= v0 && id < v0 + Vs) ? to_f32<T>(zr[id - v0]) : -INFINITY;
+    out[row] = make_float4(st.x, st.y, zid, 0.f);
+  }
+}
+
+// Merged (M, S, z(id)) of one row over the G shards (shard order).
+__device__ __forceinline__ float3 vp_merge(const float4* parts, int rows, int row, int G, float c) {
+  float m = -INFINITY, s = 0.f, z = -INFINITY;
+  bool nan = false;
+  for (int g = 0; g < G; ++g) {
+    const float4 v = parts[static_cast<size_t>(g) * rows + row];
+    nan |= isnan(v.y);
+    merge_stat(m, s, v.x, v.y, c);
+    z = fmaxf(z, v.z);
+  }
+  return make_float3(m, nan ? NAN : s, z);
+}
+
+// One warp per sequence: lane j tests position j (as verify_finalize).
+__global__ void __launch_bounds__(32) vp_decide_kernel(const VpParams a) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x, j = threadIdx.x, k = a.k;
+  const int rows_p = a.B * a.k_p, rows_q = a.B * k;
+  const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
+  bool acc = true, bad = false, nan = false;
+  if (j < k) {
+    const int d = a.draft[b * k + j];
+    bad = d < 0 || d >= a.V;
+    const float3 sp = vp_merge(a.parts_p, rows_p, b * a.k_p + j, a.G, a.c);
+    const float3 sq = vp_merge(a.parts_q, rows_q, b * k + j, a.G, a.c);
+    nan = isnan(sp.y) || isnan(sq.y);
+    if (!bad && !nan) {
+      const float pd = sp.z > -INFINITY ? fast_exp2((sp.z - sp.x) * a.c) / sp.y : 0.f;
+      const float qd = sq.z > -INFINITY ? fast_exp2((sq.z - sq.x) * a.c) / sq.y : 0.f;
+      const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + j);
+      const float u1 = uniform24(philox_word0(a.seed, a.step, kStreamAccept, idx));
+      acc = (qd == 0.f) || (u1 * qd < pd);
+    }
+  }
+  const uint32_t in_k = k >= 32 ? 0xffffffffu : ((1u << k) - 1u);
+  const uint32_t rej = __ballot_sync(0xffffffffu, !acc) & in_k;
+  const uint32_t badm = __ballot_sync(0xffffffffu, bad) & in_k;
+  const uint32_t nanm = __ballot_sync(0xffffffffu, nan) & in_k;
+  const int n = rej ? __ffs(rej) - 1 : k;
+  int32_t* tok = a.out_tokens + static_cast<size_t>(b) * (k + 1);
+  if (badm || nanm) {
+    if (j == 0) {
+      a.accepted_len[b] = -1;
+      a.out_count[b] = -1;
+      a.draw[b] = -1;
+      raise_status(a.status, (badm ? kDevBadDraft : 0) | (nanm ? kDevNaN : 0));
+    }
+    for (int i = j; i <= k; i += 32) tok[i] = -1;
+    return;
+  }
+  const int pos = n < k ? n : (a.k_p == k + 1 ? k : -1);
+  for (int i = j; i <= k; i += 32) tok[i] = i < n ? a.draft[b * k + i] : -1;
+  if (j == 0) {
+    a.accepted_len[b] = n;
+    a.out_count[b] = n + (pos >= 0 ? 1 : 0);
+    a.draw[b] = pos;
+    if (pos >= 0) {
+      const float3 sp = vp_merge(a.parts_p, rows_p, b * a.k_p + pos, a.G, a.c);
+      float3 sq = make_float3(0.f, 1.f, 0.f);
+      if (pos < k) sq = vp_merge(a.parts_q, rows_q, b * k + pos, a.G, a.c);
+      a.draw_stats[b] = make_float4(sp.x, sp.y, sq.x, sq.y);
+    }
+  }
+}
+
+// Sum of one double per thread over the CTA (valid in every thread).
+__device__ __forceinline__ double block_sum(double v, double* slots) {
+  v = warp_sum(v);
+  if ((threadIdx.x & 31) == 0) slots[threadIdx.x >> 5] = v;
+  cta_sync();
+  double t = 0.0;
+  for (int w = 0; w < kDrawThreads / 32; ++w) t += slots[w];
+  cta_sync();
+  return t;
+}
+
+// One CTA per sequence: (residual or bonus mass, p mass) of its draw row over the shard.
+template <typename T>
+__global__ void __launch_bounds__(kDrawThreads)
+    vp_masses_kernel(const T* __restrict__ p, const T* __restrict__ q, const VpParams a) {
+  __shared__ double slots[kDrawThreads / 32];
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x, pos = a.draw[b];
+  if (pos < 0) {
+    if (threadIdx.x == 0) a.masses[b] = make_double2(0.0, 0.0);
+    return;
+  }
+  const bool residual = pos < a.k;
+  const float4 st = a.draw_stats[b];
+  const T* pr = p + (static_cast<size_t>(b) * a.k_p + pos) * a.Vs;
+  const T* qr = q + (static_cast<size_t>(b) * a.k + (residual ? pos : 0)) * a.Vs;
+  const float inv_sp = 1.f / st.y, inv_sq = residual ? 1.f / st.w : 0.f;
+  double r = 0.0, pm = 0.0;
+  for (int v = threadIdx.x; v < a.Vs; v += blockDim.x) {
+    const float pv = fast_exp2((to_f32<T>(pr[v]) - st.x) * a.c) * inv_sp;
+    const float qv = residual ? fast_exp2((to_f32<T>(qr[v]) - st.z) * a.c) * inv_sq : 0.f;
+    r += static_cast<double>(fmaxf(pv - qv, 0.f));
+    pm += static_cast<double>(pv);
+  }
+  r = block_sum(r, slots);
+  pm = block_sum(pm, slots);
+  if (threadIdx.x == 0) a.masses[b] = make_double2(residual ? r : pm, pm);
+}
+
+// Owner shard of a draw: the last shard with positive mass w(g) whose
+// exclusive prefix (shard order) is <= u Z. Returns it; *tl = u Z - its prefix.
+template <typename WFn>
+__device__ __forceinline__ int vp_owner(const WFn& w, int G, double u, double* tl) {
+  double Z = 0.0;
+  for (int g = 0; g < G; ++g) Z += w(g);
+  const double thr = u * Z;
+  double pre = 0.0, own_pre = 0.0;
+  int own = -1;
+  for (int g = 0; g < G; ++g) {
+    const double wg = w(g);
+    if (wg > 0.0 && pre <= thr) {
+      own = g;
+      own_pre = pre;
+    }
+    pre += wg;
+  }
+  *tl = thr - own_pre;
+  return own;
+}
+
+// One CTA per sequence with a draw: the owner shard writes the drawn token
+// (global id) at out_tokens[b, pos]; the other shards leave it -1.
+template <typename T>
+__global__ void __launch_bounds__(kDrawThreads)
+    vp_draw_kernel(const T* __restrict__ p, const T* __restrict__ q, const VpParams a) {
+  __shared__ DrawSmem sh;
+  __shared__ int s_own;
+  __shared__ double s_tl;
+  __shared__ int s_res;
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x, pos = a.draw[b], k = a.k;
+  if (pos < 0) return;
+  const bool residual = pos < k;
+  if (threadIdx.x == 0) {
+    double z0 = 0.0;
+    for (int g = 0; g < a.G; ++g) z0 += a.masses[static_cast<size_t>(g) * a.B + b].x;
+    const bool use_res = residual && z0 > 0.0;   // zero residual mass: draw from p
+    auto w = [&](int g) {
+      const double2 m = a.masses[static_cast<size_t>(g) * a.B + b];
+      return use_res ? m.x : m.y;
+    };
+    const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
+    const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + pos);
+    const double u = static_cast<double>(
+        uniform24(philox_word0(a.seed, a.step, residual ? kStreamResidual : kStreamBonus, idx)));
+    double tl = 0.0;
+    s_own = vp_owner(w, a.G, u, &tl);
+    s_tl = tl;
+    s_res = use_res ? 1 : 0;
+  }
+  cta_sync();
+  if (s_own != a.rank) return;   // uniform over the CTA
+  const float4 st = a.draw_stats[b];
+  const T* pr = p + (static_cast<size_t>(b) * a.k_p + pos) * a.Vs;
+  const T* qr = q + (static_cast<size_t>(b) * k + (residual ? pos : 0)) * a.Vs;
+  const float inv_sp = 1.f / st.y, inv_sq = residual ? 1.f / st.w : 0.f;
+  const float c = a.c;
+  int v;
+  if (s_res) {
+    auto w_res = [&](int i) {
+      const float pv = fast_exp2((to_f32<T>(pr[i]) - st.x) * c) * inv_sp;
+      const float qv = fast_exp2((to_f32<T>(qr[i]) - st.z) * c) * inv_sq;
+      return fmaxf(pv - qv, 0.f);
+    };
+    v = block_draw(sh, w_res, a.Vs, s_tl);
+  } else {
+    auto w_p = [&](int i) { return fast_exp2((to_f32<T>(pr[i]) - st.x) * c) * inv_sp; };
+    v = block_draw(sh, w_p, a.Vs, s_tl);
+  }
+  if (threadIdx.x == 0 && v >= 0) a.out_tokens[static_cast<size_t>(b) * (k + 1) + pos] = a.v0 + v;
+}
+
+// One CTA per draft row: from all shards' partials of the row (taken with the
+// float-pair scale), the owner shard draws d ~ softmax(z / T) inside its range
+// (stream 0, index (seq_offset + b) k + j); the others write -1.
+template <typename T>
+__global__ void __launch_bounds__(kDrawThreads)
+    vp_draft_draw_kernel(const T* __restrict__ q, const VpParams a) {
+  __shared__ DrawSmem sh;
+  __shared__ int s_own;
+  __shared__ double s_tl;
+  __shared__ float s_M;
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x;
+  const int rows = a.B * a.k;
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    bool nan = false;
+    for (int g = 0; g < a.G; ++g) {
+      const float4 v = a.parts_q[static_cast<size_t>(g) * rows + row];
+      nan |= isnan(v.y);
+      M = fmaxf(M, v.x);
+    }
+    s_own = -2;
+    if (nan || M == -INFINITY) {
+      a.draft_out[row] = -1;
+      raise_status(a.status, kDevNaN);
+    } else {
+      const double cdd = static_cast<double>(a.cd.hi) + static_cast<double>(a.cd.lo);
+      auto w = [&](int g) {
+        const float4 v = a.parts_q[static_cast<size_t>(g) * rows + row];
+        return v.x == -INFINITY ? 0.0
+                                : static_cast<double>(v.y) * exp2(static_cast<double>(v.x - M) * cdd);
+      };
+      const int b = row / a.k, j = row - b * a.k;
+      const uint64_t bg = a.seq_offset + static_cast<uint64_t>(b);
+      const uint32_t idx = static_cast<uint32_t>(bg * static_cast<uint64_t>(a.k) + j);
+      const double u = static_cast<double>(uniform24(philox_word0(a.seed, a.step, kStreamDraft, idx)));
+      double tl = 0.0;
+      s_own = vp_owner(w, a.G, u, &tl);
+      s_tl = tl;
+      s_M = M;
+      if (s_own != a.rank) a.draft_out[row] = -1;
+    }
+  }
+  cta_sync();
+  if (s_own != a.rank) return;   // uniform over the CTA
+  const T* zr = q + static_cast<size_t>(row) * a.Vs;
+  const float M = s_M;
+  const TScale c = a.cd;
+  auto w = [&](int i) { return fast_exp2((to_f32<T>(zr[i]) - M) * c); };
+  const int v = block_draw(sh, w, a.Vs, s_tl);
+  if (threadIdx.x == 0) a.draft_out[row] = v >= 0 ? a.v0 + v : -1;
+}
+
 __global__ void philox_kernel(uint64_t seed, uint64_t step, uint32_t stream, uint32_t index0,
                               int64_t n, uint32_t* words, float* u) {
   if (threadIdx.x == 0) pdl_trigger();
@@ -1397,6 +1728,106 @@ uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
   }
   if (e != cudaSuccess) return cuda_error(e, "draft launch");
   return UNO_OK;
+}
+
+namespace {
+VpParams vp_params(const VpArgs& a) {
+  VpParams p{};
+  p.B = a.B;
+  p.k = a.k;
+  p.k_p = a.k_p;
+  p.Vs = a.Vs;
+  p.v0 = a.v0;
+  p.V = a.V;
+  p.G = a.G;
+  p.rank = a.rank;
+  p.c = make_scale(a.temperature);
+  p.cd = make_tscale(a.temperature);
+  p.seed = a.seed;
+  p.step = a.step;
+  p.seq_offset = a.seq_offset;
+  p.draft = a.draft;
+  p.parts_p = reinterpret_cast<const float4*>(a.parts_p);
+  p.parts_q = reinterpret_cast<const float4*>(a.parts_q);
+  p.accepted_len = a.accepted_len;
+  p.out_tokens = a.out_tokens;
+  p.out_count = a.out_count;
+  p.draw = a.draw;
+  p.draw_stats = reinterpret_cast<float4*>(a.draw_stats);
+  p.masses = reinterpret_cast<double2*>(a.masses);
+  p.draft_out = a.draft_out;
+  p.status = a.dev_status;
+  return p;
+}
+}  // namespace
+
+uno_status vp_partials_launch(uno_dtype dt, int rows, int Vs, int v0, const void* z,
+                              const int32_t* draft, int k, int k_p, int id_kind, bool precise,
+                              float temperature, float* out, cudaStream_t s) {
+  if (rows == 0) return UNO_OK;
+  float4* o = reinterpret_cast<float4*>(out);
+  cudaError_t e;
+  const float c = make_scale(temperature);
+  const TScale cd = make_tscale(temperature);
+  if (dt == UNO_F32) {
+    const float* zz = static_cast<const float*>(z);
+    e = precise ? launch_kernel(vp_partials_kernel<float, TScale>, dim3(rows), dim3(kStatThreads), 0, s,
+                                1, zz, Vs, v0, draft, k, k_p, id_kind, cd, o)
+                : launch_kernel(vp_partials_kernel<float, float>, dim3(rows), dim3(kStatThreads), 0, s,
+                                1, zz, Vs, v0, draft, k, k_p, id_kind, c, o);
+  } else {
+    const __nv_bfloat16* zz = static_cast<const __nv_bfloat16*>(z);
+    e = precise ? launch_kernel(vp_partials_kernel<__nv_bfloat16, TScale>, dim3(rows),
+                                dim3(kStatThreads), 0, s, 1, zz, Vs, v0, draft, k, k_p, id_kind, cd, o)
+                : launch_kernel(vp_partials_kernel<__nv_bfloat16, float>, dim3(rows),
+                                dim3(kStatThreads), 0, s, 1, zz, Vs, v0, draft, k, k_p, id_kind, c, o);
+  }
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "vocab-shard partials launch");
+}
+
+uno_status vp_decide_launch(const VpArgs& a, cudaStream_t s) {
+  if (a.B == 0) return UNO_OK;
+  const cudaError_t e = launch_kernel(vp_decide_kernel, dim3(a.B), dim3(32), 0, s, 1, vp_params(a));
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "vocab-shard decide launch");
+}
+
+uno_status vp_masses_launch(const VpArgs& a, cudaStream_t s) {
+  if (a.B == 0) return UNO_OK;
+  cudaError_t e;
+  if (a.dt == UNO_F32)
+    e = launch_kernel(vp_masses_kernel<float>, dim3(a.B), dim3(kDrawThreads), 0, s, 1,
+                      static_cast<const float*>(a.p), static_cast<const float*>(a.q), vp_params(a));
+  else
+    e = launch_kernel(vp_masses_kernel<__nv_bfloat16>, dim3(a.B), dim3(kDrawThreads), 0, s, 1,
+                      static_cast<const __nv_bfloat16*>(a.p), static_cast<const __nv_bfloat16*>(a.q),
+                      vp_params(a));
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "vocab-shard masses launch");
+}
+
+uno_status vp_draw_launch(const VpArgs& a, cudaStream_t s) {
+  if (a.B == 0) return UNO_OK;
+  cudaError_t e;
+  if (a.dt == UNO_F32)
+    e = launch_kernel(vp_draw_kernel<float>, dim3(a.B), dim3(kDrawThreads), 0, s, 1,
+                      static_cast<const float*>(a.p), static_cast<const float*>(a.q), vp_params(a));
+  else
+    e = launch_kernel(vp_draw_kernel<__nv_bfloat16>, dim3(a.B), dim3(kDrawThreads), 0, s, 1,
+                      static_cast<const __nv_bfloat16*>(a.p), static_cast<const __nv_bfloat16*>(a.q),
+                      vp_params(a));
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "vocab-shard draw launch");
+}
+
+uno_status vp_draft_draw_launch(const VpArgs& a, cudaStream_t s) {
+  const int rows = a.B * a.k;
+  if (rows == 0) return UNO_OK;
+  cudaError_t e;
+  if (a.dt == UNO_F32)
+    e = launch_kernel(vp_draft_draw_kernel<float>, dim3(rows), dim3(kDrawThreads), 0, s, 1,
+                      static_cast<const float*>(a.q), vp_params(a));
+  else
+    e = launch_kernel(vp_draft_draw_kernel<__nv_bfloat16>, dim3(rows), dim3(kDrawThreads), 0, s, 1,
+                      static_cast<const __nv_bfloat16*>(a.q), vp_params(a));
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "vocab-shard draft launch");
 }
 
 uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint32_t index0,
