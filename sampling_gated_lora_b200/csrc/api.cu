@@ -149,6 +149,34 @@ GemmProblem down_problem(uno_dtype dt, int64_t M, int64_t K, int32_t r, const vo
   return d;
 }
 
+// Decode-size batches whose t the decode down-projection computes: marks
+// `pm` as taking a given t and says whether the weight-only kernel takes it.
+bool decode_down_suits(GemmProblem* pm, int G) {
+  if (!lora_down_dec_suits(pm->M, pm->K, pm->r, G)) return false;
+  pm->t_given = true;
+  if (gemm_dect_suits(*pm)) return true;
+  pm->t_given = false;
+  return false;
+}
+
+// The decode down-projection writing t for the linear(s) of `pm`.
+DownDecArgs decode_down(const GemmProblem& pm, const void* const* A, int G, const uint8_t* gate,
+                        int64_t gate_row0) {
+  DownDecArgs d{};
+  d.x = pm.x;
+  for (int i = 0; i < kMaxGroups; ++i) d.A[i] = A[i < G ? i : 0];
+  d.t = const_cast<void*>(pm.t);
+  d.gate = gate;
+  d.M = pm.M;
+  d.K = pm.K;
+  d.ldt = pm.ldt;
+  d.gate_row0 = gate_row0;
+  d.r = pm.r;
+  d.G = G;
+  d.scale = pm.scale;
+  return d;
+}
+
 }  // namespace
 
 }  // namespace uno
@@ -221,11 +249,17 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   pm.gate = gate;
   pm.scale = scale;
   if (use_ws) attach_sk(&pm, L, workspace);
+  const void* As[1] = {A};
+  if (r > 0 && decode_down_suits(&pm, 1)) {   // t once, then the weight-only kernel
+    if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
+    if ((s = lora_down_dec_launch(decode_down(pm, As, 1, gate, 0), as_stream(stream))) != UNO_OK)
+      return s;
+    return gemm_run(main, as_stream(stream));
+  }
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
   if (r > 0 && !fused) {
-    const void* As[1] = {A};
     if ((s = prepare_down(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), main,
                           &down)) != UNO_OK)
       return s;
@@ -287,6 +321,12 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   pm.gate = gate;
   pm.scale = scale;
   if (use_ws) attach_sk(&pm, L, workspace);
+  if (r > 0 && decode_down_suits(&pm, G)) {   // t once, then the weight-only kernel
+    if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
+    if ((s = lora_down_dec_launch(decode_down(pm, A, G, gate, 0), as_stream(stream))) != UNO_OK)
+      return s;
+    return gemm_run(main, as_stream(stream));
+  }
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
@@ -717,11 +757,13 @@ struct StepLayout {
 
 // One operation of a step plan.
 struct StepOp {
-  int kind;            // 0 GEMM, 1 rmsnorm, 2 rmsnorm + LoRA down-projection
+  int kind;            // 0 GEMM, 1 rmsnorm, 2 rmsnorm + LoRA down-projection,
+                       // 3 decode-size LoRA down-projection
   GemmLaunch gemm;
   const void* x;
   void* y;
   NormDownArgs nd;
+  DownDecArgs dd;
   PrefetchRange w[kMaxPrefetch];    // the weights this op streams, cut into its K-slices
   PrefetchRange pf[kMaxPrefetch];   // the next weight-streaming op's, asked into L2 by this one
 };
@@ -923,6 +965,21 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       pm.sk_slots = pair_sk_slots();
       ++main_launches;
     }
+    if (r > 0 && decode_down_suits(&pm, G)) {   // t once (here or by the RMSNorm before)
+      if (!t_ready) {
+        StepOp op{};
+        op.kind = 3;
+        op.dd = decode_down(pm, As, G, nullptr, Mv);
+        P->ops.push_back(op);
+      }
+      const void* Ws[kMaxGroups];
+      int64_t w_rows[kMaxGroups];
+      for (int i = 0; i < G; ++i) {
+        Ws[i] = pm.g[i].W;
+        w_rows[i] = pm.g[i].N;
+      }
+      return gemm(pm, Ws, w_rows, G);
+    }
     pm.x_ready = r > 0 && !gemm_dec_suits(pm) && !t_ready;
     const int64_t a_rows[kMaxGroups] = {r, r, r};
     if (pm.x_ready &&
@@ -1019,6 +1076,16 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     return s;
   plan_prefetch(P, M);
   return UNO_OK;
+}
+
+// Launches one op of a step plan on `st` (M rows of width `hidden`).
+uno_status run_op(const StepOp& op, int64_t M, int64_t hidden, cudaStream_t st) {
+  switch (op.kind) {
+    case 0: return gemm_run(op.gemm, st);
+    case 1: return rmsnorm_launch(M, hidden, op.x, op.y, 1e-6f, st, op.pf);
+    case 2: return norm_down_launch(op.nd, M, st);
+    default: return lora_down_dec_launch(op.dd, st);
+  }
 }
 
 uno_model::Plan* find_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
@@ -1134,12 +1201,8 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   if (e != cudaSuccess) return cuda_error(e, "copying h_in");
   if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
     return cuda_error(e, "clearing the stream-K flags");
-  for (const StepOp& op : P->ops) {
-    s = op.kind == 0 ? gemm_run(op.gemm, st)
-        : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st, op.pf)
-                       : norm_down_launch(op.nd, M, st);
-    if (s != UNO_OK) return s;
-  }
+  for (const StepOp& op : P->ops)
+    if ((s = run_op(op, M, m->hidden, st)) != UNO_OK) return s;
 
   VerifyArgs va{};
   va.dt = UNO_BF16;
@@ -1208,14 +1271,8 @@ uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h
   if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
     return cuda_error(e, "clearing the stream-K flags");
   const size_t n_ops = n_blocks > 0 ? P->block_end[static_cast<size_t>(n_blocks) - 1] : 0;
-  for (size_t i = 0; i < n_ops; ++i) {
-    const StepOp& op = P->ops[i];
-    s = op.kind == 0 ? gemm_run(op.gemm, st)
-        : op.kind == 1 ? rmsnorm_launch(static_cast<int64_t>(M), m->hidden, op.x, op.y, 1e-6f, st,
-                                        op.pf)
-                       : norm_down_launch(op.nd, static_cast<int64_t>(M), st);
-    if (s != UNO_OK) return s;
-  }
+  for (size_t i = 0; i < n_ops; ++i)
+    if ((s = run_op(P->ops[i], static_cast<int64_t>(M), m->hidden, st)) != UNO_OK) return s;
   // the step's buffers still hold the last sub-blocks' products
   const struct { void* dst; size_t off, width; } outs[] = {
       {h_out, L.h, static_cast<size_t>(m->hidden)}, {q_out, L.q, static_cast<size_t>(m->q_out)},

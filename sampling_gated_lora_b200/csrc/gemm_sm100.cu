@@ -487,6 +487,7 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
                         reinterpret_cast<uintptr_t>(pb.zero_flags) % 16))
     return set_error(UNO_ERR_INVALID_ARG, "only a large-batch down-projection clears flags");
   if (gemm_pair_suits(pb)) return gemm_pair_prepare(pb, out);
+  if (pb.t_given && gemm_dect_suits(pb)) return gemm_dect_prepare(pb, out);
   if (gemm_dec_suits(pb)) return gemm_dec_prepare(pb, out);
   if (pb.mode == kEpiSiluPair && pb.M > 256)
     return set_error(UNO_ERR_UNSUPPORTED, "silu-pair with M > 256 needs the bf16 pair kernel");
@@ -611,6 +612,7 @@ void gemm_set_prefetch(GemmLaunch* l, const PrefetchRange* pf) {
 uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream) {
   if (l.kind == 1) return gemm_pair_run(l, stream);
   if (l.kind == 2) return gemm_dec_run(l, stream);
+  if (l.kind == 3) return gemm_dect_run(l, stream);
   void* fn = pick_kernel(static_cast<uno_dtype>(l.dtype), l.swap != 0);
   cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, l.smem_bytes);

@@ -86,6 +86,9 @@ struct GemmProblem {
   // down-projection clears the stream-K flags of the GEMM launched behind it.
   int32_t* zero_flags;
   int zero_words;
+  // t holds the gated rank-r activations already (written by the launch
+  // before this one): a decode-size batch then runs the weight-only kernel.
+  bool t_given;
 };
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
@@ -133,6 +136,25 @@ uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
 bool gemm_dec_suits(const GemmProblem& pb);
 uno_status gemm_dec_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_dec_run(const GemmLaunch& l, cudaStream_t stream);
+// The decode kernel for a precomputed t (gemm_decode_t.cu): bf16, M <= 32,
+// r <= 128, W and x in the pipeline stages, Bl t^T added by K-slice 0.
+bool gemm_dect_suits(const GemmProblem& pb);
+uno_status gemm_dect_prepare(const GemmProblem& pb, GemmLaunch* out);
+uno_status gemm_dect_run(const GemmLaunch& l, cudaStream_t stream);
+// t = scale * gate (.) (x A_g^T) for decode-size batches (M <= 32, r <= 128),
+// written side by side for G adapters into t [M, ldt] bf16.
+struct DownDecArgs {
+  const void* x;          // [M, K]
+  const void* A[kMaxGroups];
+  void* t;
+  const uint8_t* gate;    // NULL: gate[m] = (m >= gate_row0)
+  int64_t M, K, ldt, gate_row0;
+  int32_t r;
+  int G;
+  float scale;
+};
+bool lora_down_dec_suits(int64_t M, int64_t K, int32_t r, int G);
+uno_status lora_down_dec_launch(const DownDecArgs& d, cudaStream_t s);
 
 // ---------------------------------------------------------------- sampler
 
