@@ -149,34 +149,6 @@ GemmProblem down_problem(uno_dtype dt, int64_t M, int64_t K, int32_t r, const vo
   return d;
 }
 
-// Decode-size batches whose t the decode down-projection computes: marks
-// `pm` as taking a given t and says whether the weight-only kernel takes it.
-bool decode_down_suits(GemmProblem* pm, int G) {
-  if (!lora_down_dec_suits(pm->M, pm->K, pm->r, G)) return false;
-  pm->t_given = true;
-  if (gemm_dect_suits(*pm)) return true;
-  pm->t_given = false;
-  return false;
-}
-
-// The decode down-projection writing t for the linear(s) of `pm`.
-DownDecArgs decode_down(const GemmProblem& pm, const void* const* A, int G, const uint8_t* gate,
-                        int64_t gate_row0) {
-  DownDecArgs d{};
-  d.x = pm.x;
-  for (int i = 0; i < kMaxGroups; ++i) d.A[i] = A[i < G ? i : 0];
-  d.t = const_cast<void*>(pm.t);
-  d.gate = gate;
-  d.M = pm.M;
-  d.K = pm.K;
-  d.ldt = pm.ldt;
-  d.gate_row0 = gate_row0;
-  d.r = pm.r;
-  d.G = G;
-  d.scale = pm.scale;
-  return d;
-}
-
 }  // namespace
 
 }  // namespace uno
@@ -249,17 +221,11 @@ uno_status uno_gated_lora_linear(uno_dtype dt, int64_t M, int64_t K, int64_t N, 
   pm.gate = gate;
   pm.scale = scale;
   if (use_ws) attach_sk(&pm, L, workspace);
-  const void* As[1] = {A};
-  if (r > 0 && decode_down_suits(&pm, 1)) {   // t once, then the weight-only kernel
-    if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
-    if ((s = lora_down_dec_launch(decode_down(pm, As, 1, gate, 0), as_stream(stream))) != UNO_OK)
-      return s;
-    return gemm_run(main, as_stream(stream));
-  }
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
   if (r > 0 && !fused) {
+    const void* As[1] = {A};
     if ((s = prepare_down(down_problem(dt, M, K, r, x, As, 1, gate, 0, scale, t_buf), main,
                           &down)) != UNO_OK)
       return s;
@@ -321,12 +287,6 @@ uno_status uno_gated_lora_linear_group(uno_dtype dt, int64_t M, int64_t K, int32
   pm.gate = gate;
   pm.scale = scale;
   if (use_ws) attach_sk(&pm, L, workspace);
-  if (r > 0 && decode_down_suits(&pm, G)) {   // t once, then the weight-only kernel
-    if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
-    if ((s = lora_down_dec_launch(decode_down(pm, A, G, gate, 0), as_stream(stream))) != UNO_OK)
-      return s;
-    return gemm_run(main, as_stream(stream));
-  }
   const bool fused = r > 0 && gemm_dec_suits(pm);
   pm.x_ready = r > 0 && !fused;
   if ((s = gemm_prepare(pm, &main)) != UNO_OK) return s;
@@ -757,22 +717,12 @@ struct StepLayout {
 
 // One operation of a step plan.
 struct StepOp {
-  int kind;            // 0 GEMM, 1 rmsnorm, 2 rmsnorm + LoRA down-projection,
-                       // 3 decode-size LoRA down-projection
+  int kind;            // 0 GEMM, 1 rmsnorm, 2 rmsnorm + LoRA down-projection
   GemmLaunch gemm;
   const void* x;
   void* y;
   NormDownArgs nd;
-  DownDecArgs dd;
-  PrefetchRange w[kMaxPrefetch];    // the weights this op streams, cut into its K-slices
-  PrefetchRange pf[kMaxPrefetch];   // the next weight-streaming op's, asked into L2 by this one
 };
-
-// Decode-size steps (every launch streams its weights once) hand each launch
-// the next weight-streaming launch's weights to prefetch into L2 when they
-// fit in this many bytes (half of the 126 MB L2).
-constexpr int64_t kPrefetchMaxRows = 256;
-constexpr double kPrefetchBudget = 64.0 * (1 << 20);
 
 // Decode-size batches fold the LoRA down-projection of an input that an
 // RMSNorm produces into that RMSNorm's launch (one launch instead of two).
@@ -847,32 +797,6 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
 //   down(act; A_down) -> t; gemm(act, t; down) += h
 // then rmsnorm(h) -> n, the LM head's down-projection and GEMM (AR rows ->
 // logits, mask rows -> q_next). Rows >= B(k+1) carry the adapter (gate 1).
-// Decode-size plans: every op asks L2 for the leading part of each K-slice
-// of the next op that streams at least 4 MB of weights, up to kPrefetchBudget
-// bytes in all (see PrefetchRange).
-void plan_prefetch(uno_model::Plan* P, int64_t M) {
-  if (M > kPrefetchMaxRows) return;
-  auto bytes_of = [](const StepOp& o) {
-    double b = 0;
-    for (const PrefetchRange& r : o.w) b += static_cast<double>(r.rows) * static_cast<double>(r.row_bytes);
-    return b;
-  };
-  const size_t n = P->ops.size();
-  for (size_t i = 0; i < n; ++i) {
-    StepOp& op = P->ops[i];
-    size_t j = i + 1;
-    while (j < n && bytes_of(P->ops[j]) < 4.0 * (1 << 20)) ++j;
-    if (j == n) continue;
-    // whole weight matrices only: a partial prefetch needs one small request
-    // per row segment, and that many requests hold up the issuing thread
-    if (bytes_of(P->ops[j]) > kPrefetchBudget) continue;
-    for (int r = 0; r < kMaxPrefetch; ++r) op.pf[r] = P->ops[j].w[r];
-    if (op.kind == 0) gemm_set_prefetch(&op.gemm, op.pf);
-    if (op.kind == 2)
-      for (int r = 0; r < kMaxPrefetch; ++r) op.nd.pf[r] = op.pf[r];
-  }
-}
-
 uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
                       void* logits_out, uno_model::Plan* P) {
   const StepLayout L = step_layout(m, B, k);
@@ -896,26 +820,12 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     op.y = y;
     P->ops.push_back(op);
   };
-  // a GEMM launch; `wts` / `rows`: the weight matrices it streams (K columns each)
-  auto gemm = [&](const GemmProblem& pb, const void* const* wts, const int64_t* rows,
-                  int nw) -> uno_status {
+  auto gemm = [&](const GemmProblem& pb) -> uno_status {
     StepOp op{};
     op.kind = 0;
     const uno_status s = gemm_prepare(pb, &op.gemm);
-    if (s != UNO_OK) return s;
-    const unsigned long long row_bytes = static_cast<unsigned long long>(pb.K) * 2;
-    const unsigned long long seg =
-        std::min<unsigned long long>(row_bytes, static_cast<unsigned long long>(op.gemm.kb_per_split) * 128ull);
-    for (int i = 0; i < nw && i < kMaxPrefetch; ++i) {
-      op.w[i].p = wts[i];
-      op.w[i].row_bytes = row_bytes;
-      op.w[i].seg_stride = seg;
-      op.w[i].rows = static_cast<unsigned>(rows[i]);
-      op.w[i].nseg = static_cast<unsigned>((row_bytes + seg - 1) / seg);
-      op.w[i].seg_bytes = static_cast<unsigned>(seg);
-    }
-    P->ops.push_back(op);
-    return UNO_OK;
+    if (s == UNO_OK) P->ops.push_back(op);
+    return s;
   };
   // gated linear(s) on input x (width K): down-projections then the main GEMM.
   // t_ready: the preceding launch wrote t as well as x (no down-projection here).
@@ -965,34 +875,11 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       pm.sk_slots = pair_sk_slots();
       ++main_launches;
     }
-    if (r > 0 && decode_down_suits(&pm, G)) {   // t once (here or by the RMSNorm before)
-      if (!t_ready) {
-        StepOp op{};
-        op.kind = 3;
-        op.dd = decode_down(pm, As, G, nullptr, Mv);
-        P->ops.push_back(op);
-      }
-      const void* Ws[kMaxGroups];
-      int64_t w_rows[kMaxGroups];
-      for (int i = 0; i < G; ++i) {
-        Ws[i] = pm.g[i].W;
-        w_rows[i] = pm.g[i].N;
-      }
-      return gemm(pm, Ws, w_rows, G);
-    }
     pm.x_ready = r > 0 && !gemm_dec_suits(pm) && !t_ready;
-    const int64_t a_rows[kMaxGroups] = {r, r, r};
     if (pm.x_ready &&
-        (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t), As, a_rows,
-                  G)) != UNO_OK)
+        (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
       return s;
-    const void* Ws[kMaxGroups];
-    int64_t w_rows[kMaxGroups];
-    for (int i = 0; i < G; ++i) {
-      Ws[i] = pm.g[i].W;
-      w_rows[i] = pm.g[i].N;
-    }
-    return gemm(pm, Ws, w_rows, G);
+    return gemm(pm);
   };
   uno_status s;
   for (int l = 0; l < m->n_layers; ++l) {
@@ -1063,29 +950,13 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     }
     P->block_end.push_back(P->ops.size());
   }
-  if (!q_next) {   // decoder layers only
-    plan_prefetch(P, M);
-    return UNO_OK;
-  }
+  if (!q_next) return UNO_OK;   // decoder layers only
   norm(base + L.h, base + L.n);
   void* p_dst = logits_out ? logits_out : base + L.logits;
   const int which[1] = {0};
   void* y[1] = {p_dst};
   const int64_t ld[1] = {m->vocab};
-  if ((s = linear(base + L.n, m->hidden, 1, which, -1, y, ld, kEpiStore, q_next, Mv)) != UNO_OK)
-    return s;
-  plan_prefetch(P, M);
-  return UNO_OK;
-}
-
-// Launches one op of a step plan on `st` (M rows of width `hidden`).
-uno_status run_op(const StepOp& op, int64_t M, int64_t hidden, cudaStream_t st) {
-  switch (op.kind) {
-    case 0: return gemm_run(op.gemm, st);
-    case 1: return rmsnorm_launch(M, hidden, op.x, op.y, 1e-6f, st, op.pf);
-    case 2: return norm_down_launch(op.nd, M, st);
-    default: return lora_down_dec_launch(op.dd, st);
-  }
+  return linear(base + L.n, m->hidden, 1, which, -1, y, ld, kEpiStore, q_next, Mv);
 }
 
 uno_model::Plan* find_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
@@ -1201,8 +1072,12 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   if (e != cudaSuccess) return cuda_error(e, "copying h_in");
   if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
     return cuda_error(e, "clearing the stream-K flags");
-  for (const StepOp& op : P->ops)
-    if ((s = run_op(op, M, m->hidden, st)) != UNO_OK) return s;
+  for (const StepOp& op : P->ops) {
+    s = op.kind == 0 ? gemm_run(op.gemm, st)
+        : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st)
+                       : norm_down_launch(op.nd, M, st);
+    if (s != UNO_OK) return s;
+  }
 
   VerifyArgs va{};
   va.dt = UNO_BF16;
@@ -1271,8 +1146,13 @@ uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h
   if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
     return cuda_error(e, "clearing the stream-K flags");
   const size_t n_ops = n_blocks > 0 ? P->block_end[static_cast<size_t>(n_blocks) - 1] : 0;
-  for (size_t i = 0; i < n_ops; ++i)
-    if ((s = run_op(P->ops[i], static_cast<int64_t>(M), m->hidden, st)) != UNO_OK) return s;
+  for (size_t i = 0; i < n_ops; ++i) {
+    const StepOp& op = P->ops[i];
+    s = op.kind == 0 ? gemm_run(op.gemm, st)
+        : op.kind == 1 ? rmsnorm_launch(static_cast<int64_t>(M), m->hidden, op.x, op.y, 1e-6f, st)
+                       : norm_down_launch(op.nd, static_cast<int64_t>(M), st);
+    if (s != UNO_OK) return s;
+  }
   // the step's buffers still hold the last sub-blocks' products
   const struct { void* dst; size_t off, width; } outs[] = {
       {h_out, L.h, static_cast<size_t>(m->hidden)}, {q_out, L.q, static_cast<size_t>(m->q_out)},

@@ -256,14 +256,6 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
                : "memory");
 }
 
-// Ask L2 to fetch [p, p + bytes) from global memory: a hint with nothing to
-// wait for. p and bytes: multiples of 16.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
-               "r"(bytes)
-               : "memory");
-}
-
 // Contiguous copy global -> this CTA's shared memory (no tensor map),
 // completion counted on `bar`. dst, src and bytes: multiples of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,

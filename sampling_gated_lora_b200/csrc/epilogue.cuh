@@ -33,47 +33,7 @@ struct GemmArgs {
   int32_t* status;
   int x_ready;    // x complete at launch: wait for the predecessor only before reading t
   GroupArgs g[kMaxGroups];
-  PrefetchRange pf[kMaxPrefetch];   // weights of the next launch (L2 hint)
 };
-
-// Issuer `i` of `n` asks L2 for its share of the next launch's weights. The
-// GEMM kernels issue from the thread that issues the CTA's loads, after its
-// last one (one issuer per CTA); the glue kernels from every thread.
-__device__ __forceinline__ void prefetch_next(const PrefetchRange (&pf)[kMaxPrefetch], long long i,
-                                              long long n) {
-  constexpr unsigned long long kPiece = 32768ull;
-#pragma unroll
-  for (int r = 0; r < kMaxPrefetch; ++r) {
-    const PrefetchRange& R = pf[r];
-    if (R.rows == 0 || R.seg_bytes == 0) continue;
-    const char* base = static_cast<const char*>(R.p);
-    if (static_cast<unsigned long long>(R.seg_bytes) >= R.seg_stride &&
-        static_cast<unsigned long long>(R.nseg) * R.seg_stride >= R.row_bytes) {
-      // whole rows: one contiguous range, in pieces
-      const unsigned long long total = static_cast<unsigned long long>(R.rows) * R.row_bytes;
-      const long long pieces = static_cast<long long>((total + kPiece - 1) / kPiece);
-      for (long long q = i; q < pieces; q += n) {
-        const unsigned long long off = static_cast<unsigned long long>(q) * kPiece;
-        const unsigned long long left = total - off;
-        prefetch_l2_bulk(base + off, static_cast<uint32_t>(left < kPiece ? left : kPiece));
-      }
-      continue;
-    }
-    const long long items = static_cast<long long>(R.rows) * R.nseg;
-    for (long long it = i; it < items; it += n) {
-      const long long row = it / R.nseg, seg = it - row * R.nseg;
-      const unsigned long long off = static_cast<unsigned long long>(seg) * R.seg_stride;
-      if (off >= R.row_bytes) continue;
-      const unsigned long long left = R.row_bytes - off;
-      const unsigned long long bytes = left < R.seg_bytes ? left : R.seg_bytes;
-      const char* src = base + static_cast<unsigned long long>(row) * R.row_bytes + off;
-      for (unsigned long long o = 0; o < bytes; o += kPiece) {
-        const unsigned long long piece = bytes - o < kPiece ? bytes - o : kPiece;
-        prefetch_l2_bulk(src + o, static_cast<uint32_t>(piece));
-      }
-    }
-  }
-}
 
 // Host: the device-side description of a problem; `tile_n` is the number of
 // output features per feature tile (silu-pair tiles count output features).

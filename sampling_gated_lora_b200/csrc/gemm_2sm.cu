@@ -244,8 +244,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!waited) pdl_wait();
-    // every load of this CTA is issued: ask L2 for the next launch's weights
-    prefetch_next(a.pf, blockIdx.x, gridDim.x);
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer (leader)
     const uint32_t idesc = idesc_f32acc(kTile, kTile, false);
@@ -474,7 +472,6 @@ uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
   }
   std::memcpy(out->params, &pp, sizeof(pp));
   out->kind = 1;
-  out->kb_per_split = 1 << 30;   // whole rows of K per tile
   out->swap = 0;
   out->grid_x = 2 * pairs;
   out->grid_y = 1;

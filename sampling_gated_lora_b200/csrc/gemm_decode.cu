@@ -46,7 +46,7 @@ struct DecParams {
   int bn, stages, tmem_cols, kb_per_split, splits, nkr;
   uint32_t stage_bytes, bl_off, tq_off, bar_off;
 };
-static_assert(sizeof(DecParams) <= kLaunchParamBytes, "DecParams must fit GemmLaunch::params");
+static_assert(sizeof(DecParams) <= 256, "DecParams must fit GemmLaunch::params");
 
 __device__ __forceinline__ void epi_bar() { named_sync(1, 128); }
 
@@ -161,9 +161,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_const(kb, st, fb);
       tma_load_2d(st + x_off, &tm.x, kb * 64, tok0, fb);
     }
-    // every load of this CTA is issued: ask L2 for the next launch's weights
-    prefetch_next(a.pf, static_cast<long long>(blockIdx.y) * gridDim.z + blockIdx.z,
-                  static_cast<long long>(gridDim.y) * gridDim.z);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_f32acc(kRows, bn, false);
@@ -476,7 +473,6 @@ uno_status gemm_dec_prepare(const GemmProblem& pb, GemmLaunch* out) {
   }
   std::memcpy(out->params, &dp, sizeof(dp));
   out->kind = 2;
-  out->kb_per_split = dp.kb_per_split;
   out->swap = silu ? 1 : 0;   // kernel variant
   out->grid_x = 1;
   out->grid_y = feat_tiles;

@@ -61,7 +61,7 @@ struct Gemm1Params {
   int32_t* zero_flags;    // cleared by CTA (0,0,0) after its wait (or NULL); 16-byte aligned
   int zero_words;         // a multiple of 4
 };
-static_assert(sizeof(Gemm1Params) <= kLaunchParamBytes, "Gemm1Params must fit GemmLaunch::params");
+static_assert(sizeof(Gemm1Params) <= 256, "Gemm1Params must fit GemmLaunch::params");
 
 __host__ __device__ constexpr uint32_t stage_bytes_for(int bn) {
   return ((kTileP + bn) * kRowBytes + 1023u) & ~1023u;
@@ -210,10 +210,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       load_tok(kb, kSwap ? sp + p_bytes : sp, fb);
     }
     if (down) wait_pred();   // a CTA with no K-blocks still triggers
-    // every load of this CTA is issued: ask L2 for the next launch's weights
-    prefetch_next(a.pf,
-                  (static_cast<long long>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x,
-                  static_cast<long long>(gridDim.x) * gridDim.y * gridDim.z);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_f32acc(kTileP, bn, kTf32);
@@ -487,7 +483,6 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
                         reinterpret_cast<uintptr_t>(pb.zero_flags) % 16))
     return set_error(UNO_ERR_INVALID_ARG, "only a large-batch down-projection clears flags");
   if (gemm_pair_suits(pb)) return gemm_pair_prepare(pb, out);
-  if (pb.t_given && gemm_dect_suits(pb)) return gemm_dect_prepare(pb, out);
   if (gemm_dec_suits(pb)) return gemm_dec_prepare(pb, out);
   if (pb.mode == kEpiSiluPair && pb.M > 256)
     return set_error(UNO_ERR_UNSUPPORTED, "silu-pair with M > 256 needs the bf16 pair kernel");
@@ -593,7 +588,6 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   }
   std::memcpy(out->params, &gp, sizeof(gp));
   out->kind = 0;
-  out->kb_per_split = gp.kb_per_split;
   out->swap = swap;
   out->grid_x = tok_tiles;
   out->grid_y = feat_tiles;
@@ -603,16 +597,9 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   return UNO_OK;
 }
 
-void gemm_set_prefetch(GemmLaunch* l, const PrefetchRange* pf) {
-  // every kernel's parameter block starts with its GemmArgs
-  GemmArgs* a = reinterpret_cast<GemmArgs*>(l->params);
-  for (int i = 0; i < kMaxPrefetch; ++i) a->pf[i] = pf ? pf[i] : PrefetchRange{nullptr, 0};
-}
-
 uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream) {
   if (l.kind == 1) return gemm_pair_run(l, stream);
   if (l.kind == 2) return gemm_dec_run(l, stream);
-  if (l.kind == 3) return gemm_dect_run(l, stream);
   void* fn = pick_kernel(static_cast<uno_dtype>(l.dtype), l.swap != 0);
   cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, l.smem_bytes);

@@ -1,7 +1,6 @@
 // Glue between the gated projections of the synthetic decode step (bf16,
 // HBM-bound): RMSNorm without weight and silu(gate) * up.
 #include "common.cuh"
-#include "epilogue.cuh"
 #include "internal.h"
 
 namespace uno {
@@ -10,18 +9,11 @@ namespace {
 
 constexpr int kNormThreads = 256;
 
-struct PrefetchSet {
-  PrefetchRange r[kMaxPrefetch];
-};
-
-// One CTA per row: y = x / sqrt(mean(x^2) + eps), fp32 arithmetic. The
-// weights of the launch after it (constant) are asked into L2 first.
+// One CTA per row: y = x / sqrt(mean(x^2) + eps), fp32 arithmetic.
 __global__ void __launch_bounds__(kNormThreads)
     rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y, int D,
-                   float eps, const PrefetchSet pf) {
+                   float eps) {
   if (threadIdx.x == 0) pdl_trigger();
-  prefetch_next(pf.r, static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x,
-                static_cast<long long>(gridDim.x) * blockDim.x);
   pdl_wait();
   const size_t row = blockIdx.x;
   const __nv_bfloat16* xr = x + row * D;
@@ -86,9 +78,6 @@ constexpr int kNdRows = 32;
 __global__ void __launch_bounds__(kNormThreads)
     rmsnorm_down_kernel(const NormDownArgs a) {
   if (threadIdx.x == 0) pdl_trigger();
-  prefetch_next(a.pf,
-                (static_cast<long long>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x,
-                static_cast<long long>(gridDim.x) * gridDim.y * blockDim.x);
   pdl_wait();
   const size_t row = blockIdx.x;
   const int D = a.D;
@@ -197,15 +186,11 @@ __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
 }  // namespace
 
 uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
-                          cudaStream_t s, const PrefetchRange* pf) {
+                          cudaStream_t s) {
   if (M == 0) return UNO_OK;
-  PrefetchSet ps{};
-  if (pf)
-    for (int i = 0; i < kMaxPrefetch; ++i) ps.r[i] = pf[i];
   const cudaError_t e = launch_kernel(
       rmsnorm_kernel, dim3(static_cast<unsigned>(M)), dim3(kNormThreads), 0, s, 1,
-      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), static_cast<int>(D), eps,
-      ps);
+      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), static_cast<int>(D), eps);
   return e == cudaSuccess ? UNO_OK : cuda_error(e, "rmsnorm launch");
 }
 

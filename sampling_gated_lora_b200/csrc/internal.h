@@ -26,22 +26,6 @@ enum EpilogueMode : int {
 
 constexpr int kMaxGroups = 3;
 
-// Constant weights that the launch after this one reads: a launch asks L2 to
-// fetch them once its own loads are issued, so the HBM keeps streaming while
-// this launch drains and the next one starts. The region is `rows` rows of
-// `row_bytes`, each cut into `nseg` segments `seg_stride` bytes apart (the
-// K-slices the next launch's CTAs stream, in order); the first `seg_bytes` of
-// every segment are fetched, so every consuming CTA finds the same leading
-// share of its slice in L2. Pointers and byte counts: multiples of 16;
-// rows == 0: no region.
-struct PrefetchRange {
-  const void* p;
-  unsigned long long row_bytes;
-  unsigned long long seg_stride;
-  unsigned rows, nseg, seg_bytes, pad;
-};
-constexpr int kMaxPrefetch = 3;
-
 // One output group of a GEMM launch: its weights, adapter and output.
 struct GemmGroup {
   const void* W;          // [N, K]
@@ -86,9 +70,6 @@ struct GemmProblem {
   // down-projection clears the stream-K flags of the GEMM launched behind it.
   int32_t* zero_flags;
   int zero_words;
-  // t holds the gated rank-r activations already (written by the launch
-  // before this one): a decode-size batch then runs the weight-only kernel.
-  bool t_given;
 };
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
@@ -97,7 +78,7 @@ struct TensorMaps {
   CUtensorMap x, t, w[kMaxGroups], b[kMaxGroups], a[kMaxGroups];
 };
 
-constexpr size_t kLaunchParamBytes = 512;
+constexpr size_t kLaunchParamBytes = 320;
 
 // Cached launch of a GemmProblem (tensor maps + grid); valid while the
 // pointers of the problem stay the same.
@@ -111,12 +92,9 @@ struct GemmLaunch {
   int dtype;
   int32_t* sk_flag;       // stream-K flags this launch reads: zero them before it runs (or NULL)
   size_t sk_flag_bytes;
-  int kb_per_split;       // K-blocks of one split (the K-slice a CTA streams)
 };
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out);
-// Sets the ranges a prepared launch prefetches for its successor (NULL: none).
-void gemm_set_prefetch(GemmLaunch* l, const PrefetchRange* pf);
 uno_status gemm_run(const GemmLaunch& l, cudaStream_t stream);
 // Row-major [rows, inner] tensor map: box = 128 bytes of K x box_rows rows, 128-byte swizzle.
 uno_status make_map(CUtensorMap* tm, uno_dtype dt, const void* base, uint64_t inner, uint64_t rows,
@@ -136,25 +114,6 @@ uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
 bool gemm_dec_suits(const GemmProblem& pb);
 uno_status gemm_dec_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_dec_run(const GemmLaunch& l, cudaStream_t stream);
-// The decode kernel for a precomputed t (gemm_decode_t.cu): bf16, M <= 32,
-// r <= 128, W and x in the pipeline stages, Bl t^T added by K-slice 0.
-bool gemm_dect_suits(const GemmProblem& pb);
-uno_status gemm_dect_prepare(const GemmProblem& pb, GemmLaunch* out);
-uno_status gemm_dect_run(const GemmLaunch& l, cudaStream_t stream);
-// t = scale * gate (.) (x A_g^T) for decode-size batches (M <= 32, r <= 128),
-// written side by side for G adapters into t [M, ldt] bf16.
-struct DownDecArgs {
-  const void* x;          // [M, K]
-  const void* A[kMaxGroups];
-  void* t;
-  const uint8_t* gate;    // NULL: gate[m] = (m >= gate_row0)
-  int64_t M, K, ldt, gate_row0;
-  int32_t r;
-  int G;
-  float scale;
-};
-bool lora_down_dec_suits(int64_t M, int64_t K, int32_t r, int G);
-uno_status lora_down_dec_launch(const DownDecArgs& d, cudaStream_t s);
 
 // ---------------------------------------------------------------- sampler
 
@@ -219,7 +178,7 @@ uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint3
 
 // ---------------------------------------------------------------- glue
 uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
-                          cudaStream_t s, const PrefetchRange* pf = nullptr);
+                          cudaStream_t s);
 uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s);
 
 // RMSNorm of x into y plus the gated LoRA down-projection of y for G adapters
@@ -235,7 +194,6 @@ struct NormDownArgs {   // bf16 tensors
   int ldt;
   float scale;
   int64_t gate_row0;
-  PrefetchRange pf[kMaxPrefetch];   // weights of the next launch (L2 hint)
 };
 uno_status norm_down_launch(const NormDownArgs& a, int64_t M, cudaStream_t s);
 
