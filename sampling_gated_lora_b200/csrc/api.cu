@@ -96,7 +96,10 @@ uno_status prepare_down(GemmProblem d, const GemmLaunch& main, GemmLaunch* out) 
 
 // Runs the down-projection (if any) and the main launch of a gated linear.
 // The main launch's stream-K flags are cleared by the down-projection (see
-// prepare_down); without one, by a memset first.
+// prepare_down); without one, by a memset first. (Single calls leave
+// GemmProblem::t_ready unset: back to back, a separate down-projection that
+// overlaps the previous call's tail measured faster than a GEMM that
+// computes t itself behind a memset.)
 uno_status run_linear(const GemmLaunch* down, const GemmLaunch& main, cudaStream_t st) {
   if (main.sk_flag && !down) {
     const cudaError_t e = cudaMemsetAsync(main.sk_flag, 0, main.sk_flag_bytes, st);
@@ -712,7 +715,8 @@ constexpr int kLinPerLayer = 7;   // q, k, v, o, gate, up, down
 enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
 
 struct StepLayout {
-  size_t h, n, q, k, v, act, t, logits, vstat, dstat, sk_part, sk_flag, sk_flag_bytes, total;
+  size_t h, n, q, k, v, act, t, logits, vstat, dstat, sk_part, sk_flag, sk_flag_bytes, flag_block,
+      total;
 };
 
 // One operation of a step plan.
@@ -780,10 +784,12 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
   L.vstat = take(verify_workspace(B, k, k + 1, m->vocab));
   L.dstat = take(draft_workspace(B, k, m->vocab));
   // stream-K scratch of the CTA-pair GEMMs (M > 256): partial sums shared by
-  // the step's launches, one block of flags per launch (4 per layer + head)
+  // the step's launches, one block of stream-K flags and t counters per
+  // launch (4 per layer + head), all cleared at the start of a step
   if (M > 256) {
     L.sk_part = take(pair_sk_part_bytes());
-    L.sk_flag_bytes = (static_cast<size_t>(m->n_layers) * 4 + 1) * align_up(pair_sk_flag_bytes());
+    L.flag_block = align_up(pair_sk_flag_bytes()) + align_up(pair_t_ready_bytes(M));
+    L.sk_flag_bytes = (static_cast<size_t>(m->n_layers) * 4 + 1) * L.flag_block;
     L.sk_flag = take(L.sk_flag_bytes);
   }
   L.total = off;
@@ -827,8 +833,9 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     if (s == UNO_OK) P->ops.push_back(op);
     return s;
   };
-  // gated linear(s) on input x (width K): down-projections then the main GEMM.
-  // t_ready: the preceding launch wrote t as well as x (no down-projection here).
+  // gated linear(s) on input x (width K): down-projections then the main GEMM
+  // (or the main GEMM alone, when it computes t itself or is the fused
+  // decode kernel). t_ready: the preceding launch wrote t as well as x.
   auto linear = [&](const void* x, int64_t K, int G, const int* which, int layer, void* const* y,
                     const int64_t* ldy, int mode, void* y1, int64_t M0,
                     bool t_ready = false) -> uno_status {
@@ -868,18 +875,23 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     pm.gate_row0 = Mv;
     pm.scale = m->scale;
     for (int i = 0; i < G; ++i) pm.A[i] = r > 0 ? As[i] : nullptr;
+    pm.x_ready = r > 0 && !gemm_dec_suits(pm) && !t_ready;
     if (L.sk_flag_bytes) {
+      char* blk = base + L.sk_flag + static_cast<size_t>(main_launches) * L.flag_block;
       pm.sk_part = reinterpret_cast<float*>(base + L.sk_part);
-      pm.sk_flag = reinterpret_cast<int32_t*>(
-          base + L.sk_flag + static_cast<size_t>(main_launches) * align_up(pair_sk_flag_bytes()));
+      pm.sk_flag = reinterpret_cast<int32_t*>(blk);
       pm.sk_slots = pair_sk_slots();
+      if (pm.x_ready) pm.t_ready = reinterpret_cast<int32_t*>(blk + align_up(pair_sk_flag_bytes()));
       ++main_launches;
     }
-    pm.x_ready = r > 0 && !gemm_dec_suits(pm) && !t_ready;
-    if (pm.x_ready &&
+    StepOp op{};
+    op.kind = 0;
+    if ((s = gemm_prepare(pm, &op.gemm)) != UNO_OK) return s;
+    if (pm.x_ready && !op.gemm.computes_t &&
         (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
       return s;
-    return gemm(pm);
+    P->ops.push_back(op);
+    return UNO_OK;
   };
   uno_status s;
   for (int l = 0; l < m->n_layers; ++l) {
@@ -1029,8 +1041,8 @@ size_t uno_psi_step_workspace(const uno_model* m, int32_t B, int32_t k) {
 int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k) {
   if (!m || B < 1 || k < 1) return 0;
   // per layer: 2 rmsnorm + 4 GEMM launches, each with a separate
-  // down-projection launch unless the fused decode kernel takes it; then
-  // rmsnorm + LM head; verify (2 kernels) + draft (2)
+  // down-projection launch unless the GEMM computes t itself; then rmsnorm +
+  // LM head; verify (2 kernels) + draft (2)
   std::lock_guard<std::mutex> lock(const_cast<uno_model*>(m)->mu);
   for (const auto& p : m->plans)
     if (p->B == B && p->k == k && p->q_next) return static_cast<int32_t>(p->ops.size()) + 4;

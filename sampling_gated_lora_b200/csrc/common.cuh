@@ -61,6 +61,21 @@ __device__ __forceinline__ bool flag_wait(const int32_t* f, int32_t v,
   }
 }
 
+// A counter that several writers raise by one each and a reader waits on
+// until it reaches a target (bounded, like flag_wait).
+__device__ __forceinline__ void counter_add_release(int32_t* f, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool counter_wait(const int32_t* f, int32_t target,
+                                             uint64_t limit_ns = kWaitLimitNs) {
+  if (flag_acquire(f) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (flag_acquire(f) >= target) return true;
+    if ((i & 63u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // Kernels of this library are launched so that the next kernel on the stream
 // may start its prologue while this one finishes. Each kernel triggers its

@@ -29,6 +29,19 @@
 // would leave the last round part-empty, the K-blocks of the last tiles are
 // shared out evenly (stream-K); the two pairs that cut a tile meet through
 // fp32 partial sums and flags in the caller's workspace.
+//
+// Down tiles. When the kernel also computes t (r <= 128), the work list opens
+// with the down tiles of every 256-row token block:
+// t[:, g r + j] = scale * gate(m) * (x A_g^T)[m, j], the same K-loop over x
+// with adapter rows on the B side. Groups go two to a tile (A_2j in CTA 0's
+// half, A_2j+1 in CTA 1's, an N = 256 MMA); an odd last group takes a
+// 256 x 128 tile (64 of its rows per CTA, an N = 128 MMA). The epilogue
+// stores t in bf16 and adds one per epilogue warp to the token block's
+// counter; a main tile's producer waits for that count (bounded)
+// before its first adapter K-block only. Every pair takes its down tiles
+// before its main tiles and down tiles wait for nothing, so the waits end.
+// One launch replaces the separate down-projection launch, whose CTAs held
+// SMs that the pairs could not use while it ran.
 #include <algorithm>
 #include <cstring>
 
@@ -63,6 +76,12 @@ struct PairParams {
   long long sk_iters;
   float* sk_part;       // [pairs][2 CTAs][4 epilogue warps][256 columns][32 rows] fp32
   int32_t* sk_flag;     // [pairs][2 CTAs][4 epilogue warps], zero once the predecessor is done
+  // Down tiles [0, down_tiles): groups 2j and 2j + 1 (j = tile / tiles_m),
+  // token block tile % tiles_m (0 when t comes from an earlier launch); main
+  // tile i is tile down_tiles + i.
+  int down_tiles, down_expect, r, ldt;
+  __nv_bfloat16* t;
+  int32_t* t_ready;     // [tiles_m] finished down-tile epilogue warps per token block
 };
 static_assert(sizeof(PairParams) <= kLaunchParamBytes, "PairParams must fit GemmLaunch::params");
 
@@ -86,12 +105,13 @@ __device__ __forceinline__ WorkCursor work_begin(const PairParams& p, int pair, 
   return c;
 }
 
+template <bool kDown>
 __device__ __forceinline__ bool work_next(const PairParams& p, int pairs, int nkb, WorkCursor& c,
                                           int& tile, int& kb0, int& kb1) {
   if (c.tile < p.dp_tiles) {
     tile = c.tile;
     kb0 = 0;
-    kb1 = nkb;
+    kb1 = kDown && tile < p.down_tiles ? p.a.nkb_main : nkb;
     c.tile += pairs;
     return true;
   }
@@ -105,6 +125,40 @@ __device__ __forceinline__ bool work_next(const PairParams& p, int pairs, int nk
   return true;
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Token block, feature tile (main) or first group (down) of a work item;
+// `wide`: a down tile with two groups.
+struct TileId {
+  bool down, wide;
+  int mb, ft, g;
+};
+
+template <bool kDown>
+__device__ __forceinline__ TileId tile_id(const PairParams& p, int tile) {
+  TileId t;
+  t.down = kDown && tile < p.down_tiles;
+  t.wide = false;
+  if (t.down) {
+    t.mb = tile % p.tiles_m;
+    t.g = 2 * (tile / p.tiles_m);
+    t.wide = t.g + 1 < p.a.ngroups;
+    t.ft = 0;
+  } else {
+    const int mt = kDown ? tile - p.down_tiles : tile;
+    t.mb = mt % p.tiles_m;
+    t.ft = mt / p.tiles_m;
+    t.g = group_of(p.a, t.ft);
+  }
+  return t;
+}
+
+// kDown: the launch has down tiles (a separate instance, so that launches
+// without them run none of their code).
+template <bool kDown>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ TensorMaps tm, const PairParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -170,16 +224,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool waited = false;
     WorkCursor wc = work_begin(p, pair, num_pairs);
     int tile, kb0, kb1;
-    while (ok && work_next(p, num_pairs, nkb, wc, tile, kb0, kb1)) {
-      const int mb = tile % p.tiles_m, ft = tile / p.tiles_m;
-      const int g = group_of(a, ft);
+    while (ok && work_next<kDown>(p, num_pairs, nkb, wc, tile, kb0, kb1)) {
+      const TileId id = tile_id<kDown>(p, tile);
+      const int mb = id.mb, ft = id.ft, g = id.g;
       const int m0 = mb * kTile + static_cast<int>(rank) * kHalf;
+      // a down tile's B side: 64 rows of A_g per CTA
+      const uint32_t tx = id.down && !id.wide ? 3 * kHalfBytes : 2 * kStageBytes;
+      bool t_seen = !kDown;   // t of this token block is complete
       // B rows of this CTA's half: its 128 features of group g, or (silu) the
       // tile's 128 features of group `rank` (gate for CTA 0, up for CTA 1)
       const int gb = silu ? static_cast<int>(rank) : g;
       const int n0 = silu ? ft * kHalf : (ft - a.g[g].tile0) * kTile + static_cast<int>(rank) * kHalf;
       auto load_b = [&](int kb, uint32_t sb, uint32_t fb) {
-        if (kb < a.nkb_main) {
+        if (id.down) {   // wide: A_{g + rank}, all rows; else rows [64 rank, 64 rank + 64) of A_g
+          if (id.wide)
+            tma_load_2d_pair(sb, &tm.a[g + static_cast<int>(rank)], kb * 64, 0, fb);
+          else
+            tma_load_2d_pair(sb, &tm.a[g], kb * 64, static_cast<int>(rank) * (kHalf / 2), fb);
+        } else if (kb < a.nkb_main) {
           tma_load_2d_pair(sb, &tm.w[gb], kb * 64, n0, fb);
         } else {
           const int l = kb - a.nkb_main;
@@ -190,15 +252,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d_pair(sb, &tm.b[gb], j * 64, row, fb);
         }
       };
-      auto load_a = [&](int kb, uint32_t sa, uint32_t fb) {
+      auto load_a = [&](int kb, uint32_t sa, uint32_t fb) -> bool {
         if (kb < a.nkb_main) {
           tma_load_2d_pair(sa, &tm.x, kb * 64, m0, fb);
         } else {
+          if (!t_seen) {   // the down tiles of this token block wrote t with generic stores
+            if (!counter_wait(p.t_ready + mb, p.down_expect)) return false;
+            fence_proxy_async_global();
+            t_seen = true;
+          }
           const int l = kb - a.nkb_main;
           const int h = silu ? l / a.nkb_r : 0;
           const int j = silu ? l % a.nkb_r : l;
           tma_load_2d_pair(sa, &tm.t, a.g[silu ? h : g].t_col + j * 64, m0, fb);
         }
+        return true;
       };
       int kb_next = kb0;
       if (first) {
@@ -207,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pre = min(S, kb1 - kb0);
         for (int q = 0; q < pre; ++q) {
           const uint32_t sa = smem_u32(smem + q * kStageBytes);
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full[q]), 2 * kStageBytes);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[q]), tx);
           load_b(kb0 + q, sa + kHalfBytes, map_shared_rank(smem_u32(&full[q]), 0));
         }
         if (!a.x_ready) {
@@ -219,8 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             pdl_wait();
             waited = true;
           }
-          load_a(kb0 + q, smem_u32(smem + q * kStageBytes), map_shared_rank(smem_u32(&full[q]), 0));
+          if (!load_a(kb0 + q, smem_u32(smem + q * kStageBytes), map_shared_rank(smem_u32(&full[q]), 0))) {
+            fail();
+            ok = false;
+            break;
+          }
         }
+        if (!ok) break;
         it = pre;
         kb_next = kb0 + pre;
       }
@@ -233,13 +306,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t fb = map_shared_rank(smem_u32(&full[s]), 0);
-        if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * kStageBytes);
+        if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
         const uint32_t sa = smem_u32(smem + s * kStageBytes);
         if (!waited && kb >= a.nkb_main) {
           pdl_wait();
           waited = true;
         }
-        load_a(kb, sa, fb);
+        if (!load_a(kb, sa, fb)) {
+          fail();
+          ok = false;
+          break;
+        }
         load_b(kb, sa + kHalfBytes, fb);
       }
     }
@@ -247,11 +324,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer (leader)
     const uint32_t idesc = idesc_f32acc(kTile, kTile, false);
+    const uint32_t idesc_down = idesc_f32acc(kTile, kHalf, false);
     int it = 0, lt = 0;
     bool ok = true;
     WorkCursor wc = work_begin(p, pair, num_pairs);
     int tile, kb0, kb1;
-    for (; ok && work_next(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
+    for (; ok && work_next<kDown>(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
       const int b = lt & 1;
       const uint32_t aph = (lt >> 1) & 1u;
       if (!mbar_wait_cluster(smem_u32(&acce[b]), aph ^ 1u)) {
@@ -260,6 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t dacc = tmem + static_cast<uint32_t>(b * kAccCols);
+      const TileId id = tile_id<kDown>(p, tile);
+      const uint32_t id_k = id.down && !id.wide ? idesc_down : idesc;
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1u;
@@ -275,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_pair_bf16(dacc, ad + static_cast<uint64_t>(2 * kk), bd + static_cast<uint64_t>(2 * kk),
-                        idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                        id_k, (kb > kb0 || kk > 0) ? 1u : 0u);
         const uint32_t eb = smem_u32(&empty[s]);
         mma_commit_pair(map_shared_rank(eb, 0));
         mma_commit_pair(map_shared_rank(eb, 1));
@@ -292,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int lt = 0;
     WorkCursor wc = work_begin(p, pair, num_pairs);
     int tile, kb0, kb1;
-    for (; work_next(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
+    for (; work_next<kDown>(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
       const int b = lt & 1;
       const uint32_t aph = (lt >> 1) & 1u;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&accf[b]), aph));
@@ -301,12 +381,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int mb = tile % p.tiles_m, ft = tile / p.tiles_m;
-      const int g = group_of(a, ft);
+      const TileId id = tile_id<kDown>(p, tile);
+      const int mb = id.mb, ft = id.ft, g = id.g;
       const int m = mb * kTile + static_cast<int>(rank) * kHalf + i;
       const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                             static_cast<uint32_t>(b * kAccCols);
-      if (kb0 > 0) {
+      if (id.down) {
+        // t[m, g r + j] = scale * gate(m) * acc[128 (g - id.g) + j], j < r, in bf16
+        const float f = m < a.M ? a.scale * row_gate(a, m) : 0.f;
+        for (int gg = 0; gg < (id.wide ? 2 : 1); ++gg) {
+          __nv_bfloat16* dst = p.t + static_cast<size_t>(m) * p.ldt + a.g[g + gg].t_col;
+          for (int c = 0; c < p.r; c += 16) {
+            float v[16];
+            tmem_ld16(trow + static_cast<uint32_t>(gg * kHalf + c), v);
+            if (m < a.M) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                if (c + 8 * h >= p.r) break;
+                uint4 w;
+                w.x = pack_bf16x2(f * v[8 * h + 0], f * v[8 * h + 1]);
+                w.y = pack_bf16x2(f * v[8 * h + 2], f * v[8 * h + 3]);
+                w.z = pack_bf16x2(f * v[8 * h + 4], f * v[8 * h + 5]);
+                w.w = pack_bf16x2(f * v[8 * h + 6], f * v[8 * h + 7]);
+                *reinterpret_cast<uint4*>(dst + c + 8 * h) = w;
+              }
+            }
+          }
+        }
+        // t is read by the main tiles' bulk tensor copies (the async proxy)
+        fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) counter_add_release(p.t_ready + mb, 1);
+      } else if (kb0 > 0) {
         // second part of a stream-K tile: hand this warp's partial sum (its
         // 32 rows, all 256 columns) to the pair that holds the first part
         const int fi = ((pair - 1) * 2 + static_cast<int>(rank)) * 4 + quarter;
@@ -327,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // stage ring is idle): copy the next pair's partial sum for this
         // warp's rows into shared memory, then add it
         const float* part = nullptr;
-        if (kb1 < nkb) {
+        if (kb1 < nkb) {   // (down tiles took the branch above)
           const int fi = (pair * 2 + static_cast<int>(rank)) * 4 + quarter;
           pdl_wait();   // the flags were cleared by the preceding launch
           bool got = __all_sync(0xffffffffu, flag_wait(p.sk_flag + fi, 1));
@@ -417,18 +524,58 @@ size_t pair_sk_part_bytes() {
 
 size_t pair_sk_flag_bytes() { return static_cast<size_t>(pair_sk_slots()) * 2 * 4 * sizeof(int32_t); }
 
+size_t pair_t_ready_bytes(int64_t M) {
+  return static_cast<size_t>((M + kTile - 1) / kTile) * sizeof(int32_t);
+}
+
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
   const bool silu = pb.mode == kEpiSiluPair;
   const int tile_n = silu ? kHalf : kTile;
   PairParams pp{};
   pp.a = make_gemm_args(pb, tile_n, 128);
   pp.tiles_m = static_cast<int>((pb.M + kTile - 1) / kTile);
-  const int64_t tiles = static_cast<int64_t>(pp.tiles_m) * feature_tiles(pp.a, tile_n);
+  // t computed here: down tiles ahead of the main tiles, for 16 or more token
+  // blocks (M > 3840) when the down tiles fit in the pairs that the last round
+  // of main tiles leaves idle (same number of rounds). Same-box A/B on the
+  // Qwen3-8B-shaped step: 3 % faster at M = 4352 (B = 256), where every linear
+  // passes; taken at every M it was 3-4 % slower at M = 1088 and 2176. There
+  // the separate down-projection is short and hides under the previous
+  // launch's tail, while the main tiles of the first round wait for t here
+  // (~7 us: a down tile streams as long a K-loop as a main tile).
+  const int main_tiles = static_cast<int>(std::min<int64_t>(
+      static_cast<int64_t>(pp.tiles_m) * feature_tiles(pp.a, tile_n), 1ll << 30));
+  const int all_pairs = std::max(1, device_sm_count() / 2);
+  const int down_per_block = (pb.ngroups + 1) / 2;   // two groups per down tile
+  const int n_down = pp.tiles_m * down_per_block;
+  bool down = pb.t_ready && pb.t && pb.r > 0 && pb.r <= kHalf && pp.tiles_m >= 16 &&
+              (main_tiles + all_pairs - 1) / all_pairs ==
+                  (main_tiles + n_down + all_pairs - 1) / all_pairs;
+  for (int i = 0; i < pb.ngroups; ++i) down = down && pb.A[i];
+  if (down && reinterpret_cast<uintptr_t>(pb.t_ready) % 4)
+    return set_error(UNO_ERR_INVALID_ARG, "t counters must be 4-byte aligned");
+  pp.down_tiles = down ? n_down : 0;
+  pp.down_expect = 8 * down_per_block;               // 8 epilogue warps per down tile
+  pp.r = pb.r;
+  pp.ldt = static_cast<int>(pb.ldt);
+  pp.t = down ? static_cast<__nv_bfloat16*>(const_cast<void*>(pb.t)) : nullptr;
+  pp.t_ready = down ? pb.t_ready : nullptr;
+  if (down) pp.a.x_ready = 0;   // x comes from the launch right before
+  const int64_t tiles = static_cast<int64_t>(pp.tiles_m) * feature_tiles(pp.a, tile_n) + pp.down_tiles;
   if (tiles > (1ll << 30)) return set_error(UNO_ERR_UNSUPPORTED, "too many tiles");
   pp.num_tiles = static_cast<int>(tiles);
   pp.stages = 6;
   uno_status s;
   TensorMaps& tm = out->tm;
+  for (int i = 0; i < kMaxGroups; ++i) {
+    if (down) {   // A_g, rows >= r read zeros: 128 rows in one CTA (paired groups) or 64 in each
+      const bool single = i == pb.ngroups - 1 && pb.ngroups % 2 == 1;
+      if ((s = make_map(&tm.a[i], pb.dt, pb.A[i < pb.ngroups ? i : 0], pb.K, pb.r, pb.K,
+                        single ? kHalf / 2 : kHalf)) != UNO_OK)
+        return s;
+    } else {
+      std::memset(&tm.a[i], 0, sizeof(tm.a[i]));
+    }
+  }
   if ((s = make_map(&tm.x, pb.dt, pb.x, pb.K, pb.M, pb.K, kHalf)) != UNO_OK) return s;
   if (pb.r > 0) {
     if ((s = make_map(&tm.t, pb.dt, pb.t, pb.ldt, pb.M, pb.ldt, kHalf)) != UNO_OK) return s;
@@ -461,7 +608,7 @@ uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
   out->sk_flag = nullptr;
   out->sk_flag_bytes = 0;
   if (pb.sk_part && pb.sk_flag && pairs <= pb.sk_slots && rem > 0 && 5 * rem <= 4 * pairs &&
-      nkb >= 128) {
+      nkb >= 128 && pp.num_tiles - (pairs + rem) >= pp.down_tiles) {
     const int sk_tiles = pairs + rem;
     pp.dp_tiles = pp.num_tiles - sk_tiles;
     pp.sk_iters = static_cast<long long>(sk_tiles) * nkb;
@@ -470,6 +617,9 @@ uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
     out->sk_flag = pb.sk_flag;
     out->sk_flag_bytes = pair_sk_flag_bytes();
   }
+  out->computes_t = down;
+  out->t_ready = pp.t_ready;
+  out->t_ready_bytes = down ? pair_t_ready_bytes(pb.M) : 0;
   std::memcpy(out->params, &pp, sizeof(pp));
   out->kind = 1;
   out->swap = 0;
@@ -482,7 +632,10 @@ uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out) {
 }
 
 uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream) {
-  void* fn = reinterpret_cast<void*>(&gemm_pair_kernel);
+  PairParams pp;
+  std::memcpy(&pp, l.params, sizeof(pp));
+  void* fn = pp.down_tiles > 0 ? reinterpret_cast<void*>(&gemm_pair_kernel<true>)
+                               : reinterpret_cast<void*>(&gemm_pair_kernel<false>);
   cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, l.smem_bytes);
   if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute(pair smem)");
@@ -494,8 +647,6 @@ uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream) {
   cudaLaunchAttribute attr[2];
   cfg.numAttrs = launch_attrs(attr, 2, 1, 1);
   cfg.attrs = attr;
-  PairParams pp;
-  std::memcpy(&pp, l.params, sizeof(pp));
   void* args[2] = {const_cast<TensorMaps*>(&l.tm), &pp};
   e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e != cudaSuccess) return cuda_error(e, "pair GEMM launch");

@@ -475,6 +475,9 @@ int device_sm_count() {
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
   out->sk_flag = nullptr;
   out->sk_flag_bytes = 0;
+  out->t_ready = nullptr;
+  out->t_ready_bytes = 0;
+  out->computes_t = false;
   if (pb.ngroups < 1 || pb.ngroups > kMaxGroups)
     return set_error(UNO_ERR_INVALID_ARG, "1..3 output groups per GEMM launch");
   if (pb.mode == kEpiSiluPair && (pb.ngroups != 2 || pb.g[0].N != pb.g[1].N))

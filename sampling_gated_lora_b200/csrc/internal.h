@@ -70,10 +70,16 @@ struct GemmProblem {
   // down-projection clears the stream-K flags of the GEMM launched behind it.
   int32_t* zero_flags;
   int zero_words;
+  // Non-NULL: the CTA-pair kernel may compute t = scale * gate * (x A_g^T)
+  // itself (A[] and t above; r <= 128, 16 or more 256-row blocks, see
+  // gemm_pair_prepare), counting the finished parts of each 256-row block
+  // here: ceil(M / 256) words that are zero when the launch starts.
+  // GemmLaunch::computes_t tells the caller whether it does.
+  int32_t* t_ready;
 };
 
 // All tensor maps of one launch (passed to the kernel as one parameter).
-// a[] (the adapters' A matrices) is used by the fused decode kernel only.
+// a[] (the adapters' A matrices) is used by the kernels that compute t themselves.
 struct TensorMaps {
   CUtensorMap x, t, w[kMaxGroups], b[kMaxGroups], a[kMaxGroups];
 };
@@ -92,6 +98,9 @@ struct GemmLaunch {
   int dtype;
   int32_t* sk_flag;       // stream-K flags this launch reads: zero them before it runs (or NULL)
   size_t sk_flag_bytes;
+  int32_t* t_ready;       // the t counters (computes_t): zero them before it runs
+  size_t t_ready_bytes;
+  bool computes_t;        // the launch writes t itself: no separate down-projection
 };
 
 uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out);
@@ -107,6 +116,8 @@ bool gemm_pair_suits(const GemmProblem& pb);
 size_t pair_sk_part_bytes();
 size_t pair_sk_flag_bytes();
 int pair_sk_slots();
+// The t counters of a CTA-pair launch over M rows (GemmProblem::t_ready).
+size_t pair_t_ready_bytes(int64_t M);
 uno_status gemm_pair_prepare(const GemmProblem& pb, GemmLaunch* out);
 uno_status gemm_pair_run(const GemmLaunch& l, cudaStream_t stream);
 // The fused decode kernel (bf16, M <= 256, r <= 128): computes t = scale * gate

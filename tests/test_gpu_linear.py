@@ -121,6 +121,25 @@ def test_stream_k_flags_cleared_by_the_call(r):
         check_close(host_f64(y), ref, what=f"r={r} call {call}")
 
 
+@pytest.mark.parametrize("G", [1, 2, 3])
+def test_stale_workspace_grouped_calls(G):
+    """Grouped calls on the CTA-pair kernel with every workspace byte at 0x7f (stale
+    stream-K flags would never read "ready"), twice in a row: each call clears its flags
+    before the pairs use them. 1 to 3 groups of the qkv shapes, 16 token blocks."""
+    import torch
+    import sampling_gated_lora_b200 as U
+    M, K = 4000, 1024
+    Ns = (4096, 1024, 1024)[:G]
+    x, gate, cases = _group_case(M, K, Ns, 128, seed=40 + G)
+    refs = [_oracle_group(x, gate, c) for c in cases]
+    need = U.load().uno_gated_lora_linear_group_workspace(U.UNO_BF16, M, 128, G)
+    ws = torch.full((need,), 0x7F, dtype=torch.uint8, device="cuda")
+    for call in range(2):
+        ys = _run_group(x, gate, cases, False, workspace=ws)
+        for y, ref, c in zip(ys, refs, cases):
+            check_close(y, ref, what=f"G={G} N={c.N} call {call}")
+
+
 def test_stream_k_without_workspace_scratch():
     """r = 0: with the workspace the size query asks for, the pair kernel cuts tiles; with
     none it runs whole tiles only. Both match the oracle."""
@@ -167,12 +186,12 @@ def _group_case(M, K, Ns, r, seed, b_std=0.01):
     return x, gate, cases
 
 
-def _run_group(x, gate, cases, silu_pair):
+def _run_group(x, gate, cases, silu_pair, workspace=None):
     import sampling_gated_lora_b200 as U
     t = lambda a: dev_tensor(a, "bf16")
     ys = U.gated_lora_linear_group(t(x), [t(c.W) for c in cases], [t(c.A) for c in cases],
                                    [t(c.Bl) for c in cases], dev_tensor(gate, "u8"), 1.0,
-                                   silu_pair=silu_pair)
+                                   silu_pair=silu_pair, workspace=workspace)
     return [host_f64(y) for y in ys]
 
 
