@@ -18,6 +18,7 @@ Every step streams 15.1 GB of weights, far larger than the 126 MB L2.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -51,7 +52,7 @@ def parse():
     ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
     ap.add_argument("--no-kernels", action="store_true", help="skip the per-config kernel lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
-    ap.add_argument("--profile", choices=["gemm_up", "gemm_small", "verify", "draft"],
+    ap.add_argument("--profile", choices=["gemm_up", "gemm_small", "step_up", "verify", "draft"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
@@ -303,8 +304,9 @@ def kernel_lines(U, torch, pk):
             "TFLOPs": round(flops / us / 1e6, 1), "roofline_us": round(t_roof, 2),
             "frac_of_roofline": round(t_roof / us, 3), "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3)}
         del sets
-    for name, K, N in (("up", 4096, 12288), ("down", 12288, 4096)):
-        M, r = 2048, 128
+    for name, K, N, M in (("up", 4096, 12288, 2048), ("down", 12288, 4096, 2048),
+                          ("up", 4096, 12288, 4352)):
+        r = 128
         sets = [(dev((N, K), K ** -0.5), dev((r, K), K ** -0.5), dev((N, r), 0.01)) for _ in range(3)]
         x = dev((M, K), 1)
         g = torch.cat([torch.zeros(M // 2, dtype=torch.uint8), torch.ones(M // 2, dtype=torch.uint8)]).cuda()
@@ -317,7 +319,7 @@ def kernel_lines(U, torch, pk):
         single = timed(calls[0], reps=10)
         us = chained(calls)
         flops = 2 * M * K * N + 2 * (M // 2) * r * (K + N)
-        out[f"gated_linear_mlp_{name}_M2048"] = {
+        out[f"gated_linear_mlp_{name}_M{M}"] = {
             "us": round(us, 2), "single_us": round(single, 2), "TFLOPs": round(flops / us / 1e6, 1),
             "tensor_frac": round(flops / us / 1e6 / pk["bf16_tflops"], 3)}
         del sets
@@ -479,9 +481,10 @@ def run_uno(args):
     ws = torch.empty(model.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
     B, seq_off = shard(B, rank)
 
-    def step(t):
+    def step(t):   # outputs of step t in row t % n_total (steps past the timed ones reuse rows)
+        i = t % n_total
         model.step(B, k, h, qb[t % 2], db[t % 2], T, 2026, t, qb[(t + 1) % 2], db[(t + 1) % 2],
-                   acc[t], tok[t], cnt[t], ws, dev_status=status, seq_offset=seq_off)
+                   acc[i], tok[i], cnt[i], ws, dev_status=status, seq_offset=seq_off)
 
     def barrier():
         if world > 1:
@@ -536,48 +539,11 @@ def run_uno(args):
            "h2d_bytes_per_step": h_host.numel() * 2,
            "d2h_bytes_per_step": (acc_h[0].numel() + tok_h[0].numel() + cnt_h[0].numel()) * 4}
 
-    # dominant kernel: the gated linear of the MLP up projection at this step's M
-    # (gate/up/down carry 78 % of the step's flops), timed alone with events.
+    # dominant kernel: the launch of the step with the largest share of its time,
+    # timed inside the step (CUDA events after every launch of a few extra steps)
     roof = None
     if rank == 0:
-        Kd, Nd, r = shape.hidden, shape.inter, shape.r
-        x = torch.randn((M, Kd), device="cuda").to(torch.bfloat16)
-        lw = layers[0]["up"]
-        g = torch.from_numpy(W.step_gate(B, k)).cuda()
-        y = torch.empty((M, Nd), dtype=torch.bfloat16, device="cuda")
-        wsl = torch.zeros(U.load().uno_gated_lora_linear_workspace(0, M, Kd, Nd, r),
-                          dtype=torch.uint8, device="cuda")
-        f = lambda: U.gated_lora_linear(x, lw[0], lw[1], lw[2], g, 1.0, y=y, workspace=wsl)
-        for _ in range(3):
-            f()
-        reps = 20
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            f()
-        b.record()
-        b.synchronize()
-        us = a.elapsed_time(b) * 1e3 / reps
-        Mg = B * k
-        flops = 2 * M * Kd * Nd + 2 * Mg * r * (Kd + Nd)
-        byts = 2 * (Nd * Kd + r * Kd + Nd * r + M * Kd + M * Nd)
-        tensor_bound = flops / (pk["bf16_tflops"] * 1e12) > byts / (pk["hbm_gbs"] * 1e9)
-        if tensor_bound:
-            ach = flops / us / 1e6
-            roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 3), "traffic": None,
-                    "peak_sustained": pk["bf16_tflops_sustained"],
-                    "frac_sustained": round(ach / pk["bf16_tflops_sustained"], 3)}
-        else:
-            ach = byts / us / 1e3
-            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(ach / pk["hbm_gbs"], 3), "traffic": None}
-        kname = f"gated_lora_linear up 4096->12288 M={M} (LoRA down + fused GEMM)"
-        roof["traffic"] = recorded_traffic(kname)
-        roof.update({"kernel": kname,
-                     "us_per_launch": round(us, 2), "peak_source": pk_src + " burst",
-                     "algorithmic_flops": flops, "algorithmic_bytes": byts})
-        del x, y
+        roof = step_roofline(model, step, n_total + args.steps, shape, B, k, pk, pk_src)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -620,6 +586,67 @@ def run_uno(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# (N, K) of the step's linears -> (name, groups, output width)
+def linear_names(shape):
+    return {(shape.q_out + 2 * shape.kv_out, shape.hidden): ("qkv", 3, shape.q_out + 2 * shape.kv_out),
+            (shape.hidden, shape.q_out): ("o", 1, shape.hidden),
+            (2 * shape.inter, shape.hidden): ("gate/up silu pair", 2, shape.inter),
+            (shape.hidden, shape.inter): ("down", 1, shape.hidden),
+            (shape.vocab, shape.hidden): ("LM head", 1, shape.vocab)}
+
+
+def launch_work(shape, B, k, kind, dims):
+    """Algorithmic flops and bytes of one GEMM launch of the step: x W^T over all M rows,
+    the adapter (x A^T, t Bl^T) over the B k gated rows; bytes = W, A, Bl, x, y once (y
+    also read when the launch adds into it), t not counted (it stays on chip or in L2)."""
+    M, N, K, mode = dims
+    name, G, n_out = linear_names(shape).get((N, K), ("?", 1, N))
+    r, Mg = shape.r, B * k
+    flops = 2 * M * N * K + 2 * Mg * r * (G * K + N)
+    byts = 2 * (N * K + G * r * K + N * r + M * K + M * n_out * (2 if mode == 1 else 1))
+    return name, flops, byts
+
+
+def step_roofline(model, step, t0, shape, B, k, pk, pk_src, n_prof=3):
+    """Roofline line of the step's dominant launch: per (kind, shape) group of launches
+    the summed in-step time over n_prof profiled steps; the largest group's average launch
+    time against its algorithmic work."""
+    groups = {}
+    model.profile(True)
+    for i in range(n_prof):
+        step(t0 + i)
+        for kind, ms, dims in model.last_profile():
+            g = groups.setdefault((kind, dims), [0.0, 0])
+            g[0] += ms
+            g[1] += 1
+    model.profile(False)
+    total = sum(v[0] for v in groups.values())
+    (kind, dims), (ms_sum, n) = max(groups.items(), key=lambda kv: kv[1][0])
+    us = ms_sum / n * 1e3
+    name, flops, byts = launch_work(shape, B, k, kind, dims)
+    tensor_bound = flops / (pk["bf16_tflops"] * 1e12) > byts / (pk["hbm_gbs"] * 1e9)
+    # timed inside a long step: the sustained peak (the burst one for context)
+    if tensor_bound:
+        ach = flops / us / 1e6
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops_sustained"], 3),
+                "traffic": None, "peak_burst": pk["bf16_tflops"],
+                "frac_burst": round(ach / pk["bf16_tflops"], 3)}
+    else:
+        ach = byts / us / 1e3
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 3), "traffic": None}
+    M, N, K, _ = dims
+    kname = f"{kind} {name} {K}->{N} M={M}, in the step"
+    roof["traffic"] = recorded_traffic(kname)
+    roof.update({"kernel": kname, "us_per_launch": round(us, 2), "launches_per_step": n // n_prof,
+                 "share_of_step": round(ms_sum / total, 3),
+                 "timing": f"CUDA events after every launch of {n_prof} extra steps",
+                 "peak_source": pk_src + (" sustained" if tensor_bound else ""),
+                 "algorithmic_flops": flops, "algorithmic_bytes": byts})
+    return roof
 
 
 def sweep_point(U, torch, W, model, B, k, T, V, shape):
@@ -697,6 +724,10 @@ def run_profile(args):
     """A few launches of one hot kernel on a small case, for an ncu capture.
 
     gemm_up:    gated linear 4096 -> 12288, M = B(2k+1) rows (the step's MLP shape)
+    step_up:    two steps of a 1-layer Qwen3-8B-shaped model at B (M = B(2k+1)); with
+                M > 3840 each step runs 5 CTA-pair launches (qkv, o, the gate/up silu
+                pair computing t itself, down, LM head): launch 7 is the second
+                step's silu pair
     gemm_small: gated linear 4096 -> 4096, M = 9 (split-K cluster path)
     verify:     psi_verify B=32, k=16, V=151936 (311 MB of logits)
     draft:      draft sampler B=32, k=8, V=151936
@@ -706,6 +737,26 @@ def run_profile(args):
     import workloads as W
     torch.cuda.set_device(0)
     dev = lambda shape, std: (torch.randn(shape, device="cuda") * std).to(torch.bfloat16)
+    if args.profile == "step_up":
+        shape = dataclasses.replace(W.QWEN3_8B_SHAPE, n_layers=1)
+        layers, head = W.model_weights_torch(shape, "cuda", seed=0)
+        m = U.Model(layers, head, shape.hidden, shape.q_out, shape.kv_out, shape.inter,
+                    shape.vocab, shape.r, shape.scale)
+        B, k, V = args.B, args.k, shape.vocab
+        i32 = dict(dtype=torch.int32, device="cuda")
+        h = W.to_torch_bf16(W.step_hidden(B, k, shape.hidden, seed=7), "cuda")
+        qb = [torch.zeros((B, k, V), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        db = [torch.zeros((B, k), **i32) for _ in range(2)]
+        acc, tok, cnt = torch.empty(B, **i32), torch.empty((B, k + 1), **i32), torch.empty(B, **i32)
+        ws = torch.empty(m.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
+        for t in range(2):
+            m.step(B, k, h, qb[t % 2], db[t % 2], 1.0, 5, t, qb[(t + 1) % 2], db[(t + 1) % 2], acc,
+                   tok, cnt, ws)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": args.profile, "status": U.device_status(),
+                          "launches_per_step": m.kernel_count(B, k)}))
+        m.close()
+        return
     if args.profile in ("gemm_up", "gemm_small"):
         M, K, N = ((args.B * (2 * args.k + 1), 4096, 12288) if args.profile == "gemm_up"
                    else (9, 4096, 4096))

@@ -428,6 +428,31 @@ uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h
  * 0 until such a step has been run (the launch plan is built on first use). */
 int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k);
 
+/* Launch timing of uno_psi_step (a library addition for measurement; the
+ * pages have no counterpart). With enable != 0, every later uno_psi_step on
+ * this model records a CUDA event on its stream before its first launch and
+ * after each launch of its plan, after the verification's two kernels and
+ * after the draft's two; uno_model_last_profile then waits for the last
+ * profiled step and reports, per entry i in launch order:
+ *   ms[i]    the time between the event before and the event after it (the
+ *            time the entry adds to the stream; the events themselves can
+ *            cost some of the overlap between consecutive launches);
+ *   kind[i]  0 one-CTA GEMM, 1 CTA-pair GEMM, 2 CTA-pair GEMM that computes
+ *            the LoRA activations t itself, 3 fused decode-size GEMM,
+ *            10 RMSNorm, 11 RMSNorm + LoRA down-projection,
+ *            20 verification (stats + finalize), 21 draft (stats + draw);
+ *   dims[4i .. 4i+3] (optional, may be NULL) for GEMMs: M, the summed N of
+ *            its output groups, K and the epilogue mode (0 store, 1 residual
+ *            add, 2 gated down-projection, 3 silu pair); zeros otherwise.
+ * *n_out receives the number of entries (0 before a profiled step); with
+ * ms == NULL nothing else is written (a count query); otherwise cap is the
+ * length of ms and kind (dims: 4 cap) and must hold every entry. Events are created on the device
+ * of the first profiled step; profiled steps and the read must use that
+ * device (UNO_ERR_INVALID_ARG otherwise). enable = 0 stops recording. */
+uno_status uno_model_profile(uno_model* m, int32_t enable);
+uno_status uno_model_last_profile(uno_model* m, int32_t cap, float* ms, int32_t* kind,
+                                  int64_t* dims, int32_t* n_out);
+
 /* ---------------------------------------------------------------------------
  * Self-test of the bounded waits (a library addition; the pages have no
  * counterpart). Every spin in the library's kernels gives up after a time

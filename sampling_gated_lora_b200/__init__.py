@@ -35,7 +35,8 @@ EXPORTS = [
     "uno_tree_verify_workspace", "uno_tree_verify",
     "uno_philox_uniforms",
     "uno_model_create", "uno_model_destroy", "uno_psi_step_workspace", "uno_psi_step",
-    "uno_psi_step_hidden", "uno_psi_step_kernel_count",
+    "uno_psi_step_hidden", "uno_psi_step_kernel_count", "uno_model_profile",
+    "uno_model_last_profile",
     "uno_rmsnorm", "uno_silu_mul", "uno_wait_selftest",
     "uno_vp_partials", "uno_vp_verify_decide", "uno_vp_draw_masses", "uno_vp_draw",
     "uno_vp_draft_draw",
@@ -95,6 +96,8 @@ def load():
                                vp, vp, vp, sz, vp]),
         "uno_psi_step_hidden": (i32, [vp, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
         "uno_psi_step_kernel_count": (i32, [vp, i32, i32]),
+        "uno_model_profile": (i32, [vp, i32]),
+        "uno_model_last_profile": (i32, [vp, i32, vp, vp, vp, vp]),
         "uno_rmsnorm": (i32, [i64, i64, vp, vp, f32, vp]),
         "uno_silu_mul": (i32, [i64, vp, vp, vp, vp]),
         "uno_wait_selftest": (i32, [i32, u64, vp, vp, vp]),
@@ -564,6 +567,30 @@ class Model:
     def kernel_count(self, B, k):
         """Kernel launches issued by one step for (B, k) (0 before the first such step)."""
         return load().uno_psi_step_kernel_count(self._h, B, k)
+
+    PROFILE_KINDS = {0: "gemm_one_cta", 1: "gemm_pair", 2: "gemm_pair_computes_t",
+                     3: "gemm_decode", 10: "rmsnorm", 11: "rmsnorm_down", 20: "verify",
+                     21: "draft"}
+
+    def profile(self, enable=True):
+        """uno_model_profile: time every launch of the following steps with CUDA events."""
+        _check(load().uno_model_profile(self._h, 1 if enable else 0))
+
+    def last_profile(self):
+        """uno_model_last_profile: [(kind name, ms, (M, N, K, mode))] of the last profiled step,
+        in launch order (waits for that step)."""
+        L = load()
+        n = ctypes.c_int32(0)
+        _check(L.uno_model_last_profile(self._h, 0, None, None, None, ctypes.byref(n)))
+        cap = n.value
+        if cap == 0:
+            return []
+        ms = (ctypes.c_float * cap)()
+        kind = (ctypes.c_int32 * cap)()
+        dims = (ctypes.c_int64 * (4 * cap))()
+        _check(L.uno_model_last_profile(self._h, cap, ms, kind, dims, ctypes.byref(n)))
+        return [(self.PROFILE_KINDS.get(kind[i], str(kind[i])), float(ms[i]),
+                 tuple(int(d) for d in dims[4 * i: 4 * i + 4])) for i in range(n.value)]
 
     def hidden_state(self, B, k, h_in, n_blocks, workspace, h_out=None, inter=False, stream=None):
         """uno_psi_step_hidden: the step's hidden state after its first n_blocks residual

@@ -726,7 +726,36 @@ struct StepOp {
   const void* x;
   void* y;
   NormDownArgs nd;
+  int64_t dims[4];     // M, total N, K, epilogue mode (GEMMs; what uno_model_last_profile reports)
 };
+
+// Launch kinds of uno_model_last_profile.
+enum ProfKind : int32_t {
+  kProfGemmOne = 0,      // one-CTA tcgen05 GEMM (down-projections, mid-size batches)
+  kProfGemmPair = 1,     // CTA-pair GEMM
+  kProfGemmPairT = 2,    // CTA-pair GEMM that computes t itself
+  kProfGemmDecode = 3,   // fused decode-size GEMM
+  kProfNorm = 10,        // RMSNorm
+  kProfNormDown = 11,    // RMSNorm + LoRA down-projection
+  kProfVerify = 20,      // row stats + verify finalize
+  kProfDraft = 21,       // draft stats + draft draw
+};
+
+int32_t prof_kind(const StepOp& op) {
+  if (op.kind == 1) return kProfNorm;
+  if (op.kind == 2) return kProfNormDown;
+  if (op.gemm.kind == 1) return op.gemm.computes_t ? kProfGemmPairT : kProfGemmPair;
+  return op.gemm.kind == 2 ? kProfGemmDecode : kProfGemmOne;
+}
+
+void set_dims(StepOp* op, const GemmProblem& pb) {
+  int64_t n = 0;
+  for (int i = 0; i < pb.ngroups; ++i) n += pb.g[i].N;
+  op->dims[0] = pb.M;
+  op->dims[1] = n;
+  op->dims[2] = pb.K;
+  op->dims[3] = pb.mode;
+}
 
 // Decode-size batches fold the LoRA down-projection of an input that an
 // RMSNorm produces into that RMSNorm's launch (one launch instead of two).
@@ -751,6 +780,23 @@ struct uno_model {
   };
   std::mutex mu;
   std::vector<std::unique_ptr<Plan>> plans;   // most recently used last
+
+  // Launch timing (uno_model_profile): an event after each launch of a step.
+  bool profiling = false;
+  int prof_device = -1;
+  std::vector<cudaEvent_t> events;
+  std::vector<int32_t> prof_kinds;
+  std::vector<int64_t> prof_dims;
+  size_t prof_n = 0;   // events recorded by the last profiled step (launches + 1)
+
+  ~uno_model() {
+    if (events.empty()) return;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (prof_device >= 0) cudaSetDevice(prof_device);
+    for (cudaEvent_t e : events) cudaEventDestroy(e);
+    if (cur >= 0) cudaSetDevice(cur);
+  }
 
   const void* wp(int layer, int i, int part) const {
     return w[static_cast<size_t>(layer * uno::kLinPerLayer + i) * 3 + part];
@@ -829,6 +875,7 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
   auto gemm = [&](const GemmProblem& pb) -> uno_status {
     StepOp op{};
     op.kind = 0;
+    set_dims(&op, pb);
     const uno_status s = gemm_prepare(pb, &op.gemm);
     if (s == UNO_OK) P->ops.push_back(op);
     return s;
@@ -886,6 +933,7 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     }
     StepOp op{};
     op.kind = 0;
+    set_dims(&op, pm);
     if ((s = gemm_prepare(pm, &op.gemm)) != UNO_OK) return s;
     if (pm.x_ready && !op.gemm.computes_t &&
         (s = gemm(down_problem(UNO_BF16, M, K, r, x, As, G, nullptr, Mv, m->scale, t))) != UNO_OK)
@@ -1084,11 +1132,41 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   if (e != cudaSuccess) return cuda_error(e, "copying h_in");
   if (L.sk_flag_bytes && (e = cudaMemsetAsync(base + L.sk_flag, 0, L.sk_flag_bytes, st)) != cudaSuccess)
     return cuda_error(e, "clearing the stream-K flags");
+  // launch timing: event 0 before the first launch, event i + 1 after launch i
+  const size_t n_ev = P->ops.size() + 3;
+  const bool prof = m->profiling;
+  if (prof) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (m->prof_device >= 0 && m->prof_device != dev)
+      return set_error(UNO_ERR_INVALID_ARG, "profiling on device %d, step on device %d",
+                       m->prof_device, dev);
+    m->prof_device = dev;
+    while (m->events.size() < n_ev) {
+      cudaEvent_t ev;
+      if ((e = cudaEventCreate(&ev)) != cudaSuccess) return cuda_error(e, "creating a timing event");
+      m->events.push_back(ev);
+    }
+    m->prof_kinds.clear();
+    m->prof_dims.clear();
+    m->prof_n = 0;
+    if ((e = cudaEventRecord(m->events[0], st)) != cudaSuccess) return cuda_error(e, "recording an event");
+  }
+  auto mark = [&](int32_t kind, const int64_t* dims) -> uno_status {
+    if (!prof) return UNO_OK;
+    m->prof_kinds.push_back(kind);
+    for (int i = 0; i < 4; ++i) m->prof_dims.push_back(dims ? dims[i] : 0);
+    const cudaError_t er = cudaEventRecord(m->events[m->prof_kinds.size()], st);
+    if (er != cudaSuccess) return cuda_error(er, "recording an event");
+    m->prof_n = m->prof_kinds.size() + 1;
+    return UNO_OK;
+  };
   for (const StepOp& op : P->ops) {
     s = op.kind == 0 ? gemm_run(op.gemm, st)
         : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st)
                        : norm_down_launch(op.nd, M, st);
     if (s != UNO_OK) return s;
+    if ((s = mark(prof_kind(op), op.kind == 0 ? op.dims : nullptr)) != UNO_OK) return s;
   }
 
   VerifyArgs va{};
@@ -1109,6 +1187,7 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   va.out_count = out_count;
   va.dev_status = dev_status;
   if ((s = verify_launch(va, base + L.vstat, st)) != UNO_OK) return s;
+  if ((s = mark(kProfVerify, nullptr)) != UNO_OK) return s;
 
   DraftArgs da{};
   da.dt = UNO_BF16;
@@ -1122,7 +1201,41 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   da.seq_offset = seq_offset;
   da.draft = d_next;
   da.dev_status = dev_status;
-  return draft_launch(da, base + L.dstat, st);
+  if ((s = draft_launch(da, base + L.dstat, st)) != UNO_OK) return s;
+  return mark(kProfDraft, nullptr);
+}
+
+uno_status uno_model_profile(uno_model* m, int32_t enable) {
+  if (!m) return set_error(UNO_ERR_INVALID_ARG, "model is NULL");
+  std::lock_guard<std::mutex> lock(m->mu);
+  m->profiling = enable != 0;
+  m->prof_n = 0;
+  return UNO_OK;
+}
+
+uno_status uno_model_last_profile(uno_model* m, int32_t cap, float* ms, int32_t* kind,
+                                  int64_t* dims, int32_t* n_out) {
+  if (!m || !n_out) return set_error(UNO_ERR_INVALID_ARG, "model or n_out is NULL");
+  std::lock_guard<std::mutex> lock(m->mu);
+  const int32_t n = m->prof_n > 0 ? static_cast<int32_t>(m->prof_n - 1) : 0;
+  *n_out = n;
+  if (n == 0 || !ms) return UNO_OK;   // ms == NULL: the count only
+  if (cap < n || !kind) return set_error(UNO_ERR_INVALID_ARG, "cap=%d below the %d entries", cap, n);
+  int cur = -1;
+  cudaGetDevice(&cur);
+  if (m->prof_device >= 0 && (cur != m->prof_device))
+    return set_error(UNO_ERR_INVALID_ARG, "read the profile on device %d", m->prof_device);
+  cudaError_t e = cudaEventSynchronize(m->events[static_cast<size_t>(n)]);
+  if (e != cudaSuccess) return cuda_error(e, "waiting for the profiled step");
+  for (int32_t i = 0; i < n; ++i) {
+    if ((e = cudaEventElapsedTime(&ms[i], m->events[static_cast<size_t>(i)],
+                                  m->events[static_cast<size_t>(i) + 1])) != cudaSuccess)
+      return cuda_error(e, "reading a timing event");
+    kind[i] = m->prof_kinds[static_cast<size_t>(i)];
+    if (dims)
+      for (int j = 0; j < 4; ++j) dims[4 * i + j] = m->prof_dims[static_cast<size_t>(4 * i + j)];
+  }
+  return UNO_OK;
 }
 
 uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h_in,

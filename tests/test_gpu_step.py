@@ -118,3 +118,48 @@ def test_zero_adapter_step_accepts_its_own_drafts():
     acc, tok, cnt = U.psi_verify(p[:, 1:].contiguous(), buf["q_next"], buf["d_next"], 1.0, 3, 1)
     assert np.all(acc.cpu().numpy() == k)
     m.close()
+
+
+@pytest.mark.parametrize("B", [2, 40])
+def test_launch_profile(B):
+    """uno_model_profile / uno_model_last_profile: one entry per launch of the plan plus
+    the verification and the draft, GEMM entries carrying the step's M, the entries adding
+    up to the time between events around the whole step, and a step's results unchanged by
+    profiling (same tokens and draft as an unprofiled step on the same inputs)."""
+    import torch
+    import sampling_gated_lora_b200 as U
+    shape, k = W.TINY_SHAPE, 4
+    m, _, _ = _model(shape, seed=6)
+    V, M = shape.vocab, B * (2 * k + 1)
+    h = dev_tensor(W.step_hidden(B, k, shape.hidden, seed=7), "bf16")
+    gen = torch.Generator(device="cuda").manual_seed(8)
+    q0 = (2.0 * torch.randn((B, k, V), generator=gen, device="cuda")).to(torch.bfloat16)
+    d0 = dev_tensor(W.draft_ids(B, k, V, seed=9), "i32")
+    ws = torch.empty(m.workspace_bytes(B, k), dtype=torch.uint8, device="cuda")
+    outs = []
+    for prof in (False, True):
+        m.profile(prof)
+        buf = _buffers(B, k, V)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        m.step(B, k, h, q0, d0, 1.0, 11, 2, buf["q_next"], buf["d_next"], buf["acc"], buf["tok"],
+               buf["cnt"], ws)
+        b.record()
+        b.synchronize()
+        outs.append((buf["tok"].cpu().numpy(), buf["cnt"].cpu().numpy(), buf["d_next"].cpu().numpy(),
+                     a.elapsed_time(b)))
+    prof = m.last_profile()
+    assert len(prof) == m.kernel_count(B, k) - 2          # verify and draft: two kernels each
+    kinds = [p[0] for p in prof]
+    assert kinds[-2:] == ["verify", "draft"]
+    assert kinds.count("rmsnorm") + kinds.count("rmsnorm_down") == 2 * shape.n_layers + 1
+    for name, ms, dims in prof:
+        assert ms >= 0.0
+        if name.startswith("gemm"):
+            assert dims[0] == M and dims[1] > 0 and dims[2] in (shape.hidden, shape.q_out, shape.inter)
+    total = sum(p[1] for p in prof)
+    assert 0.3 * outs[1][3] <= total <= 1.05 * outs[1][3], (total, outs[1][3])
+    for x, y in zip(outs[0][:3], outs[1][:3]):
+        np.testing.assert_array_equal(x, y)
+    m.profile(False)
+    m.close()
