@@ -65,7 +65,7 @@ float make_scale(float temperature) {
 }
 
 template <typename T>
-struct Vec;   // 16-byte vector of logits
+struct Vec;   // 16-byte vector of logits (global-memory loads through the read-only path)
 template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int n = 8;
@@ -266,6 +266,138 @@ __global__ void __launch_bounds__(kStatThreads)
     st.pad = 0.f;
     st.s = acc;
     stats[w] = st;
+  }
+}
+
+// The same statistics, with the chunks staged in shared memory by bulk
+// copies (rows whose byte length is a multiple of 16 and a 16-byte aligned
+// base): a persistent grid of one CTA per SM, each of its kStagedWarps warps
+// walking the chunks w, w + W, ... (W = all warps of the grid) with a private
+// ring of kDraftSlots slots. Lane 0 keeps the ring's next copies in flight
+// (an mbarrier per slot), so an SM has kStagedWarps * kDraftSlots chunks of
+// loads outstanding while its warps compute. A warp reads its slot twice
+// (the max, then the sums), one 16-byte vector per lane at a time, so a
+// thread holds a few registers and many warps fit beside the copies. A slot
+// is refilled only after the warp has read it (an async-proxy fence orders
+// the reads before the copy). Waits are bounded: on a timeout the warp
+// records UNO_DEV_TIMEOUT, waits (bounded) for its copies still in flight
+// and stops.
+constexpr int kStagedWarps = 24;
+constexpr int kStagedThreads = kStagedWarps * 32;
+constexpr int kDraftSlots = 2;
+constexpr uint32_t kDraftSlotBytes = kSubLen * 2;   // one bf16 chunk (4 KB)
+
+__device__ __forceinline__ void unpack8(const uint4 w, float (&v)[8]) {
+  v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+  v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+}
+
+__global__ void __launch_bounds__(kStagedThreads, 1)
+    draft_stats_staged_kernel(const __nv_bfloat16* __restrict__ z_all, int rows, int V, int nsub,
+                              TScale c, DraftStat* __restrict__ stats, int32_t* status) {
+  extern __shared__ __align__(128) uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t bars[kStagedWarps][kDraftSlots];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint8_t* ring = dsmem + static_cast<size_t>(warp) * kDraftSlots * kDraftSlotBytes;
+  const int64_t units = static_cast<int64_t>(rows) * nsub;
+  const int64_t W = static_cast<int64_t>(gridDim.x) * kStagedWarps;
+  const int64_t w0 = static_cast<int64_t>(blockIdx.x) * kStagedWarps + warp;
+  if (lane == 0) {
+    for (int q = 0; q < kDraftSlots; ++q) mbar_init(smem_u32(&bars[warp][q]), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  // unit u -> (row, chunk, ids) and its copy into slot q
+  auto issue = [&](int64_t u, int q) {
+    const int row = static_cast<int>(u / nsub);
+    const int sc = static_cast<int>(u - static_cast<int64_t>(row) * nsub);
+    const int lo = sc * kSubLen;
+    const int len = min(V, lo + kSubLen) - lo;
+    const uint32_t bytes = static_cast<uint32_t>(len) * 2u;
+    const uint32_t bar = smem_u32(&bars[warp][q]);
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(smem_u32(ring + static_cast<size_t>(q) * kDraftSlotBytes),
+              z_all + static_cast<size_t>(row) * V + lo, bytes, bar);
+  };
+  if (lane == 0)
+    for (int q = 0; q < kDraftSlots; ++q)
+      if (w0 + q * W < units) issue(w0 + q * W, q);
+  constexpr int kPerLane = kSubLen / 8 / 32;   // 16-byte vectors per lane
+  int it = 0;
+  bool ok = true;
+  for (int64_t u = w0; u < units; u += W, ++it) {
+    const int q = it % kDraftSlots;
+    const uint32_t phase = static_cast<uint32_t>(it / kDraftSlots) & 1u;
+    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars[warp][q]), phase));
+    if (!ok) break;
+    const int row = static_cast<int>(u / nsub);
+    const int sc = static_cast<int>(u - static_cast<int64_t>(row) * nsub);
+    const int len = min(V, sc * kSubLen + kSubLen) - sc * kSubLen;
+    const __nv_bfloat16* slot =
+        reinterpret_cast<const __nv_bfloat16*>(ring + static_cast<size_t>(q) * kDraftSlotBytes);
+    // 16-byte vector k of this lane from the slot (shared-memory loads), -inf past the chunk
+    auto vec = [&](int k, float (&v)[8]) {
+      const int e = (lane + k * 32) * 8;
+      if (e + 8 <= len) {
+        unpack8(*reinterpret_cast<const uint4*>(slot + e), v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = e + j < len ? to_f32<__nv_bfloat16>(slot[e + j]) : -INFINITY;
+      }
+    };
+    float m = -INFINITY;
+    bool nan = false;
+#pragma unroll
+    for (int k = 0; k < kPerLane; ++k) {
+      float v[8];
+      vec(k, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        nan |= isnan(v[j]);
+        m = fmaxf(m, v[j]);
+      }
+    }
+    m = warp_max(m);
+    nan = __any_sync(0xffffffffu, nan);
+    double acc = 0.0;
+    if (m != -INFINITY) {
+#pragma unroll
+      for (int k = 0; k < kPerLane; ++k) {
+        float v[8];
+        vec(k, v);
+        float part = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part += fast_exp2((v[j] - m) * c);
+        acc += static_cast<double>(part);
+      }
+    }
+    // every lane has read the slot: it may be refilled
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && u + static_cast<int64_t>(kDraftSlots) * W < units)
+      issue(u + static_cast<int64_t>(kDraftSlots) * W, q);
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      DraftStat st;
+      st.m = nan ? NAN : m;
+      st.pad = 0.f;
+      st.s = acc;
+      stats[u] = st;
+    }
+  }
+  if (!ok) {
+    // the copies this warp still has in flight land before it leaves
+    if (lane == 0) {
+      raise_status(status, kDevTimeout);
+      int k = it;
+      for (int64_t u = w0 + static_cast<int64_t>(it) * W; u < units && k < it + kDraftSlots;
+           u += W, ++k)
+        (void)mbar_wait(smem_u32(&bars[warp][k % kDraftSlots]),
+                        static_cast<uint32_t>(k / kDraftSlots) & 1u);
+    }
+    __syncwarp();
   }
 }
 
@@ -1720,8 +1852,21 @@ uno_status draft_launch(const DraftArgs& a, void* ws, cudaStream_t s) {
       e = launch_kernel(draft_draw_kernel<float>, dim3(rows), dim3(kDrawThreads), 0, s, 1, q, dp);
   } else {
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_logits);
-    e = launch_kernel(draft_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1, q,
-                      rows, a.V, chunks, c, stats);
+    const bool staged = (reinterpret_cast<uintptr_t>(q) & 15u) == 0 && a.V % 8 == 0;
+    if (staged) {
+      const uint32_t smem = kStagedWarps * kDraftSlots * kDraftSlotBytes;
+      const int64_t per_cta = kStagedWarps;
+      const int ctas = static_cast<int>(std::max<int64_t>(
+          1, std::min<int64_t>(device_sm_count(), (warps + per_cta - 1) / per_cta)));
+      e = cudaFuncSetAttribute(draft_stats_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+      if (e == cudaSuccess)
+        e = launch_kernel(draft_stats_staged_kernel, dim3(ctas), dim3(kStagedThreads), smem, s, 1, q,
+                          rows, a.V, chunks, c, stats, a.dev_status);
+    } else {
+      e = launch_kernel(draft_stats_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, 1, q,
+                        rows, a.V, chunks, c, stats);
+    }
     if (e == cudaSuccess)
       e = launch_kernel(draft_draw_kernel<__nv_bfloat16>, dim3(rows), dim3(kDrawThreads), 0, s, 1,
                         q, dp);
