@@ -439,7 +439,9 @@ int32_t uno_psi_step_kernel_count(const uno_model* m, int32_t B, int32_t k);
  *            cost some of the overlap between consecutive launches);
  *   kind[i]  0 one-CTA GEMM, 1 CTA-pair GEMM, 2 CTA-pair GEMM that computes
  *            the LoRA activations t itself, 3 fused decode-size GEMM,
- *            10 RMSNorm, 11 RMSNorm + LoRA down-projection,
+ *            10 RMSNorm, 11 RMSNorm + LoRA down-projection, 12 rows' sums
+ *            of squares (steps of 512 rows and more fold RMSNorm into
+ *            their GEMMs and launch this once for the input),
  *            20 verification (stats + finalize), 21 draft (stats + draw);
  *   dims[4i .. 4i+3] (optional, may be NULL) for GEMMs: M, the summed N of
  *            its output groups, K and the epilogue mode (0 store, 1 residual

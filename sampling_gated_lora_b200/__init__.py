@@ -569,7 +569,7 @@ class Model:
         return load().uno_psi_step_kernel_count(self._h, B, k)
 
     PROFILE_KINDS = {0: "gemm_one_cta", 1: "gemm_pair", 2: "gemm_pair_computes_t",
-                     3: "gemm_decode", 10: "rmsnorm", 11: "rmsnorm_down", 20: "verify",
+                     3: "gemm_decode", 10: "rmsnorm", 11: "rmsnorm_down", 12: "row_sumsq", 20: "verify",
                      21: "draft"}
 
     def profile(self, enable=True):

@@ -716,12 +716,12 @@ enum { kQ = 0, kK, kV, kO, kGate, kUp, kDown };
 
 struct StepLayout {
   size_t h, n, q, k, v, act, t, logits, vstat, dstat, sk_part, sk_flag, sk_flag_bytes, flag_block,
-      total;
+      ss, ss_block, total;
 };
 
 // One operation of a step plan.
 struct StepOp {
-  int kind;            // 0 GEMM, 1 rmsnorm, 2 rmsnorm + LoRA down-projection
+  int kind;            // 0 GEMM, 1 rmsnorm, 2 rmsnorm + LoRA down-projection, 3 row sums of squares
   GemmLaunch gemm;
   const void* x;
   void* y;
@@ -737,6 +737,7 @@ enum ProfKind : int32_t {
   kProfGemmDecode = 3,   // fused decode-size GEMM
   kProfNorm = 10,        // RMSNorm
   kProfNormDown = 11,    // RMSNorm + LoRA down-projection
+  kProfSumSq = 12,       // rows' sums of squares (the first folded RMSNorm)
   kProfVerify = 20,      // row stats + verify finalize
   kProfDraft = 21,       // draft stats + draft draw
 };
@@ -744,6 +745,7 @@ enum ProfKind : int32_t {
 int32_t prof_kind(const StepOp& op) {
   if (op.kind == 1) return kProfNorm;
   if (op.kind == 2) return kProfNormDown;
+  if (op.kind == 3) return kProfSumSq;
   if (op.gemm.kind == 1) return op.gemm.computes_t ? kProfGemmPairT : kProfGemmPair;
   return op.gemm.kind == 2 ? kProfGemmDecode : kProfGemmOne;
 }
@@ -760,6 +762,13 @@ void set_dims(StepOp* op, const GemmProblem& pb) {
 // Decode-size batches fold the LoRA down-projection of an input that an
 // RMSNorm produces into that RMSNorm's launch (one launch instead of two).
 constexpr int64_t kNormDownMaxRows = 32;
+
+// From this many rows every main GEMM of a step is a CTA-pair launch, and the
+// step folds its RMSNorms into the GEMMs around them (GemmProblem::in_ss):
+// the residual-add launches write their rows' sums of squares, the next
+// launch scales its output rows. No RMSNorm launch and no normalised copy.
+constexpr int64_t kFoldNormMinRows = 512;
+constexpr float kNormEps = 1e-6f;
 
 }  // namespace
 }  // namespace uno
@@ -838,6 +847,12 @@ StepLayout step_layout(const uno_model* m, int32_t B, int32_t k) {
     L.sk_flag_bytes = (static_cast<size_t>(m->n_layers) * 4 + 1) * L.flag_block;
     L.sk_flag = take(L.sk_flag_bytes);
   }
+  // folded RMSNorm: per residual stream state (2 per layer + the input) the
+  // rows' sums of squares in 256-column partials
+  if (static_cast<int64_t>(M) >= kFoldNormMinRows) {
+    L.ss_block = align_up(M * ((static_cast<size_t>(m->hidden) + 255) / 256) * sizeof(float));
+    L.ss = take((static_cast<size_t>(m->n_layers) * 2 + 1) * L.ss_block);
+  }
   L.total = off;
   return L;
 }
@@ -883,9 +898,13 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
   // gated linear(s) on input x (width K): down-projections then the main GEMM
   // (or the main GEMM alone, when it computes t itself or is the fused
   // decode kernel). t_ready: the preceding launch wrote t as well as x.
+  const bool fold_norm = L.ss_block != 0;
+  auto ss_at = [&](int i) { return reinterpret_cast<float*>(base + L.ss + static_cast<size_t>(i) * L.ss_block); };
+  const int ss_cols = (m->hidden + 255) / 256;
+  // in_ss / out_ss: the folded RMSNorm's sums of squares read / written (or NULL)
   auto linear = [&](const void* x, int64_t K, int G, const int* which, int layer, void* const* y,
-                    const int64_t* ldy, int mode, void* y1, int64_t M0,
-                    bool t_ready = false) -> uno_status {
+                    const int64_t* ldy, int mode, void* y1, int64_t M0, bool t_ready = false,
+                    const float* in_ss = nullptr, float* out_ss = nullptr) -> uno_status {
     uno_status s;
     const void* As[kMaxGroups] = {nullptr, nullptr, nullptr};
     for (int i = 0; i < G; ++i)
@@ -922,6 +941,11 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     pm.gate_row0 = Mv;
     pm.scale = m->scale;
     for (int i = 0; i < G; ++i) pm.A[i] = r > 0 ? As[i] : nullptr;
+    pm.in_ss = in_ss;
+    pm.in_ss_cols = in_ss ? ss_cols : 0;
+    pm.out_ss = out_ss;
+    pm.norm_dim = m->hidden;
+    pm.norm_eps = kNormEps;
     pm.x_ready = r > 0 && !gemm_dec_suits(pm) && !t_ready;
     if (L.sk_flag_bytes) {
       char* blk = base + L.sk_flag + static_cast<size_t>(main_launches) * L.flag_block;
@@ -942,20 +966,29 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
     return UNO_OK;
   };
   uno_status s;
+  if (fold_norm) {   // the input's sums of squares (the later ones come from the residual adds)
+    StepOp op{};
+    op.kind = 3;
+    op.x = base + L.h;
+    op.y = ss_at(0);
+    P->ops.push_back(op);
+  }
   for (int l = 0; l < m->n_layers; ++l) {
-    norm(base + L.h, base + L.n);
+    if (!fold_norm) norm(base + L.h, base + L.n);
     {
       const int which[3] = {kQ, kK, kV};
       void* y[3] = {base + L.q, base + L.k, base + L.v};
       const int64_t ld[3] = {m->q_out, m->kv_out, m->kv_out};
-      if ((s = linear(base + L.n, m->hidden, 3, which, l, y, ld, kEpiStore, nullptr, M)) != UNO_OK)
+      if ((s = linear(fold_norm ? base + L.h : base + L.n, m->hidden, 3, which, l, y, ld, kEpiStore,
+                      nullptr, M, false, fold_norm ? ss_at(2 * l) : nullptr)) != UNO_OK)
         return s;
     }
     {
       const int which[1] = {kO};
       void* y[1] = {base + L.h};
       const int64_t ld[1] = {m->hidden};
-      if ((s = linear(base + L.q, m->q_out, 1, which, l, y, ld, kEpiAdd, nullptr, M)) != UNO_OK)
+      if ((s = linear(base + L.q, m->q_out, 1, which, l, y, ld, kEpiAdd, nullptr, M, false, nullptr,
+                      fold_norm ? ss_at(2 * l + 1) : nullptr)) != UNO_OK)
         return s;
     }
     P->block_end.push_back(P->ops.size());
@@ -975,7 +1008,7 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
       probe.A[0] = m->wp(l, kGate, 1);
       probe.A[1] = m->wp(l, kUp, 1);
       probe.g[0].N = probe.g[1].N = m->inter;
-      const bool fold = r > 0 && M <= kNormDownMaxRows && m->hidden % 8 == 0 &&
+      const bool fold = !fold_norm && r > 0 && M <= kNormDownMaxRows && m->hidden % 8 == 0 &&
                         !gemm_dec_suits(probe);
       if (fold) {
         StepOp op{};
@@ -994,29 +1027,31 @@ uno_status build_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next
         op.nd.scale = m->scale;
         op.nd.gate_row0 = Mv;
         P->ops.push_back(op);
-      } else {
+      } else if (!fold_norm) {
         norm(base + L.h, base + L.n);
       }
-      if ((s = linear(base + L.n, m->hidden, 2, which, l, y, ld, kEpiSiluPair, nullptr, M,
-                      fold)) != UNO_OK)
+      if ((s = linear(fold_norm ? base + L.h : base + L.n, m->hidden, 2, which, l, y, ld,
+                      kEpiSiluPair, nullptr, M, fold, fold_norm ? ss_at(2 * l + 1) : nullptr)) != UNO_OK)
         return s;
     }
     {
       const int which[1] = {kDown};
       void* y[1] = {base + L.h};
       const int64_t ld[1] = {m->hidden};
-      if ((s = linear(base + L.act, m->inter, 1, which, l, y, ld, kEpiAdd, nullptr, M)) != UNO_OK)
+      if ((s = linear(base + L.act, m->inter, 1, which, l, y, ld, kEpiAdd, nullptr, M, false,
+                      nullptr, fold_norm ? ss_at(2 * l + 2) : nullptr)) != UNO_OK)
         return s;
     }
     P->block_end.push_back(P->ops.size());
   }
   if (!q_next) return UNO_OK;   // decoder layers only
-  norm(base + L.h, base + L.n);
+  if (!fold_norm) norm(base + L.h, base + L.n);
   void* p_dst = logits_out ? logits_out : base + L.logits;
   const int which[1] = {0};
   void* y[1] = {p_dst};
   const int64_t ld[1] = {m->vocab};
-  return linear(base + L.n, m->hidden, 1, which, -1, y, ld, kEpiStore, q_next, Mv);
+  return linear(fold_norm ? base + L.h : base + L.n, m->hidden, 1, which, -1, y, ld, kEpiStore,
+                q_next, Mv, false, fold_norm ? ss_at(2 * m->n_layers) : nullptr);
 }
 
 uno_model::Plan* find_plan(uno_model* m, int32_t B, int32_t k, void* ws, void* q_next,
@@ -1163,8 +1198,9 @@ uno_status uno_psi_step(uno_model* m, int32_t B, int32_t k, const void* h_in, co
   };
   for (const StepOp& op : P->ops) {
     s = op.kind == 0 ? gemm_run(op.gemm, st)
-        : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, 1e-6f, st)
-                       : norm_down_launch(op.nd, M, st);
+        : op.kind == 1 ? rmsnorm_launch(M, m->hidden, op.x, op.y, kNormEps, st)
+        : op.kind == 2 ? norm_down_launch(op.nd, M, st)
+                       : row_sumsq_launch(M, m->hidden, op.x, static_cast<float*>(op.y), st);
     if (s != UNO_OK) return s;
     if ((s = mark(prof_kind(op), op.kind == 0 ? op.dims : nullptr)) != UNO_OK) return s;
   }
@@ -1274,8 +1310,10 @@ uno_status uno_psi_step_hidden(uno_model* m, int32_t B, int32_t k, const void* h
   for (size_t i = 0; i < n_ops; ++i) {
     const StepOp& op = P->ops[i];
     s = op.kind == 0 ? gemm_run(op.gemm, st)
-        : op.kind == 1 ? rmsnorm_launch(static_cast<int64_t>(M), m->hidden, op.x, op.y, 1e-6f, st)
-                       : norm_down_launch(op.nd, static_cast<int64_t>(M), st);
+        : op.kind == 1 ? rmsnorm_launch(static_cast<int64_t>(M), m->hidden, op.x, op.y, kNormEps, st)
+        : op.kind == 2 ? norm_down_launch(op.nd, static_cast<int64_t>(M), st)
+                       : row_sumsq_launch(static_cast<int64_t>(M), m->hidden, op.x,
+                                          static_cast<float*>(op.y), st);
     if (s != UNO_OK) return s;
   }
   // the step's buffers still hold the last sub-blocks' products

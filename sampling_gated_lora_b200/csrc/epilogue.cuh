@@ -32,8 +32,24 @@ struct GemmArgs {
   const uint8_t* gate;
   int32_t* status;
   int x_ready;    // x complete at launch: wait for the predecessor only before reading t
+  // folded RMSNorm (see GemmProblem): input row scales from in_ss, and the
+  // output rows' sums of squares to out_ss
+  const float* in_ss;
+  float* out_ss;
+  int in_ss_cols, out_ss_cols;   // partials per row: of the input, of this launch (its feature tiles)
+  float norm_inv_d, norm_eps;
   GroupArgs g[kMaxGroups];
 };
+
+// 1 / sqrt(mean square + eps) of input row m from its in_ss partials, added
+// in order (so every launch and every tile of the row gets the same scale).
+__device__ __forceinline__ float in_row_scale(const GemmArgs& a, int m) {
+  if (!a.in_ss || m >= a.M) return 1.0f;
+  const float* p = a.in_ss + static_cast<size_t>(m) * a.in_ss_cols;
+  float ss = 0.f;
+  for (int c = 0; c < a.in_ss_cols; ++c) ss += p[c];
+  return rsqrtf(ss * a.norm_inv_d + a.norm_eps);
+}
 
 // Host: the device-side description of a problem; `tile_n` is the number of
 // output features per feature tile (silu-pair tiles count output features).
@@ -52,6 +68,11 @@ inline GemmArgs make_gemm_args(const GemmProblem& pb, int tile_n, int row_bytes)
   a.gate = pb.gate;
   a.status = nullptr;
   a.x_ready = pb.x_ready ? 1 : 0;
+  a.in_ss = pb.in_ss;
+  a.out_ss = pb.out_ss;
+  a.in_ss_cols = pb.in_ss_cols;
+  a.norm_inv_d = pb.norm_dim > 0 ? 1.0f / static_cast<float>(pb.norm_dim) : 0.f;
+  a.norm_eps = pb.norm_eps;
   int tiles = 0;
   for (int i = 0; i < pb.ngroups; ++i) {
     a.g[i].y = pb.g[i].y;
@@ -63,6 +84,7 @@ inline GemmArgs make_gemm_args(const GemmProblem& pb, int tile_n, int row_bytes)
     if (pb.mode != kEpiSiluPair || i == 0) tiles += static_cast<int>((pb.g[i].N + tile_n - 1) / tile_n);
   }
   if (pb.mode == kEpiSiluPair) a.g[1].tile0 = tiles;   // the up group shares group 0's tiles
+  a.out_ss_cols = static_cast<int>((pb.g[0].N + tile_n - 1) / tile_n);
   return a;
 }
 
@@ -133,13 +155,20 @@ __device__ __forceinline__ void epi_store4(const GemmArgs& a, int g, int m, int 
 
 // 16 consecutive features n0..n0+15 of token row m (n0 % 16 == 0): two
 // 16-byte stores for bf16, four for f32; element by element at a ragged end.
+// sq (optional, bf16 only): adds the squares of the values stored.
 template <typename T>
 __device__ __forceinline__ void epi_store16(const GemmArgs& a, int g, int m, int n0,
-                                            const float (&v)[16]) {
+                                            const float (&v)[16], float* sq = nullptr) {
   if (m >= a.M) return;
   if (n0 + 16 > a.g[g].N) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) epi_store1<T>(a, g, m, n0 + j, v[j]);
+    for (int j = 0; j < 16; ++j) {
+      epi_store1<T>(a, g, m, n0 + j, v[j]);
+      if (sq && n0 + j < a.g[g].N) {
+        const float s = to_f32<T>(*out_ptr<T>(a, g, m, n0 + j));
+        *sq += s * s;
+      }
+    }
     return;
   }
   T* dst = out_ptr<T>(a, g, m, n0);
@@ -176,6 +205,10 @@ __device__ __forceinline__ void epi_store16(const GemmArgs& a, int g, int m, int
       for (int e = 0; e < 4; ++e) {
         __nv_bfloat162 h = __floats2bfloat162_rn(w[8 * q + 2 * e], w[8 * q + 2 * e + 1]);
         pk[e] = *reinterpret_cast<uint32_t*>(&h);
+        if (sq) {
+          const float lo = bf16_lo(pk[e]), hi = bf16_hi(pk[e]);
+          *sq += lo * lo + hi * hi;
+        }
       }
       d4[q] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }

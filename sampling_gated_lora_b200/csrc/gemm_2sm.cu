@@ -455,8 +455,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           else if (lane == 0)
             fail();
         }
+        // the folded RMSNorm of the input rows (1 without one)
+        const float rs = in_row_scale(a, m);
         if (!silu) {
           const int nb0 = (ft - a.g[g].tile0) * kTile;
+          float sq = 0.f;
+          float* sqp = a.out_ss ? &sq : nullptr;
           for (int c = 0; c < kTile; c += 16) {
             float v[16];
             tmem_ld16(trow + c, v);
@@ -464,8 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int j = 0; j < 16; ++j) v[j] += part[(c + j) * 32 + lane];
             }
-            if (nb0 + c < a.g[g].N) epi_store16<__nv_bfloat16>(a, g, m, nb0 + c, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] *= rs;
+            if (nb0 + c < a.g[g].N) epi_store16<__nv_bfloat16>(a, g, m, nb0 + c, v, sqp);
           }
+          // this tile's share of the stored rows' sums of squares (group 0 only)
+          if (a.out_ss && m < a.M)
+            a.out_ss[static_cast<size_t>(m) * a.out_ss_cols + (ft - a.g[g].tile0)] = sq;
         } else {
           const int f0 = ft * kHalf;
           for (int c = 0; c < kHalf; c += 16) {
@@ -480,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) gv[j] = silu_f(gv[j]) * uv[j];
+            for (int j = 0; j < 16; ++j) gv[j] = silu_f(gv[j] * rs) * (uv[j] * rs);
             if (f0 + c < a.g[0].N) epi_store16<__nv_bfloat16>(a, 0, m, f0 + c, gv);
           }
         }

@@ -185,6 +185,40 @@ __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
 
 }  // namespace
 
+// One warp per (row, 256-column tile): the sum of the squares of the tile's
+// bf16 values, fp32, in the layout of a residual-add GEMM's out_ss (so the
+// first GEMM of a step with folded RMSNorm reads its input's scales the same
+// way as every later one).
+__global__ void __launch_bounds__(kNormThreads)
+    row_sumsq_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int D, int cols,
+                     float* __restrict__ out) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * (kNormThreads / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= M * cols) return;
+  const int64_t m = w / cols;
+  const int c = static_cast<int>(w - m * cols);
+  const __nv_bfloat16* xr = x + m * D;
+  float ss = 0.f;
+  for (int i = c * 256 + lane; i < min(D, c * 256 + 256); i += 32) {
+    const float v = __bfloat162float(xr[i]);
+    ss += v * v;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) out[w] = ss;
+}
+
+uno_status row_sumsq_launch(int64_t M, int64_t D, const void* x, float* out, cudaStream_t s) {
+  if (M == 0) return UNO_OK;
+  const int cols = static_cast<int>((D + 255) / 256);
+  const int64_t warps = M * cols;
+  const cudaError_t e = launch_kernel(
+      row_sumsq_kernel, dim3(static_cast<unsigned>((warps + kNormThreads / 32 - 1) / (kNormThreads / 32))),
+      dim3(kNormThreads), 0, s, 1, static_cast<const __nv_bfloat16*>(x), M, static_cast<int>(D), cols, out);
+  return e == cudaSuccess ? UNO_OK : cuda_error(e, "row sum-of-squares launch");
+}
+
 uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
                           cudaStream_t s) {
   if (M == 0) return UNO_OK;

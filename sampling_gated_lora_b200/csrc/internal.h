@@ -70,6 +70,19 @@ struct GemmProblem {
   // down-projection clears the stream-K flags of the GEMM launched behind it.
   int32_t* zero_flags;
   int zero_words;
+  // RMSNorm folded into the GEMMs around it (CTA-pair kernel only). in_ss:
+  // x is an unnormalised residual stream whose rows' sums of squares come as
+  // in_ss_cols partials per row ([M, in_ss_cols] floats, added in order); every
+  // output row is scaled by 1 / sqrt(sum / norm_dim + norm_eps), which equals
+  // the GEMM of the normalised rows (the adapter term included, t being
+  // computed from the same unnormalised x). out_ss (kEpiAdd): the launch
+  // writes, per row and 256-column feature tile, the sum of squares of the
+  // bf16 values it stores ([M, feature tiles] floats).
+  const float* in_ss;
+  int in_ss_cols;
+  float* out_ss;
+  int64_t norm_dim;
+  float norm_eps;
   // Non-NULL: the CTA-pair kernel may compute t = scale * gate * (x A_g^T)
   // itself (A[] and t above; r <= 128, 16 or more 256-row blocks, see
   // gemm_pair_prepare), counting the finished parts of each 256-row block
@@ -188,6 +201,10 @@ uno_status philox_launch(uint64_t seed, uint64_t step, uint32_t stream_id, uint3
                          int64_t n, uint32_t* words, float* u, cudaStream_t s);
 
 // ---------------------------------------------------------------- glue
+// Per row m and 256-column tile c of x [M, D] bf16: out[m * ceil(D / 256) + c]
+// = sum of the squares of the tile's values (fp32), the layout a residual-add
+// GEMM writes with GemmProblem::out_ss.
+uno_status row_sumsq_launch(int64_t M, int64_t D, const void* x, float* out, cudaStream_t s);
 uno_status rmsnorm_launch(int64_t M, int64_t D, const void* x, void* y, float eps,
                           cudaStream_t s);
 uno_status silu_mul_launch(int64_t n, const void* a, const void* b, void* y, cudaStream_t s);
