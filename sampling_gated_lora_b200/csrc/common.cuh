@@ -366,6 +366,22 @@ __device__ __forceinline__ void cluster_sync() {
 // Barrier of all threads of the CTA (per-thread form, see cluster_sync).
 __device__ __forceinline__ void cta_sync() { asm volatile("barrier.sync 0;" ::: "memory"); }
 
+// The aligned forms of the two barriers, for the points after a kernel's
+// role branches: a role runs on one lane while its warp-mates go ahead, so
+// each warp first reconverges (__syncwarp), and the warp then reaches the
+// barrier as one. Without the __syncwarp the aligned forms count a warp as
+// arrived when its first lanes do, and release the barrier too early.
+__device__ __forceinline__ void cta_sync_converged() {
+  __syncwarp();
+  asm volatile("bar.sync 0;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync_converged() {
+  __syncwarp();
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Named barrier `id` of `n` threads (per-thread form).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t n) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory");

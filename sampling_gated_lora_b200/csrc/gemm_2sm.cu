@@ -503,8 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Everything issued has been waited for by the epilogues (or given up on);
   // meet the peer before freeing the pair's TMEM.
   tc_fence_before();
-  __syncwarp();
-  cluster_sync();
+  cluster_sync_converged();
   if (warp == 0) {
     __syncwarp();
     tc_fence_after();

@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   if (p.splits > 1) {
-    cluster_sync();
+    cluster_sync_converged();
     const uint32_t rank = cluster_ctarank();
     const int Sp = p.splits;
     const int groups = kSilu ? bn * (kRows / 8) : bn * (kRows / 4);
@@ -330,11 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               silu_f(gv.z) * uv.z, silu_f(gv.w) * uv.w));
       }
     }
-    cluster_sync();
+    cluster_sync_converged();
   }
 
   tc_fence_before();
-  cta_sync();
+  cta_sync_converged();
   if (warp == 0) {
     __syncwarp();
     tc_fence_after();

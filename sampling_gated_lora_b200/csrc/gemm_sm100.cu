@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (p.splits > 1) {
     // Sum the cluster's partial tiles. CTA `rank` reduces a contiguous range
     // of 4-element groups, reading the same group from every CTA.
-    cluster_sync();
+    cluster_sync_converged();
     const uint32_t rank = cluster_ctarank();
     const int S = p.splits;
     const int groups = kSwap ? (silu ? bn * (kTileP / 8) : bn * (kTileP / 4)) : kTileP * bn / 4;
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                   silu_f(gv.w) * uv.w));
       }
     }
-    cluster_sync();
+    cluster_sync_converged();
   }
 
   // Drain: if the MMA side gave up, wait (bounded) for TMA copies still in flight.
@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_wait(smem_u32(&full[it % p.stages]), (it / p.stages) & 1u, kWaitLimitNs / 4);
   }
   tc_fence_before();
-  cta_sync();   // every warp is done with TMEM before it is freed
+  cta_sync_converged();   // every warp is done with TMEM before it is freed
   if (warp == 0) {
     __syncwarp();
     tc_fence_after();
