@@ -236,7 +236,7 @@ def cpu_cores():
 
 # ---------------------------------------------------------------- kernel lines
 
-def kernel_lines(U, torch, pk):
+def kernel_lines(U, torch, pk, with_oracle=True):
     """Per-config kernel measurements (gated GEMM small M and M=2048, psi_verify).
 
     Gated linears are timed back to back, the way a decode step runs them: one
@@ -248,6 +248,23 @@ def kernel_lines(U, torch, pk):
     import workloads as W
     out = {}
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    if with_oracle:
+        from oracle import distill as OD
+        from oracle import gated_linear as OG
+        from oracle import sampling as OS
+        from oracle import tree as OT
+    host = lambda t: t.float().cpu().numpy()   # bf16 values are exact in float32
+
+    def oracle_line(line, fn, scale, sample):
+        """The fp64 oracle on a bounded sample of a kernel line's work (host arrays copied
+        before timing), scaled to the whole line: oracle_us beside the kernel's us."""
+        if not with_oracle:
+            return
+        t0 = time.perf_counter()
+        fn()
+        line["oracle_us"] = round((time.perf_counter() - t0) * 1e6 * scale, 1)
+        line["oracle_sample"] = sample
+        line["oracle_cores"] = cpu_cores()
 
     def timed(fn, reps=20):
         ts = []
@@ -299,10 +316,13 @@ def kernel_lines(U, torch, pk):
         byts = 2 * (N * K + r * K + N * r + M * K + M * N)
         flops = 2 * M * K * N + 2 * Mg * r * (K + N)
         t_roof = max(byts / (pk["hbm_gbs"] * 1e9), flops / (pk["bf16_tflops"] * 1e12)) * 1e6
-        out[f"gated_linear_4096x4096_M{M}"] = {
+        line = out[f"gated_linear_4096x4096_M{M}"] = {
             "us": round(us, 2), "single_us": round(single, 2), "GBps": round(byts / us / 1e3, 1),
             "TFLOPs": round(flops / us / 1e6, 1), "roofline_us": round(t_roof, 2),
             "frac_of_roofline": round(t_roof / us, 3), "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3)}
+        rs = min(M, 72)
+        ho = [host(a) for a in (x[:rs], sets[0][0], sets[0][1], sets[0][2])] + [g[:rs].cpu().numpy()]
+        oracle_line(line, lambda: OG.gated_linear(*ho, 1.0), M / rs, f"{rs} of {M} rows, scaled")
         del sets
     for name, K, N, M in (("up", 4096, 12288, 2048), ("down", 12288, 4096, 2048),
                           ("up", 4096, 12288, 4352)):
@@ -319,9 +339,12 @@ def kernel_lines(U, torch, pk):
         single = timed(calls[0], reps=10)
         us = chained(calls)
         flops = 2 * M * K * N + 2 * (M // 2) * r * (K + N)
-        out[f"gated_linear_mlp_{name}_M{M}"] = {
+        line = out[f"gated_linear_mlp_{name}_M{M}"] = {
             "us": round(us, 2), "single_us": round(single, 2), "TFLOPs": round(flops / us / 1e6, 1),
             "tensor_frac": round(flops / us / 1e6 / pk["bf16_tflops"], 3)}
+        rs = 64
+        ho = [host(a) for a in (x[M - rs:], sets[0][0], sets[0][1], sets[0][2])] + [g[M - rs:].cpu().numpy()]
+        oracle_line(line, lambda: OG.gated_linear(*ho, 1.0), M / rs, f"{rs} of {M} rows, scaled")
         del sets
     del x, y
     # adapter gradients (the training layout, MLP up shape): M = 2048 rows, 1024 of them
@@ -343,9 +366,14 @@ def kernel_lines(U, torch, pk):
     flops = 2 * Mg * r * (2 * K + 2 * N)
     byts = 2 * (Mg * K + Mg * N + 2 * (r * K + N * r))
     t_roof = max(byts / (pk["hbm_gbs"] * 1e9), flops / (pk["bf16_tflops"] * 1e12)) * 1e6
-    out["adapter_grads_mlp_up_M2048"] = {
+    line = out["adapter_grads_mlp_up_M2048"] = {
         "us": round(us, 1), "TFLOPs": round(flops / us / 1e6, 1), "GBps": round(byts / us / 1e3, 1),
         "roofline_us": round(t_roof, 2), "frac_of_roofline": round(t_roof / us, 3)}
+    rs = 64
+    ho = [host(x[M - rs:]), host(A), host(Bl), g[M - rs:].cpu().numpy()]
+    hdy = host(dy[M - rs:])
+    oracle_line(line, lambda: OG.gated_linear_adapter_grads(*ho, 1.0, hdy), M / rs,
+                f"{rs} of {M} rows (gated), scaled")
     del x, dy, A, Bl, bws
     # psi_verify at B=256, k=16, V=151936 (sigma 1.0 and 0.25, T = 1)
     B, k, V = 256, 16, 151936
@@ -361,10 +389,13 @@ def kernel_lines(U, torch, pk):
         f()
         us = timed(f, reps=10)
         byts = 2 * B * k * V * 2
-        out[f"psi_verify_B256_k16_sigma{sigma}"] = {
+        line = out[f"psi_verify_B256_k16_sigma{sigma}"] = {
             "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
             "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3),
             "mean_accepted": round(float(outs[0].float().mean()), 3)}
+        hp, hq, hd = host(p[:2]), host(q[:2]), d[:2].cpu().numpy()
+        oracle_line(line, lambda: OS.psi_verify(hp, hq, hd, 1.0, 1234, 0), B / 2,
+                    f"2 of {B} sequences, scaled")
         del p, q
     # linear-sampler draft of the step at B=256, k=8: 2048 rows of V=151936 bf16 logits.
     # Algorithmic bytes: one read of every logit (the draw re-reads one vocab chunk a row).
@@ -377,9 +408,11 @@ def kernel_lines(U, torch, pk):
     f()
     us = timed(f, reps=10)
     byts = Bd * kd * V * 2
-    out[f"draft_sample_B{Bd}_k{kd}"] = {
+    line = out[f"draft_sample_B{Bd}_k{kd}"] = {
         "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
         "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3)}
+    hq = host(qd[:2])
+    oracle_line(line, lambda: OS.draft_sample(hq, 1.0, 99, 0), Bd / 2, f"2 of {Bd} sequences, scaled")
     del qd
     # tree_verify at low batch: B=8 sequences, N=4 candidate blocks of k=8, V=151936.
     # Candidates: the linear sampler on q repeated N times per sequence (Philox index
@@ -392,6 +425,7 @@ def kernel_lines(U, torch, pk):
     R = N * k + 1
     depth_idx = torch.zeros((B, R), dtype=torch.long)
     nodes = 0
+    nodes_0 = 0
     for b in range(B):
         ids = {(): 0}
         for i in range(N):
@@ -401,6 +435,7 @@ def kernel_lines(U, torch, pk):
                     ids[pre] = len(ids)
                     depth_idx[b, ids[pre]] = min(j + 1, k - 1)
         nodes += len(ids)
+        nodes_0 = nodes_0 or len(ids)
     gen = torch.Generator(device="cuda").manual_seed(78)
     qf = q.float()
     p_nodes = (torch.gather(qf, 1, depth_idx.cuda()[:, :, None].expand(B, R, V))
@@ -415,10 +450,13 @@ def kernel_lines(U, torch, pk):
     f()
     us = timed(f, reps=10)
     byts = (nodes + B * k) * V * 2
-    out[f"tree_verify_B{B}_N{N}_k{k}"] = {
+    line = out[f"tree_verify_B{B}_N{N}_k{k}"] = {
         "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
         "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3), "trie_nodes": nodes,
         "mean_accepted": round(float(touts[0].float().mean()), 3)}
+    hp, hq = host(p_nodes[0, :nodes_0]), host(q[0])
+    oracle_line(line, lambda: OT.tree_verify_sequence(hp, hq, c_host[0], 1.0, 1234, 0, 0, bonus=True),
+                B, f"1 of {B} sequences, scaled")
     del p_nodes, q
     # distillation losses + gradient on the MLP batch layout: 1024 clean (teacher) rows
     # against 1024 noisy (student) rows, V=151936, bf16 logits, fp32 gradient.
@@ -433,9 +471,12 @@ def kernel_lines(U, torch, pk):
     f()
     us = timed(f, reps=10)
     byts = rows * V * (2 + 2 + 4)
-    out[f"distill_rows{rows}_V{V}"] = {
+    line = out[f"distill_rows{rows}_V{V}"] = {
         "us": round(us, 1), "GBps": round(byts / us / 1e3, 1),
         "hbm_frac": round(byts / us / 1e3 / pk["hbm_gbs"], 3)}
+    ht, hs = host(zt[:8]), host(zs[:8])
+    oracle_line(line, lambda: (OD.distill_losses(ht, hs, 1.0), OD.distill_grad(ht, hs, 1.0, 1.0, 1.0)),
+                rows / 8, f"8 of {rows} row pairs, scaled")
     del zt, zs, dg
     torch.cuda.empty_cache()
     return out
@@ -563,7 +604,7 @@ def run_uno(args):
         result["sweep_tokens_per_s"] = sweep
         del ws, qb, db
         torch.cuda.empty_cache()
-        result["kernels"] = kernel_lines(U, torch, pk)
+        result["kernels"] = kernel_lines(U, torch, pk, with_oracle=not args.no_cpu)
     if rank == 0 and world == 1 and not args.no_cpu:
         # the oracle's time per sequence-step, over several sampled sequences, converted
         # with this run's measured tokens per sequence-step (a single sample's 1..k+1
