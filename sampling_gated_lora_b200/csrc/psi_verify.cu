@@ -1006,7 +1006,11 @@ __global__ void __launch_bounds__(kDrawThreads)
 // (hyper.ai page, section "方法": the distillation and total-variation
 // losses), and the gradient w.r.t. the student logits:
 //   (alpha (q - p) + beta q (s - sum_v s_v q_v) / 2) / (T rows),  s = sign(q - p).
-// One cluster per row pair; each CTA stages its vocab chunk of both rows.
+// One cluster per row pair; each CTA stages its vocab chunk of both rows and
+// makes three passes over it (partition sums, loss terms, gradient), the
+// per-element arithmetic in float and every sum in double, with one exchange
+// of CTA totals over the cluster after each of the first two (added in rank
+// order, so every CTA holds the same bits).
 
 struct DistillParams {
   int V, chunk_elems;
@@ -1019,47 +1023,18 @@ struct DistillParams {
   int32_t* status;
 };
 
-// Cluster-wide sums of kN doubles per thread; the CTAs' block sums are added
-// in rank order, so every CTA gets the same bits. Every thread of every CTA
-// of the cluster must call it.
-template <int kN>
-__device__ void cluster_sums(double (&v)[kN], double (*warp_slots)[kN], double* cta_slot) {
-#pragma unroll
-  for (int i = 0; i < kN; ++i) v[i] = warp_sum(v[i]);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < kN; ++i) warp_slots[warp][i] = v[i];
-  }
-  cta_sync();
-  if (threadIdx.x < kN) {
-    double t = 0.0;
-    for (int w = 0; w < kDrawThreads / 32; ++w) t += warp_slots[w][threadIdx.x];
-    cta_slot[threadIdx.x] = t;
-  }
-  cluster_sync();
-  const uint32_t nrank = cluster_nctarank();
-#pragma unroll
-  for (int i = 0; i < kN; ++i) {
-    const uint32_t addr = smem_u32(&cta_slot[i]);
-    double total = 0.0;
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r < static_cast<int>(nrank)) total += ld_cluster_f64(map_shared_rank(addr, static_cast<uint32_t>(r)));
-    v[i] = total;
-  }
-  cluster_sync();   // every CTA has read the slots before they are written again
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kDrawThreads)
     distill_kernel(const T* __restrict__ z_teacher, const T* __restrict__ z_student,
                    const DistillParams a) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ double s_warp[kDrawThreads / 32][3];
-  __shared__ double s_cta[3];
-  __shared__ float s_wmax[kDrawThreads / 32][2];
-  __shared__ float s_max[2];
+  constexpr int kWarps = kDrawThreads / 32;
+  __shared__ float s_wm[kWarps][2];       // per warp: maxima (teacher, student)
+  __shared__ double s_ws[kWarps][3];      // per warp: sums
+  __shared__ float s_m[2];                // this CTA's maxima      } read by the
+  __shared__ double s_s[2];               // and sums relative to them } whole cluster
+  __shared__ double s_terms[3];           // this CTA's KL, sum |p - q|, sum s q
+  __shared__ __align__(8) uint64_t s_bar;   // the chunks' bulk copies
 
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
@@ -1067,15 +1042,41 @@ __global__ void __launch_bounds__(kDrawThreads)
   const uint32_t rank = cluster_ctarank();
   const int row = blockIdx.x / nrank;
   const int V = a.V;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int lo, len;
   chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
   T* zt = reinterpret_cast<T*>(dyn);
   T* zs = zt + a.chunk_elems;
-  load_chunk(zt, z_teacher + static_cast<size_t>(row) * V + lo, len);
-  load_chunk(zs, z_student + static_cast<size_t>(row) * V + lo, len);
+  const T* src_t = z_teacher + static_cast<size_t>(row) * V + lo;
+  const T* src_s = z_student + static_cast<size_t>(row) * V + lo;
+  const uint32_t bytes = static_cast<uint32_t>(len) * sizeof(T);
+  // both chunks by two bulk copies when they are 16-byte aligned whole vectors
+  // (all of them in flight at once), else by the threads
+  const bool bulk = ((reinterpret_cast<uintptr_t>(src_t) | reinterpret_cast<uintptr_t>(src_s)) & 15u) == 0 &&
+                    bytes % 16 == 0 && bytes > 0;
+  if (bulk) {
+    if (threadIdx.x == 0) {
+      mbar_init(smem_u32(&s_bar), 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(smem_u32(&s_bar), 2 * bytes);
+      bulk_load(smem_u32(zt), src_t, bytes, smem_u32(&s_bar));
+      bulk_load(smem_u32(zs), src_s, bytes, smem_u32(&s_bar));
+    }
+    cta_sync();   // the barrier is initialised before anyone waits on it
+    if (!mbar_wait(smem_u32(&s_bar), 0) && threadIdx.x == 0) {
+      raise_status(a.status, kDevTimeout);   // the copies still land before the CTA goes on
+      (void)mbar_wait(smem_u32(&s_bar), 0);
+    }
+  } else {
+    load_chunk(zt, src_t, len);
+    load_chunk(zs, src_s, len);
+  }
   cta_sync();
+  const float c = a.c;
 
-  // 1. the rows' maxima over the cluster (NaN kept)
+  // 1. both rows' maxima and partition sums: per warp the maxima, then each
+  // thread's sums of 2^((z - m) c) relative to its warp's maxima (float), the
+  // warps merged per CTA (double), the CTAs over the cluster in rank order
   float mt = -INFINITY, ms = -INFINITY;
   bool nan = false;
   for (int i = threadIdx.x; i < len; i += blockDim.x) {
@@ -1087,32 +1088,54 @@ __global__ void __launch_bounds__(kDrawThreads)
   mt = warp_max(mt);
   ms = warp_max(ms);
   nan = __any_sync(0xffffffffu, nan);
-  if ((threadIdx.x & 31) == 0) {
-    s_wmax[threadIdx.x >> 5][0] = nan ? NAN : mt;
-    s_wmax[threadIdx.x >> 5][1] = ms;
+  float st = 0.f, ss = 0.f;
+  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+    if (mt != -INFINITY) st += fast_exp2((to_f32<T>(zt[i]) - mt) * c);
+    if (ms != -INFINITY) ss += fast_exp2((to_f32<T>(zs[i]) - ms) * c);
+  }
+  const double wst = warp_sum(static_cast<double>(st)), wss = warp_sum(static_cast<double>(ss));
+  if (lane == 0) {
+    s_wm[warp][0] = nan ? NAN : mt;
+    s_wm[warp][1] = ms;
+    s_ws[warp][0] = wst;
+    s_ws[warp][1] = wss;
   }
   cta_sync();
-  if (threadIdx.x < 2) {
+  const double cd = static_cast<double>(c);
+  if (threadIdx.x < 2) {   // thread 0: teacher, thread 1: student
+    const int t = threadIdx.x;
     float m = -INFINITY;
     bool any = false;
-    for (int w = 0; w < kDrawThreads / 32; ++w) {
-      any |= isnan(s_wmax[w][threadIdx.x]);
-      m = fmaxf(m, s_wmax[w][threadIdx.x]);
+    for (int w = 0; w < kWarps; ++w) {
+      any |= isnan(s_wm[w][t]);
+      m = fmaxf(m, s_wm[w][t]);
     }
-    s_max[threadIdx.x] = any ? NAN : m;
+    double sum = 0.0;
+    for (int w = 0; w < kWarps; ++w)
+      if (s_wm[w][t] != -INFINITY && !any)
+        sum += s_ws[w][t] * exp2(static_cast<double>(s_wm[w][t] - m) * cd);
+    s_m[t] = any ? NAN : m;
+    s_s[t] = sum;
   }
-  cluster_sync();
+  cluster_sync();   // exchange 1: every CTA's maxima and sums
   float Mt = -INFINITY, Ms = -INFINITY;
   bool any_nan = false;
-  for (uint32_t r = 0; r < nrank; ++r) {
-    const float x = ld_cluster_f32(map_shared_rank(smem_u32(&s_max[0]), r));
-    const float y = ld_cluster_f32(map_shared_rank(smem_u32(&s_max[1]), r));
-    any_nan |= isnan(x);
-    Mt = fmaxf(Mt, x);
-    Ms = fmaxf(Ms, y);
+  float cm[2][8];
+  double csum[2][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r >= static_cast<int>(nrank)) break;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      cm[t][r] = ld_cluster_f32(map_shared_rank(smem_u32(&s_m[t]), static_cast<uint32_t>(r)));
+      csum[t][r] = ld_cluster_f64(map_shared_rank(smem_u32(&s_s[t]), static_cast<uint32_t>(r)));
+    }
+    any_nan |= isnan(cm[0][r]);
+    Mt = fmaxf(Mt, cm[0][r]);
+    Ms = fmaxf(Ms, cm[1][r]);
   }
-  cluster_sync();
   if (any_nan) {   // uniform over the cluster
+    cluster_sync();   // every CTA has read the others' slots before any leaves
     if (rank == 0 && threadIdx.x == 0) {
       a.losses[2 * row] = NAN;
       a.losses[2 * row + 1] = NAN;
@@ -1123,47 +1146,65 @@ __global__ void __launch_bounds__(kDrawThreads)
         a.grad[static_cast<size_t>(row) * V + lo + i] = NAN;
     return;
   }
-
-  // 2. the partition sums, then KL, TV and sum(sign(q - p) q)
-  const float c = a.c;
-  double sums[3] = {0.0, 0.0, 0.0};
-  for (int i = threadIdx.x; i < len; i += blockDim.x) {
-    sums[0] += static_cast<double>(fast_exp2((to_f32<T>(zt[i]) - Mt) * c));
-    sums[1] += static_cast<double>(fast_exp2((to_f32<T>(zs[i]) - Ms) * c));
+  double St = 0.0, Ss = 0.0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r >= static_cast<int>(nrank)) break;
+    if (cm[0][r] != -INFINITY) St += csum[0][r] * exp2(static_cast<double>(cm[0][r] - Mt) * cd);
+    if (cm[1][r] != -INFINITY) Ss += csum[1][r] * exp2(static_cast<double>(cm[1][r] - Ms) * cd);
   }
-  cluster_sums<3>(sums, s_warp, s_cta);
-  const double St = sums[0], Ss = sums[1];
-  const double ln_st = log(St), ln_ss = log(Ss);
-  const double inv_st = 1.0 / St, inv_ss = 1.0 / Ss;
-  const double inv_t = a.inv_t;
-  double acc[3] = {0.0, 0.0, 0.0};   // KL, sum |p - q|, sum s q
+
+  // 2. KL, sum |p - q| and sum sign(q - p) q: per element in float (log p -
+  // log q = (x - y) / T - dconst), per thread in float, then in double
+  const float inv_st = static_cast<float>(1.0 / St), inv_ss = static_cast<float>(1.0 / Ss);
+  const float inv_t = a.inv_t;
+  const float dconst = static_cast<float>(static_cast<double>(Mt - Ms) * inv_t + (log(St) - log(Ss)));
+  float k0 = 0.f, k1 = 0.f, k2 = 0.f;
   for (int i = threadIdx.x; i < len; i += blockDim.x) {
     const float x = to_f32<T>(zt[i]), y = to_f32<T>(zs[i]);
-    const double p = fast_exp2((x - Mt) * c) * inv_st;
-    const double q = fast_exp2((y - Ms) * c) * inv_ss;
-    const double lp = (static_cast<double>(x) - Mt) * inv_t - ln_st;
-    const double lq = (static_cast<double>(y) - Ms) * inv_t - ln_ss;
-    if (p > 0.0) acc[0] += p * (lp - lq);
-    acc[1] += fabs(p - q);
-    acc[2] += q > p ? q : (q < p ? -q : 0.0);
+    const float p = fast_exp2((x - Mt) * c) * inv_st;
+    const float q = fast_exp2((y - Ms) * c) * inv_ss;
+    if (p > 0.f) k0 += p * ((x - y) * inv_t - dconst);
+    k1 += fabsf(p - q);
+    k2 += q > p ? q : (q < p ? -q : 0.f);
   }
-  cluster_sums<3>(acc, s_warp, s_cta);
+  double v[3] = {warp_sum(static_cast<double>(k0)), warp_sum(static_cast<double>(k1)),
+                 warp_sum(static_cast<double>(k2))};
+  if (lane == 0)
+#pragma unroll
+    for (int i = 0; i < 3; ++i) s_ws[warp][i] = v[i];
+  cta_sync();
+  if (threadIdx.x < 3) {
+    double t = 0.0;
+    for (int w = 0; w < kWarps; ++w) t += s_ws[w][threadIdx.x];
+    s_terms[threadIdx.x] = t;
+  }
+  cluster_sync();   // exchange 2: every CTA's terms
+  double tot[3] = {0.0, 0.0, 0.0};
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r >= static_cast<int>(nrank)) break;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      tot[i] += ld_cluster_f64(map_shared_rank(smem_u32(&s_terms[i]), static_cast<uint32_t>(r)));
+  }
+  cluster_sync();   // every CTA has read the others' slots: nothing remote after this
   if (rank == 0 && threadIdx.x == 0) {
-    a.losses[2 * row] = static_cast<float>(acc[0]);
-    a.losses[2 * row + 1] = static_cast<float>(0.5 * acc[1]);
+    a.losses[2 * row] = static_cast<float>(tot[0]);
+    a.losses[2 * row + 1] = static_cast<float>(0.5 * tot[1]);
   }
   if (!a.grad) return;
 
-  // 3. the gradient w.r.t. the student logits, this CTA's chunk
-  const double sq = acc[2];
-  const double ka = static_cast<double>(a.alpha) * a.grad_scale;
-  const double kb = 0.5 * static_cast<double>(a.beta) * a.grad_scale;
+  // 3. the gradient w.r.t. the student logits, this CTA's chunk (float)
+  const float sq = static_cast<float>(tot[2]);
+  const float ka = a.alpha * a.grad_scale;
+  const float kb = 0.5f * a.beta * a.grad_scale;
   float* g = a.grad + static_cast<size_t>(row) * V + lo;
   for (int i = threadIdx.x; i < len; i += blockDim.x) {
-    const double p = fast_exp2((to_f32<T>(zt[i]) - Mt) * c) * inv_st;
-    const double q = fast_exp2((to_f32<T>(zs[i]) - Ms) * c) * inv_ss;
-    const double s = q > p ? 1.0 : (q < p ? -1.0 : 0.0);
-    g[i] = static_cast<float>(ka * (q - p) + kb * q * (s - sq));
+    const float p = fast_exp2((to_f32<T>(zt[i]) - Mt) * c) * inv_st;
+    const float q = fast_exp2((to_f32<T>(zs[i]) - Ms) * c) * inv_ss;
+    const float sgn = q > p ? 1.f : (q < p ? -1.f : 0.f);
+    g[i] = ka * (q - p) + kb * q * (sgn - sq);
   }
 }
 
