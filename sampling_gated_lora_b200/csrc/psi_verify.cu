@@ -579,6 +579,40 @@ __device__ __forceinline__ void load_chunk(T* dst, const T* src, int len) {
   }
 }
 
+// Stage `len` logits of s0 (and of s1 when it is not NULL) into d0 (d1) with
+// all of their bytes in flight at once: bulk copies completing on the
+// mbarrier `bar` when the sources are 16-byte aligned and len * sizeof(T) is
+// a multiple of 16, the threads' loads otherwise. `bar` has been initialised
+// (count 1) before a block barrier; `phase` is its next phase, and the phase
+// after is returned. The wait is bounded: on a timeout the status word gets
+// UNO_DEV_TIMEOUT and thread 0 waits for the copies once more before the CTA
+// goes on. Every thread calls it; it ends with a block barrier.
+template <typename T>
+__device__ uint32_t stage_chunks(T* d0, const T* s0, T* d1, const T* s1, int len, uint64_t* bar,
+                                 uint32_t phase, int32_t* status) {
+  const uint32_t bytes = static_cast<uint32_t>(len) * sizeof(T);
+  const uintptr_t addr = reinterpret_cast<uintptr_t>(s0) | (s1 ? reinterpret_cast<uintptr_t>(s1) : 0);
+  if ((addr & 15u) != 0 || bytes % 16 != 0 || bytes == 0) {
+    load_chunk(d0, s0, len);
+    if (s1) load_chunk(d1, s1, len);
+    cta_sync();
+    return phase;
+  }
+  cta_sync();   // earlier reads of d0 / d1 (generic proxy) are done
+  if (threadIdx.x == 0) {
+    fence_proxy_async_smem();   // and ordered before the copies' writes
+    mbar_arrive_expect_tx(smem_u32(bar), (s1 ? 2u : 1u) * bytes);
+    bulk_load(smem_u32(d0), s0, bytes, smem_u32(bar));
+    if (s1) bulk_load(smem_u32(d1), s1, bytes, smem_u32(bar));
+  }
+  if (!mbar_wait(smem_u32(bar), phase) && threadIdx.x == 0) {
+    raise_status(status, kDevTimeout);
+    (void)mbar_wait(smem_u32(bar), phase);
+  }
+  cta_sync();
+  return phase ^ 1u;
+}
+
 struct FinalizeParams {
   int B, k, k_p, V, chunks;
   float c;   // log2(e) / T
@@ -601,8 +635,13 @@ __global__ void __launch_bounds__(kDrawThreads)
   __shared__ DrawSmem sh;
   __shared__ int s_n, s_bad, s_nan;
   __shared__ float s_stat[4];   // Mp, Sp, Mq, Sq of the drawing row(s)
+  __shared__ __align__(8) uint64_t s_bar;   // the staged rows' bulk copies
 
-  if (threadIdx.x == 0) pdl_trigger();
+  if (threadIdx.x == 0) {
+    pdl_trigger();
+    mbar_init(smem_u32(&s_bar), 1);
+    fence_mbar_init();
+  }
   pdl_wait();
   const uint32_t nrank = cluster_nctarank();
   const uint32_t rank = cluster_ctarank();
@@ -687,9 +726,9 @@ __global__ void __launch_bounds__(kDrawThreads)
   chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
   T* zp = reinterpret_cast<T*>(dyn);
   T* zq = zp + a.chunk_elems;
-  load_chunk(zp, p_logits + static_cast<size_t>(prow) * V + lo, len);
-  if (residual) load_chunk(zq, q_logits + static_cast<size_t>(qrow_local) * V + lo, len);
-  cta_sync();
+  stage_chunks(zp, p_logits + static_cast<size_t>(prow) * V + lo, zq,
+               residual ? q_logits + static_cast<size_t>(qrow_local) * V + lo : nullptr, len, &s_bar,
+               0u, a.status);
   const float Mp = s_stat[0], inv_sp = 1.f / s_stat[1];
   const float Mq = s_stat[2], inv_sq = residual ? 1.f / s_stat[3] : 0.f;
   const float c = a.c;
@@ -1047,31 +1086,13 @@ __global__ void __launch_bounds__(kDrawThreads)
   chunk_range(V, static_cast<int>(nrank), static_cast<int>(rank), &lo, &len);
   T* zt = reinterpret_cast<T*>(dyn);
   T* zs = zt + a.chunk_elems;
-  const T* src_t = z_teacher + static_cast<size_t>(row) * V + lo;
-  const T* src_s = z_student + static_cast<size_t>(row) * V + lo;
-  const uint32_t bytes = static_cast<uint32_t>(len) * sizeof(T);
-  // both chunks by two bulk copies when they are 16-byte aligned whole vectors
-  // (all of them in flight at once), else by the threads
-  const bool bulk = ((reinterpret_cast<uintptr_t>(src_t) | reinterpret_cast<uintptr_t>(src_s)) & 15u) == 0 &&
-                    bytes % 16 == 0 && bytes > 0;
-  if (bulk) {
-    if (threadIdx.x == 0) {
-      mbar_init(smem_u32(&s_bar), 1);
-      fence_mbar_init();
-      mbar_arrive_expect_tx(smem_u32(&s_bar), 2 * bytes);
-      bulk_load(smem_u32(zt), src_t, bytes, smem_u32(&s_bar));
-      bulk_load(smem_u32(zs), src_s, bytes, smem_u32(&s_bar));
-    }
-    cta_sync();   // the barrier is initialised before anyone waits on it
-    if (!mbar_wait(smem_u32(&s_bar), 0) && threadIdx.x == 0) {
-      raise_status(a.status, kDevTimeout);   // the copies still land before the CTA goes on
-      (void)mbar_wait(smem_u32(&s_bar), 0);
-    }
-  } else {
-    load_chunk(zt, src_t, len);
-    load_chunk(zs, src_s, len);
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&s_bar), 1);
+    fence_mbar_init();
   }
-  cta_sync();
+  cta_sync();   // the barrier is initialised before anyone waits on it
+  stage_chunks(zt, z_teacher + static_cast<size_t>(row) * V + lo, zs,
+               z_student + static_cast<size_t>(row) * V + lo, len, &s_bar, 0u, a.status);
   const float c = a.c;
 
   // 1. both rows' maxima and partition sums: per warp the maxima, then each
