@@ -31,7 +31,7 @@ namespace {
 constexpr int kTile = 64;
 
 // out[c, r] = f(r) in[r, c] for r < R, c < C (out row stride ld_out >= R);
-// out[c, r] = 0 for R <= r < ld_out. f(r) = scale * gate(r) when gated
+// out[c, r] = 0 for R <= r < ld_out, and rows with f(r) = 0 are not read. f(r) = scale * gate(r) when gated
 // (gate[r], or r >= gate_row0 without a gate vector), else 1. One 64 x 64
 // tile per CTA of 256 threads, staged in shared memory so that both the
 // reads and the writes are row-contiguous.
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(256)
     for (int h = 0; h < 2; ++h) {
       const int cl = 2 * tx + h, c = c0 + cl;
       float v = 0.f;
-      if (r < R && c < C) v = f * __bfloat162float(in[static_cast<size_t>(r) * ld_in + c]);
+      if (r < R && c < C && f != 0.f) v = f * __bfloat162float(in[static_cast<size_t>(r) * ld_in + c]);
       tile[rl][cl] = v;
     }
   }

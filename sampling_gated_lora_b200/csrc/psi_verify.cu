@@ -953,8 +953,14 @@ __global__ void __launch_bounds__(kDrawThreads)
   __shared__ double s_part, s_warp[kDrawThreads / 32];
   __shared__ float s_stat[4];
   __shared__ int s_flag[4];   // [0] decision, [1] bad candidate, [2] trie nodes, [3] NaN
+  __shared__ __align__(8) uint64_t s_bar;   // bulk copies of the staged rows
+  uint32_t bar_phase = 0;
 
-  if (threadIdx.x == 0) pdl_trigger();
+  if (threadIdx.x == 0) {
+    pdl_trigger();
+    mbar_init(smem_u32(&s_bar), 1);
+    fence_mbar_init();
+  }
   pdl_wait();
   const uint32_t nrank = cluster_nctarank();
   const uint32_t rank = cluster_ctarank();
@@ -1071,9 +1077,7 @@ __global__ void __launch_bounds__(kDrawThreads)
       }
       // rejected: the residual mass Z of this test, over the whole vocabulary
       if (!staged) {
-        load_chunk(zp, prow + lo, len);
-        load_chunk(zq, qrow + lo, len);
-        cta_sync();
+        bar_phase = stage_chunks(zp, prow + lo, zq, qrow + lo, len, &s_bar, bar_phase, a.status);
         staged = true;
       }
       double part = 0.0;
@@ -1148,8 +1152,9 @@ __global__ void __launch_bounds__(kDrawThreads)
     return;
   }
   const float Mp = s_stat[0];
-  load_chunk(zp, p_logits + (static_cast<size_t>(b) * R + node) * V + lo, len);
-  cta_sync();
+  bar_phase = stage_chunks(zp, p_logits + (static_cast<size_t>(b) * R + node) * V + lo,
+                           static_cast<T*>(nullptr), static_cast<const T*>(nullptr), len, &s_bar,
+                           bar_phase, a.status);
   const uint32_t idx3 = static_cast<uint32_t>(bg * static_cast<uint64_t>(k) + static_cast<uint64_t>(k));
   const double u = static_cast<double>(uniform24(philox_word0(a.seed, a.step, kStreamBonus, idx3)));
   auto w_p = [&](int v) { return fast_exp2((to_f32<T>(zp[v]) - Mp) * c); };
