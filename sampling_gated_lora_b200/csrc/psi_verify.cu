@@ -932,10 +932,12 @@ __device__ double cluster_sum(double* part_slot, double* warp_slots, double v) {
 
 // Target of a test at one vocab entry after `n` rejections at the node:
 // r_1 = p, r_{t+1} = max(r_t - q, 0) / Z_t (unchanged when Z_t = 0).
-__device__ __forceinline__ double tree_target(float p, float q, const double* Z, int n) {
+// Zinv[t] = 1 / Z[t] (0 when Z[t] = 0, which leaves r unchanged), taken once
+// per rejection so the per-entry chain multiplies instead of dividing.
+__device__ __forceinline__ double tree_target(float p, float q, const double* Zinv, int n) {
   double r = p;
   for (int t = 0; t < n; ++t)
-    if (Z[t] > 0.0) r = fmax(r - static_cast<double>(q), 0.0) / Z[t];
+    if (Zinv[t] > 0.0) r = fmax(r - static_cast<double>(q), 0.0) * Zinv[t];
   return r;
 }
 
@@ -949,7 +951,8 @@ __global__ void __launch_bounds__(kDrawThreads)
   __shared__ int s_node[kTreeMaxN][kTreeMaxK + 1];   // trie node after j tokens of candidate i
   __shared__ int s_id[kTreeMaxN * kTreeMaxK];
   __shared__ int s_tok[kTreeMaxK];
-  __shared__ double s_Z[kTreeMaxN];
+  __shared__ double s_Z[kTreeMaxN];      // residual masses of the rejections at this node
+  __shared__ double s_Zinv[kTreeMaxN];   // and their reciprocals (0 for a zero mass)
   __shared__ double s_part, s_warp[kDrawThreads / 32];
   __shared__ float s_stat[4];
   __shared__ int s_flag[4];   // [0] decision, [1] bad candidate, [2] trie nodes, [3] NaN
@@ -1061,7 +1064,7 @@ __global__ void __launch_bounds__(kDrawThreads)
         const int x = cand[i * k + j];
         const float px = fast_exp2((to_f32<T>(prow[x]) - Mp) * c) * inv_sp;
         const float qx = fast_exp2((to_f32<T>(qrow[x]) - Mq) * c) * inv_sq;
-        const float r = static_cast<float>(tree_target(px, qx, s_Z, nz));
+        const float r = static_cast<float>(tree_target(px, qx, s_Zinv, nz));
         const uint32_t idx = static_cast<uint32_t>(
             (bg * static_cast<uint64_t>(k) + static_cast<uint64_t>(j)) * static_cast<uint64_t>(N) +
             static_cast<uint64_t>(i));
@@ -1084,10 +1087,13 @@ __global__ void __launch_bounds__(kDrawThreads)
       for (int v = threadIdx.x; v < len; v += blockDim.x) {
         const float p = fast_exp2((to_f32<T>(zp[v]) - Mp) * c) * inv_sp;
         const float q = fast_exp2((to_f32<T>(zq[v]) - Mq) * c) * inv_sq;
-        part += fmax(tree_target(p, q, s_Z, nz) - static_cast<double>(q), 0.0);
+        part += fmax(tree_target(p, q, s_Zinv, nz) - static_cast<double>(q), 0.0);
       }
       const double Z = cluster_sum(&s_part, s_warp, part);
-      if (threadIdx.x == 0) s_Z[nz] = Z;
+      if (threadIdx.x == 0) {
+        s_Z[nz] = Z;
+        s_Zinv[nz] = Z > 0.0 ? 1.0 / Z : 0.0;
+      }
       ++nz;
       cta_sync();
     }
@@ -1118,7 +1124,7 @@ __global__ void __launch_bounds__(kDrawThreads)
     auto w_res = [&](int v) {
       const float p = fast_exp2((to_f32<T>(zp[v]) - Mp) * c) * inv_sp;
       const float q = fast_exp2((to_f32<T>(zq[v]) - Mq) * c) * inv_sq;
-      const double r = tree_target(p, q, s_Z, last);
+      const double r = tree_target(p, q, s_Zinv, last);
       return static_cast<float>(s_Z[last] > 0.0 ? fmax(r - static_cast<double>(q), 0.0) : r);
     };
     bool zero = false;
