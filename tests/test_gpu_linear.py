@@ -140,6 +140,49 @@ def test_stale_workspace_grouped_calls(G):
             check_close(y, ref, what=f"G={G} N={c.N} call {call}")
 
 
+@pytest.mark.parametrize("G,M", [(1, 9), (3, 17), (1, 72)])
+def test_decode_calls_reused_workspace_and_graph_replay(G, M):
+    """Decode-size calls (the fused decode kernel): a workspace filled with 0x7f and one
+    filled with zeros, each used by two calls in a row, and a CUDA graph of one call
+    replayed three times. Every output matches the oracle, and the replays are
+    bit-identical to the eager call."""
+    import torch
+    import sampling_gated_lora_b200 as U
+    K = 4096
+    Ns = (4096, 1024, 1024)[:G]
+    x, gate, cases = _group_case(M, K, Ns, 128, seed=60 + G + M, b_std=0.05)
+    refs = [_oracle_group(x, gate, c) for c in cases]
+    need = U.load().uno_gated_lora_linear_group_workspace(U.UNO_BF16, M, 128, G)
+    for fill in (0x7F, 0):
+        ws = torch.full((need,), fill, dtype=torch.uint8, device="cuda")
+        for call in range(2):
+            ys = _run_group(x, gate, cases, False, workspace=ws)
+            for y, ref, c in zip(ys, refs, cases):
+                check_close(y, ref, what=f"G={G} M={M} N={c.N} fill={fill:#x} call {call}")
+    t = lambda a: dev_tensor(a, "bf16")
+    args = (t(x), [t(c.W) for c in cases], [t(c.A) for c in cases], [t(c.Bl) for c in cases],
+            dev_tensor(gate, "u8"), 1.0)
+    outs = [torch.empty((M, n), dtype=torch.bfloat16, device="cuda") for n in Ns]
+    ws = torch.full((need,), 0x7F, dtype=torch.uint8, device="cuda")
+    U.gated_lora_linear_group(*args, ys=outs, workspace=ws)
+    eager = [host_f64(o) for o in outs]
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        U.gated_lora_linear_group(*args, ys=outs, workspace=ws,
+                                  stream=torch.cuda.current_stream())
+    for rep in range(3):
+        for o in outs:
+            o.fill_(0)
+        graph.replay()
+        torch.cuda.synchronize()
+        for o, e, ref, c in zip(outs, eager, refs, cases):
+            got = host_f64(o)
+            np.testing.assert_array_equal(got, e)
+            check_close(got, ref, what=f"G={G} M={M} N={c.N} graph replay {rep}")
+
+
 def test_stream_k_without_workspace_scratch():
     """r = 0: with the workspace the size query asks for, the pair kernel cuts tiles; with
     none it runs whole tiles only. Both match the oracle."""
