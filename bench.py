@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--impl", choices=["uno", "reference"], default="uno")
     ap.add_argument("--no-kernels", action="store_true", help="skip the per-config kernel lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
-    ap.add_argument("--profile", choices=["gemm_up", "gemm_small", "step_up", "verify", "draft"],
+    ap.add_argument("--profile", choices=["gemm_up", "gemm_small", "step_up", "verify", "draft",
+                                          "draft_full", "gemm_down", "backward"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
@@ -795,6 +796,11 @@ def run_profile(args):
     gemm_small: gated linear 4096 -> 4096, M = 9 (split-K cluster path)
     verify:     psi_verify B=32, k=16, V=151936 (311 MB of logits)
     draft:      draft sampler B=32, k=8, V=151936
+    draft_full: draft sampler at B (default 256), k=8, V=151936 (622 MB of logits at B=256)
+    gemm_down:  gated linear 12288 -> 4096, M = 2048, half the rows gated (the MLP-down
+                kernel line)
+    backward:   adapter gradients, MLP-up shape 4096 -> 12288, r = 128, M = 2048, half the
+                rows gated (the adapter-gradient kernel line)
     """
     import torch
     import sampling_gated_lora_b200 as U
@@ -821,7 +827,19 @@ def run_profile(args):
                           "launches_per_step": m.kernel_count(B, k)}))
         m.close()
         return
-    if args.profile in ("gemm_up", "gemm_small"):
+    if args.profile == "gemm_down":
+        M, K, N, r = 2048, 12288, 4096, 128
+        x, Wt, A, Bl = dev((M, K), 1), dev((N, K), K ** -0.5), dev((r, K), K ** -0.5), dev((N, r), 0.01)
+        g = (torch.arange(M, device="cuda") >= M // 2).to(torch.uint8)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        f = lambda: U.gated_lora_linear(x, Wt, A, Bl, g, 1.0, y=y)
+    elif args.profile == "backward":
+        M, K, N, r = 2048, 4096, 12288, 128
+        x, dy = dev((M, K), 1), dev((M, N), 1)
+        A, Bl = dev((r, K), K ** -0.5), dev((N, r), 0.01)
+        g = (torch.arange(M, device="cuda") >= M // 2).to(torch.uint8)
+        f = lambda: U.gated_lora_adapter_grads(x, dy, A, Bl, g, 1.0)
+    elif args.profile in ("gemm_up", "gemm_small"):
         M, K, N = ((args.B * (2 * args.k + 1), 4096, 12288) if args.profile == "gemm_up"
                    else (9, 4096, 4096))
         r = 128
@@ -834,7 +852,8 @@ def run_profile(args):
         d = U.draft_sample(q, 1.0, 99, 0)
         f = lambda: U.psi_verify(p, q, d, 1.0, 1234, 0)
     else:
-        _, q = W.logits_case_torch(32, 8, 151936, sigma=1.0, seed=1234)
+        _, q = W.logits_case_torch(args.B if args.profile == "draft_full" else 32, 8, 151936,
+                                   sigma=1.0, seed=1234)
         f = lambda: U.draft_sample(q, 1.0, 99, 0)
     for _ in range(4):
         f()

@@ -293,6 +293,49 @@ __device__ __forceinline__ void unpack8(const uint4 w, float (&v)[8]) {
   v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
 }
 
+// Two bf16 maxima per instruction; a NaN operand gives NaN (so the chunk max
+// also tells whether the chunk holds a NaN).
+__device__ __forceinline__ uint32_t bmax2_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Two floats in one 64-bit register (element 0 in the low half) and the
+// packed fp32 arithmetic of sm_100 on them: one instruction per two elements,
+// each with the rounding of its scalar counterpart.
+using f32x2 = unsigned long long;
+__device__ __forceinline__ f32x2 f2_make(float a, float b) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(f32x2 v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ f32x2 f2_sub(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// The two elements of a bf16x2 word as floats.
+__device__ __forceinline__ f32x2 f2_from_bf16x2(uint32_t w) { return f2_make(bf16_lo(w), bf16_hi(w)); }
+
 __global__ void __launch_bounds__(kStagedThreads, 1)
     draft_stats_staged_kernel(const __nv_bfloat16* __restrict__ z_all, int rows, int V, int nsub,
                               TScale c, DraftStat* __restrict__ stats, int32_t* status) {
@@ -348,30 +391,60 @@ __global__ void __launch_bounds__(kStagedThreads, 1)
         for (int j = 0; j < 8; ++j) v[j] = e + j < len ? to_f32<__nv_bfloat16>(slot[e + j]) : -INFINITY;
       }
     };
-    float m = -INFINITY;
-    bool nan = false;
+    // the chunk max, two bf16 per instruction (a NaN makes it NaN); rows are
+    // whole 16-byte vectors, so a vector lies wholly inside or past the chunk
+    uint32_t m2 = 0xFF80FF80u;   // (-inf, -inf)
 #pragma unroll
     for (int k = 0; k < kPerLane; ++k) {
-      float v[8];
-      vec(k, v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        nan |= isnan(v[j]);
-        m = fmaxf(m, v[j]);
-      }
-    }
-    m = warp_max(m);
-    nan = __any_sync(0xffffffffu, nan);
-    double acc = 0.0;
-    if (m != -INFINITY) {
-#pragma unroll
-      for (int k = 0; k < kPerLane; ++k) {
+      const int e = (lane + k * 32) * 8;
+      if (e + 8 <= len) {
+        const uint4 w = *reinterpret_cast<const uint4*>(slot + e);
+        m2 = bmax2_nan(m2, bmax2_nan(bmax2_nan(w.x, w.y), bmax2_nan(w.z, w.w)));
+      } else if (e < len) {
         float v[8];
         vec(k, v);
-        float part = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) part += fast_exp2((v[j] - m) * c);
-        acc += static_cast<double>(part);
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t b = __float_as_uint(v[j]) >> 16;
+          m2 = bmax2_nan(m2, b | (b << 16));
+        }
+      }
+    }
+    const float mlo = bf16_lo(m2), mhi = bf16_hi(m2);
+    bool nan = isnan(mlo) || isnan(mhi);
+    float m = fmaxf(mlo, mhi);
+    m = warp_max(m);
+    nan = __any_sync(0xffffffffu, nan);
+    // sum of 2^((z - m) c): the difference, the float-pair scale and the sum of
+    // each 16-byte vector two elements per instruction, across vectors in double
+    double acc = 0.0;
+    if (m != -INFINITY && !nan) {
+      const f32x2 mm = f2_make(m, m), chi = f2_make(c.hi, c.hi), clo = f2_make(c.lo, c.lo);
+#pragma unroll
+      for (int k = 0; k < kPerLane; ++k) {
+        const int e = (lane + k * 32) * 8;
+        if (e + 8 <= len) {
+          const uint4 w = *reinterpret_cast<const uint4*>(slot + e);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+          f32x2 part = f2_make(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const f32x2 d = f2_sub(f2_from_bf16x2(ws[j]), mm);
+            float x0, x1;
+            f2_split(f2_fma(d, chi, f2_mul(d, clo)), x0, x1);
+            part = f2_add(part, f2_make(fast_exp2(x0), fast_exp2(x1)));
+          }
+          float p0, p1;
+          f2_split(part, p0, p1);
+          acc += static_cast<double>(p0 + p1);
+        } else if (e < len) {
+          float v[8];
+          vec(k, v);
+          float part = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) part += fast_exp2((v[j] - m) * c);
+          acc += static_cast<double>(part);
+        }
       }
     }
     // every lane has read the slot: it may be refilled
