@@ -1302,9 +1302,29 @@ __global__ void __launch_bounds__(kDrawThreads)
   // 1. both rows' maxima and partition sums: per warp the maxima, then each
   // thread's sums of 2^((z - m) c) relative to its warp's maxima (float), the
   // warps merged per CTA (double), the CTAs over the cluster in rank order
+  // bf16 chunks are read as 16-byte vectors of 8 (the chunks start 16-byte
+  // aligned in shared memory), two elements per instruction where the
+  // arithmetic allows it; a ragged end of the chunk and f32 rows one by one
+  constexpr bool kVec = std::is_same<T, __nv_bfloat16>::value;
+  const int nvec = kVec ? len / 8 : 0;
+  const int tail0 = nvec * 8;
+  const uint4* vt = reinterpret_cast<const uint4*>(zt);
+  const uint4* vs = reinterpret_cast<const uint4*>(zs);
   float mt = -INFINITY, ms = -INFINITY;
   bool nan = false;
-  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+  if (kVec) {   // maxima two at a time; a NaN makes the max NaN
+    uint32_t mt2 = 0xFF80FF80u, ms2 = 0xFF80FF80u;
+    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+      const uint4 a = vt[i], b = vs[i];
+      mt2 = bmax2_nan(mt2, bmax2_nan(bmax2_nan(a.x, a.y), bmax2_nan(a.z, a.w)));
+      ms2 = bmax2_nan(ms2, bmax2_nan(bmax2_nan(b.x, b.y), bmax2_nan(b.z, b.w)));
+    }
+    const float t0 = bf16_lo(mt2), t1 = bf16_hi(mt2), s0 = bf16_lo(ms2), s1 = bf16_hi(ms2);
+    nan = isnan(t0) || isnan(t1) || isnan(s0) || isnan(s1);
+    mt = fmaxf(t0, t1);
+    ms = fmaxf(s0, s1);
+  }
+  for (int i = tail0 + static_cast<int>(threadIdx.x); i < len; i += blockDim.x) {
     const float x = to_f32<T>(zt[i]), y = to_f32<T>(zs[i]);
     nan |= isnan(x) || isnan(y);
     mt = fmaxf(mt, x);
@@ -1314,7 +1334,33 @@ __global__ void __launch_bounds__(kDrawThreads)
   ms = warp_max(ms);
   nan = __any_sync(0xffffffffu, nan);
   float st = 0.f, ss = 0.f;
-  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+  if (kVec) {
+    const f32x2 c2 = f2_make(c, c), mt2 = f2_make(mt, mt), ms2 = f2_make(ms, ms);
+    const bool dt = mt != -INFINITY, ds = ms != -INFINITY;
+    f32x2 st2 = f2_make(0.f, 0.f), ss2 = f2_make(0.f, 0.f);
+    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+      const uint4 a = vt[i], b = vs[i];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float e0, e1;
+        if (dt) {
+          f2_split(f2_mul(f2_sub(f2_from_bf16x2(wa[q]), mt2), c2), e0, e1);
+          st2 = f2_add(st2, f2_make(fast_exp2(e0), fast_exp2(e1)));
+        }
+        if (ds) {
+          f2_split(f2_mul(f2_sub(f2_from_bf16x2(wb[q]), ms2), c2), e0, e1);
+          ss2 = f2_add(ss2, f2_make(fast_exp2(e0), fast_exp2(e1)));
+        }
+      }
+    }
+    float a0, a1, b0, b1;
+    f2_split(st2, a0, a1);
+    f2_split(ss2, b0, b1);
+    st = a0 + a1;
+    ss = b0 + b1;
+  }
+  for (int i = tail0 + static_cast<int>(threadIdx.x); i < len; i += blockDim.x) {
     if (mt != -INFINITY) st += fast_exp2((to_f32<T>(zt[i]) - mt) * c);
     if (ms != -INFINITY) ss += fast_exp2((to_f32<T>(zs[i]) - ms) * c);
   }
@@ -1385,7 +1431,47 @@ __global__ void __launch_bounds__(kDrawThreads)
   const float inv_t = a.inv_t;
   const float dconst = static_cast<float>(static_cast<double>(Mt - Ms) * inv_t + (log(St) - log(Ss)));
   float k0 = 0.f, k1 = 0.f, k2 = 0.f;
-  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+  const f32x2 c2 = f2_make(c, c), Mt2 = f2_make(Mt, Mt), Ms2 = f2_make(Ms, Ms);
+  const f32x2 ist2 = f2_make(inv_st, inv_st), iss2 = f2_make(inv_ss, inv_ss);
+  // p and q of the two elements of bf16x2 words wx (teacher) and wy (student)
+  auto pq2 = [&](uint32_t wx, uint32_t wy, f32x2* x, f32x2* y, f32x2* p, f32x2* q) {
+    *x = f2_from_bf16x2(wx);
+    *y = f2_from_bf16x2(wy);
+    float ex0, ex1, ey0, ey1;
+    f2_split(f2_mul(f2_sub(*x, Mt2), c2), ex0, ex1);
+    f2_split(f2_mul(f2_sub(*y, Ms2), c2), ey0, ey1);
+    *p = f2_mul(f2_make(fast_exp2(ex0), fast_exp2(ex1)), ist2);
+    *q = f2_mul(f2_make(fast_exp2(ey0), fast_exp2(ey1)), iss2);
+  };
+  if (kVec) {
+    const f32x2 it2 = f2_make(inv_t, inv_t), dc2 = f2_make(dconst, dconst);
+    f32x2 K0 = f2_make(0.f, 0.f), K1 = K0, K2 = K0;
+    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+      const uint4 a = vt[i], b = vs[i];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f32x2 x, y, p, q;
+        pq2(wa[j], wb[j], &x, &y, &p, &q);
+        float p0, p1, q0, q1, t0, t1, d0, d1;
+        f2_split(p, p0, p1);
+        f2_split(q, q0, q1);
+        f2_split(f2_sub(f2_mul(f2_sub(x, y), it2), dc2), t0, t1);
+        K0 = f2_fma(p, f2_make(p0 > 0.f ? t0 : 0.f, p1 > 0.f ? t1 : 0.f), K0);   // 0 log 0 = 0
+        f2_split(f2_sub(p, q), d0, d1);
+        K1 = f2_add(K1, f2_make(fabsf(d0), fabsf(d1)));
+        K2 = f2_add(K2, f2_make(q0 > p0 ? q0 : (q0 < p0 ? -q0 : 0.f), q1 > p1 ? q1 : (q1 < p1 ? -q1 : 0.f)));
+      }
+    }
+    float u0, u1;
+    f2_split(K0, u0, u1);
+    k0 = u0 + u1;
+    f2_split(K1, u0, u1);
+    k1 = u0 + u1;
+    f2_split(K2, u0, u1);
+    k2 = u0 + u1;
+  }
+  for (int i = tail0 + static_cast<int>(threadIdx.x); i < len; i += blockDim.x) {
     const float x = to_f32<T>(zt[i]), y = to_f32<T>(zs[i]);
     const float p = fast_exp2((x - Mt) * c) * inv_st;
     const float q = fast_exp2((y - Ms) * c) * inv_ss;
@@ -1425,7 +1511,36 @@ __global__ void __launch_bounds__(kDrawThreads)
   const float ka = a.alpha * a.grad_scale;
   const float kb = 0.5f * a.beta * a.grad_scale;
   float* g = a.grad + static_cast<size_t>(row) * V + lo;
-  for (int i = threadIdx.x; i < len; i += blockDim.x) {
+  if (kVec) {
+    const f32x2 ka2 = f2_make(ka, ka), kb2 = f2_make(kb, kb), sq2 = f2_make(sq, sq);
+    const bool g16 = (reinterpret_cast<uintptr_t>(g) & 15u) == 0;
+    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+      const uint4 a = vt[i], b = vs[i];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+      float out[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f32x2 x, y, p, q;
+        pq2(wa[j], wb[j], &x, &y, &p, &q);
+        float p0, p1, q0, q1;
+        f2_split(p, p0, p1);
+        f2_split(q, q0, q1);
+        const f32x2 sgn = f2_make(q0 > p0 ? 1.f : (q0 < p0 ? -1.f : 0.f),
+                                  q1 > p1 ? 1.f : (q1 < p1 ? -1.f : 0.f));
+        f2_split(f2_fma(f2_mul(kb2, q), f2_sub(sgn, sq2), f2_mul(ka2, f2_sub(q, p))), out[2 * j],
+                 out[2 * j + 1]);
+      }
+      float* gi = g + 8 * i;
+      if (g16) {
+        reinterpret_cast<float4*>(gi)[0] = make_float4(out[0], out[1], out[2], out[3]);
+        reinterpret_cast<float4*>(gi)[1] = make_float4(out[4], out[5], out[6], out[7]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) gi[j] = out[j];
+      }
+    }
+  }
+  for (int i = tail0 + static_cast<int>(threadIdx.x); i < len; i += blockDim.x) {
     const float p = fast_exp2((to_f32<T>(zt[i]) - Mt) * c) * inv_st;
     const float q = fast_exp2((to_f32<T>(zs[i]) - Ms) * c) * inv_ss;
     const float sgn = q > p ? 1.f : (q < p ? -1.f : 0.f);
