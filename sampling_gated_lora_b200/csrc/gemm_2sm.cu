@@ -88,20 +88,33 @@ static_assert(sizeof(PairParams) <= kLaunchParamBytes, "PairParams must fit Gemm
 // The work of one pair: its whole tiles, then its stream-K share cut at tile
 // boundaries. Each share spans at least one tile's worth of K-blocks (the
 // stream-K tiles number at least as many as the pairs), so a tile that two
-// shares cut has exactly two parts: the first (kb0 = 0, kb1 < nkb) belongs
-// to pair p, which finishes the tile with the partial sum of the second
-// (kb0 > 0, kb1 = nkb), the first part of pair p + 1's share. Pair p reaches
-// its part last in its share, pair p + 1 first in its own.
+// shares cut has exactly two parts: the first (kb0 = 0, kb1 < nkb) ends pair
+// p's share, the second (kb0 > 0, kb1 = nkb) begins pair p + 1's. A share is
+// walked as: the tiles wholly inside it, then its first part (the head, which
+// starts at K-block 0), then its second part (the tail) last. Every pair
+// enters its share at the same time, so at any moment the pairs stand at one
+// of a few common K offsets (the heads and whole tiles at the offset of the
+// clock, the tails at the clock minus a constant), and the tiles they run at
+// once share their x and W K-slices in L2; walked in index order instead, the
+// parts start at scattered K offsets and the same slices stream from HBM once
+// per pair. The head's pair hands its partial sum to pair p + 1, which adds it
+// when it finishes the tile with the tail, its last item (its stage ring is
+// idle then).
 struct WorkCursor {
   int tile;
-  long long it, it_end;
+  int phase;              // stream-K share: 0 whole tiles, 1 head, 2 tail, 3 done
+  long long it, it_end;   // the share [it, it_end) in K-block iterations
+  long long w, w_end;     // its whole tiles [w, w_end) (tile aligned)
 };
 
-__device__ __forceinline__ WorkCursor work_begin(const PairParams& p, int pair, int pairs) {
+__device__ __forceinline__ WorkCursor work_begin(const PairParams& p, int pair, int pairs, int nkb) {
   WorkCursor c;
   c.tile = pair;
+  c.phase = 0;
   c.it = p.sk_iters * pair / pairs;
   c.it_end = p.sk_iters * (pair + 1) / pairs;
+  c.w = (c.it + nkb - 1) / nkb * nkb;
+  c.w_end = max(c.w, c.it_end / nkb * nkb);
   return c;
 }
 
@@ -116,13 +129,37 @@ __device__ __forceinline__ bool work_next(const PairParams& p, int pairs, int nk
     return true;
   }
   if (c.it >= c.it_end) return false;
-  const long long rel = c.it / nkb;
-  const long long end = min((rel + 1) * nkb, c.it_end);
-  tile = p.dp_tiles + static_cast<int>(rel);
-  kb0 = static_cast<int>(c.it - rel * nkb);
-  kb1 = static_cast<int>(end - rel * nkb);
-  c.it = end;
-  return true;
+  if (c.phase == 0) {   // the tiles wholly inside the share
+    if (c.w < c.w_end) {
+      tile = p.dp_tiles + static_cast<int>(c.w / nkb);
+      kb0 = 0;
+      kb1 = nkb;
+      c.w += nkb;
+      return true;
+    }
+    c.phase = 1;
+  }
+  if (c.phase == 1) {   // the head: the first part of the tile the share ends in
+    c.phase = 2;
+    if (c.it_end % nkb != 0) {
+      const long long rel = c.it_end / nkb;
+      tile = p.dp_tiles + static_cast<int>(rel);
+      kb0 = 0;
+      kb1 = static_cast<int>(c.it_end - rel * nkb);
+      return true;
+    }
+  }
+  if (c.phase == 2) {   // the tail: the second part of the tile the share starts in
+    c.phase = 3;
+    if (c.it % nkb != 0) {
+      const long long rel = c.it / nkb;
+      tile = p.dp_tiles + static_cast<int>(rel);
+      kb0 = static_cast<int>(c.it - rel * nkb);
+      kb1 = nkb;
+      return true;
+    }
+  }
+  return false;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -222,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     bool first = true;
     bool waited = false;
-    WorkCursor wc = work_begin(p, pair, num_pairs);
+    WorkCursor wc = work_begin(p, pair, num_pairs, nkb);
     int tile, kb0, kb1;
     while (ok && work_next<kDown>(p, num_pairs, nkb, wc, tile, kb0, kb1)) {
       const TileId id = tile_id<kDown>(p, tile);
@@ -327,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t idesc_down = idesc_f32acc(kTile, kHalf, false);
     int it = 0, lt = 0;
     bool ok = true;
-    WorkCursor wc = work_begin(p, pair, num_pairs);
+    WorkCursor wc = work_begin(p, pair, num_pairs, nkb);
     int tile, kb0, kb1;
     for (; ok && work_next<kDown>(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
       const int b = lt & 1;
@@ -370,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int i = quarter * 32 + lane;
     int lt = 0;
-    WorkCursor wc = work_begin(p, pair, num_pairs);
+    WorkCursor wc = work_begin(p, pair, num_pairs, nkb);
     int tile, kb0, kb1;
     for (; work_next<kDown>(p, num_pairs, nkb, wc, tile, kb0, kb1); ++lt) {
       const int b = lt & 1;
@@ -413,11 +450,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         __threadfence();
         __syncwarp();
         if (lane == 0) counter_add_release(p.t_ready + mb, 1);
-      } else if (kb0 > 0) {
-        // second part of a stream-K tile: hand this warp's partial sum (its
-        // 32 rows, all 256 columns) to the pair that holds the first part
-        const int fi = ((pair - 1) * 2 + static_cast<int>(rank)) * 4 + quarter;
+      } else if (kb1 < nkb) {
+        // first part of a stream-K tile (this pair's head): hand this warp's
+        // partial sum (its 32 rows, all 256 columns) to the next pair, which
+        // finishes the tile. The partial sums are shared by the launches of a
+        // stream and the flags cleared by the preceding launch: both wait
+        // until that launch has finished.
+        const int fi = (pair * 2 + static_cast<int>(rank)) * 4 + quarter;
         float* part = p.sk_part + static_cast<size_t>(fi) * kSkWarpFloats;
+        pdl_wait();
         for (int c = 0; c < kTile; c += 16) {
           float v[16];
           tmem_ld16(trow + c, v);
@@ -427,15 +468,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_global();   // the reader copies them with the async proxy
         __threadfence();
         __syncwarp();
-        pdl_wait();   // the flags were cleared by the preceding launch
         if (lane == 0) flag_release(p.sk_flag + fi, 1);
       } else {
-        // first part of a stream-K tile (the pair's last work item, so the
-        // stage ring is idle): copy the next pair's partial sum for this
-        // warp's rows into shared memory, then add it
+        // a whole tile, or the second part of a stream-K tile (the pair's last
+        // work item, so the stage ring is idle): copy the previous pair's
+        // partial sum for this warp's rows into shared memory, then add it
         const float* part = nullptr;
-        if (kb1 < nkb) {   // (down tiles took the branch above)
-          const int fi = (pair * 2 + static_cast<int>(rank)) * 4 + quarter;
+        if (kb0 > 0) {
+          const int fi = ((pair - 1) * 2 + static_cast<int>(rank)) * 4 + quarter;
           pdl_wait();   // the flags were cleared by the preceding launch
           bool got = __all_sync(0xffffffffu, flag_wait(p.sk_flag + fi, 1));
           const uint32_t dst = smem_u32(smem + static_cast<uint32_t>(quarter) * kSkWarpBytes);
