@@ -59,6 +59,29 @@ def test_flat_rows_full_vocabulary(T):
     _check_parity(q, T, 23, 6, "bf16")
 
 
+def test_masked_chunk_and_nan_rows_full_vocabulary():
+    """V = 151936 bf16 rows (16-byte rows: the staged stats pass, 2048-id chunks): a row
+    whose ids [10240, 12288) (one whole chunk) are -inf draws like the oracle and never
+    inside the masked chunk; a row holding one NaN is flagged (draft -1, DEV_NAN) and its
+    neighbours still match the oracle."""
+    import torch
+    import sampling_gated_lora_b200 as U
+    gen = torch.Generator().manual_seed(44)
+    q = W.from_torch_bf16((2.0 * torch.randn((4, 8, 151936), generator=gen)).to(torch.bfloat16))
+    q[0, :, 10240:12288] = W.from_torch_bf16(torch.full((8, 2048), float("-inf")).to(torch.bfloat16))
+    ok_rows = [0, 1, 3]
+    g = _check_parity(q[ok_rows], 1.0, 29, 2, "bf16")
+    assert not np.any((g[0] >= 10240) & (g[0] < 12288))
+    q_nan = q.copy()
+    q_nan[2, 5, 77777] = W.from_torch_bf16(torch.tensor([float("nan")]).to(torch.bfloat16))[0]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    d = U.draft_sample(dev_tensor(q_nan, "bf16"), 1.0, 29, 2, dev_status=status).cpu().numpy()
+    assert d[2, 5] == -1 and int(status.item()) & U.DEV_NAN
+    assert np.all(np.delete(d[2], 5) >= 0)
+    # the other sequences draw exactly as in the same call without the NaN
+    np.testing.assert_array_equal(d[ok_rows], _gpu_draft(q, 1.0, 29, 2)[ok_rows])
+
+
 def _replicate(row_bits, n):
     import torch
     t = W.to_torch_bf16(row_bits, "cuda")
