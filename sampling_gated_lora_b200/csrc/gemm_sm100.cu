@@ -519,8 +519,9 @@ uno_status gemm_prepare(const GemmProblem& pb, GemmLaunch* out) {
 
   const int nkb = ga.nkb_main + (silu ? 2 : 1) * ga.nkb_r;
 
-  // Shared memory: ~96 KB (two or three CTAs per SM) for narrow decode tiles,
-  // ~200 KB otherwise.
+  // Shared memory: ~96 KB for narrow decode tiles, ~200 KB otherwise. (Shared
+  // memory would fit two or three narrow CTAs per SM; the swap variant's 142
+  // registers a thread allow two.)
   // Down-projections of large batches take the full ring: their cluster grid
   // is sized to one CTA per SM, and each CTA streams a long K-slice whose
   // rate is set by the bytes it keeps in flight.
